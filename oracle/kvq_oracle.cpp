@@ -1,0 +1,606 @@
+// Plain CPU oracle for the rotated token-wise INT4 paged KV cache.
+//
+// TEST INFRASTRUCTURE ONLY. Nothing in the product path may include, link or
+// call this file: only tests/, the smoke check and the benchmark's CPU
+// baseline use it. It shares no source, header, table or helper with the CUDA
+// library; the two meet only through seeded inputs generated elsewhere.
+//
+// What it follows:
+//  * "SAW-INT4: System-Aware 4-Bit KV-Cache Quantization for Real-World LLM
+//    Serving", Summary and Method: token-wise INT4 quantization of the KV cache
+//    behind a block-diagonal Hadamard rotation, fused into paged KV-cache
+//    layouts.
+//  * "UltraQuant: 4-bit KV caching for long agents" (Traditional Chinese page),
+//    section on how the method works: a Walsh-Hadamard rotation of the K/V
+//    vectors spreads outlier channels before quantization.
+//  * "IsoQuant: Hardware-Aligned SO(4) Isoclinic Rotations for LLM KV Cache
+//    Compression", Abstract: each 4-D block is a quaternion v and is mapped to
+//    qL * v * conj(qR).
+// Where the pages leave a step open, the reading taken is the one written
+// beside the step below; the same readings are listed in the design notes.
+//
+// Build: g++ -O2 -ffp-contract=off -fno-fast-math -frounding-math -fopenmp
+// -shared -fPIC. No fused multiply-add is formed implicitly
+// (-ffp-contract=off), so every float expression below is a sequence of
+// IEEE-754 binary32 operations with round-to-nearest-even, exactly as
+// written; the two operations that round upward switch the hardware rounding
+// mode around themselves (-frounding-math keeps the compiler from moving or
+// folding them).
+
+#include <cfenv>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <vector>
+#include <algorithm>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+extern "C" {
+
+// ---------------------------------------------------------------------------
+// IEEE-754 binary16, written from the format definition (1 sign bit, 5
+// exponent bits with bias 15, 10 fraction bits; subnormals have quantum 2^-24).
+// ---------------------------------------------------------------------------
+
+double orc_half_to_double(uint16_t h) {
+  const int sign = h >> 15;
+  const int e = (h >> 10) & 0x1f;
+  const int m = h & 0x3ff;
+  double v;
+  if (e == 0) {
+    v = std::ldexp((double)m, -24);
+  } else if (e == 31) {
+    v = m ? NAN : INFINITY;
+  } else {
+    v = std::ldexp((double)(1024 + m), e - 25);
+  }
+  return sign ? -v : v;
+}
+
+// Rounding modes for binary32 -> binary16.
+enum { ORC_RN = 0, ORC_RD = 1, ORC_RU = 2 };
+
+// Converts a value to binary16 bits under one of three rounding modes: to
+// nearest (ties to even), toward -inf, toward +inf. All double arithmetic
+// below is exact: x is only scaled by powers of two, floored, subtracted from
+// its own floor and compared.
+uint16_t orc_double_to_half(double x, int mode) {
+  if (std::isnan(x)) return 0x7e00;
+  const bool neg = std::signbit(x);
+  const uint16_t sign = neg ? 0x8000 : 0;
+  if (std::isinf(x)) return sign | 0x7c00;
+  double a = std::fabs(x);
+  if (a == 0.0) return sign;
+  // Direction in which the MAGNITUDE moves: toward -inf on a negative number
+  // makes the magnitude larger.
+  enum { NEAREST, DOWN, UP } dir = NEAREST;
+  if (mode == ORC_RD) dir = neg ? UP : DOWN;
+  if (mode == ORC_RU) dir = neg ? DOWN : UP;
+
+  int e2;
+  std::frexp(a, &e2);              // a = f * 2^e2 with f in [0.5, 1)
+  int E = e2 - 1;                  // a in [2^E, 2^(E+1))
+  if (E < -14) E = -14;            // subnormals share the quantum of binade -14
+  const double q = std::ldexp(1.0, E - 10);  // spacing of binary16 values here
+  const double n = a / q;          // exact
+  const double fl = std::floor(n);
+  double r;
+  if (dir == DOWN) {
+    r = fl;
+  } else if (dir == UP) {
+    r = (n == fl) ? fl : fl + 1.0;
+  } else {
+    const double frac = n - fl;
+    if (frac > 0.5) r = fl + 1.0;
+    else if (frac < 0.5) r = fl;
+    else r = (std::fmod(fl, 2.0) == 0.0) ? fl : fl + 1.0;
+  }
+  const double v = r * q;
+  if (v > 65504.0) {               // past the largest finite binary16
+    if (dir == DOWN) return sign | 0x7bff;
+    return sign | 0x7c00;          // nearest: only reached when a >= 65520
+  }
+  // r in [0, 2048]; r == 2048 carries into the next binade naturally.
+  const int bits = ((E + 15) << 10) + ((int)r - 1024);
+  return (uint16_t)(sign | (uint16_t)bits);
+}
+
+uint16_t orc_float_to_half(float x, int mode) { return orc_double_to_half((double)x, mode); }
+
+float orc_half_to_float(uint16_t h) { return (float)orc_half_to_double(h); }
+
+// ---------------------------------------------------------------------------
+// Block-diagonal Walsh-Hadamard rotation (SAW-INT4 Summary/Method; UltraQuant
+// method section). Blocks are contiguous runs of b channels; within a block
+// y = (1/sqrt(b)) * H_b * x with H_b the Sylvester Hadamard matrix,
+// H_b[i][j] = (-1)^popcount(i & j). It is computed by the fast transform:
+// stages h = 1, 2, 4, ..., b/2 in ascending order; at each stage every pair
+// (i, i+h) with (i & h) == 0 becomes (x_i + x_{i+h}, x_i - x_{i+h}), each one
+// binary32 operation; then every element is multiplied by c_b, the binary32
+// value nearest 1/sqrt(b).
+// ---------------------------------------------------------------------------
+
+float orc_hadamard_scale(int b) {
+  // 1/sqrt(b) for b a power of two: 2^(-k) when b = 4^k, sqrt(2) * 2^(-k)
+  // when b = 2 * 4^(k-1) (i.e. b = 2^(2k-1)). sqrt(2.0) is correctly rounded
+  // in double and lies far from a binary32 rounding boundary, so this is the
+  // binary32 value nearest 1/sqrt(b).
+  int lg = 0;
+  while ((1 << lg) < b) ++lg;
+  if (lg % 2 == 0) return std::ldexp(1.0f, -lg / 2);
+  return (float)std::ldexp(std::sqrt(2.0), -(lg + 1) / 2);
+}
+
+void orc_fwht_unscaled(float* x, int b) {
+  for (int h = 1; h < b; h <<= 1) {
+    for (int i = 0; i < b; ++i) {
+      if ((i & h) == 0) {
+        const float a = x[i];
+        const float c = x[i + h];
+        x[i] = a + c;
+        x[i + h] = a - c;
+      }
+    }
+  }
+}
+
+void orc_rotate_hadamard_f32(float* x, int d, int b) {
+  const float cb = orc_hadamard_scale(b);
+  for (int t = 0; t < d; t += b) {
+    orc_fwht_unscaled(x + t, b);
+    for (int i = 0; i < b; ++i) x[t + i] = x[t + i] * cb;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Quaternion block rotation (IsoQuant Abstract: T(v) = qL v conj(qR), full
+// SO(4) variant). Channels 4j..4j+3 of a head are the quaternion
+// (w, x, y, z). The table holds, per block j, qL[j] then qR[j], each as
+// (w, x, y, z) in binary32. Each component of a Hamilton product a*b is the
+// textbook formula evaluated as fma(t3, fma(t2, fma(t1, t0))) with t0 a plain
+// product and the terms in this order:
+//   w: ( a.w b.w, -a.x b.x, -a.y b.y, -a.z b.z)
+//   x: ( a.w b.x,  a.x b.w,  a.y b.z, -a.z b.y)
+//   y: ( a.w b.y, -a.x b.z,  a.y b.w,  a.z b.x)
+//   z: ( a.w b.z,  a.x b.y, -a.y b.x,  a.z b.w)
+// ---------------------------------------------------------------------------
+
+void orc_hamilton_f32(const float* a, const float* b, float* out) {
+  const float aw = a[0], ax = a[1], ay = a[2], az = a[3];
+  const float bw = b[0], bx = b[1], by = b[2], bz = b[3];
+  float w = aw * bw;
+  w = std::fma(-ax, bx, w);
+  w = std::fma(-ay, by, w);
+  w = std::fma(-az, bz, w);
+  float x = aw * bx;
+  x = std::fma(ax, bw, x);
+  x = std::fma(ay, bz, x);
+  x = std::fma(-az, by, x);
+  float y = aw * by;
+  y = std::fma(-ax, bz, y);
+  y = std::fma(ay, bw, y);
+  y = std::fma(az, bx, y);
+  float z = aw * bz;
+  z = std::fma(ax, by, z);
+  z = std::fma(-ay, bx, z);
+  z = std::fma(az, bw, z);
+  out[0] = w; out[1] = x; out[2] = y; out[3] = z;
+}
+
+void orc_rotate_quat_f32(float* x, int d, const float* quat) {
+  for (int j = 0; j < d / 4; ++j) {
+    const float* qL = quat + j * 8;
+    const float* qR = quat + j * 8 + 4;
+    const float qRc[4] = {qR[0], -qR[1], -qR[2], -qR[3]};
+    float t[4];
+    orc_hamilton_f32(qL, x + 4 * j, t);
+    orc_hamilton_f32(t, qRc, x + 4 * j);
+  }
+}
+
+// Rotation kinds (same numbering as the library's public enum, restated).
+enum { ORC_ROT_NONE = 0, ORC_ROT_HADAMARD = 1, ORC_ROT_QUAT = 2 };
+
+void orc_rotate_f32(float* x, int d, int kind, int b, const float* quat) {
+  if (kind == ORC_ROT_HADAMARD) orc_rotate_hadamard_f32(x, d, b);
+  else if (kind == ORC_ROT_QUAT) orc_rotate_quat_f32(x, d, quat);
+}
+
+// ---------------------------------------------------------------------------
+// Token-wise asymmetric INT4 quantizer (SAW-INT4 Summary: "token-wise INT4";
+// one scale and one zero-point per (token, head) row).
+// Readings: the minimum is stored rounded toward -inf; the scale is
+// (max - m16)/15 with the binary32 subtraction, the binary32 division and the
+// final binary16 conversion all rounded toward +inf, so every x lies in
+// [m16, m16 + 15 s16] exactly; the code is round-half-even of
+// RN(RN(x - m16) * RN(1/s16)) clamped to [0, 15] (the clamp never acts given
+// that range, and is kept as the definition); a row
+// with max == m16 has s16 = 0 and all codes 0; -0 is normalised to +0 in both
+// the minimum and the maximum so the stored bits do not depend on reduction
+// order.
+// ---------------------------------------------------------------------------
+
+// Binary32 subtraction and division rounded toward +inf (IEEE-754 directed
+// rounding, done by the FPU in that mode).
+float orc_sub_ru(float a, float b) {
+  const int old = std::fegetround();
+  std::fesetround(FE_UPWARD);
+  volatile float va = a, vb = b;
+  volatile float r = va - vb;
+  std::fesetround(old);
+  return r;
+}
+
+float orc_div_ru(float a, float b) {
+  const int old = std::fegetround();
+  std::fesetround(FE_UPWARD);
+  volatile float va = a, vb = b;
+  volatile float r = va / vb;
+  std::fesetround(old);
+  return r;
+}
+
+static float rint_half_even(float t) {
+  const float fl = std::floor(t);
+  const float fr = t - fl;  // exact for |t| < 2^23
+  if (fr > 0.5f) return fl + 1.0f;
+  if (fr < 0.5f) return fl;
+  return (std::fmod(fl, 2.0f) == 0.0f) ? fl : fl + 1.0f;
+}
+
+void orc_quantize_row(const float* y, int d, uint8_t* codes,
+                      uint16_t* s16_out, uint16_t* m16_out) {
+  float mn = y[0], mx = y[0];
+  for (int i = 1; i < d; ++i) {
+    if (y[i] < mn) mn = y[i];
+    if (y[i] > mx) mx = y[i];
+  }
+  mn = mn + 0.0f;
+  mx = mx + 0.0f;
+  const uint16_t m16 = orc_float_to_half(mn, ORC_RD);
+  const float m = orc_half_to_float(m16);
+  const float diff = orc_sub_ru(mx, m);
+  const float s32 = orc_div_ru(diff, 15.0f);
+  const uint16_t s16 = orc_float_to_half(s32, ORC_RU);
+  const float s = orc_half_to_float(s16);
+  std::vector<int> c(d, 0);
+  if (s != 0.0f) {
+    const float inv = 1.0f / s;
+    for (int i = 0; i < d; ++i) {
+      const float t0 = y[i] - m;
+      const float t1 = t0 * inv;
+      float r = rint_half_even(t1);
+      if (r < 0.0f) r = 0.0f;
+      if (r > 15.0f) r = 15.0f;
+      c[i] = (int)r;
+    }
+  }
+  // Two 4-bit codes per byte, the even channel in the low nibble.
+  for (int k = 0; k < d / 2; ++k)
+    codes[k] = (uint8_t)(c[2 * k] | (c[2 * k + 1] << 4));
+  *s16_out = s16;
+  *m16_out = m16;
+}
+
+// Unpacks one row of codes (d/2 bytes) into d integers.
+void orc_unpack_row(const uint8_t* codes, int d, int* c) {
+  for (int k = 0; k < d / 2; ++k) {
+    c[2 * k] = codes[k] & 0xf;
+    c[2 * k + 1] = codes[k] >> 4;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Paged placement (SAW-INT4 Summary: the quantizer writes straight into paged
+// KV-cache layouts). Reading: pools are [page][kv_head][slot][d/2] bytes of
+// codes and [page][kv_head][slot] pairs (s16, m16) of binary16 (scale first);
+// K and V have separate pools; page = block_table[seq][pos / P], slot =
+// pos % P.
+// Error flags (OR-ed into *err): 1 = block-table entry outside [0, NP),
+// 2 = position outside the table (pos < 0 or pos / P >= bt_stride),
+// 4 = sequence index outside [0, num_seqs), 8 = sequence length invalid.
+// ---------------------------------------------------------------------------
+
+enum { ORC_ERR_PAGE = 1, ORC_ERR_POS = 2, ORC_ERR_SEQ = 4, ORC_ERR_LEN = 8 };
+
+void orc_quantize_append(int d, int H, int P, int NP, int rot_kind, int rot_block,
+                         const float* quat, int T, const uint16_t* k, const uint16_t* v,
+                         int64_t tok_stride, const int32_t* token_seq,
+                         const int32_t* token_pos, int num_seqs,
+                         const int32_t* block_table, int bt_stride, uint8_t* k_codes,
+                         uint16_t* k_params, uint8_t* v_codes, uint16_t* v_params,
+                         int32_t* err) {
+  int32_t flags = 0;
+  std::vector<float> row(d);
+  for (int t = 0; t < T; ++t) {
+    const int seq = token_seq[t];
+    if (seq < 0) continue;
+    if (seq >= num_seqs) { flags |= ORC_ERR_SEQ; continue; }
+    const int pos = token_pos[t];
+    if (pos < 0 || pos / P >= bt_stride) { flags |= ORC_ERR_POS; continue; }
+    const int page = block_table[(int64_t)seq * bt_stride + pos / P];
+    if (page < 0 || page >= NP) { flags |= ORC_ERR_PAGE; continue; }
+    const int slot = pos % P;
+    for (int kv = 0; kv < 2; ++kv) {
+      const uint16_t* src = kv == 0 ? k : v;
+      uint8_t* codes = kv == 0 ? k_codes : v_codes;
+      uint16_t* params = kv == 0 ? k_params : v_params;
+      for (int h = 0; h < H; ++h) {
+        const uint16_t* x = src + (int64_t)t * tok_stride + (int64_t)h * d;
+        for (int i = 0; i < d; ++i) row[i] = orc_half_to_float(x[i]);
+        orc_rotate_f32(row.data(), d, rot_kind, rot_block, quat);
+        const int64_t r = ((int64_t)page * H + h) * P + slot;
+        uint16_t s16, m16;
+        orc_quantize_row(row.data(), d, codes + r * (d / 2), &s16, &m16);
+        params[2 * r] = s16;
+        params[2 * r + 1] = m16;
+      }
+    }
+  }
+  *err |= flags;
+}
+
+// ---------------------------------------------------------------------------
+// Inverse rotation in double precision, used after attention and by the
+// dense export. Hadamard: R is symmetric and R R = I for the exact
+// orthonormal R, so R^-1 = R (computed with the exact 1/sqrt(b)).
+// Quaternion: T(v) = qL v conj(qR) is inverted by
+// v = qL^-1 w conj(qR)^-1 = (conj(qL)/|qL|^2) w (qR/|qR|^2).
+// ---------------------------------------------------------------------------
+
+static void hamilton_f64(const double* a, const double* b, double* o) {
+  o[0] = a[0] * b[0] - a[1] * b[1] - a[2] * b[2] - a[3] * b[3];
+  o[1] = a[0] * b[1] + a[1] * b[0] + a[2] * b[3] - a[3] * b[2];
+  o[2] = a[0] * b[2] - a[1] * b[3] + a[2] * b[0] + a[3] * b[1];
+  o[3] = a[0] * b[3] + a[1] * b[2] - a[2] * b[1] + a[3] * b[0];
+}
+
+void orc_rotate_f64(double* x, int d, int kind, int b, const float* quat) {
+  if (kind == ORC_ROT_HADAMARD) {
+    const double cb = 1.0 / std::sqrt((double)b);
+    std::vector<double> y(b);
+    for (int t = 0; t < d; t += b) {
+      for (int i = 0; i < b; ++i) {
+        double acc = 0.0;
+        for (int j = 0; j < b; ++j)
+          acc += (__builtin_popcount(i & j) & 1) ? -x[t + j] : x[t + j];
+        y[i] = acc * cb;
+      }
+      for (int i = 0; i < b; ++i) x[t + i] = y[i];
+    }
+  } else if (kind == ORC_ROT_QUAT) {
+    for (int j = 0; j < d / 4; ++j) {
+      const double qL[4] = {quat[8 * j], quat[8 * j + 1], quat[8 * j + 2], quat[8 * j + 3]};
+      const double qR[4] = {quat[8 * j + 4], -(double)quat[8 * j + 5], -(double)quat[8 * j + 6],
+                            -(double)quat[8 * j + 7]};
+      double t[4];
+      hamilton_f64(qL, x + 4 * j, t);
+      hamilton_f64(t, qR, x + 4 * j);
+    }
+  }
+}
+
+void orc_unrotate_f64(double* x, int d, int kind, int b, const float* quat) {
+  if (kind == ORC_ROT_HADAMARD) {
+    orc_rotate_f64(x, d, kind, b, quat);  // R^-1 = R
+  } else if (kind == ORC_ROT_QUAT) {
+    for (int j = 0; j < d / 4; ++j) {
+      const double L[4] = {quat[8 * j], quat[8 * j + 1], quat[8 * j + 2], quat[8 * j + 3]};
+      const double R[4] = {quat[8 * j + 4], quat[8 * j + 5], quat[8 * j + 6], quat[8 * j + 7]};
+      const double nL = L[0] * L[0] + L[1] * L[1] + L[2] * L[2] + L[3] * L[3];
+      const double nR = R[0] * R[0] + R[1] * R[1] + R[2] * R[2] + R[3] * R[3];
+      const double Linv[4] = {L[0] / nL, -L[1] / nL, -L[2] / nL, -L[3] / nL};
+      const double Rinv[4] = {R[0] / nR, R[1] / nR, R[2] / nR, R[3] / nR};  // (conj qR)^-1
+      double t[4];
+      hamilton_f64(Linv, x + 4 * j, t);
+      hamilton_f64(t, Rinv, x + 4 * j);
+    }
+  }
+}
+
+// Dequantized value of one stored element: c * s16 + m16 (exact in double).
+static inline double deq(int c, uint16_t s16, uint16_t m16) {
+  return (double)c * orc_half_to_double(s16) + orc_half_to_double(m16);
+}
+
+// Dense export of cached tokens: out[s][j][h][:] for j < seq_lens[s]
+// (rows at or past seq_lens[s] are left untouched). Values are computed in
+// double, optionally un-rotated, then rounded once to binary32 (out_fp32) or
+// to binary16 with round-to-nearest-even.
+void orc_dequantize_pages(int d, int H, int P, int NP, int rot_kind, int rot_block,
+                          const float* quat, int S, const int32_t* seq_lens,
+                          int max_seq_len, const int32_t* block_table, int bt_stride,
+                          const uint8_t* codes, const uint16_t* params, int unrotate,
+                          int out_fp32, void* out, int32_t* err) {
+  int32_t flags = 0;
+  std::vector<int> c(d);
+  std::vector<double> x(d);
+  for (int s = 0; s < S; ++s) {
+    int L = seq_lens[s];
+    if (L < 0 || L > max_seq_len || (L + P - 1) / P > bt_stride) { flags |= ORC_ERR_LEN; continue; }
+    for (int j = 0; j < L; ++j) {
+      const int page = block_table[(int64_t)s * bt_stride + j / P];
+      if (page < 0 || page >= NP) { flags |= ORC_ERR_PAGE; continue; }
+      for (int h = 0; h < H; ++h) {
+        const int64_t r = ((int64_t)page * H + h) * P + j % P;
+        orc_unpack_row(codes + r * (d / 2), d, c.data());
+        for (int i = 0; i < d; ++i) x[i] = deq(c[i], params[2 * r], params[2 * r + 1]);
+        if (unrotate) orc_unrotate_f64(x.data(), d, rot_kind, rot_block, quat);
+        const int64_t o = (((int64_t)s * max_seq_len + j) * H + h) * d;
+        if (out_fp32) {
+          float* of = (float*)out;
+          for (int i = 0; i < d; ++i) of[o + i] = (float)x[i];
+        } else {
+          uint16_t* oh = (uint16_t*)out;
+          for (int i = 0; i < d; ++i) oh[o + i] = orc_double_to_half(x[i], ORC_RN);
+        }
+      }
+    }
+  }
+  *err |= flags;
+}
+
+
+// ---------------------------------------------------------------------------
+// Decode attention over the INT4 pages (SAW-INT4 Key takeaway: the rotated
+// INT4 cache must serve fused attention). Everything is in double precision:
+// for sequence s and query head g (KV head h = g / (Hq/H), contiguous
+// grouping),
+//   qhat = R q_g, z_j = sm_scale * (qhat . khat_j) for every cached j < L_s,
+//   p = softmax(z) (maximum subtracted first), otilde = sum_j p_j vhat_j,
+//   o = R^-1 otilde,
+// where khat_j, vhat_j are the dequantized rotated rows. Because R is
+// orthogonal, qhat . (R k) = q . k: the query is rotated by the same R that
+// the keys were quantized behind. A page whose block-table entry is outside
+// [0, NP) contributes no token and sets flag 1; an invalid length sets flag 8
+// and gives a zero output; a sequence with no token gives a zero output.
+// ---------------------------------------------------------------------------
+
+void orc_paged_decode_attn(int d, int H, int P, int NP, int rot_kind, int rot_block,
+                           const float* quat, int S, int Hq, const uint16_t* q,
+                           const int32_t* seq_lens, int max_seq_len,
+                           const int32_t* block_table, int bt_stride, double sm_scale,
+                           const uint8_t* k_codes, const uint16_t* k_params,
+                           const uint8_t* v_codes, const uint16_t* v_params, double* out,
+                           int32_t* err) {
+  const int G = Hq / H;
+  int32_t flags = 0;
+#pragma omp parallel for schedule(dynamic) reduction(| : flags)
+  for (int sg = 0; sg < S * Hq; ++sg) {
+    const int s = sg / Hq, g = sg % Hq, h = g / G;
+    double* o = out + (int64_t)sg * d;
+    for (int i = 0; i < d; ++i) o[i] = 0.0;
+    const int L = seq_lens[s];
+    if (L < 0 || L > max_seq_len || (L + P - 1) / P > bt_stride) { flags |= ORC_ERR_LEN; continue; }
+    std::vector<double> qh(d), kh(d), acc(d, 0.0);
+    std::vector<int> c(d);
+    for (int i = 0; i < d; ++i) qh[i] = orc_half_to_double(q[(int64_t)sg * d + i]);
+    orc_rotate_f64(qh.data(), d, rot_kind, rot_block, quat);
+    std::vector<double> z;
+    std::vector<int64_t> rows;
+    z.reserve(L);
+    rows.reserve(L);
+    for (int j = 0; j < L; ++j) {
+      const int page = block_table[(int64_t)s * bt_stride + j / P];
+      if (page < 0 || page >= NP) { flags |= ORC_ERR_PAGE; continue; }
+      const int64_t r = ((int64_t)page * H + h) * P + j % P;
+      orc_unpack_row(k_codes + r * (d / 2), d, c.data());
+      double dot = 0.0;
+      for (int i = 0; i < d; ++i) dot += qh[i] * deq(c[i], k_params[2 * r], k_params[2 * r + 1]);
+      z.push_back(sm_scale * dot);
+      rows.push_back(r);
+    }
+    if (z.empty()) continue;
+    const double zmax = *std::max_element(z.begin(), z.end());
+    double denom = 0.0;
+    for (size_t j = 0; j < z.size(); ++j) { z[j] = std::exp(z[j] - zmax); denom += z[j]; }
+    for (size_t j = 0; j < z.size(); ++j) {
+      const int64_t r = rows[j];
+      orc_unpack_row(v_codes + r * (d / 2), d, c.data());
+      const double p = z[j] / denom;
+      for (int i = 0; i < d; ++i) acc[i] += p * deq(c[i], v_params[2 * r], v_params[2 * r + 1]);
+    }
+    orc_unrotate_f64(acc.data(), d, rot_kind, rot_block, quat);
+    for (int i = 0; i < d; ++i) o[i] = acc[i];
+  }
+  *err |= flags;
+}
+
+// The same attention over an unquantized binary16 paged cache
+// ([page][kv_head][slot][d]), without rotation: the full-precision baseline
+// the INT4 cache is compared against.
+void orc_paged_decode_attn_fp16(int d, int H, int P, int NP, int S, int Hq, const uint16_t* q,
+                                const int32_t* seq_lens, int max_seq_len,
+                                const int32_t* block_table, int bt_stride, double sm_scale,
+                                const uint16_t* k16, const uint16_t* v16, double* out,
+                                int32_t* err) {
+  const int G = Hq / H;
+  int32_t flags = 0;
+#pragma omp parallel for schedule(dynamic) reduction(| : flags)
+  for (int sg = 0; sg < S * Hq; ++sg) {
+    const int s = sg / Hq, g = sg % Hq, h = g / G;
+    double* o = out + (int64_t)sg * d;
+    for (int i = 0; i < d; ++i) o[i] = 0.0;
+    const int L = seq_lens[s];
+    if (L < 0 || L > max_seq_len || (L + P - 1) / P > bt_stride) { flags |= ORC_ERR_LEN; continue; }
+    std::vector<double> qh(d), acc(d, 0.0);
+    for (int i = 0; i < d; ++i) qh[i] = orc_half_to_double(q[(int64_t)sg * d + i]);
+    std::vector<double> z;
+    std::vector<int64_t> rows;
+    for (int j = 0; j < L; ++j) {
+      const int page = block_table[(int64_t)s * bt_stride + j / P];
+      if (page < 0 || page >= NP) { flags |= ORC_ERR_PAGE; continue; }
+      const int64_t r = ((int64_t)page * H + h) * P + j % P;
+      double dot = 0.0;
+      for (int i = 0; i < d; ++i) dot += qh[i] * orc_half_to_double(k16[r * d + i]);
+      z.push_back(sm_scale * dot);
+      rows.push_back(r);
+    }
+    if (z.empty()) continue;
+    const double zmax = *std::max_element(z.begin(), z.end());
+    double denom = 0.0;
+    for (size_t j = 0; j < z.size(); ++j) { z[j] = std::exp(z[j] - zmax); denom += z[j]; }
+    for (size_t j = 0; j < z.size(); ++j) {
+      const double p = z[j] / denom;
+      for (int i = 0; i < d; ++i) acc[i] += p * orc_half_to_double(v16[rows[j] * d + i]);
+    }
+    for (int i = 0; i < d; ++i) o[i] = acc[i];
+  }
+  *err |= flags;
+}
+
+// Number of threads the parallel loops above use (1 without OpenMP).
+int orc_num_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+void orc_set_num_threads(int n) {
+#ifdef _OPENMP
+  if (n > 0) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
+// ---------------------------------------------------------------------------
+// Row-array helpers for the Python wrapper (loops over the functions above).
+// ---------------------------------------------------------------------------
+
+void orc_float_to_half_array(const float* x, int64_t n, int mode, uint16_t* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_float_to_half(x[i], mode);
+}
+
+void orc_double_to_half_array(const double* x, int64_t n, int mode, uint16_t* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_double_to_half(x[i], mode);
+}
+
+void orc_half_to_double_array(const uint16_t* h, int64_t n, double* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_half_to_double(h[i]);
+}
+
+void orc_rotate_rows_f32(float* x, int64_t rows, int d, int kind, int b, const float* quat) {
+  for (int64_t r = 0; r < rows; ++r) orc_rotate_f32(x + r * d, d, kind, b, quat);
+}
+
+void orc_rotate_rows_f64(double* x, int64_t rows, int d, int kind, int b, const float* quat) {
+  for (int64_t r = 0; r < rows; ++r) orc_rotate_f64(x + r * d, d, kind, b, quat);
+}
+
+void orc_unrotate_rows_f64(double* x, int64_t rows, int d, int kind, int b, const float* quat) {
+  for (int64_t r = 0; r < rows; ++r) orc_unrotate_f64(x + r * d, d, kind, b, quat);
+}
+
+void orc_quantize_rows(const float* y, int64_t rows, int d, uint8_t* codes, uint16_t* s16,
+                       uint16_t* m16) {
+  for (int64_t r = 0; r < rows; ++r)
+    orc_quantize_row(y + r * d, d, codes + r * (d / 2), s16 + r, m16 + r);
+}
+
+}  // extern "C"
