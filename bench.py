@@ -1,0 +1,440 @@
+"""Benchmark of the rotated INT4 paged KV-cache hot path on B200.
+
+One step = one pass of the whole path over one batch of the Llama-3-8B-shaped
+decode layer (32 sequences x 4096 cached tokens, 8 KV heads, 32 query heads,
+head_dim 128, Hadamard block 64, page 16, shuffled block table): append one
+new token per sequence (fused rotate -> INT4 -> pack -> page scatter), then
+paged decode attention over the 4097 cached INT4 tokens. Inputs are seeded
+synthetic draws of that shape (no dataset exists for this).
+
+The device-timed region covers exactly --steps steps between a barrier and a
+synchronize on both sides; consecutive steps alternate between two cache
+replicas (2 x 143 MB > the 126 MB L2), so every step reads its pages from HBM.
+Also measured (outside that region): the bulk prefill append of the same
+layer (131072 tokens) in GB/s.
+
+Multi-GPU: one process per GPU (torchrun); every rank runs an independent
+shard of sequences (weak scaling, no collective on the data path); the
+reported time is the max over ranks.
+
+--impl reference times the CPU oracle (the only reference this method has) on
+rank 0 on a bounded sample of the same workload.
+
+Prints one JSON line.
+"""
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+WORKLOAD = "llama8b"
+METRIC = "INT4 paged decode-attn tokens/s (append + decode step, one layer)"
+UNIT = "tokens/s"
+BYTES_PER_TOKEN_HEAD = 136  # decode: 2 * (64 code bytes + 4 param bytes), head_dim 128
+APPEND_BYTES_PER_TOKEN_HEAD = 648  # append: 2 * 256 B read + 2 * 68 B written
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
+    return ap.parse_args()
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, world, device):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x, world, device):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "20"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        if not rows:
+            return None
+        sm = np.array([float(r[1]) for r in rows if r[1].replace(".", "").isdigit()])
+        mx = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        loaded = sm[sm > 0.5 * mx] if sm.size else sm
+        med = float(np.median(loaded)) if loaded.size else (float(np.median(sm)) if sm.size else None)
+        return {"sm_mhz": med, "sm_max_mhz": mx, "reasons": reasons, "samples": int(sm.size)}
+
+
+# ---------------------------------------------------------------- peaks
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_traffic(kernel):
+    """DRAM bytes per launch from the committed ncu summary, valid only while
+    the kernel's source is unchanged since the capture (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    d = json.load(open(path)).get(kernel)
+    if not d:
+        return None
+    src = os.path.join(ROOT, d["source"])
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return float(d["bytes_per_launch"]) if h == d["source_sha256_16"] else None
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args, world, rank, local):
+    from bit_rotated_kv_block_b200 import kvq, workloads
+    from bit_rotated_kv_block_b200 import build as kbuild
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if rank == 0 or not os.path.exists(kbuild.LIB):
+        kbuild.build()
+    barrier(world)
+    kvq.lib()
+    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(device)
+
+    # each rank owns an independent shard of 32 sequences (seeded per rank)
+    w = workloads.llama8b(seed=args.seed + 1000 * rank)
+    S, H, Hq, d, ctx = w.S, w.H, w.Hq, w.d, int(w.seq_lens[0])
+    k, v, ts, tp = w.prefill_tokens()
+    K, V, TS, TP = dev(k), dev(v), dev(ts), dev(tp)
+    BT = dev(w.block_table)
+    caches = []
+    for rep in range(2):
+        c = kvq.Cache(w.d, w.H, w.P, w.NP, w.rot_kind, w.rot_block)
+        kc, kp = c.new_pools(device=device, fill=0)
+        vc, vp = c.new_pools(device=device, fill=0)
+        kvq.quantize_append(c, K, V, TS, TP, BT, kc, kp, vc, vp)
+        caches.append((c, kc, kp, vc, vp))
+    torch.cuda.synchronize()
+
+    # bulk prefill append throughput (131072 tokens, inputs 268 MB > L2)
+    c0, kc0, kp0, vc0, vp0 = caches[0]
+    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(8)]
+    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(8)]
+    for i in range(3):
+        kvq.quantize_append(c0, K, V, TS, TP, BT, kc0, kp0, vc0, vp0)
+    for i in range(8):
+        e0[i].record()
+        kvq.quantize_append(c0, K, V, TS, TP, BT, kc0, kp0, vc0, vp0)
+        e1[i].record()
+    torch.cuda.synchronize()
+    t_app = float(np.median([a.elapsed_time(b) for a, b in zip(e0, e1)])) * 1e-3
+    app_bytes = len(ts) * H * APPEND_BYTES_PER_TOKEN_HEAD
+    del K, V
+
+    # step inputs: one new token per sequence at position ctx, and queries
+    ks, vs, sts, stp = w.step_tokens(0)
+    q = w.queries(0)
+    lens = (w.seq_lens + 1).astype(np.int32)
+    SK, SV, STS, STP, Q, LENS = dev(ks), dev(vs), dev(sts), dev(stp), dev(q), dev(lens)
+    L = int(lens.max())
+    out = torch.empty((S, Hq, d), dtype=torch.float32, device=device)
+    ws = torch.zeros(kvq.decode_workspace_bytes(c0, S, Hq, L), dtype=torch.uint8, device=device)
+    err = torch.zeros(1, dtype=torch.int32, device=device)
+    stream = torch.cuda.current_stream()
+    launches_per_step = 1 + 3
+
+    def step(i):
+        c, kc, kp, vc, vp = caches[i % 2]
+        kvq.quantize_append(c, SK, SV, STS, STP, BT, kc, kp, vc, vp, err=err)
+        kvq.paged_decode_attn(c, Q, LENS, L, BT, kc, kp, vc, vp, out=out, workspace=ws, err=err)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+
+    steps = args.steps
+    dec0 = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    dec1 = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for i in range(steps):
+        c, kc, kp, vc, vp = caches[i % 2]
+        kvq.quantize_append(c, SK, SV, STS, STP, BT, kc, kp, vc, vp, err=err)
+        dec0[i].record(stream)
+        kvq.paged_decode_attn(c, Q, LENS, L, BT, kc, kp, vc, vp, out=out, workspace=ws, err=err)
+        dec1[i].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    elapsed = t0.elapsed_time(t1) * 1e-3
+    t_dec = float(np.mean([a.elapsed_time(b) for a, b in zip(dec0, dec1)])) * 1e-3
+    assert int(err.item()) == 0, f"device error flags {int(err.item())}"
+
+    elapsed_max = max_over_ranks(elapsed, world, device)
+    units = sum_over_ranks(float(S * steps), world, device)
+    value = units / elapsed_max
+    ms_per_step = elapsed_max / steps * 1e3
+
+    # end to end through the public API with host buffers: pinned inputs in,
+    # result out, every step
+    hk = torch.from_numpy(ks).pin_memory()
+    hv = torch.from_numpy(vs).pin_memory()
+    hq = torch.from_numpy(q).pin_memory()
+    hout = torch.empty((S, Hq, d), dtype=torch.float32).pin_memory()
+    h2d = hk.numel() * 2 + hv.numel() * 2 + hq.numel() * 2
+    d2h = hout.numel() * 4
+    e2e_steps = min(steps, 500)
+    for i in range(3):
+        SK.copy_(hk, non_blocking=True); SV.copy_(hv, non_blocking=True)
+        Q.copy_(hq, non_blocking=True); step(i); hout.copy_(out, non_blocking=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    a0 = torch.cuda.Event(enable_timing=True)
+    a1 = torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for i in range(e2e_steps):
+        SK.copy_(hk, non_blocking=True)
+        SV.copy_(hv, non_blocking=True)
+        Q.copy_(hq, non_blocking=True)
+        step(i)
+        hout.copy_(out, non_blocking=True)
+    a1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_t = max_over_ranks(a0.elapsed_time(a1) * 1e-3, world, device)
+    e2e_value = sum_over_ranks(float(S * e2e_steps), world, device) / e2e_t
+
+    if rank != 0:
+        return None
+    peak, peak_kind = measured_peaks()
+    dec_bytes = S * L * H * BYTES_PER_TOKEN_HEAD
+    achieved = dec_bytes / t_dec / 1e9
+    traffic = kernel_traffic("decode_llama8b")
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "u4 codes / f16 params / f32 math",
+        "data": "synthetic",
+        "config": {"workload": "Llama-3-8B-shaped decode layer: 32 seqs x 4096 ctx (+1 appended),"
+                               " 8 KV heads, 32 q heads, d 128, Hadamard b 64, page 16",
+                   "global_batch": S * world, "seq_len": L, "parallelism": f"replicas x{world}",
+                   "l2": "steps alternate between 2 cache replicas (2 x 143 MB > 126 MB L2)"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic, "kernel": "decode attention",
+                     "bytes_per_launch": dec_bytes, "peak_source": peak_kind},
+        "append_prefill": {"gbs": app_bytes / t_app / 1e9, "frac": app_bytes / t_app / 1e9 / peak,
+                           "us": t_app * 1e6, "bytes": app_bytes, "tokens": len(ts)},
+        "decode": {"us": t_dec * 1e6, "kv_tokens_per_s": S * L / t_dec,
+                   "gbs": achieved},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * steps,
+        "clocks": clk,
+    }
+    return line, w
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def oracle_step_sample(w, n_heads_budget, seed_rank=0):
+    """Set up the oracle's cache for one sequence; returns a closure that runs
+    one bounded sample (the step append of that sequence's token and decode
+    attention for ``n_heads_budget`` query heads) and the number of query
+    tokens (in units of a full 32-head token) it covers."""
+    import oracle
+    s = 0
+    k, v, ts, tp = w.prefill_tokens(seqs=[s])
+    oc = oracle.Cache(w.d, w.H, w.P, w.NP, w.rot_kind, w.rot_block)
+    kc, kp = oc.alloc_pools(0)
+    vc, vp = oc.alloc_pools(0)
+    oracle.quantize_append(oc, k.view(np.uint16), v.view(np.uint16), ts, tp, w.block_table,
+                           kc, kp, vc, vp)
+    ks, vs, sts, stp = w.step_tokens(0)
+    q = w.queries(0)
+    lens = np.array([int(w.seq_lens[s]) + 1], np.int32)
+    nh = max(1, min(w.Hq, n_heads_budget))
+    q_s = np.ascontiguousarray(q[s:s + 1, :nh])
+    # attention over the first nh query heads: a cache view whose query-head
+    # count is nh requires nh to be a multiple of H; round to whole groups
+    G = w.Hq // w.H
+    nkv = max(1, nh // G)
+    nh = nkv * G
+    q_s = np.ascontiguousarray(q[s:s + 1, :nh])
+    oc_sub = oracle.Cache(w.d, nkv, w.P, w.NP, w.rot_kind, w.rot_block)
+    kc_s = np.ascontiguousarray(kc[:, :nkv])
+    kp_s = np.ascontiguousarray(kp[:, :nkv])
+    vc_s = np.ascontiguousarray(vc[:, :nkv])
+    vp_s = np.ascontiguousarray(vp[:, :nkv])
+
+    def run():
+        oracle.quantize_append(oc, ks[s:s + 1].view(np.uint16), vs[s:s + 1].view(np.uint16),
+                               np.array([0], np.int32), stp[s:s + 1], w.block_table[s:s + 1],
+                               kc, kp, vc, vp)
+        oracle.paged_decode_attn(oc_sub, q_s.view(np.uint16), lens, int(lens[0]),
+                                 w.block_table[s:s + 1], 1 / math.sqrt(w.d), kc_s, kp_s, vc_s,
+                                 vp_s)
+
+    return run, nh / w.Hq
+
+
+def cpu_baseline(w, budget_s):
+    import oracle
+    run, frac = oracle_step_sample(w, w.Hq)
+    t = time.perf_counter()
+    run()
+    one = time.perf_counter() - t
+    reps = max(1, int(budget_s / max(one, 1e-3)))
+    t = time.perf_counter()
+    for _ in range(reps):
+        run()
+    el = time.perf_counter() - t
+    return {"value": reps * frac / el, "unit": UNIT, "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{reps} x (append of 1 token + decode attention of 1 sequence x "
+                      f"{int(frac * w.Hq)} query heads over {int(w.seq_lens[0]) + 1} INT4 "
+                      f"tokens), fp64 attention, OpenMP over heads"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    import oracle
+    from bit_rotated_kv_block_b200 import workloads
+    w = workloads.llama8b(seed=args.seed)
+    # size each step's sample so warmup + steps of oracle work take ~2 minutes
+    budget = 120.0
+    per_step = budget / max(1, args.steps + args.warmup)
+    run_full, _ = oracle_step_sample(w, w.Hq)
+    t = time.perf_counter()
+    run_full()
+    full = time.perf_counter() - t
+    heads = int(max(w.Hq // w.H, min(w.Hq, w.Hq * per_step / max(full, 1e-6))))
+    run, frac = oracle_step_sample(w, heads)
+    for _ in range(args.warmup):
+        run()
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    el = time.perf_counter() - t
+    value = args.steps * frac / el
+    sample = (f"per step: append of 1 token + decode attention of 1 sequence x "
+              f"{int(round(frac * w.Hq))} query heads over {int(w.seq_lens[0]) + 1} tokens")
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32 quantize / f64 attention (CPU oracle)", "data": "synthetic",
+        "config": {"workload": "Llama-3-8B-shaped decode layer (bounded sample per step)",
+                   "global_batch": 32, "seq_len": int(w.seq_lens[0]) + 1,
+                   "parallelism": "rank 0 CPU"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, world, rank)
+            if line is not None:
+                print(json.dumps(line), flush=True)
+            return
+        res = run_ours(args, world, rank, local)
+        if res is None:
+            return
+        line, w = res
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w, args.cpu_budget)
+        print(json.dumps(line), flush=True)
+    finally:
+        if world > 1 and torch.distributed.is_initialized():
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

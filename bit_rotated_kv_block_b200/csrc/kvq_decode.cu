@@ -1,0 +1,690 @@
+// Paged decode attention over the rotated INT4 cache.
+//
+// Method: "SAW-INT4: System-Aware 4-Bit KV-Cache Quantization for Real-World
+// LLM Serving" (Summary, Key takeaway): the INT4 cache is read by attention in
+// its paged layout; the query is rotated by the same orthogonal block
+// Hadamard (or quaternion) map as the keys, so q . k is unchanged, and the
+// output is rotated back once per query head.
+//
+// Three kernels on the caller's stream:
+//  1. qprep:   qhat = R q for every (sequence, query head), binary32, into the
+//              workspace.
+//  2. split:   one warp per (sequence, KV head, split of the page range). The
+//              warp streams its (page, KV head) chunks (codes + params of K
+//              and V, contiguous in the pool) into a 2-4 stage shared-memory
+//              ring with cp.async, and runs both contractions on tensor cores
+//              (mma.sync m16n8k16, f16 x f16 -> f32):
+//                QK^T: A = [qhat_hi ; qhat_lo] rows of the query heads, B =
+//                      K codes (c - 8, exact in f16) as columns, so the score
+//                      fragment of head r for tokens {2j, 2j+1, 2j+8, 2j+9}
+//                      already sits in lane (r, j) -- exactly the B operand
+//                      layout of the PV product, no transposes;
+//                PV:   A = V codes transposed (channels x tokens) built from
+//                      nibbles with prmt/lop3, B = p * s_v split into f16
+//                      hi + lo columns.
+//              Scale and zero-point are applied algebraically:
+//                qhat . khat = s_k * sum (c - 8) qhat + (m_k + 8 s_k) sum qhat,
+//                sum p vhat  = sum (p s_v)(c - 8)     + sum p (m_v + 8 s_v).
+//              Online softmax in base 2; the warp writes (acc, max, sum) per
+//              query head to the workspace.
+//  3. combine: log-sum-exp merge of the splits, normalisation, R^-1 in
+//              binary32 registers, float32 output.
+// No kernel waits on another CTA; completion of async copies is tracked by
+// the hardware commit groups, so nothing spins.
+
+#include <cuda_runtime.h>
+
+#include "kvq_device.cuh"
+#include "kvq_launch.h"
+#include "kvq_rotate.cuh"
+
+namespace kvq {
+
+constexpr int kDecWarps = 4;
+constexpr int kMaxPagesPerSplit = 256;  // page ids of one work item live in shared memory
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct DecodeArgs {
+  int S, Hq, H, G, P, NP, bt_stride, max_seq_len, splits, pages_per_split;
+  float scale2;  // sm_scale * log2(e)
+  const int32_t* seq_lens;
+  const int32_t* block_table;
+  const uint8_t* k_codes;
+  const uint32_t* k_params;
+  const uint8_t* v_codes;
+  const uint32_t* v_params;
+  const float* qhat;  // [S][Hq][D]
+  float* part;        // [S][Hq][splits][D + 2]
+  int32_t* err;
+};
+
+// ---------------------------------------------------------------------------
+// 1. query rotation: one thread per E channels of a (sequence, query head) row
+// ---------------------------------------------------------------------------
+
+template <int D, int ROT, int LGB>
+__global__ void __launch_bounds__(128) qprep_kernel(const __half* __restrict__ q, int rows,
+                                                    const float* __restrict__ quat,
+                                                    float* __restrict__ qhat) {
+  constexpr int E = D < 128 ? D : 128;
+  constexpr int TPR = D / E;
+  const int gt = blockIdx.x * blockDim.x + threadIdx.x;
+  const int row = gt / TPR, part = gt % TPR;
+  // rows of a d = 256 head are lane pairs; keep whole pairs in or out
+  if (row >= rows) return;
+  float x[E];
+  const uint4* src = reinterpret_cast<const uint4*>(q + (int64_t)row * D + part * E);
+#pragma unroll
+  for (int c = 0; c < E / 8; ++c) {
+    const uint4 u = src[c];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __half22float2(u32_as_h2(w[i]));
+      x[8 * c + 2 * i] = f.x;
+      x[8 * c + 2 * i + 1] = f.y;
+    }
+  }
+  const unsigned pair_mask = 3u << ((threadIdx.x % kWarp) & ~1);
+  if (ROT == KVQ_ROT_HADAMARD) hadamard_regs<E, LGB>(x, part, pair_mask);
+  if (ROT == KVQ_ROT_QUAT) quat_regs<E>(x, quat, part * E);
+  float4* dst = reinterpret_cast<float4*>(qhat + (int64_t)row * D + part * E);
+#pragma unroll
+  for (int c = 0; c < E / 4; ++c) dst[c] = make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]);
+}
+
+// ---------------------------------------------------------------------------
+// 2. split kernel
+// ---------------------------------------------------------------------------
+
+template <int D, int P, int GP>
+struct DecCfg {
+  static constexpr int NKS = D / 16;           // QK k-steps over channels
+  static constexpr int NMT = D / 16;           // PV m-tiles over channels
+  static constexpr int TILES = P / 16;         // 16-token tiles per page
+  static constexpr int NPV = GP == 8 ? 2 : 1;  // PV n-tiles (hi / lo columns)
+  static constexpr int QW = D / 4;             // query channels per lane
+  static constexpr int ROWB = D / 2;           // code bytes per token
+  static constexpr int CODE_B = P * ROWB;      // code bytes per (page, head)
+  static constexpr int STAGE_B = 2 * CODE_B + 8 * P;
+  // pipeline depth: about 8-13 KB of pages in flight per warp
+  static constexpr int NST = STAGE_B <= 2304 ? 4 : (STAGE_B <= 4608 ? 3 : 2);
+  static constexpr int IDS_B = kMaxPagesPerSplit * 4;
+  static constexpr int WARP_B = NST * STAGE_B + IDS_B;
+};
+
+// Swizzled position of the 16-byte unit `u` of token `t` in the V code
+// buffer (conflict-free transposing reads; see the PV fragment loads).
+template <int D>
+__device__ __forceinline__ int v_unit_off(int t, int u) {
+  if (D == 128) {  // 64-byte rows: line = t / 2 holds tokens 2l, 2l+1
+    const int line = t >> 1, un = ((t & 1) << 2) | u;
+    return line * 128 + ((un ^ ((line & 3) << 1)) << 4);
+  } else {  // D == 256: 128-byte rows
+    return t * 128 + ((u ^ (t & 7)) << 4);
+  }
+}
+// Position of the 16-byte unit `u` of token `t` in the K code buffer.
+template <int D>
+__device__ __forceinline__ int k_unit_off(int t, int u) {
+  if (D == 256) return t * 128 + ((u ^ (t & 1)) << 4);
+  return t * (D / 2) + (u << 4);
+}
+
+template <int D, int P, int GP>
+__global__ void __launch_bounds__(kDecWarps * kWarp) decode_split_kernel(const DecodeArgs a) {
+  static_assert(D == 128 || D == 256, "decode attention supports head_dim 128 and 256");
+  using C = DecCfg<D, P, GP>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
+  const int r = lane >> 2, j = lane & 3;
+  const int item = blockIdx.x * kDecWarps + warp;
+  const int per_seq = a.H * a.splits;
+  if (item >= a.S * per_seq) return;
+  const int s = item / per_seq;
+  const int h = (item / a.splits) % a.H;
+  const int split = item % a.splits;
+  uint8_t* ring = smem + warp * C::WARP_B;
+
+  // ---- sequence length and page range of this work item
+  int L = a.seq_lens[s];
+  bool len_ok = L >= 0 && L <= a.max_seq_len && (L + a.P - 1) / a.P <= a.bt_stride;
+  if (!len_ok) {
+    if (lane == 0 && h == 0 && split == 0) raise_flag(a.err, KVQ_ERRF_LEN);
+    L = 0;
+  }
+  const int npages = (L + P - 1) / P;
+  const int pbeg = split * a.pages_per_split;
+  int pend = pbeg + a.pages_per_split;
+  if (pend > npages) pend = npages;
+  const int nmine = pend > pbeg ? pend - pbeg : 0;
+
+  // block-table entries of the item's pages, loaded once (independent loads)
+  int32_t* ids = reinterpret_cast<int32_t*>(ring + C::NST * C::STAGE_B);
+  for (int c = lane; c < nmine; c += kWarp) ids[c] = a.block_table[(int64_t)s * a.bt_stride + pbeg + c];
+  __syncwarp();
+
+  // ---- query fragments: rows = [hi ; lo] of the GP heads of this KV head
+  // lane (r, j) handles query head hr and channels [j*QW, (j+1)*QW)
+  const int hr = (GP == 8) ? r : (r & 3);
+  const bool lo_row = (GP == 4) && (r >= 4);
+  const int g = h * a.G + hr;           // global query head
+  const bool head_ok = hr < a.G;
+  float qs;  // sum of qhat over all channels of head hr
+  uint32_t qa[C::NKS][4];
+  {
+    float x[C::QW];
+    const float* src = a.qhat + ((int64_t)s * a.Hq + g) * D + j * C::QW;
+#pragma unroll
+    for (int c = 0; c < C::QW / 4; ++c) {
+      float4 f = head_ok ? reinterpret_cast<const float4*>(src)[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+      x[4 * c] = f.x; x[4 * c + 1] = f.y; x[4 * c + 2] = f.z; x[4 * c + 3] = f.w;
+    }
+    float part = 0.f;
+#pragma unroll
+    for (int i = 0; i < C::QW; ++i) part += x[i];
+    part += __shfl_xor_sync(0xffffffffu, part, 1);
+    part += __shfl_xor_sync(0xffffffffu, part, 2);
+    qs = part;
+    __half hi[C::QW], lo[C::QW];
+#pragma unroll
+    for (int i = 0; i < C::QW; ++i) split_hl(x[i], hi[i], lo[i]);
+    // k-step kk, column 2j(+1) <- local channel 8(kk/2) + 2(kk%2) (+4);
+    // column 2j+8(+9) <- local channel 8(kk/2) + 2(kk%2) + 1 (+4)
+#pragma unroll
+    for (int kk = 0; kk < C::NKS; ++kk) {
+      const int c0 = 8 * (kk >> 1) + 2 * (kk & 1);
+      const int c1 = c0 + 1;
+      if (GP == 8) {
+        qa[kk][0] = h2_as_u32(__halves2half2(hi[c0], hi[c0 + 4]));
+        qa[kk][1] = h2_as_u32(__halves2half2(lo[c0], lo[c0 + 4]));
+        qa[kk][2] = h2_as_u32(__halves2half2(hi[c1], hi[c1 + 4]));
+        qa[kk][3] = h2_as_u32(__halves2half2(lo[c1], lo[c1 + 4]));
+      } else {
+        const __half* sel = lo_row ? lo : hi;
+        qa[kk][0] = h2_as_u32(__halves2half2(sel[c0], sel[c0 + 4]));
+        qa[kk][1] = 0u;
+        qa[kk][2] = h2_as_u32(__halves2half2(sel[c1], sel[c1 + 4]));
+        qa[kk][3] = 0u;
+      }
+    }
+  }
+
+  // ---- page ring
+  const int64_t head_chunk = (int64_t)C::CODE_B;
+  auto issue = [&](int i) {
+    if (i < nmine) {
+      const int page = ids[i];
+      if (page >= 0 && page < a.NP) {
+        uint8_t* st = ring + (i % C::NST) * C::STAGE_B;
+        const int64_t row = (int64_t)page * a.H + h;
+        const uint8_t* kc = a.k_codes + row * head_chunk;
+        const uint8_t* vc = a.v_codes + row * head_chunk;
+        constexpr int UNITS = C::CODE_B / 16;
+        constexpr int UPT = (D / 2) / 16;  // 16-byte units per token
+#pragma unroll
+        for (int c = lane; c < UNITS; c += kWarp) {
+          const int t = c / UPT, u = c % UPT;
+          cp_async16(st + k_unit_off<D>(t, u), kc + c * 16);
+          cp_async16(st + C::CODE_B + v_unit_off<D>(t, u), vc + c * 16);
+        }
+        constexpr int PU = P * 4 / 16;  // 16-byte units of params per pool
+        if (lane < PU) {
+          cp_async16(st + 2 * C::CODE_B + lane * 16,
+                     reinterpret_cast<const uint8_t*>(a.k_params + row * P) + lane * 16);
+        } else if (lane < 2 * PU) {
+          cp_async16(st + 2 * C::CODE_B + P * 4 + (lane - PU) * 16,
+                     reinterpret_cast<const uint8_t*>(a.v_params + row * P) + (lane - PU) * 16);
+        }
+      }
+    }
+    cp_async_commit();
+  };
+
+  // ---- state
+  float acc[C::NMT][C::NPV][4];
+#pragma unroll
+  for (int mt = 0; mt < C::NMT; ++mt)
+#pragma unroll
+    for (int n = 0; n < C::NPV; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[mt][n][e] = 0.f;
+  float M = -INFINITY;  // running max (base-2 scaled scores) of head hr
+  float Lp = 0.f;       // this lane's share of sum p
+  float Op = 0.f;       // this lane's share of sum p (m_v + 8 s_v)
+
+  for (int i = 0; i < C::NST - 1; ++i) issue(i);
+
+  for (int i = 0; i < nmine; ++i) {
+    issue(i + C::NST - 1);
+    cp_async_wait<C::NST - 1>();
+    __syncwarp();
+    const int pidx = pbeg + i;
+    const int page = ids[i];
+    const bool page_ok = page >= 0 && page < a.NP;
+    if (!page_ok && lane == 0) raise_flag(a.err, KVQ_ERRF_PAGE);
+    const uint8_t* st = ring + (i % C::NST) * C::STAGE_B;
+    const uint8_t* kbuf = st;
+    const uint8_t* vbuf = st + C::CODE_B;
+    const uint2* kpar = reinterpret_cast<const uint2*>(st + 2 * C::CODE_B);
+    const uint2* vpar = reinterpret_cast<const uint2*>(st + 2 * C::CODE_B + P * 4);
+
+    // ---- scores of all tiles of the page: z[tile][0..3] for tokens
+    // 16*tile + {2j, 2j+1, 2j+8, 2j+9}
+    float z[C::TILES][4];
+#pragma unroll
+    for (int tt = 0; tt < C::TILES; ++tt) {
+      float cacc[2][4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) cacc[nt][e] = 0.f;
+        const int tok = 16 * tt + 8 * nt + r;
+        uint32_t w[D / 32];
+#pragma unroll
+        for (int u = 0; u < D / 128; ++u) {
+          const uint4 v4 = *reinterpret_cast<const uint4*>(kbuf + k_unit_off<D>(tok, (D / 128) * j + u));
+          w[4 * u] = v4.x; w[4 * u + 1] = v4.y; w[4 * u + 2] = v4.z; w[4 * u + 3] = v4.w;
+        }
+#pragma unroll
+        for (int kk = 0; kk < C::NKS; ++kk) {
+          const uint32_t wd = w[kk >> 1];
+          const uint32_t b0 = (kk & 1) ? nib_pair<2>(wd) : nib_pair<0>(wd);
+          const uint32_t b1 = (kk & 1) ? nib_pair<3>(wd) : nib_pair<1>(wd);
+          mma16816(cacc[nt], qa[kk], b0, b1);
+        }
+      }
+      // dot products of head hr with the four tokens of this lane
+      float dt[4] = {cacc[0][0], cacc[0][1], cacc[1][0], cacc[1][1]};
+      if (GP == 8) {
+        dt[0] += cacc[0][2]; dt[1] += cacc[0][3]; dt[2] += cacc[1][2]; dt[3] += cacc[1][3];
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dt[e] += __shfl_xor_sync(0xffffffffu, dt[e], 16);
+      }
+      const uint2 kp01 = kpar[8 * tt + j];      // tokens 16tt + 2j, 2j+1
+      const uint2 kp89 = kpar[8 * tt + 4 + j];  // tokens 16tt + 2j+8, 2j+9
+      const uint32_t kp[4] = {kp01.x, kp01.y, kp89.x, kp89.y};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 sm = __half22float2(u32_as_h2(kp[e]));  // (scale, min)
+        const int tok = pidx * P + 16 * tt + 2 * j + (e & 1) + 8 * (e >> 1);
+        const float sc = (sm.x * dt[e] + (sm.y + 8.f * sm.x) * qs) * a.scale2;
+        z[tt][e] = (page_ok && tok < L) ? sc : -INFINITY;
+      }
+    }
+
+    // ---- online softmax update for head hr (max over the 4 lanes j)
+    float mloc = -INFINITY;
+#pragma unroll
+    for (int tt = 0; tt < C::TILES; ++tt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) mloc = fmaxf(mloc, z[tt][e]);
+    mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
+    mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
+    const float Mn = fmaxf(M, mloc);
+    const float alpha = (Mn == -INFINITY) ? 1.f : fast_exp2(M - Mn);
+    M = Mn;
+    Lp *= alpha;
+    Op *= alpha;
+    // rescale the output accumulators: lane (r, j) holds columns of heads
+    // c0 = 2(j & (GP/2 - 1)), c0 + 1 -> their alpha from lanes r = c0, c0 + 1
+    {
+      const int c0 = (GP == 8) ? 2 * j : 2 * (j & 1);
+      const float a0 = __shfl_sync(0xffffffffu, alpha, 4 * c0);
+      const float a1 = __shfl_sync(0xffffffffu, alpha, 4 * c0 + 4);
+#pragma unroll
+      for (int mt = 0; mt < C::NMT; ++mt)
+#pragma unroll
+        for (int n = 0; n < C::NPV; ++n) {
+          acc[mt][n][0] *= a0; acc[mt][n][1] *= a1;
+          acc[mt][n][2] *= a0; acc[mt][n][3] *= a1;
+        }
+    }
+
+    // ---- PV per tile
+#pragma unroll
+    for (int tt = 0; tt < C::TILES; ++tt) {
+      const uint2 vp01 = vpar[8 * tt + j];
+      const uint2 vp89 = vpar[8 * tt + 4 + j];
+      const uint32_t vp[4] = {vp01.x, vp01.y, vp89.x, vp89.y};
+      __half phi[4], plo[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        // masked tokens may sit on stale or never-written shared memory:
+        // their terms are forced to exact zeros rather than p * (params)
+        const bool live = z[tt][e] != -INFINITY;
+        const float2 sm = __half22float2(u32_as_h2(vp[e]));
+        const float p = live ? fast_exp2(z[tt][e] - M) : 0.f;
+        Lp += p;
+        Op += live ? p * (sm.y + 8.f * sm.x) : 0.f;
+        split_hl(live ? p * sm.x : 0.f, phi[e], plo[e]);
+      }
+      // B operand columns: GP = 8: n-tile 0 = hi, 1 = lo (col r = head r);
+      // GP = 4: col r < 4 = hi of head r, r >= 4 = lo of head r - 4
+      uint32_t pb[C::NPV][2];
+      if (GP == 8) {
+        pb[0][0] = h2_as_u32(__halves2half2(phi[0], phi[1]));
+        pb[0][1] = h2_as_u32(__halves2half2(phi[2], phi[3]));
+        pb[C::NPV - 1][0] = h2_as_u32(__halves2half2(plo[0], plo[1]));
+        pb[C::NPV - 1][1] = h2_as_u32(__halves2half2(plo[2], plo[3]));
+      } else {
+        const __half* sel = lo_row ? plo : phi;
+        pb[0][0] = h2_as_u32(__halves2half2(sel[0], sel[1]));
+        pb[0][1] = h2_as_u32(__halves2half2(sel[2], sel[3]));
+      }
+      if (!head_ok) {
+#pragma unroll
+        for (int n = 0; n < C::NPV; ++n) pb[n][0] = pb[n][1] = 0u;
+      }
+      // A operand: V codes of tokens {2j, 2j+1} and {2j+8, 2j+9}, channels of
+      // lane row r: [r*D/8, (r+1)*D/8)
+      constexpr int WPT = D / 64;  // 32-bit words per token per lane
+      uint32_t vw[4][WPT];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int tok = 16 * tt + 2 * j + (e & 1) + 8 * (e >> 1);
+        if (D == 128) {
+          const uint2 v2 = *reinterpret_cast<const uint2*>(vbuf + v_unit_off<D>(tok, r >> 1) + 8 * (r & 1));
+          vw[e][0] = v2.x; vw[e][1] = v2.y;
+        } else {
+          const uint4 v4 = *reinterpret_cast<const uint4*>(vbuf + v_unit_off<D>(tok, r));
+          vw[e][0] = v4.x; vw[e][1] = v4.y; vw[e][2] = v4.z; vw[e][3] = v4.w;
+        }
+      }
+      // m-tile mt: group gq = mt / 8 (words 2gq, 2gq+1), nibble e = mt % 8;
+      // row slot r <- word 2gq, slot r+8 <- word 2gq+1
+#pragma unroll
+      for (int gq = 0; gq < WPT / 2; ++gq) {
+        uint32_t pr[2][2][2];  // [token pair][word in group][lo/hi bytes]
+#pragma unroll
+        for (int tp = 0; tp < 2; ++tp)
+#pragma unroll
+          for (int wi = 0; wi < 2; ++wi) {
+            const int wd = 2 * gq + wi;
+            const uint32_t X = vw[2 * tp][wd], Y = vw[2 * tp + 1][wd];
+            pr[tp][wi][0] = __byte_perm(X, Y, 0x5410);
+            pr[tp][wi][1] = __byte_perm(X, Y, 0x7632);
+          }
+#pragma unroll
+        for (int e8 = 0; e8 < 8; ++e8) {
+          const int mt = gq * 8 + e8;
+          if (mt >= C::NMT) break;
+          uint32_t av[4];
+          auto nib = [&](uint32_t z32) -> uint32_t {
+            switch (e8 & 3) {
+              case 0: return nib_pair<0>(z32);
+              case 1: return nib_pair<1>(z32);
+              case 2: return nib_pair<2>(z32);
+              default: return nib_pair<3>(z32);
+            }
+          };
+          const int bsel = e8 >> 2;
+          av[0] = nib(pr[0][0][bsel]);  // slot r,   tokens 2j, 2j+1
+          av[1] = nib(pr[0][1][bsel]);  // slot r+8, tokens 2j, 2j+1
+          av[2] = nib(pr[1][0][bsel]);  // slot r,   tokens 2j+8, 2j+9
+          av[3] = nib(pr[1][1][bsel]);  // slot r+8, tokens 2j+8, 2j+9
+#pragma unroll
+          for (int n = 0; n < C::NPV; ++n) mma16816(acc[mt][n], av, pb[n][0], pb[n][1]);
+        }
+      }
+    }
+    __syncwarp();  // stage i % C::NST is refilled by the next issue
+  }
+  cp_async_wait<0>();
+
+  // ---- partial results: (acc + sum p (m + 8 s)) per channel, M, sum p
+  Lp += __shfl_xor_sync(0xffffffffu, Lp, 1);
+  Lp += __shfl_xor_sync(0xffffffffu, Lp, 2);
+  Op += __shfl_xor_sync(0xffffffffu, Op, 1);
+  Op += __shfl_xor_sync(0xffffffffu, Op, 2);
+  if (GP == 4) {
+    // fold the lo columns (lanes j = 2, 3) onto the hi columns (j = 0, 1)
+#pragma unroll
+    for (int mt = 0; mt < C::NMT; ++mt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[mt][0][e] += __shfl_xor_sync(0xffffffffu, acc[mt][0][e], 2);
+  }
+  const int c0 = (GP == 8) ? 2 * j : 2 * (j & 1);  // heads of this lane's columns
+  const float o0 = __shfl_sync(0xffffffffu, Op, 4 * c0);
+  const float o1 = __shfl_sync(0xffffffffu, Op, 4 * c0 + 4);
+  const bool writer = (GP == 8) || (j < 2);
+  const int64_t base = ((int64_t)s * a.Hq + (int64_t)h * a.G) * a.splits + split;
+#pragma unroll
+  for (int hc = 0; hc < 2; ++hc) {
+    const int gh = c0 + hc;
+    if (!writer || gh >= a.G) continue;
+    float* dst = a.part + (base + (int64_t)gh * a.splits) * (D + 2);
+    const float ov = hc ? o1 : o0;
+#pragma unroll
+    for (int mt = 0; mt < C::NMT; ++mt) {
+      // m-tile mt, row slot r <- channel r*D/8 + 16*(mt/8) + mt%8,
+      // row slot r+8 <- that channel + 8
+      const int ch0 = r * (D / 8) + 16 * (mt / 8) + (mt % 8);
+      float v0 = 0.f, v1 = 0.f;
+#pragma unroll
+      for (int n = 0; n < C::NPV; ++n) {
+        v0 += acc[mt][n][hc];
+        v1 += acc[mt][n][2 + hc];
+      }
+      dst[ch0] = v0 + ov;
+      dst[ch0 + 8] = v1 + ov;
+    }
+  }
+  // the lanes that own head hr's softmax state write it (one lane per head)
+  if (j == 0 && !lo_row && head_ok) {
+    float* dst = a.part + (base + (int64_t)hr * a.splits) * (D + 2);
+    dst[D] = M;
+    dst[D + 1] = Lp;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// 3. combine: one thread per E channels of a (sequence, query head) row
+// ---------------------------------------------------------------------------
+
+template <int D, int ROT, int LGB>
+__global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ part, int rows,
+                                                      int splits, const float* __restrict__ quat,
+                                                      float* __restrict__ out) {
+  constexpr int E = D < 128 ? D : 128;
+  constexpr int TPR = D / E;
+  const int gt = blockIdx.x * blockDim.x + threadIdx.x;
+  const int row = gt / TPR, pt = gt % TPR;
+  if (row >= rows) return;
+  const float* src = part + (int64_t)row * splits * (D + 2);
+  float Mx = -INFINITY;
+  for (int i = 0; i < splits; ++i) Mx = fmaxf(Mx, src[(int64_t)i * (D + 2) + D]);
+  float x[E];
+#pragma unroll
+  for (int c = 0; c < E; ++c) x[c] = 0.f;
+  float Ls = 0.f;
+  if (Mx != -INFINITY) {
+    for (int i = 0; i < splits; ++i) {
+      const float* p = src + (int64_t)i * (D + 2);
+      const float Mi = p[D];
+      if (Mi == -INFINITY) continue;
+      const float w = fast_exp2(Mi - Mx);
+      Ls += w * p[D + 1];
+#pragma unroll
+      for (int c = 0; c < E; ++c) x[c] += w * p[pt * E + c];
+    }
+  }
+  const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+#pragma unroll
+  for (int c = 0; c < E; ++c) x[c] *= inv;
+  const unsigned pair_mask = 3u << ((threadIdx.x % kWarp) & ~1);
+  if (ROT == KVQ_ROT_HADAMARD) hadamard_regs<E, LGB>(x, pt, pair_mask);  // R^-1 = R
+  if (ROT == KVQ_ROT_QUAT) quat_inv_regs<E>(x, quat, pt * E);
+  float4* dst = reinterpret_cast<float4*>(out + (int64_t)row * D + pt * E);
+#pragma unroll
+  for (int c = 0; c < E / 4; ++c) dst[c] = make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]);
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+
+template <int D, int P, int GP>
+static size_t split_smem() {
+  return (size_t)kDecWarps * DecCfg<D, P, GP>::WARP_B;
+}
+
+template <int D, int P, int GP>
+static int split_resident_warps() {
+  static int cached = -1;
+  if (cached < 0) {
+    auto kern = decode_split_kernel<D, P, GP>;
+    const size_t smem = split_smem<D, P, GP>();
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    int blocks = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, kern, kDecWarps * kWarp, smem) !=
+        cudaSuccess)
+      blocks = 1;
+    const int sms = device_sm_count();
+    cached = (blocks < 1 ? 1 : blocks) * kDecWarps * (sms > 0 ? sms : 148);
+  }
+  return cached;
+}
+
+static int resident_warps(int D, int P, int GP) {
+#define KVQ_RW(d_, p_, g_) \
+  if (D == d_ && P == p_ && GP == g_) return split_resident_warps<d_, p_, g_>();
+  KVQ_RW(128, 16, 4) KVQ_RW(128, 16, 8) KVQ_RW(128, 32, 4) KVQ_RW(128, 32, 8)
+  KVQ_RW(128, 64, 4) KVQ_RW(128, 64, 8) KVQ_RW(256, 16, 4) KVQ_RW(256, 32, 4)
+  KVQ_RW(256, 64, 4)
+#undef KVQ_RW
+  return 148 * 8;
+}
+
+DecodePlan decode_plan(const kvq_cache_desc& d, int32_t S, int32_t Hq, int32_t max_seq_len) {
+  DecodePlan pl{};
+  const int P = d.page_size;
+  pl.pages_max = (max_seq_len + P - 1) / P;
+  if (pl.pages_max < 1) pl.pages_max = 1;
+  const int G = Hq / d.num_kv_heads;
+  const int GP = G <= 4 ? 4 : 8;
+  const int target = resident_warps(d.head_dim, P, GP);
+  const int pairs = S * d.num_kv_heads;
+  int splits = target / (pairs > 0 ? pairs : 1);
+  const int min_splits = (pl.pages_max + kMaxPagesPerSplit - 1) / kMaxPagesPerSplit;
+  if (splits < min_splits) splits = min_splits;
+  if (splits < 1) splits = 1;
+  if (splits > pl.pages_max) splits = pl.pages_max;
+  pl.pages_per_split = (pl.pages_max + splits - 1) / splits;
+  pl.splits = (pl.pages_max + pl.pages_per_split - 1) / pl.pages_per_split;
+  const size_t qhat = (size_t)S * Hq * d.head_dim * sizeof(float);
+  const size_t parts = (size_t)S * Hq * pl.splits * (d.head_dim + 2) * sizeof(float);
+  pl.workspace = ((qhat + 255) / 256) * 256 + parts;
+  return pl;
+}
+
+template <int D, int P, int GP>
+static cudaError_t launch_split(const DecodeArgs& a, cudaStream_t st) {
+  auto kern = decode_split_kernel<D, P, GP>;
+  const size_t smem = split_smem<D, P, GP>();
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int items = a.S * a.H * a.splits;
+  const int grid = (items + kDecWarps - 1) / kDecWarps;
+  kern<<<grid, kDecWarps * kWarp, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+static cudaError_t launch_split_any(const DecodeArgs& a, int D, int GP, cudaStream_t st) {
+#define KVQ_LS(d_, p_, g_) \
+  if (D == d_ && a.P == p_ && GP == g_) return launch_split<d_, p_, g_>(a, st);
+  KVQ_LS(128, 16, 4) KVQ_LS(128, 16, 8) KVQ_LS(128, 32, 4) KVQ_LS(128, 32, 8)
+  KVQ_LS(128, 64, 4) KVQ_LS(128, 64, 8) KVQ_LS(256, 16, 4) KVQ_LS(256, 32, 4)
+  KVQ_LS(256, 64, 4)
+#undef KVQ_LS
+  return cudaErrorInvalidValue;
+}
+
+template <int D, int ROT, int LGB>
+static cudaError_t launch_rot_pair(const __half* q, int rows, const float* quat, float* qhat,
+                                   const float* part, int splits, float* out, bool prep,
+                                   cudaStream_t st) {
+  constexpr int TPR = D <= 128 ? 1 : D / 128;
+  const int threads = rows * TPR;
+  const int grid = (threads + 127) / 128;
+  if (prep)
+    qprep_kernel<D, ROT, LGB><<<grid, 128, 0, st>>>(q, rows, quat, qhat);
+  else
+    combine_kernel<D, ROT, LGB><<<grid, 128, 0, st>>>(part, rows, splits, quat, out);
+  return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_rot(int rot, int lgb, const __half* q, int rows, const float* quat,
+                              float* qhat, const float* part, int splits, float* out, bool prep,
+                              cudaStream_t st) {
+  if (rot == KVQ_ROT_NONE)
+    return launch_rot_pair<D, KVQ_ROT_NONE, 0>(q, rows, quat, qhat, part, splits, out, prep, st);
+  if (rot == KVQ_ROT_QUAT)
+    return launch_rot_pair<D, KVQ_ROT_QUAT, 0>(q, rows, quat, qhat, part, splits, out, prep, st);
+  switch (lgb) {
+    case 4: return launch_rot_pair<D, KVQ_ROT_HADAMARD, 4>(q, rows, quat, qhat, part, splits, out, prep, st);
+    case 5: return launch_rot_pair<D, KVQ_ROT_HADAMARD, 5>(q, rows, quat, qhat, part, splits, out, prep, st);
+    case 6: return launch_rot_pair<D, KVQ_ROT_HADAMARD, 6>(q, rows, quat, qhat, part, splits, out, prep, st);
+    case 7:
+      if (D >= 128) return launch_rot_pair<D, KVQ_ROT_HADAMARD, (D >= 128 ? 7 : 6)>(q, rows, quat, qhat, part, splits, out, prep, st);
+      break;
+    case 8:
+      if (D >= 256) return launch_rot_pair<D, KVQ_ROT_HADAMARD, (D >= 256 ? 8 : 6)>(q, rows, quat, qhat, part, splits, out, prep, st);
+      break;
+  }
+  return cudaErrorInvalidValue;
+}
+
+int decode_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, const void* q,
+                  const int32_t* seq_lens, int32_t max_seq_len, const int32_t* block_table,
+                  int32_t bt_stride, float sm_scale, const uint8_t* k_codes,
+                  const void* k_params, const uint8_t* v_codes, const void* v_params,
+                  float* out, void* workspace, size_t workspace_bytes, int32_t* err,
+                  cudaStream_t st) {
+  const int D = d.head_dim;
+  const int G = Hq / d.num_kv_heads;
+  const int GP = G <= 4 ? 4 : 8;
+  if ((D != 128 && D != 256) || (D == 256 && GP != 4)) return KVQ_ERR_UNSUPPORTED;
+  const DecodePlan pl = decode_plan(d, S, Hq, max_seq_len);
+  if (workspace == nullptr || workspace_bytes < pl.workspace) return KVQ_ERR_WORKSPACE;
+  int lgb = 0;
+  while ((1 << lgb) < d.rot_block) ++lgb;
+  float* qhat = static_cast<float*>(workspace);
+  const size_t qbytes = (((size_t)S * Hq * D * sizeof(float)) + 255) / 256 * 256;
+  float* part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + qbytes);
+  const __half* qh = static_cast<const __half*>(q);
+  const int rows = S * Hq;
+
+  cudaError_t e;
+  switch (D) {
+    case 128: e = launch_rot<128>(d.rot_kind, lgb, qh, rows, d.quat, qhat, part, pl.splits, out, true, st); break;
+    case 256: e = launch_rot<256>(d.rot_kind, lgb, qh, rows, d.quat, qhat, part, pl.splits, out, true, st); break;
+    default: return KVQ_ERR_UNSUPPORTED;
+  }
+  if (e == cudaErrorInvalidValue) return KVQ_ERR_UNSUPPORTED;
+  if (e != cudaSuccess) return KVQ_ERR_CUDA;
+
+  DecodeArgs a;
+  a.S = S; a.Hq = Hq; a.H = d.num_kv_heads; a.G = G; a.P = d.page_size; a.NP = d.num_pages;
+  a.bt_stride = bt_stride; a.max_seq_len = max_seq_len; a.splits = pl.splits;
+  a.pages_per_split = pl.pages_per_split;
+  a.scale2 = sm_scale * kLog2e;
+  a.seq_lens = seq_lens; a.block_table = block_table;
+  a.k_codes = k_codes; a.k_params = static_cast<const uint32_t*>(k_params);
+  a.v_codes = v_codes; a.v_params = static_cast<const uint32_t*>(v_params);
+  a.qhat = qhat; a.part = part; a.err = err;
+  e = launch_split_any(a, D, GP, st);
+  if (e == cudaErrorInvalidValue) return KVQ_ERR_UNSUPPORTED;
+  if (e != cudaSuccess) return KVQ_ERR_CUDA;
+
+  switch (D) {
+    case 128: e = launch_rot<128>(d.rot_kind, lgb, qh, rows, d.quat, qhat, part, pl.splits, out, false, st); break;
+    default: e = launch_rot<256>(d.rot_kind, lgb, qh, rows, d.quat, qhat, part, pl.splits, out, false, st); break;
+  }
+  if (e != cudaSuccess) return KVQ_ERR_CUDA;
+  return KVQ_OK;
+}
+
+}  // namespace kvq

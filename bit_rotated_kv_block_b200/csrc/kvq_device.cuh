@@ -1,0 +1,152 @@
+// Device helpers shared by the libkvq kernels (sm_100a only).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "kvq.h"
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
+#error "libkvq is written for sm_100a (B200) only"
+#endif
+
+namespace kvq {
+
+constexpr int kWarp = 32;
+
+// ---------------------------------------------------------------------------
+// Packed binary32 pairs. add/sub/mul.rn.f32x2 round each lane as IEEE
+// binary32 with round-to-nearest-even and are never contracted into FMAs, so
+// results are identical to two scalar operations.
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint64_t pk(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 upk(uint64_t v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// Three-input minimum / maximum (exact, order-free).
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float min3(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Binary32 value nearest 1/sqrt(b) for b = 2^lg: 2^(-lg/2) for even lg,
+// sqrt(2) * 2^(-(lg+1)/2) for odd lg (sqrt(2) rounded to binary32 is
+// 0x3FB504F3; scaling by a power of two is exact).
+__host__ __device__ __forceinline__ float hadamard_scale(int lg) {
+  const float r2 = 1.41421353816986083984375f;  // binary32 nearest sqrt(2)
+  float s = (lg & 1) ? r2 : 1.0f;
+  int e = (lg & 1) ? (lg + 1) / 2 : lg / 2;
+  for (int i = 0; i < e; ++i) s *= 0.5f;
+  return s;
+}
+
+// ---------------------------------------------------------------------------
+// Error flags
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void raise_flag(int32_t* flags, int32_t bit) {
+  if (flags) atomicOr(flags, bit);
+}
+
+// ---------------------------------------------------------------------------
+// Asynchronous global -> shared copies (16 bytes per thread, no staging
+// through registers). The hardware tracks completion per commit group; no
+// software spin-wait is involved.
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)),
+               "l"(gmem_src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Warp-level tensor-core MMA: D[16x8] (f32) += A[16x16] (f16) * B[16x8] (f16).
+// Fragment ownership (lane = 4*r + j):
+//   A: a[0] = (row r,   k 2j..2j+1)   a[1] = (row r+8, k 2j..2j+1)
+//      a[2] = (row r,   k 2j+8..+9)   a[3] = (row r+8, k 2j+8..+9)
+//   B: b[0] = (k 2j..2j+1, col r)     b[1] = (k 2j+8..+9, col r)
+//   C: c[0..1] = (row r, cols 2j, 2j+1)  c[2..3] = (row r+8, cols 2j, 2j+1)
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t h2_as_u32(__half2 h) {
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ __half2 u32_as_h2(uint32_t u) {
+  return *reinterpret_cast<__half2*>(&u);
+}
+
+// Four packed 4-bit codes -> two half2 holding (code - 8), exact.
+// From a 32-bit word w of 8 nibbles n0..n7 (n_i at bits 4i) and shift e*4,
+// returns half2(n_e - 8, n_{e+4} - 8): the nibble is placed in the mantissa
+// of 1024.0 (0x6400) and 1032 is subtracted.
+template <int E>
+__device__ __forceinline__ uint32_t nib_pair(uint32_t w) {
+  uint32_t t;
+  const uint32_t x = (E == 0) ? w : (w >> (4 * E));
+  asm("lop3.b32 %0, %1, %2, %3, 0xea;" : "=r"(t) : "r"(x), "r"(0x000F000Fu), "r"(0x64006400u));
+  const __half2 h = __hsub2(u32_as_h2(t), u32_as_h2(0x64086408u));  // 1032.0 = 0x6408
+  return h2_as_u32(h);
+}
+
+// half2 (hi, lo) split of a binary32 value: hi = RN16(x), lo = RN16(x - hi).
+__device__ __forceinline__ void split_hl(float x, __half& hi, __half& lo) {
+  hi = __float2half_rn(x);
+  lo = __float2half_rn(x - __half2float(hi));
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+}  // namespace kvq

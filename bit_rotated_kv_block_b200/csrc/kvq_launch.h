@@ -1,0 +1,43 @@
+// Host-side launchers of the libkvq kernels (internal; the public ABI is
+// include/kvq.h). Each returns a kvq_status and enqueues work on `st` only.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "kvq.h"
+
+namespace kvq {
+
+// Streaming multiprocessors of the current device (cached per device).
+int device_sm_count();
+
+int append_launch(const kvq_cache_desc& d, int32_t T, const void* k, const void* v,
+                  int64_t tok_stride, const int32_t* token_seq, const int32_t* token_pos,
+                  int32_t num_seqs, const int32_t* block_table, int32_t bt_stride,
+                  uint8_t* k_codes, void* k_params, uint8_t* v_codes, void* v_params,
+                  int32_t* err, cudaStream_t st);
+
+int dequant_launch(const kvq_cache_desc& d, int32_t S, const int32_t* seq_lens,
+                   int32_t max_seq_len, const int32_t* block_table, int32_t bt_stride,
+                   const uint8_t* codes, const void* params, int32_t unrotate, int32_t out_fp32,
+                   void* out, int32_t* err, cudaStream_t st);
+
+// Split-K plan of the decode attention for these sizes.
+struct DecodePlan {
+  int pages_max;        // ceil(max_seq_len / P)
+  int splits;           // work items per (sequence, KV head)
+  int pages_per_split;  // pages one work item walks
+  size_t workspace;     // bytes of partial results
+};
+DecodePlan decode_plan(const kvq_cache_desc& d, int32_t S, int32_t Hq, int32_t max_seq_len);
+
+int decode_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, const void* q,
+                  const int32_t* seq_lens, int32_t max_seq_len, const int32_t* block_table,
+                  int32_t bt_stride, float sm_scale, const uint8_t* k_codes,
+                  const void* k_params, const uint8_t* v_codes, const void* v_params,
+                  float* out, void* workspace, size_t workspace_bytes, int32_t* err,
+                  cudaStream_t st);
+
+}  // namespace kvq

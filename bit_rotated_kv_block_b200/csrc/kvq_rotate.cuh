@@ -1,0 +1,133 @@
+// Rotation helpers shared by the append, export and attention kernels.
+//
+// Block-diagonal Walsh-Hadamard rotation ("SAW-INT4: System-Aware 4-Bit
+// KV-Cache Quantization for Real-World LLM Serving", Summary/Method;
+// "UltraQuant: 4-bit KV caching for long agents", method section) and the
+// quaternion block rotation qL v conj(qR) ("IsoQuant: Hardware-Aligned SO(4)
+// Isoclinic Rotations for LLM KV Cache Compression", Abstract), both on
+// values held in registers: a thread owns E consecutive channels of a row.
+#pragma once
+
+#include "kvq_device.cuh"
+
+namespace kvq {
+
+// In-thread Walsh-Hadamard butterflies on blocks of B = 2^LGB channels
+// (B <= E), stages h = 1, 2, ..., B/2 in ascending order.
+template <int E, int LGB>
+__device__ __forceinline__ void fwht_regs(float (&x)[E]) {
+  constexpr int B = 1 << LGB;
+  static_assert(B <= E, "block wider than a thread");
+  if (B >= 2) {
+#pragma unroll
+    for (int i = 0; i < E; i += 2) {
+      const float a = x[i], c = x[i + 1];
+      x[i] = __fadd_rn(a, c);
+      x[i + 1] = __fsub_rn(a, c);
+    }
+  }
+#pragma unroll
+  for (int h = 2; h < B; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < E; i += 2) {
+      if ((i & h) == 0) {
+        const uint64_t a = pk(x[i], x[i + 1]);
+        const uint64_t c = pk(x[i + h], x[i + h + 1]);
+        const float2 s = upk(add2(a, c));
+        const float2 d = upk(sub2(a, c));
+        x[i] = s.x;
+        x[i + 1] = s.y;
+        x[i + h] = d.x;
+        x[i + h + 1] = d.y;
+      }
+    }
+  }
+}
+
+// Multiplies by the Hadamard scale. For b a power of 4 the scale is a power
+// of two, the product is exact, and a later fusion of it into a
+// multiply-add could not change any rounding, so the packed multiply is
+// used; otherwise each product is rounded by __fmul_rn, which is never
+// contracted into a fused multiply-add.
+template <int E, int LGB>
+__device__ __forceinline__ void scale_regs(float (&x)[E], float cb) {
+  if ((LGB & 1) == 0) {
+    const uint64_t c2 = pk(cb, cb);
+#pragma unroll
+    for (int i = 0; i < E; i += 2) {
+      const float2 r = upk(mul2(pk(x[i], x[i + 1]), c2));
+      x[i] = r.x;
+      x[i + 1] = r.y;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < E; ++i) x[i] = __fmul_rn(x[i], cb);
+  }
+}
+
+// One Hamilton product a (x) b, each component as
+// fma(t3, fma(t2, fma(t1, t0))) with the term order of the definition.
+__device__ __forceinline__ void hamilton(const float a[4], const float b[4], float o[4]) {
+  o[0] = __fmaf_rn(-a[3], b[3], __fmaf_rn(-a[2], b[2], __fmaf_rn(-a[1], b[1], __fmul_rn(a[0], b[0]))));
+  o[1] = __fmaf_rn(-a[3], b[2], __fmaf_rn(a[2], b[3], __fmaf_rn(a[1], b[0], __fmul_rn(a[0], b[1]))));
+  o[2] = __fmaf_rn(a[3], b[1], __fmaf_rn(a[2], b[0], __fmaf_rn(-a[1], b[3], __fmul_rn(a[0], b[2]))));
+  o[3] = __fmaf_rn(a[3], b[0], __fmaf_rn(-a[2], b[1], __fmaf_rn(a[1], b[2], __fmul_rn(a[0], b[3]))));
+}
+
+template <int E>
+__device__ __forceinline__ void quat_regs(float (&x)[E], const float* tbl, int ch0) {
+#pragma unroll
+  for (int k = 0; k < E / 4; ++k) {
+    const float* q = tbl + (ch0 / 4 + k) * 8;
+    const float qL[4] = {q[0], q[1], q[2], q[3]};
+    const float qRc[4] = {q[4], -q[5], -q[6], -q[7]};
+    const float v[4] = {x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3]};
+    float t[4], y[4];
+    hamilton(qL, v, t);
+    hamilton(t, qRc, y);
+    x[4 * k] = y[0];
+    x[4 * k + 1] = y[1];
+    x[4 * k + 2] = y[2];
+    x[4 * k + 3] = y[3];
+  }
+}
+
+// Full Hadamard rotation of a thread's E channels, block 2^LGB. Blocks wider
+// than E (b = 256 with E = 128) finish with one stage across the lane pair
+// (2i, 2i+1) given by pair_mask; part 0 holds the lower channels.
+template <int E, int LGB>
+__device__ __forceinline__ void hadamard_regs(float (&x)[E], int part, unsigned pair_mask) {
+  constexpr int B = 1 << LGB;
+  constexpr int LGIN = (B <= E) ? LGB : (E == 128 ? 7 : 6);
+  fwht_regs<E, LGIN>(x);
+  if (B > E) {
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+      const float o = __shfl_xor_sync(pair_mask, x[i], 1);
+      x[i] = part == 0 ? __fadd_rn(x[i], o) : __fsub_rn(o, x[i]);
+    }
+  }
+  scale_regs<E, LGB>(x, hadamard_scale(LGB));
+}
+
+// Inverse quaternion rotation w -> conj(qL) w qR (the inverse of
+// v -> qL v conj(qR) for unit quaternions), plain binary32 arithmetic.
+template <int E>
+__device__ __forceinline__ void quat_inv_regs(float (&x)[E], const float* tbl, int ch0) {
+#pragma unroll
+  for (int k = 0; k < E / 4; ++k) {
+    const float* q = tbl + (ch0 / 4 + k) * 8;
+    const float qLc[4] = {q[0], -q[1], -q[2], -q[3]};
+    const float qR[4] = {q[4], q[5], q[6], q[7]};
+    const float w[4] = {x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3]};
+    float t[4], y[4];
+    hamilton(qLc, w, t);
+    hamilton(t, qR, y);
+    x[4 * k] = y[0];
+    x[4 * k + 1] = y[1];
+    x[4 * k + 2] = y[2];
+    x[4 * k + 3] = y[3];
+  }
+}
+
+}  // namespace kvq

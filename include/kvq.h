@@ -1,0 +1,192 @@
+/*
+ * kvq.h -- C ABI of libkvq: a rotated, token-wise INT4, paged KV cache for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method (page "SAW-INT4: System-Aware 4-Bit KV-Cache Quantization for
+ * Real-World LLM Serving", Summary and Method): every (token, KV head) row of
+ * K and of V is rotated by a block-diagonal Hadamard matrix, quantized to
+ * 4-bit codes with one scale and one zero-point per row, and written straight
+ * into a paged cache through a block table; attention then reads the INT4
+ * pages with the query rotated by the same orthogonal matrix, so q . k is
+ * unchanged by the rotation. The Walsh-Hadamard rotation spreads outlier
+ * channels before quantization (page "UltraQuant: 4-bit KV caching for long
+ * agents", method section). An alternative rotation maps each 4-channel block
+ * v to qL v conj(qR) with unit quaternions (page "IsoQuant: Hardware-Aligned
+ * SO(4) Isoclinic Rotations for LLM KV Cache Compression", Abstract).
+ *
+ * Conventions for every entry point:
+ *  - Every pointer argument except `desc` is a DEVICE pointer (cudaMalloc'd
+ *    or a torch CUDA tensor's data pointer) unless its comment says "host".
+ *    `desc` itself is a host pointer; `desc->quat` is a device pointer.
+ *  - The caller owns every buffer. The library never allocates, frees or
+ *    synchronises; all work is enqueued on `stream` (a cudaStream_t; NULL is
+ *    the legacy default stream). Calls on one stream run in order.
+ *  - The return value (kvq_status) is decided on the host before launch:
+ *    argument and shape checks, 16-byte alignment of pointers and strides,
+ *    workspace size, and cudaGetLastError() after the launch. A non-OK status
+ *    means nothing was launched (except KVQ_ERR_CUDA).
+ *  - Device-side problems (a block-table entry outside [0, num_pages), a
+ *    position outside the table, a sequence index or length out of range)
+ *    never fault or trap: the affected write or page is skipped and a bit is
+ *    OR-ed into *err_flags (KVQ_ERRF_*) if err_flags is not NULL. The caller
+ *    reads it after its own synchronisation.
+ *  - Inputs are never modified; pool bytes not addressed by a call are never
+ *    touched.
+ *
+ * Cache layout (per pool, K and V have separate pools):
+ *  codes  : uint8  [num_pages][num_kv_heads][page_size][head_dim/2]
+ *           two 4-bit codes per byte, even channel in the low nibble.
+ *  params : binary16 pairs [num_pages][num_kv_heads][page_size][2] =
+ *           (scale s16, minimum m16) of each row; the row dequantizes to
+ *           x_i = c_i * s16 + m16 in the rotated basis.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KVQ_OK = 0,
+  KVQ_ERR_INVALID_ARG = 1, /* a size, index or pointer argument is invalid */
+  KVQ_ERR_UNSUPPORTED = 2, /* a valid geometry this build has no kernel for */
+  KVQ_ERR_MISALIGNED = 3,  /* a pointer or stride is not 16-byte aligned   */
+  KVQ_ERR_WORKSPACE = 4,   /* workspace missing or smaller than required   */
+  KVQ_ERR_CUDA = 5         /* the CUDA runtime reported an error at launch  */
+} kvq_status;
+
+typedef enum {
+  KVQ_ROT_NONE = 0,     /* identity: the rotation-free INT4 baseline       */
+  KVQ_ROT_HADAMARD = 1, /* block-diagonal Walsh-Hadamard, block rot_block   */
+  KVQ_ROT_QUAT = 2      /* per 4-channel block v -> qL v conj(qR)          */
+} kvq_rot_kind;
+
+/* Bits OR-ed into *err_flags by the kernels. */
+#define KVQ_ERRF_PAGE 1 /* block-table entry outside [0, num_pages): page skipped */
+#define KVQ_ERRF_POS 2  /* position < 0 or position/page_size >= bt_stride       */
+#define KVQ_ERRF_SEQ 4  /* token's sequence index >= num_seqs                    */
+#define KVQ_ERRF_LEN 8  /* seq_lens[s] < 0, > max_seq_len, or past the table      */
+
+/* Geometry of one paged cache (both pools share it).
+ *  head_dim     d: 64, 128 or 256.
+ *  num_kv_heads H: >= 1.
+ *  page_size    P: tokens per page; 16, 32 or 64.
+ *  num_pages    NP: pool capacity in pages (>= 1).
+ *  rot_kind     a kvq_rot_kind.
+ *  rot_block    b, for KVQ_ROT_HADAMARD: a power of two in [16, 256]
+ *               dividing d (ignored otherwise).
+ *  quat         for KVQ_ROT_QUAT: device float [d/4][2][4], per block j
+ *               (qL[j], qR[j]) as (w, x, y, z); unit quaternions. NULL
+ *               otherwise. Channels 4j..4j+3 form block j. */
+typedef struct {
+  int32_t head_dim;
+  int32_t num_kv_heads;
+  int32_t page_size;
+  int32_t num_pages;
+  int32_t rot_kind;
+  int32_t rot_block;
+  const float* quat;
+} kvq_cache_desc;
+
+/*
+ * kvq_quantize_append -- rotate, quantize, pack and scatter new tokens of K
+ * and V into the INT4 pools ("SAW-INT4", Summary/Method: the fused
+ * rotation-quantization kernel writing into paged KV-cache layouts).
+ *
+ *  num_tokens  T >= 0 (T = 0 is a no-op returning KVQ_OK).
+ *  k, v        binary16 [T][H][d]: token t's row for head h starts at element
+ *              t*tok_stride + h*d. Both 16-byte aligned.
+ *  tok_stride  elements between consecutive tokens, >= H*d, multiple of 8.
+ *  token_seq   int32 [T]: sequence of each token; < 0 skips the token.
+ *  token_pos   int32 [T]: position of each token within its sequence.
+ *  num_seqs    rows of block_table.
+ *  block_table int32 [num_seqs][bt_stride]: page of (seq, pos / P).
+ *  k_codes ... v_params: the pools (layout above), 16-byte aligned.
+ *
+ * Per row (token t, head h), in binary32: x = widen(k[t][h]); y = R x
+ * (Hadamard: butterflies h = 1, 2, ..., b/2 on each block, pair (i, i+h)
+ * -> (x_i + x_{i+h}, x_i - x_{i+h}), then times the binary32 value nearest
+ * 1/sqrt(b); quaternion: (qL (x) v) (x) conj(qR) with the Hamilton
+ * components as fused multiply-adds in a fixed term order); mn = min y + 0,
+ * mx = max y + 0; m16 = binary16 round-down(mn); s16 = binary16 round-up of
+ * round-up32(round-up32(mx - m16) / 15); inv = round-nearest32(1/s16);
+ * code_i = round-half-even(RN(RN(y_i - m16) * inv)) in [0, 15] (all 0 when
+ * s16 = 0). Codes, scale and minimum are bit-identical to that definition.
+ * Domain: inputs finite, and every rotated value as well as the scale within
+ * the binary16 range (|y| <= 65504); outside it (e.g. a minimum that rounds
+ * to -inf) the row's codes are unspecified, but nothing outside the row's
+ * slot is written.
+ * Tokens writing the same slot in one call race (caller error).
+ */
+int kvq_quantize_append(const kvq_cache_desc* desc, int32_t num_tokens, const void* k,
+                        const void* v, int64_t tok_stride, const int32_t* token_seq,
+                        const int32_t* token_pos, int32_t num_seqs,
+                        const int32_t* block_table, int32_t bt_stride, uint8_t* k_codes,
+                        void* k_params, uint8_t* v_codes, void* v_params,
+                        int32_t* err_flags, void* stream);
+
+/*
+ * kvq_decode_workspace_bytes -- bytes of device workspace that
+ * kvq_paged_decode_attn needs for these sizes (host-only computation; 0 on
+ * invalid arguments). The workspace holds per-split partial results.
+ */
+size_t kvq_decode_workspace_bytes(const kvq_cache_desc* desc, int32_t num_seqs,
+                                  int32_t num_q_heads, int32_t max_seq_len);
+
+/*
+ * kvq_paged_decode_attn -- one query token per sequence attends over its
+ * cached INT4 tokens ("SAW-INT4", Key takeaway: serving-compatible attention
+ * over the rotated INT4 cache).
+ *
+ *  num_seqs     S >= 1; num_q_heads Hq: a multiple of H with Hq/H <= 8.
+ *  q            binary16 [S][Hq][d], not rotated (the kernel rotates it).
+ *  seq_lens     int32 [S]: cached tokens of each sequence (0 gives out = 0).
+ *  max_seq_len  upper bound of seq_lens (sizes the split-K work).
+ *  sm_scale     softmax scale (typically 1/sqrt(d)).
+ *  out          float32 [S][Hq][d], in the original (un-rotated) basis.
+ *  workspace    >= kvq_decode_workspace_bytes(...) bytes, 16-byte aligned.
+ *
+ * For query head g (KV head h = g / (Hq/H)): qhat = R q_g;
+ * z_j = sm_scale * qhat . khat_j; p = softmax(z); out = R^-1 sum_j p_j vhat_j,
+ * with khat_j, vhat_j the dequantized rows. Results match a double-precision
+ * evaluation of that definition to about 1e-4 absolute for unit-scale data
+ * (the contractions run on tensor cores with split binary16 operands).
+ */
+int kvq_paged_decode_attn(const kvq_cache_desc* desc, int32_t num_seqs, int32_t num_q_heads,
+                          const void* q, const int32_t* seq_lens, int32_t max_seq_len,
+                          const int32_t* block_table, int32_t bt_stride, float sm_scale,
+                          const uint8_t* k_codes, const void* k_params,
+                          const uint8_t* v_codes, const void* v_params, float* out,
+                          void* workspace, size_t workspace_bytes, int32_t* err_flags,
+                          void* stream);
+
+/*
+ * kvq_dequantize_pages -- dense export of the cached rows of one pool:
+ * out[s][j][h][:] = c * s16 + m16 (optionally rotated back by R^-1) for
+ * j < seq_lens[s]; rows j >= seq_lens[s] are not written.
+ *
+ *  out       float32 (out_fp32 != 0) or binary16 [S][max_seq_len][H][d].
+ *  unrotate  0: values in the rotated basis (exact in float32);
+ *            1: R^-1 applied in binary32 arithmetic.
+ */
+int kvq_dequantize_pages(const kvq_cache_desc* desc, int32_t num_seqs,
+                         const int32_t* seq_lens, int32_t max_seq_len,
+                         const int32_t* block_table, int32_t bt_stride, const uint8_t* codes,
+                         const void* params, int32_t unrotate, int32_t out_fp32, void* out,
+                         int32_t* err_flags, void* stream);
+
+/* Human-readable name of a kvq_status value (static storage). */
+const char* kvq_status_string(int status);
+
+/* Library build string (static storage). */
+const char* kvq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H */

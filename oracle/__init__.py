@@ -226,8 +226,10 @@ def quantize_append(cache, k, v, token_seq, token_pos, block_table, k_codes, k_p
     """Rotate, quantize, pack and scatter T tokens of K and V (binary16 bits,
     [T][H][d] with token stride ``tok_stride`` elements) into the pools, in
     place. Returns the OR of error flags."""
+    # converted copies are bound to names so they outlive the C call
     k, v = _c(k, np.uint16), _c(v, np.uint16)
-    T = len(token_seq)
+    ts, tp = _c(token_seq, np.int32), _c(token_pos, np.int32)
+    T = len(ts)
     if tok_stride is None:
         tok_stride = cache.H * cache.d
     bt = _c(block_table, np.int32)
@@ -238,25 +240,25 @@ def quantize_append(cache, k, v, token_seq, token_pos, block_table, k_codes, k_p
         assert a.flags.c_contiguous
     lib().orc_quantize_append(cache.d, cache.H, cache.P, cache.NP, cache.rot_kind,
                               cache.rot_block, _p(cache.quat), T, _p(k), _p(v), tok_stride,
-                              _p(_c(token_seq, np.int32)), _p(_c(token_pos, np.int32)),
-                              num_seqs, _p(bt), bt.shape[1], _p(k_codes), _p(k_params),
-                              _p(v_codes), _p(v_params), _p(err))
+                              _p(ts), _p(tp), num_seqs, _p(bt), bt.shape[1], _p(k_codes),
+                              _p(k_params), _p(v_codes), _p(v_params), _p(err))
     return int(err[0])
 
 
 def dequantize_pages(cache, seq_lens, max_seq_len, block_table, codes, params, unrotate,
                      out_fp32=True, out=None):
     bt = _c(block_table, np.int32)
+    lens = _c(seq_lens, np.int32)
+    codes, params = _c(codes, np.uint8), _c(params, np.uint16)
     S = bt.shape[0]
     shape = (S, max_seq_len, cache.H, cache.d)
     if out is None:
         out = np.zeros(shape, np.float32 if out_fp32 else np.uint16)
     err = np.zeros(1, np.int32)
     lib().orc_dequantize_pages(cache.d, cache.H, cache.P, cache.NP, cache.rot_kind,
-                               cache.rot_block, _p(cache.quat), S,
-                               _p(_c(seq_lens, np.int32)), max_seq_len, _p(bt), bt.shape[1],
-                               _p(_c(codes, np.uint8)), _p(_c(params, np.uint16)),
-                               int(bool(unrotate)), int(bool(out_fp32)), _p(out), _p(err))
+                               cache.rot_block, _p(cache.quat), S, _p(lens), max_seq_len, _p(bt),
+                               bt.shape[1], _p(codes), _p(params), int(bool(unrotate)),
+                               int(bool(out_fp32)), _p(out), _p(err))
     return out, int(err[0])
 
 
@@ -267,14 +269,15 @@ def paged_decode_attn(cache, q, seq_lens, max_seq_len, block_table, sm_scale, k_
     q = _c(q, np.uint16)
     S, Hq, d = q.shape
     bt = _c(block_table, np.int32)
+    lens = _c(seq_lens, np.int32)
+    kc, kp = _c(k_codes, np.uint8), _c(k_params, np.uint16)
+    vc, vp = _c(v_codes, np.uint8), _c(v_params, np.uint16)
     out = np.empty((S, Hq, d), np.float64)
     err = np.zeros(1, np.int32)
     lib().orc_paged_decode_attn(cache.d, cache.H, cache.P, cache.NP, cache.rot_kind,
-                                cache.rot_block, _p(cache.quat), S, Hq, _p(q),
-                                _p(_c(seq_lens, np.int32)), max_seq_len, _p(bt), bt.shape[1],
-                                float(sm_scale), _p(_c(k_codes, np.uint8)),
-                                _p(_c(k_params, np.uint16)), _p(_c(v_codes, np.uint8)),
-                                _p(_c(v_params, np.uint16)), _p(out), _p(err))
+                                cache.rot_block, _p(cache.quat), S, Hq, _p(q), _p(lens),
+                                max_seq_len, _p(bt), bt.shape[1], float(sm_scale), _p(kc),
+                                _p(kp), _p(vc), _p(vp), _p(out), _p(err))
     return out, int(err[0])
 
 
@@ -283,11 +286,12 @@ def paged_decode_attn_fp16(d, H, P, NP, q, seq_lens, max_seq_len, block_table, s
     q = _c(q, np.uint16)
     S, Hq, _ = q.shape
     bt = _c(block_table, np.int32)
+    lens = _c(seq_lens, np.int32)
+    k16, v16 = _c(k16, np.uint16), _c(v16, np.uint16)
     out = np.empty((S, Hq, d), np.float64)
     err = np.zeros(1, np.int32)
-    lib().orc_paged_decode_attn_fp16(d, H, P, NP, S, Hq, _p(q), _p(_c(seq_lens, np.int32)),
-                                     max_seq_len, _p(bt), bt.shape[1], float(sm_scale),
-                                     _p(_c(k16, np.uint16)), _p(_c(v16, np.uint16)), _p(out),
+    lib().orc_paged_decode_attn_fp16(d, H, P, NP, S, Hq, _p(q), _p(lens), max_seq_len, _p(bt),
+                                     bt.shape[1], float(sm_scale), _p(k16), _p(v16), _p(out),
                                      _p(err))
     return out, int(err[0])
 

@@ -1,0 +1,84 @@
+"""Shared set-up for the GPU parity tests: the same seeded inputs go to the
+CUDA library (through the C ABI) and to the CPU oracle."""
+
+import numpy as np
+import torch
+
+import oracle
+from bit_rotated_kv_block_b200 import kvq
+
+
+def dev(x):
+    return torch.from_numpy(np.ascontiguousarray(x)).cuda()
+
+
+class Pair:
+    """One paged cache built twice: GPU pools through libkvq, host pools through
+    the oracle, both started from the same sentinel bytes."""
+
+    def __init__(self, d, H, P, NP, rot_kind, rot_block=0, quat=None, fill=0xAA):
+        self.gpu = kvq.Cache(d, H, P, NP, rot_kind, rot_block, quat)
+        self.orc = oracle.Cache(d, H, P, NP, rot_kind, rot_block, quat)
+        self.kc, self.kp = self.gpu.new_pools(fill=fill)
+        self.vc, self.vp = self.gpu.new_pools(fill=fill)
+        self.okc, self.okp = self.orc.alloc_pools(fill)
+        self.ovc, self.ovp = self.orc.alloc_pools(fill)
+        self.err = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    @classmethod
+    def for_workload(cls, w, fill=0xAA):
+        return cls(w.d, w.H, w.P, w.NP, w.rot_kind, w.rot_block, w.quat, fill)
+
+    def append(self, k, v, token_seq, token_pos, block_table, oracle_too=True, tok_stride=None,
+               k_dev=None, v_dev=None):
+        """k, v: float16 numpy [T][H][d] (or wider rows with tok_stride)."""
+        self.err.zero_()
+        kd = dev(k) if k_dev is None else k_dev
+        vd = dev(v) if v_dev is None else v_dev
+        bt = dev(block_table.astype(np.int32))
+        kvq.quantize_append(self.gpu, kd, vd, dev(token_seq.astype(np.int32)),
+                            dev(token_pos.astype(np.int32)), bt, self.kc, self.kp, self.vc,
+                            self.vp, err=self.err, tok_stride=tok_stride)
+        oerr = 0
+        if oracle_too:
+            oerr = oracle.quantize_append(self.orc, k.view(np.uint16), v.view(np.uint16),
+                                          token_seq, token_pos, block_table, self.okc,
+                                          self.okp.reshape(self.orc.NP, self.orc.H, self.orc.P, 2),
+                                          self.ovc, self.ovp, tok_stride=tok_stride)
+        torch.cuda.synchronize()
+        return int(self.err.item()), oerr
+
+    def assert_pools_equal(self):
+        """Bit-exact comparison of codes and params (all bytes, untouched ones too)."""
+        for g, o in ((self.kc, self.okc), (self.vc, self.ovc)):
+            gh = g.cpu().numpy()
+            if not np.array_equal(gh, o):
+                bad = np.argwhere(gh != o)
+                raise AssertionError(f"code bytes differ at {len(bad)} places, first {bad[:5]}")
+        for g, o in ((self.kp, self.okp), (self.vp, self.ovp)):
+            gh = g.cpu().numpy().view(np.uint16).reshape(o.shape)
+            if not np.array_equal(gh, o):
+                bad = np.argwhere(gh != o)
+                raise AssertionError(f"param words differ at {len(bad)} places, first {bad[:5]}")
+
+    def oracle_attention(self, q, seq_lens, max_seq_len, block_table, sm_scale):
+        return oracle.paged_decode_attn(self.orc, q.view(np.uint16), seq_lens, max_seq_len,
+                                        block_table, sm_scale, self.okc, self.okp, self.ovc,
+                                        self.ovp)
+
+    def gpu_attention(self, q, seq_lens, max_seq_len, block_table, sm_scale):
+        self.err.zero_()
+        out = kvq.paged_decode_attn(self.gpu, dev(q), dev(seq_lens.astype(np.int32)), max_seq_len,
+                                    dev(block_table.astype(np.int32)), self.kc, self.kp, self.vc,
+                                    self.vp, sm_scale=sm_scale, err=self.err)
+        torch.cuda.synchronize()
+        return out.cpu().numpy().astype(np.float64), int(self.err.item())
+
+
+def fill_workload(w, seqs=None, layer=0, oracle_too=True, fill=0xAA):
+    """Pair cache holding the workload's cached tokens of the given sequences."""
+    p = Pair.for_workload(w, fill)
+    k, v, ts, tp = w.prefill_tokens(seqs, layer)
+    e, oe = p.append(k, v, ts, tp, w.block_table, oracle_too=oracle_too)
+    assert e == 0 and oe == 0
+    return p, (k, v, ts, tp)

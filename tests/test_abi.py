@@ -1,0 +1,77 @@
+"""The C-ABI library builds, loads without a GPU, exports every function that
+include/kvq.h declares, and rejects bad arguments on the host (these calls
+return before any CUDA call, so no GPU is needed)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from bit_rotated_kv_block_b200 import build, kvq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return kvq.lib()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "kvq.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(kvq_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_function_is_exported(L):
+    names = declared_functions()
+    assert "kvq_quantize_append" in names and "kvq_paged_decode_attn" in names
+    assert "kvq_dequantize_pages" in names and "kvq_decode_workspace_bytes" in names
+    for n in names:
+        assert hasattr(L, n), n
+        assert n in kvq.SIGNATURES, n
+
+
+def test_status_strings_and_version(L):
+    assert kvq.version().startswith("libkvq")
+    for code, name in kvq.STATUS.items():
+        assert L.kvq_status_string(code).decode() == name
+
+
+def _desc(**kw):
+    base = dict(head_dim=128, num_kv_heads=8, page_size=16, num_pages=16, rot_kind=1,
+                rot_block=128, quat=None)
+    base.update(kw)
+    return kvq.CacheDesc(**base)
+
+
+def _append(L, desc, T=1, k=16, v=16, stride=1024, seq=16, pos=16, S=1, bt=16, bts=1, pools=16):
+    P = ctypes.c_void_p
+    return L.kvq_quantize_append(ctypes.byref(desc), T, P(k) if k else None, P(v) if v else None,
+                                 stride, P(seq) if seq else None, P(pos) if pos else None, S,
+                                 P(bt) if bt else None, bts, P(pools), P(pools), P(pools),
+                                 P(pools), None, None)
+
+
+def test_host_validation_codes(L):
+    OK, INV, UNS, MIS = 0, 1, 2, 3
+    assert _append(L, _desc(), T=0) == OK                       # empty batch: no launch
+    assert _append(L, _desc(head_dim=100)) == UNS
+    assert _append(L, _desc(page_size=24)) == UNS
+    assert _append(L, _desc(rot_block=96)) == INV               # not a power of two
+    assert _append(L, _desc(rot_block=8)) == UNS                # below the supported blocks
+    assert _append(L, _desc(rot_block=256)) == INV              # wider than head_dim
+    assert _append(L, _desc(rot_kind=2)) == INV                 # quaternion without a table
+    assert _append(L, _desc(rot_kind=7)) == INV
+    assert _append(L, _desc(num_kv_heads=0)) == INV
+    assert _append(L, _desc(), k=0) == INV                      # null input
+    assert _append(L, _desc(), stride=1000) == INV              # stride < H * d
+    assert _append(L, _desc(), stride=1028) == MIS              # stride not a multiple of 8
+    assert _append(L, _desc(), k=24) == MIS                     # misaligned pointer
+    assert _append(L, _desc(), T=-1) == INV
+    desc = _desc()
+    assert L.kvq_decode_workspace_bytes(ctypes.byref(desc), 0, 32, 100) == 0
+    assert L.kvq_decode_workspace_bytes(ctypes.byref(desc), 2, 30, 100) == 0   # Hq % H != 0
