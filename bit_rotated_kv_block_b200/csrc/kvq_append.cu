@@ -12,21 +12,26 @@
 //    row of K or V, so every butterfly stage of a block of up to 128 channels
 //    runs in registers without shuffles; d = 256 uses two threads per row and
 //    one xor-1 shuffle stage for b = 256.
-//  * A CTA of 256 threads owns a tile of TOK tokens x {K, V} x H heads. The
-//    tile's fp16 rows are copied global -> shared with coalesced 16-byte
-//    cp.async (row pitch 2E + 16 bytes, so each thread then reads its own row
-//    with conflict-free 128-bit loads) while the previous tile is computed
-//    (two buffers). The grid is persistent: one CTA per SM walks the tiles.
+//  * A CTA of 384 threads owns a tile of TOK tokens x {K, V} x H heads. Each
+//    thread pulls its own row segment (2E contiguous bytes) global -> shared
+//    with one TMA bulk copy that completes on the buffer's mbarrier (row
+//    pitch 2E + 16 bytes, so the thread then reads it with conflict-free
+//    128-bit loads) while the previous tile is computed (two buffers). The
+//    grid is persistent: one CTA per SM walks the tiles. Waits on the
+//    mbarriers are bounded and end in KVQ_ERRF_TIMEOUT, never in a hang.
 //  * Threads are ordered head-major, token-minor, so a warp writes the codes
 //    of up to 32 consecutive slots of one (page, head) chunk.
 //  * Arithmetic is bit-exact with the published definition (see kvq.h):
 //    binary32 butterflies in ascending stage order (packed f32x2 lanes for
 //    stages >= 2), directed roundings through __fsub_ru / __fdiv_ru /
-//    __float2half_rd / __float2half_ru, RN(1/s) by __frcp_rn, and code
-//    rounding by adding 1.5 * 2^23 (exact round-half-even for values in
-//    [0, 2^22)); the [0, 15] clamp of the definition never acts because
-//    every value lies in [m16, m16 + 15 s16], so the low nibble is the code.
+//    __float2half_rd / __float2half_ru, RN(1/s) by __frcp_rn, and the code
+//    as one fused multiply-add (y - m16) * inv + 1.5 * 2^23, which rounds the
+//    exact product to the nearest integer, ties to even; the [0, 15] clamp of
+//    the definition never acts because every value lies in
+//    [m16, m16 + 15 s16], so the low nibble is the code.
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include "kvq_device.cuh"
@@ -35,13 +40,11 @@
 
 namespace kvq {
 
-constexpr int kAppendThreads = 256;
+constexpr int kAppendThreads = 384;
 
 struct AppendArgs {
-  int T, H, P, NP, num_seqs, bt_stride, tok_per_tile, num_tiles;
-  int64_t tok_stride;
-  const __half* k;
-  const __half* v;
+  int T, H, P, lg_page, NP, num_seqs, bt_stride, tok_per_tile, num_tiles;
+  int box_stride;  // bytes between TMA boxes in a tile buffer (multiple of 1024)
   const int32_t* token_seq;
   const int32_t* token_pos;
   const int32_t* block_table;
@@ -55,57 +58,69 @@ struct AppendArgs {
 
 // D: head_dim, ROT: rotation kind, LGB: log2 of the Hadamard block.
 template <int D, int ROT, int LGB>
-__global__ void __launch_bounds__(kAppendThreads, 1) append_kernel(const AppendArgs a) {
+__global__ void __launch_bounds__(kAppendThreads, 1)
+    append_kernel(const AppendArgs a, const __grid_constant__ CUtensorMap tmk,
+                  const __grid_constant__ CUtensorMap tmv) {
   constexpr int E = D < 128 ? D : 128;   // channels per thread
   constexpr int TPR = D / E;             // threads per row
-  constexpr int ROWB = 2 * E + 16;       // shared-memory pitch of a thread row
-  constexpr int CHUNKS = D / 8;          // 16-byte chunks per (token, head) row
+  constexpr int NH = D / 64;             // 64-channel boxes per row
 
-  extern __shared__ __align__(16) uint8_t smem[];
-  uint8_t* buf0 = smem;
-  uint8_t* buf1 = smem + kAppendThreads * ROWB;
-  float* qtbl = reinterpret_cast<float*>(smem + 2 * kAppendThreads * ROWB);
+  extern __shared__ uint8_t smem_raw[];
+  // 128-byte swizzled TMA boxes need 1024-byte aligned destinations
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const int H = a.H, TOK = a.tok_per_tile;
+  const int bufb = 2 * NH * a.box_stride;  // bytes of one tile buffer
+  uint8_t* const buf0 = smem;
+  uint8_t* const buf1 = smem + bufb;
+  float* qtbl = reinterpret_cast<float*>(smem + 2 * bufb);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * bufb + D * 8);
 
   const int tid = threadIdx.x;
-  const int H = a.H, TOK = a.tok_per_tile;
   const int rows_per_tile = 2 * H * TOK * TPR;
 
+  if (tid == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    mbar_fence_init();
+  }
   if (ROT == KVQ_ROT_QUAT) {
     for (int i = tid; i < D * 2; i += kAppendThreads) qtbl[i] = a.quat[i];
   }
 
-  // this thread's role, fixed for all tiles: thread row = ((kv*H + h)*TOK + t)*TPR + part
+  // this thread's role, fixed for all tiles (token-major):
+  // thread row = ((kv*TOK + t)*H + h)*TPR + part
   const bool active = tid < rows_per_tile;
   int my_part = 0, my_t = 0, my_h = 0, my_kv = 0;
   if (active) {
     my_part = tid % TPR;
     const int r = tid / TPR;
-    my_t = r % TOK;
-    my_h = (r / TOK) % H;
-    my_kv = r / (TOK * H);
+    my_h = r % H;
+    my_t = (r / H) % TOK;
+    my_kv = r / (H * TOK);
   }
+  const int my_line = my_t * H + my_h;  // 128-byte line of this row inside each box
 
-  auto issue_tile = [&](int tile, uint8_t* buf) {
-    const int t0 = tile * TOK;
-    const int warp = tid / kWarp, lane = tid % kWarp;
-    // one (kv, token) row of H*D halves per warp iteration
-    for (int r = warp; r < 2 * TOK; r += kAppendThreads / kWarp) {
-      const int kv = r / TOK, t = r % TOK;
-      if (t0 + t >= a.T) continue;
-      const __half* src = (kv ? a.v : a.k) + (int64_t)(t0 + t) * a.tok_stride;
-      for (int c = lane; c < H * CHUNKS; c += kWarp) {
-        const int h = c / CHUNKS, w = c % CHUNKS;
-        const int ch = w * 8;
-        const int tr = ((kv * H + h) * TOK + t) * TPR + ch / E;
-        cp_async16(buf + tr * ROWB + (ch % E) * 2, src + h * D + ch);
-      }
-    }
+  // One elected thread fills a tile buffer: for K and V, NH boxes of
+  // (64 channels x H heads x TOK tokens), each landing densely (swizzled) at
+  // (kv * NH + box) * box_stride. Tokens past the batch end are zero-filled by
+  // the TMA unit and counted in the transaction bytes.
+  auto issue_tile = [&](int tile, int bi) {
+    if (tile >= a.num_tiles || tid != 0) return;
+    uint8_t* buf = bi ? buf1 : buf0;
+    mbar_arrive_expect_tx(&bars[bi], (uint32_t)(2 * NH * TOK * H * 128));
+#pragma unroll
+    for (int kv = 0; kv < 2; ++kv)
+#pragma unroll
+      for (int hb = 0; hb < NH; ++hb)
+        tma_load_3d(buf + (kv * NH + hb) * a.box_stride, kv ? &tmv : &tmk, hb * 64, 0,
+                    tile * TOK, &bars[bi]);
   };
 
   // Destination of this thread's row, resolved one tile ahead so the
   // dependent metadata loads (token -> sequence/position -> block table) are
-  // in flight while the previous tile computes. row_dst < 0: no store.
+  // in flight while the previous tile computes. A result < 0: no store.
   const bool lead = my_kv == 0 && my_h == 0 && my_part == 0;  // raises the token's flags
+  const int lgP = a.lg_page, Pm = (1 << lgP) - 1;
   auto meta_load = [&](int tile, int& seq, int& pos) {
     const int tok = tile * TOK + my_t;
     seq = -1;
@@ -121,35 +136,41 @@ __global__ void __launch_bounds__(kAppendThreads, 1) append_kernel(const AppendA
       if (lead) raise_flag(a.err, KVQ_ERRF_SEQ);
       return -1;
     }
-    if (pos < 0 || pos / a.P >= a.bt_stride) {
+    if (pos < 0 || (pos >> lgP) >= a.bt_stride) {
       if (lead) raise_flag(a.err, KVQ_ERRF_POS);
       return -1;
     }
-    const int page = a.block_table[(int64_t)seq * a.bt_stride + pos / a.P];
+    const int page = a.block_table[(int64_t)seq * a.bt_stride + (pos >> lgP)];
     if (page < 0 || page >= a.NP) {
       if (lead) raise_flag(a.err, KVQ_ERRF_PAGE);
       return -1;
     }
-    return ((int64_t)page * H + my_h) * a.P + pos % a.P;
+    return (((int64_t)page * H + my_h) << lgP) + (pos & Pm);
   };
 
+  __syncthreads();  // barriers initialised, quaternion table visible
   int tile = blockIdx.x;
-  if (tile < a.num_tiles) issue_tile(tile, buf0);
-  cp_async_commit();
+  issue_tile(tile, 0);
   int seq_n, pos_n;
   meta_load(tile, seq_n, pos_n);
   int64_t dst_cur = resolve(seq_n, pos_n);
-  __syncthreads();  // quaternion table visible
+  uint32_t parity = 0;  // bit b: phase parity to wait for on buffer b
 
   for (int it = 0; tile < a.num_tiles; ++it, tile += gridDim.x) {
-    uint8_t* cur = (it & 1) ? buf1 : buf0;
-    uint8_t* nxt = (it & 1) ? buf0 : buf1;
+    const int b = it & 1;
+    uint8_t* cur = b ? buf1 : buf0;
     const int next = tile + gridDim.x;
-    if (next < a.num_tiles) issue_tile(next, nxt);
-    cp_async_commit();
+    issue_tile(next, b ^ 1);
     meta_load(next, seq_n, pos_n);  // consumed after this tile's compute
-    cp_async_wait<1>();
-    __syncthreads();
+    const bool ok = mbar_wait(&bars[b], (parity >> b) & 1u);
+    parity ^= 1u << b;
+    if (!__syncthreads_and(ok)) {
+      // a copy never completed: report, let the other buffer's copies land
+      // (bounded), and leave without touching the pools
+      if (tid == 0) raise_flag(a.err, KVQ_ERRF_TIMEOUT);
+      if (next < a.num_tiles) mbar_wait(&bars[b ^ 1], (parity >> (b ^ 1)) & 1u);
+      return;
+    }
 
     const int tok = tile * TOK + my_t;
     // rows of tokens past the batch end do nothing; every other active row
@@ -158,23 +179,35 @@ __global__ void __launch_bounds__(kAppendThreads, 1) append_kernel(const AppendA
     if (active && tok < a.T) {
       {
         float x[E];
-        const uint4* row = reinterpret_cast<const uint4*>(cur + tid * ROWB);
 #pragma unroll
         for (int c = 0; c < E / 8; ++c) {
-          const uint4 u = row[c];
+          // channel block c of this thread: box (part*E/64 + c/8), 16-byte
+          // chunk c%8 of line my_line, at its 128B-swizzled position
+          const uint8_t* box = cur + (my_kv * NH + my_part * (E / 64) + c / 8) * a.box_stride;
+          const uint4 u = *reinterpret_cast<const uint4*>(
+              box + my_line * 128 + (((c % 8) ^ (my_line & 7)) << 4));
           const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const float2 f = __half22float2(u32_as_h2(w[q]));
-            x[8 * c + 2 * q] = f.x;
-            x[8 * c + 2 * q + 1] = f.y;
+            const __half2 h2 = u32_as_h2(w[q]);
+            if (ROT == KVQ_ROT_HADAMARD) {
+              // first butterfly stage straight from binary16: widening is
+              // exact, so (x_i + x_{i+1}, x_i - x_{i+1}) round as in binary32
+              const float b = __high2float(h2);
+              x[8 * c + 2 * q] = add_h_f(__low2half(h2), b);
+              x[8 * c + 2 * q + 1] = sub_h_f(__low2half(h2), b);
+            } else {
+              const float2 f = __half22float2(h2);
+              x[8 * c + 2 * q] = f.x;
+              x[8 * c + 2 * q + 1] = f.y;
+            }
           }
         }
 
         // the two threads of a d = 256 row are lanes 2i, 2i+1 of one warp
         const unsigned pair_mask = 3u << ((tid % kWarp) & ~1);
         if (ROT == KVQ_ROT_HADAMARD) {
-          hadamard_regs<E, LGB>(x, my_part, pair_mask);
+          hadamard_regs<E, LGB, true>(x, my_part, pair_mask);
         } else if (ROT == KVQ_ROT_QUAT) {
           quat_regs<E>(x, qtbl, my_part * E);
         }
@@ -206,19 +239,18 @@ __global__ void __launch_bounds__(kAppendThreads, 1) append_kernel(const AppendA
         uint32_t packed[E / 8];
         if (s != 0.0f) {
           const float inv = __frcp_rn(s);
-          const uint64_t m2 = pk(m, m);
+          const uint64_t m2 = pk(m, m), inv2 = pk(inv, inv);
           const uint64_t magic2 = pk(12582912.0f, 12582912.0f);  // 1.5 * 2^23
 #pragma unroll
           for (int c = 0; c < E / 8; ++c) {
             uint32_t b[8];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-              // the product must be rounded on its own before the rounding
-              // add: __fmul_rn is never contracted into a fused multiply-add
-              // (the packed multiply was seen to be, at exact .5 ties)
-              const float2 t = upk(sub2(pk(x[8 * c + 2 * q], x[8 * c + 2 * q + 1]), m2));
-              const float t1x = __fmul_rn(t.x, inv), t1y = __fmul_rn(t.y, inv);
-              const float2 r = upk(add2(pk(t1x, t1y), magic2));
+              // code = nearest integer (ties to even) of the exact product
+              // t * inv: one fused multiply-add with 1.5 * 2^23 rounds it
+              // once, leaving the integer in the low mantissa bits
+              const uint64_t t = sub2(pk(x[8 * c + 2 * q], x[8 * c + 2 * q + 1]), m2);
+              const float2 r = upk(fma2(t, inv2, magic2));
               b[2 * q] = __float_as_uint(r.x);
               b[2 * q + 1] = __float_as_uint(r.y);
             }
@@ -250,30 +282,68 @@ __global__ void __launch_bounds__(kAppendThreads, 1) append_kernel(const AppendA
     dst_cur = resolve(seq_n, pos_n);  // next tile's destination (its loads were in flight)
     __syncthreads();  // buffer `cur` is refilled by the next iteration's issue
   }
-  cp_async_wait<0>();
+}
+
+// Driver entry point for tensor-map encoding (no link-time libcuda needed).
+static PFN_cuTensorMapEncodeTiled encode_fn() {
+  static PFN_cuTensorMapEncodeTiled fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled>(p);
+  }
+  return fn;
+}
+
+// [T][H][D] binary16 rows with token stride tok_stride (elements) as a 3-D
+// tensor (D innermost); box (64 channels, H heads, TOK tokens), 128B swizzle.
+static bool encode_rows(CUtensorMap* m, const void* base, int D, int H, int T,
+                        int64_t tok_stride, int TOK) {
+  PFN_cuTensorMapEncodeTiled fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)tok_stride * 2};
+  const cuuint32_t box[3] = {64u, (cuuint32_t)H, (cuuint32_t)TOK};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+static size_t append_smem(int D, int box_stride) {
+  return 1024 + 2 * (size_t)(2 * (D / 64)) * box_stride + (size_t)D * 8 + 2 * sizeof(uint64_t);
 }
 
 template <int D, int ROT, int LGB>
-static cudaError_t launch_append(const AppendArgs& a, int grid, cudaStream_t st) {
-  constexpr int E = D < 128 ? D : 128;
-  const size_t smem = 2 * kAppendThreads * (2 * E + 16) + D * 2 * sizeof(float);
+static cudaError_t launch_append(const AppendArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
+                                 int grid, cudaStream_t st) {
+  const size_t smem = append_smem(D, a.box_stride);
   auto kern = append_kernel<D, ROT, LGB>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kAppendThreads, smem, st>>>(a);
+  kern<<<grid, kAppendThreads, smem, st>>>(a, tk, tv);
   return cudaGetLastError();
 }
 
 template <int D>
-static cudaError_t dispatch_rot(const AppendArgs& a, int rot, int lgb, int grid, cudaStream_t st) {
-  if (rot == KVQ_ROT_NONE) return launch_append<D, KVQ_ROT_NONE, 0>(a, grid, st);
-  if (rot == KVQ_ROT_QUAT) return launch_append<D, KVQ_ROT_QUAT, 0>(a, grid, st);
+static cudaError_t dispatch_rot(const AppendArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
+                                int rot, int lgb, int grid, cudaStream_t st) {
+  if (rot == KVQ_ROT_NONE) return launch_append<D, KVQ_ROT_NONE, 0>(a, tk, tv, grid, st);
+  if (rot == KVQ_ROT_QUAT) return launch_append<D, KVQ_ROT_QUAT, 0>(a, tk, tv, grid, st);
   switch (lgb) {
-    case 4: return launch_append<D, KVQ_ROT_HADAMARD, 4>(a, grid, st);
-    case 5: return launch_append<D, KVQ_ROT_HADAMARD, 5>(a, grid, st);
-    case 6: return launch_append<D, KVQ_ROT_HADAMARD, 6>(a, grid, st);
-    case 7: if (D >= 128) return launch_append<D, KVQ_ROT_HADAMARD, (D >= 128 ? 7 : 6)>(a, grid, st); break;
-    case 8: if (D >= 256) return launch_append<D, KVQ_ROT_HADAMARD, (D >= 256 ? 8 : 6)>(a, grid, st); break;
+    case 4: return launch_append<D, KVQ_ROT_HADAMARD, 4>(a, tk, tv, grid, st);
+    case 5: return launch_append<D, KVQ_ROT_HADAMARD, 5>(a, tk, tv, grid, st);
+    case 6: return launch_append<D, KVQ_ROT_HADAMARD, 6>(a, tk, tv, grid, st);
+    case 7:
+      if (D >= 128) return launch_append<D, KVQ_ROT_HADAMARD, (D >= 128 ? 7 : 6)>(a, tk, tv, grid, st);
+      break;
+    case 8:
+      if (D >= 256) return launch_append<D, KVQ_ROT_HADAMARD, (D >= 256 ? 8 : 6)>(a, tk, tv, grid, st);
+      break;
   }
   return cudaErrorInvalidValue;
 }
@@ -287,7 +357,7 @@ int append_launch(const kvq_cache_desc& d, int32_t T, const void* k, const void*
   const int E = D < 128 ? D : 128;
   const int TPR = D / E;
   const int tok_max = kAppendThreads / (2 * d.num_kv_heads * TPR);
-  if (tok_max < 1) return KVQ_ERR_UNSUPPORTED;
+  if (tok_max < 1 || d.num_kv_heads > 256) return KVQ_ERR_UNSUPPORTED;
   const int sms = device_sm_count();
   if (sms <= 0) return KVQ_ERR_CUDA;
   // small batches: fewer tokens per tile so more SMs share the work
@@ -298,14 +368,14 @@ int append_launch(const kvq_cache_desc& d, int32_t T, const void* k, const void*
   a.T = T;
   a.H = d.num_kv_heads;
   a.P = d.page_size;
+  a.lg_page = 0;
+  while ((1 << a.lg_page) < d.page_size) ++a.lg_page;
   a.NP = d.num_pages;
   a.num_seqs = num_seqs;
   a.bt_stride = bt_stride;
   a.tok_per_tile = tok;
   a.num_tiles = (T + tok - 1) / tok;
-  a.tok_stride = tok_stride;
-  a.k = static_cast<const __half*>(k);
-  a.v = static_cast<const __half*>(v);
+  a.box_stride = (tok * d.num_kv_heads * 128 + 1023) / 1024 * 1024;
   a.token_seq = token_seq;
   a.token_pos = token_pos;
   a.block_table = block_table;
@@ -315,14 +385,18 @@ int append_launch(const kvq_cache_desc& d, int32_t T, const void* k, const void*
   a.v_params = static_cast<uint32_t*>(v_params);
   a.quat = d.quat;
   a.err = err;
+  CUtensorMap tk, tv;
+  if (!encode_rows(&tk, k, D, a.H, T, tok_stride, tok) ||
+      !encode_rows(&tv, v, D, a.H, T, tok_stride, tok))
+    return KVQ_ERR_CUDA;
   const int grid = a.num_tiles < sms ? a.num_tiles : sms;
   int lgb = 0;
   while ((1 << lgb) < d.rot_block) ++lgb;
   cudaError_t e;
   switch (D) {
-    case 64: e = dispatch_rot<64>(a, d.rot_kind, lgb, grid, st); break;
-    case 128: e = dispatch_rot<128>(a, d.rot_kind, lgb, grid, st); break;
-    case 256: e = dispatch_rot<256>(a, d.rot_kind, lgb, grid, st); break;
+    case 64: e = dispatch_rot<64>(a, tk, tv, d.rot_kind, lgb, grid, st); break;
+    case 128: e = dispatch_rot<128>(a, tk, tv, d.rot_kind, lgb, grid, st); break;
+    case 256: e = dispatch_rot<256>(a, tk, tv, d.rot_kind, lgb, grid, st); break;
     default: return KVQ_ERR_UNSUPPORTED;
   }
   if (e == cudaErrorInvalidValue) return KVQ_ERR_UNSUPPORTED;

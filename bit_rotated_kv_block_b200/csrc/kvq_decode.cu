@@ -6,32 +6,30 @@
 // Hadamard (or quaternion) map as the keys, so q . k is unchanged, and the
 // output is rotated back once per query head.
 //
-// Three kernels on the caller's stream:
-//  1. qprep:   qhat = R q for every (sequence, query head), binary32, into the
-//              workspace.
-//  2. split:   one warp per (sequence, KV head, split of the page range). The
-//              warp streams its (page, KV head) chunks (codes + params of K
-//              and V, contiguous in the pool) into a 2-4 stage shared-memory
-//              ring with cp.async, and runs both contractions on tensor cores
-//              (mma.sync m16n8k16, f16 x f16 -> f32):
-//                QK^T: A = [qhat_hi ; qhat_lo] rows of the query heads, B =
-//                      K codes (c - 8, exact in f16) as columns, so the score
-//                      fragment of head r for tokens {2j, 2j+1, 2j+8, 2j+9}
-//                      already sits in lane (r, j) -- exactly the B operand
-//                      layout of the PV product, no transposes;
-//                PV:   A = V codes transposed (channels x tokens) built from
-//                      nibbles with prmt/lop3, B = p * s_v split into f16
-//                      hi + lo columns.
-//              Scale and zero-point are applied algebraically:
-//                qhat . khat = s_k * sum (c - 8) qhat + (m_k + 8 s_k) sum qhat,
-//                sum p vhat  = sum (p s_v)(c - 8)     + sum p (m_v + 8 s_v).
-//              Online softmax in base 2; the warp writes (acc, max, sum) per
-//              query head to the workspace.
-//  3. combine: log-sum-exp merge of the splits, normalisation, R^-1 in
-//              binary32 registers, float32 output.
-// No kernel waits on another CTA; completion of async copies is tracked by
-// the hardware commit groups, so nothing spins.
-
+// One kernel, one warp per (sequence, KV head, split of the page range):
+//  1. The warp rotates its query heads in registers: lane (r, j) holds
+//     channels [j*d/4, (j+1)*d/4) of query head r (GP = 8) or r % 4 (GP = 4);
+//     butterfly stages inside a quarter run in registers, wider ones across
+//     lanes j by shuffles.
+//  2. It streams its (page, KV head) chunks (codes + params of K and V,
+//     contiguous in the pool) into a 2-4 stage shared-memory ring with
+//     cp.async and runs both contractions on tensor cores (mma.sync
+//     m16n8k16, f16 x f16 -> f32):
+//       QK^T: A = [qhat_hi ; qhat_lo] rows of the query heads, B = K codes
+//             (c - 8, exact in f16) as columns, so the score fragment of head
+//             r for tokens {2j, 2j+1, 2j+8, 2j+9} already sits in lane (r, j)
+//             -- exactly the B operand layout of the PV product;
+//       PV:   A = V codes transposed (channels x tokens) built from nibbles
+//             with prmt/lop3, B = p * s_v split into f16 hi + lo columns.
+//     Scale and zero-point are applied algebraically:
+//       qhat . khat = s_k * sum (c - 8) qhat + (m_k + 8 s_k) sum qhat,
+//       sum p vhat  = sum (p s_v)(c - 8)     + sum p (m_v + 8 s_v).
+//     Online softmax in base 2.
+//  3. It writes (acc, max, sum) per query head to the workspace, fences, and
+//     bumps a per-(sequence, KV head) counter; the warp that brings the
+//     counter to the number of splits merges all splits (log-sum-exp),
+//     normalises, rotates back in registers, writes the float32 output and
+//     resets the counter to zero. No warp ever waits on another.
 #include <cuda_runtime.h>
 
 #include "kvq_device.cuh"
@@ -46,52 +44,21 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 struct DecodeArgs {
   int S, Hq, H, G, P, NP, bt_stride, max_seq_len, splits, pages_per_split;
+  int rot_kind, lgb;
   float scale2;  // sm_scale * log2(e)
+  const __half* q;  // [S][Hq][D]
+  const float* quat;
   const int32_t* seq_lens;
   const int32_t* block_table;
   const uint8_t* k_codes;
   const uint32_t* k_params;
   const uint8_t* v_codes;
   const uint32_t* v_params;
-  const float* qhat;  // [S][Hq][D]
-  float* part;        // [S][Hq][splits][D + 2]
+  float* out;        // [S][Hq][D]
+  float* part;       // [S][Hq][splits][D + 4]: acc[D], max, sum, 2 pad
+  int32_t* counter;  // [S][H], zero between calls
   int32_t* err;
 };
-
-// ---------------------------------------------------------------------------
-// 1. query rotation: one thread per E channels of a (sequence, query head) row
-// ---------------------------------------------------------------------------
-
-template <int D, int ROT, int LGB>
-__global__ void __launch_bounds__(128) qprep_kernel(const __half* __restrict__ q, int rows,
-                                                    const float* __restrict__ quat,
-                                                    float* __restrict__ qhat) {
-  constexpr int E = D < 128 ? D : 128;
-  constexpr int TPR = D / E;
-  const int gt = blockIdx.x * blockDim.x + threadIdx.x;
-  const int row = gt / TPR, part = gt % TPR;
-  // rows of a d = 256 head are lane pairs; keep whole pairs in or out
-  if (row >= rows) return;
-  float x[E];
-  const uint4* src = reinterpret_cast<const uint4*>(q + (int64_t)row * D + part * E);
-#pragma unroll
-  for (int c = 0; c < E / 8; ++c) {
-    const uint4 u = src[c];
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 f = __half22float2(u32_as_h2(w[i]));
-      x[8 * c + 2 * i] = f.x;
-      x[8 * c + 2 * i + 1] = f.y;
-    }
-  }
-  const unsigned pair_mask = 3u << ((threadIdx.x % kWarp) & ~1);
-  if (ROT == KVQ_ROT_HADAMARD) hadamard_regs<E, LGB>(x, part, pair_mask);
-  if (ROT == KVQ_ROT_QUAT) quat_regs<E>(x, quat, part * E);
-  float4* dst = reinterpret_cast<float4*>(qhat + (int64_t)row * D + part * E);
-#pragma unroll
-  for (int c = 0; c < E / 4; ++c) dst[c] = make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]);
-}
 
 // ---------------------------------------------------------------------------
 // 2. split kernel
@@ -129,6 +96,43 @@ template <int D>
 __device__ __forceinline__ int k_unit_off(int t, int u) {
   if (D == 256) return t * 128 + ((u ^ (t & 1)) << 4);
   return t * (D / 2) + (u << 4);
+}
+
+// Rotation of a query (or output) row held as quarters: lane j of a group
+// of four consecutive lanes owns channels [j*QW, (j+1)*QW). Butterfly
+// stages with distance < QW run in registers, wider ones across the lanes
+// (distance QW: lane ^ 1, 2*QW: lane ^ 2); the lower-channel lane adds and
+// the upper one subtracts. All 32 lanes must call it. Binary32, not part of
+// the bit-exact quantize path.
+template <int QW>
+__device__ __forceinline__ void rotate_quarter(float (&x)[QW], int j, int rot_kind, int lgb,
+                                               const float* quat, bool inverse) {
+  if (rot_kind == KVQ_ROT_HADAMARD) {
+    constexpr int LQ = QW == 32 ? 5 : 6;
+    const int lin = lgb < LQ ? lgb : LQ;
+    switch (lin) {
+      case 4: fwht_regs<QW, 4>(x); break;
+      case 5: fwht_regs<QW, 5>(x); break;
+      default: fwht_regs<QW, (LQ > 5 ? 6 : 5)>(x); break;
+    }
+    for (int hs = QW; hs < (1 << lgb); hs <<= 1) {
+      const int m = hs / QW;  // 1 or 2: lane distance
+      const bool lower = (j & m) == 0;
+#pragma unroll
+      for (int i = 0; i < QW; ++i) {
+        const float o = __shfl_xor_sync(0xffffffffu, x[i], m);
+        x[i] = lower ? x[i] + o : o - x[i];
+      }
+    }
+    const float cb = hadamard_scale(lgb);
+#pragma unroll
+    for (int i = 0; i < QW; ++i) x[i] *= cb;
+  } else if (rot_kind == KVQ_ROT_QUAT) {
+    if (inverse)
+      quat_inv_regs<QW>(x, quat, j * QW);
+    else
+      quat_regs<QW>(x, quat, j * QW);
+  }
 }
 
 template <int D, int P, int GP>
@@ -174,12 +178,21 @@ __global__ void __launch_bounds__(kDecWarps * kWarp) decode_split_kernel(const D
   uint32_t qa[C::NKS][4];
   {
     float x[C::QW];
-    const float* src = a.qhat + ((int64_t)s * a.Hq + g) * D + j * C::QW;
+    {
+      const uint4* src = reinterpret_cast<const uint4*>(a.q + ((int64_t)s * a.Hq + g) * D + j * C::QW);
 #pragma unroll
-    for (int c = 0; c < C::QW / 4; ++c) {
-      float4 f = head_ok ? reinterpret_cast<const float4*>(src)[c] : make_float4(0.f, 0.f, 0.f, 0.f);
-      x[4 * c] = f.x; x[4 * c + 1] = f.y; x[4 * c + 2] = f.z; x[4 * c + 3] = f.w;
+      for (int c = 0; c < C::QW / 8; ++c) {
+        const uint4 u = head_ok ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __half22float2(u32_as_h2(w4[e]));
+          x[8 * c + 2 * e] = f.x;
+          x[8 * c + 2 * e + 1] = f.y;
+        }
+      }
     }
+    rotate_quarter<C::QW>(x, j, a.rot_kind, a.lgb, a.quat, false);
     float part = 0.f;
 #pragma unroll
     for (int i = 0; i < C::QW; ++i) part += x[i];
@@ -454,7 +467,7 @@ __global__ void __launch_bounds__(kDecWarps * kWarp) decode_split_kernel(const D
   for (int hc = 0; hc < 2; ++hc) {
     const int gh = c0 + hc;
     if (!writer || gh >= a.G) continue;
-    float* dst = a.part + (base + (int64_t)gh * a.splits) * (D + 2);
+    float* dst = a.part + (base + (int64_t)gh * a.splits) * (D + 4);
     const float ov = hc ? o1 : o0;
 #pragma unroll
     for (int mt = 0; mt < C::NMT; ++mt) {
@@ -473,52 +486,57 @@ __global__ void __launch_bounds__(kDecWarps * kWarp) decode_split_kernel(const D
   }
   // the lanes that own head hr's softmax state write it (one lane per head)
   if (j == 0 && !lo_row && head_ok) {
-    float* dst = a.part + (base + (int64_t)hr * a.splits) * (D + 2);
+    float* dst = a.part + (base + (int64_t)hr * a.splits) * (D + 4);
     dst[D] = M;
     dst[D + 1] = Lp;
   }
-}
 
-// ---------------------------------------------------------------------------
-// 3. combine: one thread per E channels of a (sequence, query head) row
-// ---------------------------------------------------------------------------
-
-template <int D, int ROT, int LGB>
-__global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ part, int rows,
-                                                      int splits, const float* __restrict__ quat,
-                                                      float* __restrict__ out) {
-  constexpr int E = D < 128 ? D : 128;
-  constexpr int TPR = D / E;
-  const int gt = blockIdx.x * blockDim.x + threadIdx.x;
-  const int row = gt / TPR, pt = gt % TPR;
-  if (row >= rows) return;
-  const float* src = part + (int64_t)row * splits * (D + 2);
-  float Mx = -INFINITY;
-  for (int i = 0; i < splits; ++i) Mx = fmaxf(Mx, src[(int64_t)i * (D + 2) + D]);
-  float x[E];
+  // ---- the last warp of this (sequence, KV head) merges the splits
+  __threadfence();
+  __syncwarp();
+  int last = 0;
+  if (lane == 0) last = atomicAdd(a.counter + (int64_t)s * a.H + h, 1) == a.splits - 1;
+  last = __shfl_sync(0xffffffffu, last, 0);
+  if (!last) return;
+  __threadfence();
+  const bool owner = head_ok && !lo_row;
+  float x[C::QW];
 #pragma unroll
-  for (int c = 0; c < E; ++c) x[c] = 0.f;
-  float Ls = 0.f;
-  if (Mx != -INFINITY) {
-    for (int i = 0; i < splits; ++i) {
-      const float* p = src + (int64_t)i * (D + 2);
-      const float Mi = p[D];
-      if (Mi == -INFINITY) continue;
-      const float w = fast_exp2(Mi - Mx);
-      Ls += w * p[D + 1];
+  for (int c = 0; c < C::QW; ++c) x[c] = 0.f;
+  if (owner) {
+    const float* src = a.part + ((int64_t)s * a.Hq + g) * a.splits * (D + 4);
+    float Mx = -INFINITY;
+    for (int i = 0; i < a.splits; ++i) Mx = fmaxf(Mx, __ldcg(src + (int64_t)i * (D + 4) + D));
+    float Ls = 0.f;
+    if (Mx != -INFINITY) {
+      for (int i = 0; i < a.splits; ++i) {
+        const float* pi = src + (int64_t)i * (D + 4);
+        const float Mi = __ldcg(pi + D);
+        if (Mi == -INFINITY) continue;
+        const float wgt = fast_exp2(Mi - Mx);
+        Ls += wgt * __ldcg(pi + D + 1);
+        const float4* v4 = reinterpret_cast<const float4*>(pi + j * C::QW);
 #pragma unroll
-      for (int c = 0; c < E; ++c) x[c] += w * p[pt * E + c];
+        for (int c = 0; c < C::QW / 4; ++c) {
+          const float4 f = __ldcg(v4 + c);
+          x[4 * c] += wgt * f.x;
+          x[4 * c + 1] += wgt * f.y;
+          x[4 * c + 2] += wgt * f.z;
+          x[4 * c + 3] += wgt * f.w;
+        }
+      }
     }
+    const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+#pragma unroll
+    for (int c = 0; c < C::QW; ++c) x[c] *= inv;
   }
-  const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+  rotate_quarter<C::QW>(x, j, a.rot_kind, a.lgb, a.quat, true);  // R^-1 (R^-1 = R for Hadamard)
+  if (owner) {
+    float4* dst = reinterpret_cast<float4*>(a.out + ((int64_t)s * a.Hq + g) * D + j * C::QW);
 #pragma unroll
-  for (int c = 0; c < E; ++c) x[c] *= inv;
-  const unsigned pair_mask = 3u << ((threadIdx.x % kWarp) & ~1);
-  if (ROT == KVQ_ROT_HADAMARD) hadamard_regs<E, LGB>(x, pt, pair_mask);  // R^-1 = R
-  if (ROT == KVQ_ROT_QUAT) quat_inv_regs<E>(x, quat, pt * E);
-  float4* dst = reinterpret_cast<float4*>(out + (int64_t)row * D + pt * E);
-#pragma unroll
-  for (int c = 0; c < E / 4; ++c) dst[c] = make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]);
+    for (int c = 0; c < C::QW / 4; ++c) dst[c] = make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]);
+  }
+  if (lane == 0) a.counter[(int64_t)s * a.H + h] = 0;
 }
 
 // ---------------------------------------------------------------------------
@@ -547,15 +565,19 @@ static int split_resident_warps() {
   return cached;
 }
 
+#define KVQ_DECODE_CONFIGS(X)                                                                  \
+  X(128, 16, 4) X(128, 16, 8) X(128, 32, 4) X(128, 32, 8) X(128, 64, 4) X(128, 64, 8)          \
+  X(256, 16, 4) X(256, 32, 4) X(256, 64, 4)
+
 static int resident_warps(int D, int P, int GP) {
 #define KVQ_RW(d_, p_, g_) \
   if (D == d_ && P == p_ && GP == g_) return split_resident_warps<d_, p_, g_>();
-  KVQ_RW(128, 16, 4) KVQ_RW(128, 16, 8) KVQ_RW(128, 32, 4) KVQ_RW(128, 32, 8)
-  KVQ_RW(128, 64, 4) KVQ_RW(128, 64, 8) KVQ_RW(256, 16, 4) KVQ_RW(256, 32, 4)
-  KVQ_RW(256, 64, 4)
+  KVQ_DECODE_CONFIGS(KVQ_RW)
 #undef KVQ_RW
   return 148 * 8;
 }
+
+static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 DecodePlan decode_plan(const kvq_cache_desc& d, int32_t S, int32_t Hq, int32_t max_seq_len) {
   DecodePlan pl{};
@@ -573,9 +595,9 @@ DecodePlan decode_plan(const kvq_cache_desc& d, int32_t S, int32_t Hq, int32_t m
   if (splits > pl.pages_max) splits = pl.pages_max;
   pl.pages_per_split = (pl.pages_max + splits - 1) / splits;
   pl.splits = (pl.pages_max + pl.pages_per_split - 1) / pl.pages_per_split;
-  const size_t qhat = (size_t)S * Hq * d.head_dim * sizeof(float);
-  const size_t parts = (size_t)S * Hq * pl.splits * (d.head_dim + 2) * sizeof(float);
-  pl.workspace = ((qhat + 255) / 256) * 256 + parts;
+  const size_t counters = (size_t)S * d.num_kv_heads * sizeof(int32_t);
+  const size_t parts = (size_t)S * Hq * pl.splits * (d.head_dim + 4) * sizeof(float);
+  pl.workspace = align256(counters) + parts;
   return pl;
 }
 
@@ -594,46 +616,8 @@ static cudaError_t launch_split(const DecodeArgs& a, cudaStream_t st) {
 static cudaError_t launch_split_any(const DecodeArgs& a, int D, int GP, cudaStream_t st) {
 #define KVQ_LS(d_, p_, g_) \
   if (D == d_ && a.P == p_ && GP == g_) return launch_split<d_, p_, g_>(a, st);
-  KVQ_LS(128, 16, 4) KVQ_LS(128, 16, 8) KVQ_LS(128, 32, 4) KVQ_LS(128, 32, 8)
-  KVQ_LS(128, 64, 4) KVQ_LS(128, 64, 8) KVQ_LS(256, 16, 4) KVQ_LS(256, 32, 4)
-  KVQ_LS(256, 64, 4)
+  KVQ_DECODE_CONFIGS(KVQ_LS)
 #undef KVQ_LS
-  return cudaErrorInvalidValue;
-}
-
-template <int D, int ROT, int LGB>
-static cudaError_t launch_rot_pair(const __half* q, int rows, const float* quat, float* qhat,
-                                   const float* part, int splits, float* out, bool prep,
-                                   cudaStream_t st) {
-  constexpr int TPR = D <= 128 ? 1 : D / 128;
-  const int threads = rows * TPR;
-  const int grid = (threads + 127) / 128;
-  if (prep)
-    qprep_kernel<D, ROT, LGB><<<grid, 128, 0, st>>>(q, rows, quat, qhat);
-  else
-    combine_kernel<D, ROT, LGB><<<grid, 128, 0, st>>>(part, rows, splits, quat, out);
-  return cudaGetLastError();
-}
-
-template <int D>
-static cudaError_t launch_rot(int rot, int lgb, const __half* q, int rows, const float* quat,
-                              float* qhat, const float* part, int splits, float* out, bool prep,
-                              cudaStream_t st) {
-  if (rot == KVQ_ROT_NONE)
-    return launch_rot_pair<D, KVQ_ROT_NONE, 0>(q, rows, quat, qhat, part, splits, out, prep, st);
-  if (rot == KVQ_ROT_QUAT)
-    return launch_rot_pair<D, KVQ_ROT_QUAT, 0>(q, rows, quat, qhat, part, splits, out, prep, st);
-  switch (lgb) {
-    case 4: return launch_rot_pair<D, KVQ_ROT_HADAMARD, 4>(q, rows, quat, qhat, part, splits, out, prep, st);
-    case 5: return launch_rot_pair<D, KVQ_ROT_HADAMARD, 5>(q, rows, quat, qhat, part, splits, out, prep, st);
-    case 6: return launch_rot_pair<D, KVQ_ROT_HADAMARD, 6>(q, rows, quat, qhat, part, splits, out, prep, st);
-    case 7:
-      if (D >= 128) return launch_rot_pair<D, KVQ_ROT_HADAMARD, (D >= 128 ? 7 : 6)>(q, rows, quat, qhat, part, splits, out, prep, st);
-      break;
-    case 8:
-      if (D >= 256) return launch_rot_pair<D, KVQ_ROT_HADAMARD, (D >= 256 ? 8 : 6)>(q, rows, quat, qhat, part, splits, out, prep, st);
-      break;
-  }
   return cudaErrorInvalidValue;
 }
 
@@ -651,40 +635,25 @@ int decode_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, const void* q,
   if (workspace == nullptr || workspace_bytes < pl.workspace) return KVQ_ERR_WORKSPACE;
   int lgb = 0;
   while ((1 << lgb) < d.rot_block) ++lgb;
-  float* qhat = static_cast<float*>(workspace);
-  const size_t qbytes = (((size_t)S * Hq * D * sizeof(float)) + 255) / 256 * 256;
-  float* part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + qbytes);
-  const __half* qh = static_cast<const __half*>(q);
-  const int rows = S * Hq;
-
-  cudaError_t e;
-  switch (D) {
-    case 128: e = launch_rot<128>(d.rot_kind, lgb, qh, rows, d.quat, qhat, part, pl.splits, out, true, st); break;
-    case 256: e = launch_rot<256>(d.rot_kind, lgb, qh, rows, d.quat, qhat, part, pl.splits, out, true, st); break;
-    default: return KVQ_ERR_UNSUPPORTED;
-  }
-  if (e == cudaErrorInvalidValue) return KVQ_ERR_UNSUPPORTED;
-  if (e != cudaSuccess) return KVQ_ERR_CUDA;
 
   DecodeArgs a;
   a.S = S; a.Hq = Hq; a.H = d.num_kv_heads; a.G = G; a.P = d.page_size; a.NP = d.num_pages;
   a.bt_stride = bt_stride; a.max_seq_len = max_seq_len; a.splits = pl.splits;
   a.pages_per_split = pl.pages_per_split;
+  a.rot_kind = d.rot_kind; a.lgb = lgb;
   a.scale2 = sm_scale * kLog2e;
+  a.q = static_cast<const __half*>(q); a.quat = d.quat;
   a.seq_lens = seq_lens; a.block_table = block_table;
   a.k_codes = k_codes; a.k_params = static_cast<const uint32_t*>(k_params);
   a.v_codes = v_codes; a.v_params = static_cast<const uint32_t*>(v_params);
-  a.qhat = qhat; a.part = part; a.err = err;
-  e = launch_split_any(a, D, GP, st);
+  a.out = out;
+  a.counter = static_cast<int32_t*>(workspace);
+  a.part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                    align256((size_t)S * d.num_kv_heads * sizeof(int32_t)));
+  a.err = err;
+  const cudaError_t e = launch_split_any(a, D, GP, st);
   if (e == cudaErrorInvalidValue) return KVQ_ERR_UNSUPPORTED;
-  if (e != cudaSuccess) return KVQ_ERR_CUDA;
-
-  switch (D) {
-    case 128: e = launch_rot<128>(d.rot_kind, lgb, qh, rows, d.quat, qhat, part, pl.splits, out, false, st); break;
-    default: e = launch_rot<256>(d.rot_kind, lgb, qh, rows, d.quat, qhat, part, pl.splits, out, false, st); break;
-  }
-  if (e != cudaSuccess) return KVQ_ERR_CUDA;
-  return KVQ_OK;
+  return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 
 }  // namespace kvq

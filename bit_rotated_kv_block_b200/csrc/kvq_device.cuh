@@ -15,9 +15,11 @@ namespace kvq {
 constexpr int kWarp = 32;
 
 // ---------------------------------------------------------------------------
-// Packed binary32 pairs. add/sub/mul.rn.f32x2 round each lane as IEEE
-// binary32 with round-to-nearest-even and are never contracted into FMAs, so
-// results are identical to two scalar operations.
+// Packed binary32 pairs: each lane rounds as IEEE binary32 with
+// round-to-nearest-even. A packed multiply may be fused with a following add
+// by the code generator, so mul2 is only used where the product is exact
+// (a power-of-two factor); products that must round on their own use
+// __fmul_rn, which is never contracted.
 // ---------------------------------------------------------------------------
 
 __device__ __forceinline__ uint64_t pk(float lo, float hi) {
@@ -44,6 +46,26 @@ __device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
   uint64_t r;
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
+}
+
+// Packed fused multiply-add: one rounding of a*b + c per lane.
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
+// Mixed-precision add / subtract: widen the binary16 operand exactly, then
+// one binary32 rounding (a + c, a - c).
+__device__ __forceinline__ float add_h_f(__half a, float c) {
+  float d;
+  asm("add.rn.f32.f16 %0, %1, %2;" : "=f"(d) : "h"(__half_as_ushort(a)), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float sub_h_f(__half a, float c) {
+  float d;
+  asm("sub.rn.f32.f16 %0, %1, %2;" : "=f"(d) : "h"(__half_as_ushort(a)), "f"(c));
+  return d;
 }
 
 // Three-input minimum / maximum (exact, order-free).
@@ -97,6 +119,62 @@ __device__ __forceinline__ void cp_async_commit() {
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Bulk (TMA) copies global -> shared completing on an mbarrier. No multicast.
+// Waits are bounded: after kMbarSpinLimit polls the caller gets `false` and
+// must raise KVQ_ERRF_TIMEOUT instead of hanging.
+// ---------------------------------------------------------------------------
+
+constexpr uint32_t kMbarSpinLimit = 1u << 22;
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_fence_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+// true once the phase with the given parity has completed; false on timeout
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  const uint32_t addr = smem_u32(bar);
+  for (uint32_t it = 0; it < kMbarSpinLimit; ++it) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(addr), "r"(parity)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+__device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, uint32_t bytes,
+                                         uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(smem_dst)),
+      "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Tiled TMA load of one 3-D box (coordinates in elements, innermost first)
+// into shared memory, completing on an mbarrier. No multicast.
+__device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* tmap, int x, int y, int z,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
 }
 
 // ---------------------------------------------------------------------------

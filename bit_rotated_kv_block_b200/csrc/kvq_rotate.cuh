@@ -14,11 +14,11 @@ namespace kvq {
 
 // In-thread Walsh-Hadamard butterflies on blocks of B = 2^LGB channels
 // (B <= E), stages h = 1, 2, ..., B/2 in ascending order.
-template <int E, int LGB>
+template <int E, int LGB, bool SKIP1 = false>
 __device__ __forceinline__ void fwht_regs(float (&x)[E]) {
   constexpr int B = 1 << LGB;
   static_assert(B <= E, "block wider than a thread");
-  if (B >= 2) {
+  if (B >= 2 && !SKIP1) {
 #pragma unroll
     for (int i = 0; i < E; i += 2) {
       const float a = x[i], c = x[i + 1];
@@ -94,12 +94,13 @@ __device__ __forceinline__ void quat_regs(float (&x)[E], const float* tbl, int c
 
 // Full Hadamard rotation of a thread's E channels, block 2^LGB. Blocks wider
 // than E (b = 256 with E = 128) finish with one stage across the lane pair
-// (2i, 2i+1) given by pair_mask; part 0 holds the lower channels.
-template <int E, int LGB>
+// (2i, 2i+1) given by pair_mask; part 0 holds the lower channels. With
+// STAGE1_DONE the first butterfly stage (h = 1) has already been applied.
+template <int E, int LGB, bool STAGE1_DONE = false>
 __device__ __forceinline__ void hadamard_regs(float (&x)[E], int part, unsigned pair_mask) {
   constexpr int B = 1 << LGB;
   constexpr int LGIN = (B <= E) ? LGB : (E == 128 ? 7 : 6);
-  fwht_regs<E, LGIN>(x);
+  fwht_regs<E, LGIN, STAGE1_DONE>(x);
   if (B > E) {
 #pragma unroll
     for (int i = 0; i < E; ++i) {

@@ -70,6 +70,8 @@ typedef enum {
 #define KVQ_ERRF_POS 2  /* position < 0 or position/page_size >= bt_stride       */
 #define KVQ_ERRF_SEQ 4  /* token's sequence index >= num_seqs                    */
 #define KVQ_ERRF_LEN 8  /* seq_lens[s] < 0, > max_seq_len, or past the table      */
+#define KVQ_ERRF_TIMEOUT 16 /* a bounded wait for an asynchronous copy expired; the
+                               affected tile was skipped (never expected)          */
 
 /* Geometry of one paged cache (both pools share it).
  *  head_dim     d: 64, 128 or 256.
@@ -114,8 +116,9 @@ typedef struct {
  * components as fused multiply-adds in a fixed term order); mn = min y + 0,
  * mx = max y + 0; m16 = binary16 round-down(mn); s16 = binary16 round-up of
  * round-up32(round-up32(mx - m16) / 15); inv = round-nearest32(1/s16);
- * code_i = round-half-even(RN(RN(y_i - m16) * inv)) in [0, 15] (all 0 when
- * s16 = 0). Codes, scale and minimum are bit-identical to that definition.
+ * code_i = nearest integer, ties to even, of the exact product
+ * RN(y_i - m16) * inv, in [0, 15] (all 0 when s16 = 0). Codes, scale and
+ * minimum are bit-identical to that definition.
  * Domain: inputs finite, and every rotated value as well as the scale within
  * the binary16 range (|y| <= 65504); outside it (e.g. a minimum that rounds
  * to -inf) the row's codes are unspecified, but nothing outside the row's
@@ -131,8 +134,12 @@ int kvq_quantize_append(const kvq_cache_desc* desc, int32_t num_tokens, const vo
 
 /*
  * kvq_decode_workspace_bytes -- bytes of device workspace that
- * kvq_paged_decode_attn needs for these sizes (host-only computation; 0 on
- * invalid arguments). The workspace holds per-split partial results.
+ * kvq_paged_decode_attn needs for these sizes (0 on invalid arguments). The
+ * workspace holds one counter per (sequence, KV head) followed by per-split
+ * partial results. It must be zero-filled before its first use; every call
+ * that returns KVQ_OK leaves the counters at zero again, so one zeroed
+ * workspace serves any number of later calls on the same stream. Calls that
+ * share a workspace must not overlap in time.
  */
 size_t kvq_decode_workspace_bytes(const kvq_cache_desc* desc, int32_t num_seqs,
                                   int32_t num_q_heads, int32_t max_seq_len);
@@ -148,7 +155,8 @@ size_t kvq_decode_workspace_bytes(const kvq_cache_desc* desc, int32_t num_seqs,
  *  max_seq_len  upper bound of seq_lens (sizes the split-K work).
  *  sm_scale     softmax scale (typically 1/sqrt(d)).
  *  out          float32 [S][Hq][d], in the original (un-rotated) basis.
- *  workspace    >= kvq_decode_workspace_bytes(...) bytes, 16-byte aligned.
+ *  workspace    >= kvq_decode_workspace_bytes(...) bytes, 16-byte aligned,
+ *               zero-filled before its first use (see above).
  *
  * For query head g (KV head h = g / (Hq/H)): qhat = R q_g;
  * z_j = sm_scale * qhat . khat_j; p = softmax(z); out = R^-1 sum_j p_j vhat_j,

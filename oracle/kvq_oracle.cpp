@@ -210,14 +210,15 @@ void orc_rotate_f32(float* x, int d, int kind, int b, const float* quat) {
 }
 
 // ---------------------------------------------------------------------------
-// Token-wise asymmetric INT4 quantizer (SAW-INT4 Summary: "token-wise INT4";
-// one scale and one zero-point per (token, head) row).
+// Token-wise asymmetric INT4 quantizer (SAW-INT4 page, Summary: one scale and
+// one zero-point per (token, head) row, 16 levels).
 // Readings: the minimum is stored rounded toward -inf; the scale is
 // (max - m16)/15 with the binary32 subtraction, the binary32 division and the
 // final binary16 conversion all rounded toward +inf, so every x lies in
-// [m16, m16 + 15 s16] exactly; the code is round-half-even of
-// RN(RN(x - m16) * RN(1/s16)) clamped to [0, 15] (the clamp never acts given
-// that range, and is kept as the definition); a row
+// [m16, m16 + 15 s16] exactly; the code is the nearest integer (ties to even)
+// to the exact product RN(x - m16) * RN(1/s16), clamped to [0, 15] (one
+// rounding of the product; the clamp never acts given that range, and is
+// kept as the definition); a row
 // with max == m16 has s16 = 0 and all codes 0; -0 is normalised to +0 in both
 // the minimum and the maximum so the stored bits do not depend on reduction
 // order.
@@ -243,12 +244,14 @@ float orc_div_ru(float a, float b) {
   return r;
 }
 
-static float rint_half_even(float t) {
-  const float fl = std::floor(t);
-  const float fr = t - fl;  // exact for |t| < 2^23
-  if (fr > 0.5f) return fl + 1.0f;
-  if (fr < 0.5f) return fl;
-  return (std::fmod(fl, 2.0f) == 0.0f) ? fl : fl + 1.0f;
+// Nearest integer, ties to even, of a double (exact: floor and the
+// fraction of a double below 2^52 are exact).
+static double rint_half_even(double t) {
+  const double fl = std::floor(t);
+  const double fr = t - fl;
+  if (fr > 0.5) return fl + 1.0;
+  if (fr < 0.5) return fl;
+  return (std::fmod(fl, 2.0) == 0.0) ? fl : fl + 1.0;
 }
 
 void orc_quantize_row(const float* y, int d, uint8_t* codes,
@@ -271,10 +274,10 @@ void orc_quantize_row(const float* y, int d, uint8_t* codes,
     const float inv = 1.0f / s;
     for (int i = 0; i < d; ++i) {
       const float t0 = y[i] - m;
-      const float t1 = t0 * inv;
-      float r = rint_half_even(t1);
-      if (r < 0.0f) r = 0.0f;
-      if (r > 15.0f) r = 15.0f;
+      const double prod = (double)t0 * (double)inv;  // exact: 24 x 24 bits
+      double r = rint_half_even(prod);
+      if (r < 0.0) r = 0.0;
+      if (r > 15.0) r = 15.0;
       c[i] = (int)r;
     }
   }

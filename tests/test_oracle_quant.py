@@ -22,7 +22,7 @@ def _hex_bytes(s):
     return np.array([int(t, 16) for t in s.split()], np.uint8)
 
 
-@pytest.mark.parametrize("row", ["row1", "row2"])
+@pytest.mark.parametrize("row", ["row1", "row2", "row3"])
 def test_hand_worked_rows(row):
     g = read_golden("quant_rows_hand.txt")
     x = np.array([float(t) for t in g[row + "_x"].split()], np.float32)
