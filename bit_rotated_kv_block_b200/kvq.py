@@ -30,6 +30,8 @@ SIGNATURES = {
                                              _P, _P, _P, _P, _SZ, _P, _P]),
     "kvq_dequantize_pages": (ctypes.c_int, [_P, _I32, _P, _I32, _P, _I32, _P, _P, _I32, _I32, _P,
                                             _P, _P]),
+    "kvq_paged_decode_attn_noalloc": (ctypes.c_int, [_P, _I32, _I32, _P, _P, _I32, _P, _I32, _F32,
+                                                     _P, _P, _P, _P, _P, _P, _P]),
     "kvq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "kvq_version": (ctypes.c_char_p, []),
 }
@@ -152,6 +154,25 @@ def paged_decode_attn(cache, q, seq_lens, max_seq_len, block_table, k_codes, k_p
                                      _ptr(workspace), workspace.numel() * workspace.element_size(),
                                      _ptr(err), _stream(stream))
     _check("kvq_paged_decode_attn", st)
+    return out
+
+
+def paged_decode_attn_noalloc(cache, q, seq_lens, max_seq_len, block_table, k_codes, k_params,
+                              v_codes, v_params, out=None, sm_scale=None, err=None, stream=None):
+    """Decode attention whose scratch is the library's fixed device array
+    (for callers that cannot allocate); q: float16 CUDA [S][Hq][d]."""
+    S, Hq, d = q.shape
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((S, Hq, d), dtype=torch.float32, device=q.device)
+    st = lib().kvq_paged_decode_attn_noalloc(ctypes.byref(cache.desc), S, Hq, _ptr(q),
+                                             _ptr(seq_lens), int(max_seq_len), _ptr(block_table),
+                                             int(block_table.shape[1]), float(sm_scale),
+                                             _ptr(k_codes), _ptr(k_params), _ptr(v_codes),
+                                             _ptr(v_params), _ptr(out), _ptr(err),
+                                             _stream(stream))
+    _check("kvq_paged_decode_attn_noalloc", st)
     return out
 
 

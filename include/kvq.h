@@ -187,6 +187,42 @@ int kvq_dequantize_pages(const kvq_cache_desc* desc, int32_t num_seqs,
                          const void* params, int32_t unrotate, int32_t out_fp32, void* out,
                          int32_t* err_flags, void* stream);
 
+/* Size of the fixed scratch array behind kvq_paged_decode_attn_noalloc. */
+#define KVQ_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * kvq_paged_decode_attn_noalloc -- kvq_paged_decode_attn for callers that
+ * cannot allocate device memory (no counterpart in the method's pages; it is
+ * a deployment convenience). Some callers have no way to hand over a
+ * workspace: an engine whose device memory is planned once at start-up and
+ * whose allocator refuses later requests, a plug-in living inside a host
+ * framework that owns every device allocation, or a serving path that must
+ * not call cudaMalloc/cudaFree because those calls synchronise the device.
+ *
+ * Arguments and results are those of kvq_paged_decode_attn without
+ * `workspace` / `workspace_bytes`. The scratch is a 16 MiB array compiled
+ * into the library (KVQ_NOALLOC_SCRATCH_BYTES): every GPU that loads libkvq
+ * holds it until the process exits. The call allocates and frees nothing;
+ * it enqueues one cudaMemsetAsync (clearing the split counters at the start
+ * of the scratch) and the decode kernel on `stream`.
+ *  - Sizes whose workspace (kvq_decode_workspace_bytes) exceeds
+ *    KVQ_NOALLOC_SCRATCH_BYTES are rejected with KVQ_ERR_WORKSPACE before
+ *    anything is launched.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress, once per device, with that device current); make
+ *    that first call before any stream capture on the device.
+ *  - All calls on a device share the one array and it keeps the last call's
+ *    contents: calls that overlap on the GPU (different streams, or
+ *    different host threads without ordering) race and give wrong results.
+ */
+int kvq_paged_decode_attn_noalloc(const kvq_cache_desc* desc, int32_t num_seqs,
+                                  int32_t num_q_heads, const void* q, const int32_t* seq_lens,
+                                  int32_t max_seq_len, const int32_t* block_table,
+                                  int32_t bt_stride, float sm_scale, const uint8_t* k_codes,
+                                  const void* k_params, const uint8_t* v_codes,
+                                  const void* v_params, float* out, int32_t* err_flags,
+                                  void* stream);
+
 /* Human-readable name of a kvq_status value (static storage). */
 const char* kvq_status_string(int status);
 
