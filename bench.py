@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
+    ap.add_argument("--profile-case", choices=["append", "decode"], default=None,
+                    help="run a short fixed case for an ncu capture (4 launches) and exit")
     return ap.parse_args()
 
 
@@ -66,6 +68,11 @@ def dist_setup(args):
         backend = "nccl" if torch.cuda.is_available() else "gloo"
         torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
     return world, rank, local
+
+
+def shard_seed(seed, rank):
+    """Seed of rank ``rank``'s shard: every rank draws its own sequences."""
+    return seed + 1000 * rank
 
 
 def barrier(world):
@@ -178,7 +185,7 @@ def run_ours(args, world, rank, local):
     dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(device)
 
     # each rank owns an independent shard of 32 sequences (seeded per rank)
-    w = workloads.llama8b(seed=args.seed + 1000 * rank)
+    w = workloads.llama8b(seed=shard_seed(args.seed, rank))
     S, H, Hq, d, ctx = w.S, w.H, w.Hq, w.d, int(w.seq_lens[0])
     k, v, ts, tp = w.prefill_tokens()
     K, V, TS, TP = dev(k), dev(v), dev(ts), dev(tp)
@@ -217,7 +224,7 @@ def run_ours(args, world, rank, local):
     ws = torch.zeros(kvq.decode_workspace_bytes(c0, S, Hq, L), dtype=torch.uint8, device=device)
     err = torch.zeros(1, dtype=torch.int32, device=device)
     stream = torch.cuda.current_stream()
-    launches_per_step = 1 + 3
+    launches_per_step = 2  # one append kernel + one decode kernel
 
     def step(i):
         c, kc, kp, vc, vp = caches[i % 2]
@@ -415,8 +422,43 @@ def run_reference(args, world, rank):
     }
 
 
+def profile_case(which):
+    """Short cases for ncu captures, each well above L2 and well below a few GB:
+    append = 4 bulk appends of one prefill layer (65536 tokens, Hadamard b 128,
+    268 MB in, 71 MB out); decode = 4 decode calls of the Llama-3-8B-shaped
+    layer (143 MB of INT4 pages) after filling its cache with one append."""
+    from bit_rotated_kv_block_b200 import kvq, workloads
+    torch.cuda.set_device(0)
+    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
+    w = workloads.prefill(rot_block=128) if which == "append" else workloads.llama8b()
+    k, v, ts, tp = w.prefill_tokens()
+    c = kvq.Cache(w.d, w.H, w.P, w.NP, w.rot_kind, w.rot_block)
+    kc, kp = c.new_pools(fill=0)
+    vc, vp = c.new_pools(fill=0)
+    K, V, TS, TP, BT = dev(k), dev(v), dev(ts), dev(tp), dev(w.block_table)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kvq.quantize_append(c, K, V, TS, TP, BT, kc, kp, vc, vp, err=err)
+    if which == "append":
+        for _ in range(4):
+            kvq.quantize_append(c, K, V, TS, TP, BT, kc, kp, vc, vp, err=err)
+    else:
+        del K, V
+        q, lens = dev(w.queries()), dev(w.seq_lens)
+        L = int(w.seq_lens.max())
+        ws = torch.zeros(kvq.decode_workspace_bytes(c, w.S, w.Hq, L), dtype=torch.uint8,
+                         device="cuda")
+        for _ in range(4):
+            kvq.paged_decode_attn(c, q, lens, L, BT, kc, kp, vc, vp, workspace=ws, err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0, f"device error flags {int(err.item())}"
+    print(f"profile case {which} done")
+
+
 def main():
     args = parse()
+    if args.profile_case:
+        profile_case(args.profile_case)
+        return
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":

@@ -12,15 +12,18 @@
 //    row of K or V, so every butterfly stage of a block of up to 128 channels
 //    runs in registers without shuffles; d = 256 uses two threads per row and
 //    one xor-1 shuffle stage for b = 256.
-//  * A CTA of 384 threads owns a tile of TOK tokens x {K, V} x H heads. Each
-//    thread pulls its own row segment (2E contiguous bytes) global -> shared
-//    with one TMA bulk copy that completes on the buffer's mbarrier (row
-//    pitch 2E + 16 bytes, so the thread then reads it with conflict-free
-//    128-bit loads) while the previous tile is computed (two buffers). The
-//    grid is persistent: one CTA per SM walks the tiles. Waits on the
-//    mbarriers are bounded and end in KVQ_ERRF_TIMEOUT, never in a hang.
-//  * Threads are ordered head-major, token-minor, so a warp writes the codes
-//    of up to 32 consecutive slots of one (page, head) chunk.
+//  * A CTA of 384 threads owns a tile of TOK tokens x {K, V} x H heads. One
+//    elected thread fills the tile's shared-memory buffer with TMA tensor
+//    copies (cp.async.bulk.tensor.3d, boxes of 64 channels x H heads x TOK
+//    tokens, 128-byte swizzle so that every thread's 128-bit reads of its
+//    row are bank-conflict free) that complete on the buffer's mbarrier,
+//    while the previous tile is computed (two buffers). The grid is
+//    persistent: one CTA per SM walks the tiles. Waits on the mbarriers are
+//    bounded and end in KVQ_ERRF_TIMEOUT, never in a hang.
+//  * Threads are ordered token-major, head-minor, so a warp's rows are
+//    consecutive lines of the swizzled boxes, and the destination of each
+//    row (token -> sequence, position -> block table) is resolved one tile
+//    ahead of its use.
 //  * Arithmetic is bit-exact with the published definition (see kvq.h):
 //    binary32 butterflies in ascending stage order (packed f32x2 lanes for
 //    stages >= 2), directed roundings through __fsub_ru / __fdiv_ru /

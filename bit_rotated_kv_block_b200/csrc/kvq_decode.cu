@@ -45,7 +45,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 struct DecodeArgs {
   int S, Hq, H, G, P, NP, bt_stride, max_seq_len, splits, pages_per_split;
   int rot_kind, lgb;
-  float scale2;  // sm_scale * log2(e)
+  double scale2;  // sm_scale * log2(e), in double
   const __half* q;  // [S][Hq][D]
   const float* quat;
   const int32_t* seq_lens;
@@ -55,7 +55,7 @@ struct DecodeArgs {
   const uint8_t* v_codes;
   const uint32_t* v_params;
   float* out;        // [S][Hq][D]
-  float* part;       // [S][Hq][splits][D + 4]: acc[D], max, sum, 2 pad
+  float* part;       // [S][Hq][splits][D + 4]: acc[D], max (double), sum, pad
   int32_t* counter;  // [S][H], zero between calls
   int32_t* err;
 };
@@ -66,7 +66,8 @@ struct DecodeArgs {
 
 template <int D, int P, int GP>
 struct DecCfg {
-  static constexpr int NKS = D / 16;           // QK k-steps over channels
+  static constexpr int NKS8 = D / 32;          // QK int8 k-steps over channels
+  static constexpr int NQT = GP == 8 ? 2 : 1;  // 16-row tiles of query limbs
   static constexpr int NMT = D / 16;           // PV m-tiles over channels
   static constexpr int TILES = P / 16;         // 16-token tiles per page
   static constexpr int NPV = GP == 8 ? 2 : 1;  // PV n-tiles (hi / lo columns)
@@ -174,8 +175,16 @@ __global__ void __launch_bounds__(kDecWarps * kWarp) decode_split_kernel(const D
   const bool lo_row = (GP == 4) && (r >= 4);
   const int g = h * a.G + hr;           // global query head
   const bool head_ok = hr < a.G;
-  float qs;  // sum of qhat over all channels of head hr
-  uint32_t qa[C::NKS][4];
+  // The query as a 30-bit fixed point qint = qhat * 2^30 / amax (amax = the
+  // head's largest |qhat|), split into four signed 8-bit limbs
+  // qint = l3*2^24 + l2*2^16 + l1*2^8 + l0 for the int8 tensor cores.
+  long long qsum;  // sum of qint over the head's channels (exact)
+  double zk;       // sm_scale * log2(e) * amax / 2^30
+  // A fragments per k-step kk: the lane's 8 channels j*QW + 8kk + [0, 8),
+  // even ones in a[0]/a[1], odd ones in a[2]/a[3]. Rows:
+  //   GP = 4: rows 0-3 l3, 4-7 l2, 8-11 l1, 12-15 l0 of heads 0-3;
+  //   GP = 8: tile 0 rows 0-7 l3, 8-15 l2; tile 1 rows 0-7 l1, 8-15 l0.
+  uint32_t qa[C::NQT][C::NKS8][4];
   {
     float x[C::QW];
     {
@@ -193,61 +202,90 @@ __global__ void __launch_bounds__(kDecWarps * kWarp) decode_split_kernel(const D
       }
     }
     rotate_quarter<C::QW>(x, j, a.rot_kind, a.lgb, a.quat, false);
-    float part = 0.f;
+    float amax = 0.f;
 #pragma unroll
-    for (int i = 0; i < C::QW; ++i) part += x[i];
-    part += __shfl_xor_sync(0xffffffffu, part, 1);
-    part += __shfl_xor_sync(0xffffffffu, part, 2);
-    qs = part;
-    __half hi[C::QW], lo[C::QW];
+    for (int i = 0; i < C::QW; ++i) amax = fmaxf(amax, fabsf(x[i]));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    const double mul = amax > 0.f ? 1073741824.0 / (double)amax : 0.0;  // 2^30 / amax
+    zk = a.scale2 * ((double)amax * (1.0 / 1073741824.0));
+    long long qs_l = 0;
 #pragma unroll
-    for (int i = 0; i < C::QW; ++i) split_hl(x[i], hi[i], lo[i]);
-    // k-step kk, column 2j(+1) <- local channel 8(kk/2) + 2(kk%2) (+4);
-    // column 2j+8(+9) <- local channel 8(kk/2) + 2(kk%2) + 1 (+4)
+    for (int kk = 0; kk < C::NKS8; ++kk) {
+      int li[2][4][4];  // [even/odd][l3, l2, l1, l0][4 channels]
 #pragma unroll
-    for (int kk = 0; kk < C::NKS; ++kk) {
-      const int c0 = 8 * (kk >> 1) + 2 * (kk & 1);
-      const int c1 = c0 + 1;
+      for (int od = 0; od < 2; ++od)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int q = __double2int_rn((double)x[8 * kk + 2 * i + od] * mul);  // |q| <= 2^30
+          qs_l += q;
+          const int l0 = (q << 24) >> 24;
+          const int r1 = (q - l0) >> 8;
+          const int l1 = (r1 << 24) >> 24;
+          const int r2 = (r1 - l1) >> 8;
+          const int l2 = (r2 << 24) >> 24;
+          li[od][0][i] = (r2 - l2) >> 8;
+          li[od][1][i] = l2;
+          li[od][2][i] = l1;
+          li[od][3][i] = l0;
+        }
+      auto pk4 = [&](int od, int limb) {
+        return pack_s8x4(li[od][limb][0], li[od][limb][1], li[od][limb][2], li[od][limb][3]);
+      };
       if (GP == 8) {
-        qa[kk][0] = h2_as_u32(__halves2half2(hi[c0], hi[c0 + 4]));
-        qa[kk][1] = h2_as_u32(__halves2half2(lo[c0], lo[c0 + 4]));
-        qa[kk][2] = h2_as_u32(__halves2half2(hi[c1], hi[c1 + 4]));
-        qa[kk][3] = h2_as_u32(__halves2half2(lo[c1], lo[c1 + 4]));
+        qa[0][kk][0] = pk4(0, 0);
+        qa[0][kk][1] = pk4(0, 1);
+        qa[0][kk][2] = pk4(1, 0);
+        qa[0][kk][3] = pk4(1, 1);
+        qa[C::NQT - 1][kk][0] = pk4(0, 2);
+        qa[C::NQT - 1][kk][1] = pk4(0, 3);
+        qa[C::NQT - 1][kk][2] = pk4(1, 2);
+        qa[C::NQT - 1][kk][3] = pk4(1, 3);
       } else {
-        const __half* sel = lo_row ? lo : hi;
-        qa[kk][0] = h2_as_u32(__halves2half2(sel[c0], sel[c0 + 4]));
-        qa[kk][1] = 0u;
-        qa[kk][2] = h2_as_u32(__halves2half2(sel[c1], sel[c1 + 4]));
-        qa[kk][3] = 0u;
+        // row r: l3 (r < 4) or l2 (r >= 4); row r + 8: l1 (r < 4) or l0
+        qa[0][kk][0] = lo_row ? pk4(0, 1) : pk4(0, 0);
+        qa[0][kk][2] = lo_row ? pk4(1, 1) : pk4(1, 0);
+        qa[0][kk][1] = lo_row ? pk4(0, 3) : pk4(0, 2);
+        qa[0][kk][3] = lo_row ? pk4(1, 3) : pk4(1, 2);
       }
     }
+    qs_l += __shfl_xor_sync(0xffffffffu, qs_l, 1);
+    qs_l += __shfl_xor_sync(0xffffffffu, qs_l, 2);
+    qsum = qs_l;
   }
 
-  // ---- page ring
-  const int64_t head_chunk = (int64_t)C::CODE_B;
+  // ---- page ring: each lane copies the same 16-byte units of every page,
+  // so their shared-memory destinations are computed once
+  constexpr int UNITS = C::CODE_B / 16;        // 16-byte units of codes per pool
+  constexpr int UPT = (D / 2) / 16;            // units per token
+  constexpr int UPL = (UNITS + kWarp - 1) / kWarp;  // units per lane
+  constexpr int PU = P * 4 / 16;               // 16-byte units of params per pool
+  int koff[UPL], voff[UPL];
+#pragma unroll
+  for (int i = 0; i < UPL; ++i) {
+    const int c = lane + kWarp * i;
+    koff[i] = k_unit_off<D>(c / UPT, c % UPT);
+    voff[i] = C::CODE_B + v_unit_off<D>(c / UPT, c % UPT);
+  }
+  const int par_dst = lane < PU ? 2 * C::CODE_B + lane * 16 : 2 * C::CODE_B + P * 4 + (lane - PU) * 16;
   auto issue = [&](int i) {
     if (i < nmine) {
       const int page = ids[i];
       if (page >= 0 && page < a.NP) {
         uint8_t* st = ring + (i % C::NST) * C::STAGE_B;
         const int64_t row = (int64_t)page * a.H + h;
-        const uint8_t* kc = a.k_codes + row * head_chunk;
-        const uint8_t* vc = a.v_codes + row * head_chunk;
-        constexpr int UNITS = C::CODE_B / 16;
-        constexpr int UPT = (D / 2) / 16;  // 16-byte units per token
+        const uint8_t* kc = a.k_codes + row * C::CODE_B + lane * 16;
+        const uint8_t* vc = a.v_codes + row * C::CODE_B + lane * 16;
 #pragma unroll
-        for (int c = lane; c < UNITS; c += kWarp) {
-          const int t = c / UPT, u = c % UPT;
-          cp_async16(st + k_unit_off<D>(t, u), kc + c * 16);
-          cp_async16(st + C::CODE_B + v_unit_off<D>(t, u), vc + c * 16);
+        for (int u = 0; u < UPL; ++u) {
+          if (UNITS % kWarp == 0 || lane + kWarp * u < UNITS) {
+            cp_async16(st + koff[u], kc + u * kWarp * 16);
+            cp_async16(st + voff[u], vc + u * kWarp * 16);
+          }
         }
-        constexpr int PU = P * 4 / 16;  // 16-byte units of params per pool
-        if (lane < PU) {
-          cp_async16(st + 2 * C::CODE_B + lane * 16,
-                     reinterpret_cast<const uint8_t*>(a.k_params + row * P) + lane * 16);
-        } else if (lane < 2 * PU) {
-          cp_async16(st + 2 * C::CODE_B + P * 4 + (lane - PU) * 16,
-                     reinterpret_cast<const uint8_t*>(a.v_params + row * P) + (lane - PU) * 16);
+        if (lane < 2 * PU) {
+          const uint32_t* pp = lane < PU ? a.k_params + row * P : a.v_params + row * P;
+          cp_async16(st + par_dst, reinterpret_cast<const uint8_t*>(pp) + (lane % PU) * 16);
         }
       }
     }
@@ -262,7 +300,10 @@ __global__ void __launch_bounds__(kDecWarps * kWarp) decode_split_kernel(const D
     for (int n = 0; n < C::NPV; ++n)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[mt][n][e] = 0.f;
-  float M = -INFINITY;  // running max (base-2 scaled scores) of head hr
+  // Scores are formed in double from exact integers: with a dominant (sink)
+  // token the base-2 logits reach ~100, where a binary32 rounding would
+  // already move the other tokens' weights visibly.
+  double M = -INFINITY;  // running max (base-2 scaled scores) of head hr
   float Lp = 0.f;       // this lane's share of sum p
   float Op = 0.f;       // this lane's share of sum p (m_v + 8 s_v)
 
@@ -284,14 +325,16 @@ __global__ void __launch_bounds__(kDecWarps * kWarp) decode_split_kernel(const D
 
     // ---- scores of all tiles of the page: z[tile][0..3] for tokens
     // 16*tile + {2j, 2j+1, 2j+8, 2j+9}
-    float z[C::TILES][4];
+    double z[C::TILES][4];
 #pragma unroll
     for (int tt = 0; tt < C::TILES; ++tt) {
-      float cacc[2][4];
+      int ci[C::NQT][2][4];
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) cacc[nt][e] = 0.f;
+        for (int t = 0; t < C::NQT; ++t)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) ci[t][nt][e] = 0;
         const int tok = 16 * tt + 8 * nt + r;
         uint32_t w[D / 32];
 #pragma unroll
@@ -300,20 +343,36 @@ __global__ void __launch_bounds__(kDecWarps * kWarp) decode_split_kernel(const D
           w[4 * u] = v4.x; w[4 * u + 1] = v4.y; w[4 * u + 2] = v4.z; w[4 * u + 3] = v4.w;
         }
 #pragma unroll
-        for (int kk = 0; kk < C::NKS; ++kk) {
-          const uint32_t wd = w[kk >> 1];
-          const uint32_t b0 = (kk & 1) ? nib_pair<2>(wd) : nib_pair<0>(wd);
-          const uint32_t b1 = (kk & 1) ? nib_pair<3>(wd) : nib_pair<1>(wd);
-          mma16816(cacc[nt], qa[kk], b0, b1);
+        for (int kk = 0; kk < C::NKS8; ++kk) {
+          const uint32_t b0 = w[kk] & 0x0F0F0F0Fu;         // even channels as bytes
+          const uint32_t b1 = (w[kk] >> 4) & 0x0F0F0F0Fu;  // odd channels
+#pragma unroll
+          for (int t = 0; t < C::NQT; ++t) mma16832_s8u8(ci[t][nt], qa[t][kk], b0, b1);
         }
       }
-      // dot products of head hr with the four tokens of this lane
-      float dt[4] = {cacc[0][0], cacc[0][1], cacc[1][0], cacc[1][1]};
-      if (GP == 8) {
-        dt[0] += cacc[0][2]; dt[1] += cacc[0][3]; dt[2] += cacc[1][2]; dt[3] += cacc[1][3];
-      } else {
+      // sum_i (c_i - 8) qint_i of head hr with the four tokens
+      // {2j, 2j+1, 2j+8, 2j+9}, exact in 64-bit integers (the centring keeps
+      // the two score terms small, so their binary32 rounding stays small)
+      long long dt[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) dt[e] += __shfl_xor_sync(0xffffffffu, dt[e], 16);
+      for (int e = 0; e < 4; ++e) {
+        const int nt = e >> 1, c = e & 1;
+        int l3, l2, l1, l0;
+        if (GP == 8) {
+          l3 = ci[0][nt][c];
+          l2 = ci[0][nt][2 + c];
+          l1 = ci[C::NQT - 1][nt][c];
+          l0 = ci[C::NQT - 1][nt][2 + c];
+        } else {
+          // lanes r < 4 hold the (l3, l1) rows, lanes r + 4 the (l2, l0) rows
+          const int o0 = __shfl_xor_sync(0xffffffffu, ci[0][nt][c], 16);
+          const int o2 = __shfl_xor_sync(0xffffffffu, ci[0][nt][2 + c], 16);
+          l3 = lo_row ? o0 : ci[0][nt][c];
+          l2 = lo_row ? ci[0][nt][c] : o0;
+          l1 = lo_row ? o2 : ci[0][nt][2 + c];
+          l0 = lo_row ? ci[0][nt][2 + c] : o2;
+        }
+        dt[e] = (((long long)l3 * 256ll + l2) * 256ll + l1) * 256ll + l0 - 8ll * qsum;
       }
       const uint2 kp01 = kpar[8 * tt + j];      // tokens 16tt + 2j, 2j+1
       const uint2 kp89 = kpar[8 * tt + 4 + j];  // tokens 16tt + 2j+8, 2j+9
@@ -322,27 +381,28 @@ __global__ void __launch_bounds__(kDecWarps * kWarp) decode_split_kernel(const D
       for (int e = 0; e < 4; ++e) {
         const float2 sm = __half22float2(u32_as_h2(kp[e]));  // (scale, min)
         const int tok = pidx * P + 16 * tt + 2 * j + (e & 1) + 8 * (e >> 1);
-        const float sc = (sm.x * dt[e] + (sm.y + 8.f * sm.x) * qs) * a.scale2;
+        const double sd = (double)sm.x, md = (double)sm.y;
+        const double sc = zk * (sd * (double)dt[e] + (md + 8.0 * sd) * (double)qsum);
         z[tt][e] = (page_ok && tok < L) ? sc : -INFINITY;
       }
     }
 
     // ---- online softmax update for head hr (max over the 4 lanes j)
-    float mloc = -INFINITY;
+    double mloc = -INFINITY;
 #pragma unroll
     for (int tt = 0; tt < C::TILES; ++tt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) mloc = fmaxf(mloc, z[tt][e]);
-    mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
-    mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
-    const float Mn = fmaxf(M, mloc);
-    const float alpha = (Mn == -INFINITY) ? 1.f : fast_exp2(M - Mn);
+      for (int e = 0; e < 4; ++e) mloc = fmax(mloc, z[tt][e]);
+    mloc = fmax(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
+    mloc = fmax(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
+    const double Mn = fmax(M, mloc);
+    const float alpha = (Mn == -INFINITY) ? 1.f : fast_exp2((float)(M - Mn));
     M = Mn;
     Lp *= alpha;
     Op *= alpha;
     // rescale the output accumulators: lane (r, j) holds columns of heads
     // c0 = 2(j & (GP/2 - 1)), c0 + 1 -> their alpha from lanes r = c0, c0 + 1
-    {
+    if (__any_sync(0xffffffffu, alpha != 1.f)) {  // warp-uniform: skip when no max moved
       const int c0 = (GP == 8) ? 2 * j : 2 * (j & 1);
       const float a0 = __shfl_sync(0xffffffffu, alpha, 4 * c0);
       const float a1 = __shfl_sync(0xffffffffu, alpha, 4 * c0 + 4);
@@ -361,30 +421,37 @@ __global__ void __launch_bounds__(kDecWarps * kWarp) decode_split_kernel(const D
       const uint2 vp01 = vpar[8 * tt + j];
       const uint2 vp89 = vpar[8 * tt + 4 + j];
       const uint32_t vp[4] = {vp01.x, vp01.y, vp89.x, vp89.y};
-      __half phi[4], plo[4];
+      float pv[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         // masked tokens may sit on stale or never-written shared memory:
         // their terms are forced to exact zeros rather than p * (params)
         const bool live = z[tt][e] != -INFINITY;
         const float2 sm = __half22float2(u32_as_h2(vp[e]));
-        const float p = live ? fast_exp2(z[tt][e] - M) : 0.f;
+        const float p = live ? fast_exp2((float)(z[tt][e] - M)) : 0.f;
         Lp += p;
         Op += live ? p * (sm.y + 8.f * sm.x) : 0.f;
-        split_hl(live ? p * sm.x : 0.f, phi[e], plo[e]);
+        pv[e] = live ? p * sm.x : 0.f;
       }
+      // p * s as f16 hi + lo pairs (packed conversions): hi = RN16(x),
+      // lo = RN16(x - hi), for tokens (2j, 2j+1) and (2j+8, 2j+9)
+      const __half2 h01 = __floats2half2_rn(pv[0], pv[1]);
+      const __half2 h89 = __floats2half2_rn(pv[2], pv[3]);
+      const float2 f01 = __half22float2(h01), f89 = __half22float2(h89);
+      const uint32_t hi01 = h2_as_u32(h01), hi89 = h2_as_u32(h89);
+      const uint32_t lo01 = h2_as_u32(__floats2half2_rn(pv[0] - f01.x, pv[1] - f01.y));
+      const uint32_t lo89 = h2_as_u32(__floats2half2_rn(pv[2] - f89.x, pv[3] - f89.y));
       // B operand columns: GP = 8: n-tile 0 = hi, 1 = lo (col r = head r);
       // GP = 4: col r < 4 = hi of head r, r >= 4 = lo of head r - 4
       uint32_t pb[C::NPV][2];
       if (GP == 8) {
-        pb[0][0] = h2_as_u32(__halves2half2(phi[0], phi[1]));
-        pb[0][1] = h2_as_u32(__halves2half2(phi[2], phi[3]));
-        pb[C::NPV - 1][0] = h2_as_u32(__halves2half2(plo[0], plo[1]));
-        pb[C::NPV - 1][1] = h2_as_u32(__halves2half2(plo[2], plo[3]));
+        pb[0][0] = hi01;
+        pb[0][1] = hi89;
+        pb[C::NPV - 1][0] = lo01;
+        pb[C::NPV - 1][1] = lo89;
       } else {
-        const __half* sel = lo_row ? plo : phi;
-        pb[0][0] = h2_as_u32(__halves2half2(sel[0], sel[1]));
-        pb[0][1] = h2_as_u32(__halves2half2(sel[2], sel[3]));
+        pb[0][0] = lo_row ? lo01 : hi01;
+        pb[0][1] = lo_row ? lo89 : hi89;
       }
       if (!head_ok) {
 #pragma unroll
@@ -419,26 +486,33 @@ __global__ void __launch_bounds__(kDecWarps * kWarp) decode_split_kernel(const D
             pr[tp][wi][0] = __byte_perm(X, Y, 0x5410);
             pr[tp][wi][1] = __byte_perm(X, Y, 0x7632);
           }
+        // nibbles of every (token pair, word, byte half): nb[tp][wi][bsel][k]
+        uint32_t nb[2][2][2][4];
+#pragma unroll
+        for (int tp = 0; tp < 2; ++tp)
+#pragma unroll
+          for (int wi = 0; wi < 2; ++wi)
+#pragma unroll
+            for (int bs = 0; bs < 2; ++bs) nib4(pr[tp][wi][bs], nb[tp][wi][bs]);
 #pragma unroll
         for (int e8 = 0; e8 < 8; ++e8) {
           const int mt = gq * 8 + e8;
-          if (mt >= C::NMT) break;
+          const int bsel = e8 >> 2, k = e8 & 3;
           uint32_t av[4];
-          auto nib = [&](uint32_t z32) -> uint32_t {
-            switch (e8 & 3) {
-              case 0: return nib_pair<0>(z32);
-              case 1: return nib_pair<1>(z32);
-              case 2: return nib_pair<2>(z32);
-              default: return nib_pair<3>(z32);
-            }
-          };
-          const int bsel = e8 >> 2;
-          av[0] = nib(pr[0][0][bsel]);  // slot r,   tokens 2j, 2j+1
-          av[1] = nib(pr[0][1][bsel]);  // slot r+8, tokens 2j, 2j+1
-          av[2] = nib(pr[1][0][bsel]);  // slot r,   tokens 2j+8, 2j+9
-          av[3] = nib(pr[1][1][bsel]);  // slot r+8, tokens 2j+8, 2j+9
+          av[0] = nb[0][0][bsel][k];  // slot r,   tokens 2j, 2j+1
+          av[1] = nb[0][1][bsel][k];  // slot r+8, tokens 2j, 2j+1
+          av[2] = nb[1][0][bsel][k];  // slot r,   tokens 2j+8, 2j+9
+          av[3] = nb[1][1][bsel][k];  // slot r+8, tokens 2j+8, 2j+9
+          // each 16-token product starts from zero and joins the running sum
+          // through an IEEE round-to-nearest add: accumulating inside the
+          // tensor core would round toward zero against a large running sum
 #pragma unroll
-          for (int n = 0; n < C::NPV; ++n) mma16816(acc[mt][n], av, pb[n][0], pb[n][1]);
+          for (int n = 0; n < C::NPV; ++n) {
+            float t4[4] = {0.f, 0.f, 0.f, 0.f};
+            mma16816(t4, av, pb[n][0], pb[n][1]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[mt][n][e] = __fadd_rn(acc[mt][n][e], t4[e]);
+          }
         }
       }
     }
@@ -487,8 +561,8 @@ __global__ void __launch_bounds__(kDecWarps * kWarp) decode_split_kernel(const D
   // the lanes that own head hr's softmax state write it (one lane per head)
   if (j == 0 && !lo_row && head_ok) {
     float* dst = a.part + (base + (int64_t)hr * a.splits) * (D + 4);
-    dst[D] = M;
-    dst[D + 1] = Lp;
+    *reinterpret_cast<double*>(dst + D) = M;  // 8-byte aligned: (D + 4) * 4 * k + 4 * D
+    dst[D + 2] = Lp;
   }
 
   // ---- the last warp of this (sequence, KV head) merges the splits
@@ -505,16 +579,17 @@ __global__ void __launch_bounds__(kDecWarps * kWarp) decode_split_kernel(const D
   for (int c = 0; c < C::QW; ++c) x[c] = 0.f;
   if (owner) {
     const float* src = a.part + ((int64_t)s * a.Hq + g) * a.splits * (D + 4);
-    float Mx = -INFINITY;
-    for (int i = 0; i < a.splits; ++i) Mx = fmaxf(Mx, __ldcg(src + (int64_t)i * (D + 4) + D));
+    double Mx = -INFINITY;
+    for (int i = 0; i < a.splits; ++i)
+      Mx = fmax(Mx, __ldcg(reinterpret_cast<const double*>(src + (int64_t)i * (D + 4) + D)));
     float Ls = 0.f;
     if (Mx != -INFINITY) {
       for (int i = 0; i < a.splits; ++i) {
         const float* pi = src + (int64_t)i * (D + 4);
-        const float Mi = __ldcg(pi + D);
+        const double Mi = __ldcg(reinterpret_cast<const double*>(pi + D));
         if (Mi == -INFINITY) continue;
-        const float wgt = fast_exp2(Mi - Mx);
-        Ls += wgt * __ldcg(pi + D + 1);
+        const float wgt = fast_exp2((float)(Mi - Mx));
+        Ls += wgt * __ldcg(pi + D + 2);
         const float4* v4 = reinterpret_cast<const float4*>(pi + j * C::QW);
 #pragma unroll
         for (int c = 0; c < C::QW / 4; ++c) {
@@ -641,7 +716,7 @@ int decode_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, const void* q,
   a.bt_stride = bt_stride; a.max_seq_len = max_seq_len; a.splits = pl.splits;
   a.pages_per_split = pl.pages_per_split;
   a.rot_kind = d.rot_kind; a.lgb = lgb;
-  a.scale2 = sm_scale * kLog2e;
+  a.scale2 = (double)sm_scale * 1.4426950408889634074;
   a.q = static_cast<const __half*>(q); a.quat = d.quat;
   a.seq_lens = seq_lens; a.block_table = block_table;
   a.k_codes = k_codes; a.k_params = static_cast<const uint32_t*>(k_params);

@@ -195,6 +195,29 @@ __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// Warp-level integer MMA: D[16x8] (s32) += A[16x32] (s8) * B[32x8] (u8).
+// Fragment ownership (lane = 4*r + j), four 8-bit values per register:
+//   A: a[0] = (row r,   k 4j..4j+3)     a[1] = (row r+8, k 4j..4j+3)
+//      a[2] = (row r,   k 4j+16..+19)   a[3] = (row r+8, k 4j+16..+19)
+//   B: b0 = (k 4j..4j+3, col r)         b1 = (k 4j+16..+19, col r)
+//   C: c[0..1] = (row r, cols 2j, 2j+1)  c[2..3] = (row r+8, cols 2j, 2j+1)
+// Integer accumulation is exact.
+__device__ __forceinline__ void mma16832_s8u8(int (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                              uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Packs four signed 8-bit values (given as int) into one register, first in
+// the lowest byte.
+__device__ __forceinline__ uint32_t pack_s8x4(int v0, int v1, int v2, int v3) {
+  return (uint32_t)(v0 & 0xff) | ((uint32_t)(v1 & 0xff) << 8) | ((uint32_t)(v2 & 0xff) << 16) |
+         ((uint32_t)(v3 & 0xff) << 24);
+}
+
 __device__ __forceinline__ uint32_t h2_as_u32(__half2 h) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
@@ -213,6 +236,26 @@ __device__ __forceinline__ uint32_t nib_pair(uint32_t w) {
   asm("lop3.b32 %0, %1, %2, %3, 0xea;" : "=r"(t) : "r"(x), "r"(0x000F000Fu), "r"(0x64006400u));
   const __half2 h = __hsub2(u32_as_h2(t), u32_as_h2(0x64086408u));  // 1032.0 = 0x6408
   return h2_as_u32(h);
+}
+
+// The four nibbles of each 16-bit half of z as half2 (code - 8), exact:
+// out[k] = half2(nibble k of the low half, nibble k of the high half). Nibbles
+// 0 and 2 land at 1024 + c (mantissa bits 0-3) and lose 1032; nibbles 1 and 3
+// land at 1024 + 16c (bits 4-7) and are mapped by (.)/16 - 72 = c - 8.
+__device__ __forceinline__ void nib4(uint32_t z, uint32_t (&out)[4]) {
+  const __half2 k1032 = u32_as_h2(0x64086408u);                    // 1032
+  const __half2 k16th = u32_as_h2(0x2C002C00u);                    // 1/16
+  const __half2 km72 = u32_as_h2(0xD480D480u);                     // -72
+  const uint32_t z8 = z >> 8;
+  uint32_t t0, t1, t2, t3;
+  asm("lop3.b32 %0, %1, %2, %3, 0xea;" : "=r"(t0) : "r"(z), "r"(0x000F000Fu), "r"(0x64006400u));
+  asm("lop3.b32 %0, %1, %2, %3, 0xea;" : "=r"(t1) : "r"(z), "r"(0x00F000F0u), "r"(0x64006400u));
+  asm("lop3.b32 %0, %1, %2, %3, 0xea;" : "=r"(t2) : "r"(z8), "r"(0x000F000Fu), "r"(0x64006400u));
+  asm("lop3.b32 %0, %1, %2, %3, 0xea;" : "=r"(t3) : "r"(z8), "r"(0x00F000F0u), "r"(0x64006400u));
+  out[0] = h2_as_u32(__hsub2(u32_as_h2(t0), k1032));
+  out[1] = h2_as_u32(__hfma2(u32_as_h2(t1), k16th, km72));
+  out[2] = h2_as_u32(__hsub2(u32_as_h2(t2), k1032));
+  out[3] = h2_as_u32(__hfma2(u32_as_h2(t3), k16th, km72));
 }
 
 // half2 (hi, lo) split of a binary32 value: hi = RN16(x), lo = RN16(x - hi).

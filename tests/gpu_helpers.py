@@ -62,9 +62,10 @@ class Pair:
                 raise AssertionError(f"param words differ at {len(bad)} places, first {bad[:5]}")
 
     def oracle_attention(self, q, seq_lens, max_seq_len, block_table, sm_scale):
+        # the C ABI takes sm_scale as binary32: the oracle gets that same value
         return oracle.paged_decode_attn(self.orc, q.view(np.uint16), seq_lens, max_seq_len,
-                                        block_table, sm_scale, self.okc, self.okp, self.ovc,
-                                        self.ovp)
+                                        block_table, float(np.float32(sm_scale)), self.okc,
+                                        self.okp, self.ovc, self.ovp)
 
     def gpu_attention(self, q, seq_lens, max_seq_len, block_table, sm_scale):
         self.err.zero_()
