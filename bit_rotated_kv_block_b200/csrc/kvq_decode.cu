@@ -10,27 +10,31 @@
 //  1. The warp rotates its query heads in registers: lane (r, j) holds
 //     channels [j*d/4, (j+1)*d/4) of query head r (GP = 8) or r % 4 (GP = 4);
 //     butterfly stages inside a quarter run in registers, wider ones across
-//     lanes j by shuffles.
+//     lanes j by shuffles. Each rotated head is then held as a 30-bit fixed
+//     point qint = RN(qhat * 2^30 / amax), split into four signed 8-bit limbs.
 //  2. It streams its (page, KV head) chunks (codes + params of K and V,
 //     contiguous in the pool) into a 2-4 stage shared-memory ring with
-//     cp.async and runs both contractions on tensor cores (mma.sync
-//     m16n8k16, f16 x f16 -> f32):
-//       QK^T: A = [qhat_hi ; qhat_lo] rows of the query heads, B = K codes
-//             (c - 8, exact in f16) as columns, so the score fragment of head
-//             r for tokens {2j, 2j+1, 2j+8, 2j+9} already sits in lane (r, j)
-//             -- exactly the B operand layout of the PV product;
-//       PV:   A = V codes transposed (channels x tokens) built from nibbles
-//             with prmt/lop3, B = p * s_v split into f16 hi + lo columns.
-//     Scale and zero-point are applied algebraically:
-//       qhat . khat = s_k * sum (c - 8) qhat + (m_k + 8 s_k) sum qhat,
-//       sum p vhat  = sum (p s_v)(c - 8)     + sum p (m_v + 8 s_v).
-//     Online softmax in base 2.
+//     cp.async and runs both contractions on tensor cores (mma.sync):
+//       QK^T: m16n8k32 s8 x u8 -> s32, A = the query limbs (one row per
+//             (head, limb)), B = the K codes as bytes (two lop3 per word,
+//             no unpacking to floats); the four limb dots recombine exactly
+//             into sum_i c_i qint_i, and the score
+//               z = sm_scale log2(e) (amax / 2^30) (s_k dot + m_k sum qint)
+//             is formed in double from exact integers;
+//       PV:   m16n8k16 f16 x f16 -> f32, A = V codes transposed (channels x
+//             tokens) as c - 8 (exact in binary16, built from nibbles with
+//             prmt/lop3), B = p * s_v split into binary16 hi + lo columns;
+//             each 16-token product joins the running sum through an IEEE
+//             round-to-nearest add, and sum p (m_v + 8 s_v) is added once at
+//             the end. Online softmax in base 2 (the running max in double).
 //  3. It writes (acc, max, sum) per query head to the workspace, fences, and
 //     bumps a per-(sequence, KV head) counter; the warp that brings the
 //     counter to the number of splits merges all splits (log-sum-exp),
 //     normalises, rotates back in registers, writes the float32 output and
 //     resets the counter to zero. No warp ever waits on another.
 #include <cuda_runtime.h>
+
+#include <type_traits>
 
 #include "kvq_device.cuh"
 #include "kvq_launch.h"
@@ -40,7 +44,6 @@ namespace kvq {
 
 constexpr int kDecWarps = 4;
 constexpr int kMaxPagesPerSplit = 256;  // page ids of one work item live in shared memory
-constexpr float kLog2e = 1.4426950408889634f;
 
 struct DecodeArgs {
   int S, Hq, H, G, P, NP, bt_stride, max_seq_len, splits, pages_per_split;
@@ -78,26 +81,9 @@ struct DecCfg {
   // pipeline depth: about 8-13 KB of pages in flight per warp
   static constexpr int NST = STAGE_B <= 2304 ? 4 : (STAGE_B <= 4608 ? 3 : 2);
   static constexpr int IDS_B = kMaxPagesPerSplit * 4;
-  static constexpr int WARP_B = NST * STAGE_B + IDS_B;
+  static constexpr int BAR_OFF = NST * STAGE_B + IDS_B;  // NST mbarriers
+  static constexpr int WARP_B = (BAR_OFF + NST * 8 + 127) / 128 * 128;
 };
-
-// Swizzled position of the 16-byte unit `u` of token `t` in the V code
-// buffer (conflict-free transposing reads; see the PV fragment loads).
-template <int D>
-__device__ __forceinline__ int v_unit_off(int t, int u) {
-  if (D == 128) {  // 64-byte rows: line = t / 2 holds tokens 2l, 2l+1
-    const int line = t >> 1, un = ((t & 1) << 2) | u;
-    return line * 128 + ((un ^ ((line & 3) << 1)) << 4);
-  } else {  // D == 256: 128-byte rows
-    return t * 128 + ((u ^ (t & 7)) << 4);
-  }
-}
-// Position of the 16-byte unit `u` of token `t` in the K code buffer.
-template <int D>
-__device__ __forceinline__ int k_unit_off(int t, int u) {
-  if (D == 256) return t * 128 + ((u ^ (t & 1)) << 4);
-  return t * (D / 2) + (u << 4);
-}
 
 // Rotation of a query (or output) row held as quarters: lane j of a group
 // of four consecutive lanes owns channels [j*QW, (j+1)*QW). Butterfly
@@ -175,10 +161,98 @@ __global__ void __launch_bounds__(kDecWarps * kWarp) decode_split_kernel(const D
   const bool lo_row = (GP == 4) && (r >= 4);
   const int g = h * a.G + hr;           // global query head
   const bool head_ok = hr < a.G;
+  // ---- page ring: one lane stages each (page, head) chunk with four bulk
+  // copies (K codes, V codes, K params, V params, all contiguous in the
+  // pools) that complete on the stage's mbarrier. Waits are bounded.
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + C::BAR_OFF);
+  if (lane == 0) {
+#pragma unroll
+    for (int b = 0; b < C::NST; ++b) mbar_init(&bars[b], 1);
+    mbar_fence_init();
+  }
+  __syncwarp();
+  auto page_of = [&](int i) { return i < nmine ? ids[i] : -1; };
+  uint32_t pending = 0;  // bit b: stage b has copies in flight (same in all lanes)
+  auto issue = [&](int i) {
+    const int page = page_of(i);
+    if (page < 0 || page >= a.NP) return;
+    const int sidx = i % C::NST;
+    pending |= 1u << sidx;
+    if (lane == 0) {
+      uint8_t* st = ring + sidx * C::STAGE_B;
+      const int64_t row = (int64_t)page * a.H + h;
+      // the stage was last read through ordinary loads: order those before
+      // the bulk copies that overwrite it
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive_expect_tx(&bars[sidx], (uint32_t)C::STAGE_B);
+      bulk_g2s(st, a.k_codes + row * C::CODE_B, C::CODE_B, &bars[sidx]);
+      bulk_g2s(st + C::CODE_B, a.v_codes + row * C::CODE_B, C::CODE_B, &bars[sidx]);
+      bulk_g2s(st + 2 * C::CODE_B, a.k_params + row * P, P * 4, &bars[sidx]);
+      bulk_g2s(st + 2 * C::CODE_B + P * 4, a.v_params + row * P, P * 4, &bars[sidx]);
+    }
+  };
+
+  // Tokens of a 16-token tile are visited in the order
+  //   pi(8h + n) = 8h + (n ^ ((n >> 1) & 1))      (n < 8)
+  // in both products: QK column n of half h is token pi(8h + n), and the PV
+  // k index 2j + c (+ 8h) is the same token. The swap of the pair members for
+  // odd j makes the four lanes j of a V fragment load alternate between the
+  // two 64-byte halves of a 128-byte line (no bank conflicts without a
+  // swizzle).
+  const int tk_r = r ^ ((r >> 1) & 1);        // K row of lane r within a half
+  int tk_e[4];                                 // token of score / PV slot e
+#pragma unroll
+  for (int e = 0; e < 4; ++e) tk_e[e] = 8 * (e >> 1) + 2 * j + ((e & 1) ^ (j & 1));
+  constexpr int VB = D == 128 ? 8 : 16;        // V bytes per lane per token
+  // byte offsets inside a stage (tile 0; tile tt adds 16 tt rows)
+  int k_ld[2], v_ld[4], kp_ld[4];
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) k_ld[nt] = (8 * nt + tk_r) * C::ROWB + j * 16 * (D / 128);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    v_ld[e] = C::CODE_B + tk_e[e] * C::ROWB + r * VB;
+    kp_ld[e] = 2 * C::CODE_B + tk_e[e] * 4;
+  }
+
+  constexpr int NE = GP == 8 ? 4 : 2;
+  const int own = lo_row ? 1 : 0;  // GP = 4: token half of this lane
+  int kps[NE], tks[NE];            // K-param offset and token of score e
+#pragma unroll
+  for (int e = 0; e < NE; ++e) {
+    kps[e] = GP == 8 ? kp_ld[e] : (own ? kp_ld[2 + e] : kp_ld[e]);
+    tks[e] = GP == 8 ? tk_e[e] : (own ? tk_e[2 + e] : tk_e[e]);
+  }
+
+  // ---- state
+  float acc[C::NMT][C::NPV][4];
+#pragma unroll
+  for (int mt = 0; mt < C::NMT; ++mt)
+#pragma unroll
+    for (int n = 0; n < C::NPV; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[mt][n][e] = 0.f;
+  // Scores are formed in double from exact integers: with a dominant (sink)
+  // token the base-2 logits reach ~100, where a binary32 rounding would
+  // already move the other tokens' weights visibly. The running maximum only
+  // serves as the exponent offset, so it is kept in binary32 (a value within
+  // half an ulp of the true maximum) and every weight is 2^(z - M) with the
+  // difference taken in double.
+  float M = -INFINITY;  // running max (base-2 scaled scores) of head hr
+  float Lp = 0.f;       // this lane's share of sum p
+  float Op = 0.f;       // this lane's share of sum p (m_v + 8 s_v)
+  // GP = 8: lane (r, j) scores head r with the tokens of slots e = 0..3;
+  // GP = 4: lanes r and r + 4 share head r % 4 and split those slots,
+  // {0, 1} for r < 4 and {2, 3} for r >= 4
+  uint32_t parity = 0;             // bit b: phase parity awaited on stage b
+  bool dead = false;               // a copy timed out: stop reading pages
+
+  for (int i = 0; i < C::NST - 1; ++i) issue(i);
+
+  // the first pages are in flight while the query is prepared
   // The query as a 30-bit fixed point qint = qhat * 2^30 / amax (amax = the
   // head's largest |qhat|), split into four signed 8-bit limbs
   // qint = l3*2^24 + l2*2^16 + l1*2^8 + l0 for the int8 tensor cores.
-  long long qsum;  // sum of qint over the head's channels (exact)
+  double qsum;     // sum of qint over the head's channels (exact)
   double zk;       // sm_scale * log2(e) * amax / 2^30
   // A fragments per k-step kk: the lane's 8 channels j*QW + 8kk + [0, 8),
   // even ones in a[0]/a[1], odd ones in a[2]/a[3]. Rows:
@@ -207,324 +281,308 @@ __global__ void __launch_bounds__(kDecWarps * kWarp) decode_split_kernel(const D
     for (int i = 0; i < C::QW; ++i) amax = fmaxf(amax, fabsf(x[i]));
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-    const double mul = amax > 0.f ? 1073741824.0 / (double)amax : 0.0;  // 2^30 / amax
-    zk = a.scale2 * ((double)amax * (1.0 / 1073741824.0));
+    // scale 2^k with amax * 2^k < 2^30: a power of two, so qhat * 2^k is
+    // exact in binary32 and the conversion only drops bits below 2^-k
+    const int ebits = (__float_as_int(amax) >> 23) & 0xFF;  // amax < 2^(ebits - 126)
+    int k = 30 - (ebits - 126);
+    k = k > 126 ? 126 : k;
+    const float mulf = amax > 0.f ? __int_as_float((k + 127) << 23) : 0.f;
+    zk = a.scale2 * __hiloint2double((1023 - k) << 20, 0);  // sm_scale log2(e) 2^-k
     long long qs_l = 0;
 #pragma unroll
     for (int kk = 0; kk < C::NKS8; ++kk) {
-      int li[2][4][4];  // [even/odd][l3, l2, l1, l0][4 channels]
+      // limbs of the lane's 8 channels: with t = q + 0x808080 (128 added to
+      // each of the three low bytes), q = sum_k (T_k - 128 [k < 3]) 256^k for
+      // the bytes T_k of t, so the signed limbs are the bytes of
+      // t ^ 0x00808080, byte k = limb k (|q| < 2^30 keeps the top limb in s8)
+      uint32_t u[8];
 #pragma unroll
-      for (int od = 0; od < 2; ++od)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int q = __double2int_rn((double)x[8 * kk + 2 * i + od] * mul);  // |q| <= 2^30
-          qs_l += q;
-          const int l0 = (q << 24) >> 24;
-          const int r1 = (q - l0) >> 8;
-          const int l1 = (r1 << 24) >> 24;
-          const int r2 = (r1 - l1) >> 8;
-          const int l2 = (r2 << 24) >> 24;
-          li[od][0][i] = (r2 - l2) >> 8;
-          li[od][1][i] = l2;
-          li[od][2][i] = l1;
-          li[od][3][i] = l0;
-        }
-      auto pk4 = [&](int od, int limb) {
-        return pack_s8x4(li[od][limb][0], li[od][limb][1], li[od][limb][2], li[od][limb][3]);
+      for (int c = 0; c < 8; ++c) {
+        const int q = __float2int_rn(x[8 * kk + c] * mulf);
+        qs_l += q;
+        u[c] = (uint32_t)(q + 0x808080) ^ 0x00808080u;
+      }
+      // limb `lb` (0 = lowest) of channels {o, o+2, o+4, o+6} as one s8x4 word
+      auto pk4 = [&](int o, int lb) {
+        const uint32_t lo = __byte_perm(u[o], u[o + 2], (lb) | ((4 + lb) << 4));
+        const uint32_t hi = __byte_perm(u[o + 4], u[o + 6], (lb) | ((4 + lb) << 4));
+        return __byte_perm(lo, hi, 0x5410);
       };
       if (GP == 8) {
-        qa[0][kk][0] = pk4(0, 0);
-        qa[0][kk][1] = pk4(0, 1);
-        qa[0][kk][2] = pk4(1, 0);
-        qa[0][kk][3] = pk4(1, 1);
-        qa[C::NQT - 1][kk][0] = pk4(0, 2);
-        qa[C::NQT - 1][kk][1] = pk4(0, 3);
-        qa[C::NQT - 1][kk][2] = pk4(1, 2);
-        qa[C::NQT - 1][kk][3] = pk4(1, 3);
+        qa[0][kk][0] = pk4(0, 3);
+        qa[0][kk][1] = pk4(0, 2);
+        qa[0][kk][2] = pk4(1, 3);
+        qa[0][kk][3] = pk4(1, 2);
+        qa[C::NQT - 1][kk][0] = pk4(0, 1);
+        qa[C::NQT - 1][kk][1] = pk4(0, 0);
+        qa[C::NQT - 1][kk][2] = pk4(1, 1);
+        qa[C::NQT - 1][kk][3] = pk4(1, 0);
       } else {
         // row r: l3 (r < 4) or l2 (r >= 4); row r + 8: l1 (r < 4) or l0
-        qa[0][kk][0] = lo_row ? pk4(0, 1) : pk4(0, 0);
-        qa[0][kk][2] = lo_row ? pk4(1, 1) : pk4(1, 0);
-        qa[0][kk][1] = lo_row ? pk4(0, 3) : pk4(0, 2);
-        qa[0][kk][3] = lo_row ? pk4(1, 3) : pk4(1, 2);
+        qa[0][kk][0] = lo_row ? pk4(0, 2) : pk4(0, 3);
+        qa[0][kk][2] = lo_row ? pk4(1, 2) : pk4(1, 3);
+        qa[0][kk][1] = lo_row ? pk4(0, 0) : pk4(0, 1);
+        qa[0][kk][3] = lo_row ? pk4(1, 0) : pk4(1, 1);
       }
     }
     qs_l += __shfl_xor_sync(0xffffffffu, qs_l, 1);
     qs_l += __shfl_xor_sync(0xffffffffu, qs_l, 2);
-    qsum = qs_l;
+    qsum = (double)qs_l;  // |qsum| <= 2^30 * D: exact
   }
 
-  // ---- page ring: each lane copies the same 16-byte units of every page,
-  // so their shared-memory destinations are computed once
-  constexpr int UNITS = C::CODE_B / 16;        // 16-byte units of codes per pool
-  constexpr int UPT = (D / 2) / 16;            // units per token
-  constexpr int UPL = (UNITS + kWarp - 1) / kWarp;  // units per lane
-  constexpr int PU = P * 4 / 16;               // 16-byte units of params per pool
-  int koff[UPL], voff[UPL];
-#pragma unroll
-  for (int i = 0; i < UPL; ++i) {
-    const int c = lane + kWarp * i;
-    koff[i] = k_unit_off<D>(c / UPT, c % UPT);
-    voff[i] = C::CODE_B + v_unit_off<D>(c / UPT, c % UPT);
-  }
-  const int par_dst = lane < PU ? 2 * C::CODE_B + lane * 16 : 2 * C::CODE_B + P * 4 + (lane - PU) * 16;
-  auto issue = [&](int i) {
-    if (i < nmine) {
-      const int page = ids[i];
-      if (page >= 0 && page < a.NP) {
-        uint8_t* st = ring + (i % C::NST) * C::STAGE_B;
-        const int64_t row = (int64_t)page * a.H + h;
-        const uint8_t* kc = a.k_codes + row * C::CODE_B + lane * 16;
-        const uint8_t* vc = a.v_codes + row * C::CODE_B + lane * 16;
-#pragma unroll
-        for (int u = 0; u < UPL; ++u) {
-          if (UNITS % kWarp == 0 || lane + kWarp * u < UNITS) {
-            cp_async16(st + koff[u], kc + u * kWarp * 16);
-            cp_async16(st + voff[u], vc + u * kWarp * 16);
-          }
-        }
-        if (lane < 2 * PU) {
-          const uint32_t* pp = lane < PU ? a.k_params + row * P : a.v_params + row * P;
-          cp_async16(st + par_dst, reinterpret_cast<const uint8_t*>(pp) + (lane % PU) * 16);
-        }
-      }
-    }
-    cp_async_commit();
-  };
-
-  // ---- state
-  float acc[C::NMT][C::NPV][4];
-#pragma unroll
-  for (int mt = 0; mt < C::NMT; ++mt)
-#pragma unroll
-    for (int n = 0; n < C::NPV; ++n)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[mt][n][e] = 0.f;
-  // Scores are formed in double from exact integers: with a dominant (sink)
-  // token the base-2 logits reach ~100, where a binary32 rounding would
-  // already move the other tokens' weights visibly.
-  double M = -INFINITY;  // running max (base-2 scaled scores) of head hr
-  float Lp = 0.f;       // this lane's share of sum p
-  float Op = 0.f;       // this lane's share of sum p (m_v + 8 s_v)
-
-  for (int i = 0; i < C::NST - 1; ++i) issue(i);
 
   for (int i = 0; i < nmine; ++i) {
-    issue(i + C::NST - 1);
-    cp_async_wait<C::NST - 1>();
-    __syncwarp();
+    if (!dead) issue(i + C::NST - 1);
     const int pidx = pbeg + i;
     const int page = ids[i];
-    const bool page_ok = page >= 0 && page < a.NP;
-    if (!page_ok && lane == 0) raise_flag(a.err, KVQ_ERRF_PAGE);
-    const uint8_t* st = ring + (i % C::NST) * C::STAGE_B;
-    const uint8_t* kbuf = st;
-    const uint8_t* vbuf = st + C::CODE_B;
-    const uint2* kpar = reinterpret_cast<const uint2*>(st + 2 * C::CODE_B);
-    const uint2* vpar = reinterpret_cast<const uint2*>(st + 2 * C::CODE_B + P * 4);
-
-    // ---- scores of all tiles of the page: z[tile][0..3] for tokens
-    // 16*tile + {2j, 2j+1, 2j+8, 2j+9}
-    double z[C::TILES][4];
-#pragma unroll
-    for (int tt = 0; tt < C::TILES; ++tt) {
-      int ci[C::NQT][2][4];
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-        for (int t = 0; t < C::NQT; ++t)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) ci[t][nt][e] = 0;
-        const int tok = 16 * tt + 8 * nt + r;
-        uint32_t w[D / 32];
-#pragma unroll
-        for (int u = 0; u < D / 128; ++u) {
-          const uint4 v4 = *reinterpret_cast<const uint4*>(kbuf + k_unit_off<D>(tok, (D / 128) * j + u));
-          w[4 * u] = v4.x; w[4 * u + 1] = v4.y; w[4 * u + 2] = v4.z; w[4 * u + 3] = v4.w;
-        }
-#pragma unroll
-        for (int kk = 0; kk < C::NKS8; ++kk) {
-          const uint32_t b0 = w[kk] & 0x0F0F0F0Fu;         // even channels as bytes
-          const uint32_t b1 = (w[kk] >> 4) & 0x0F0F0F0Fu;  // odd channels
-#pragma unroll
-          for (int t = 0; t < C::NQT; ++t) mma16832_s8u8(ci[t][nt], qa[t][kk], b0, b1);
-        }
-      }
-      // sum_i (c_i - 8) qint_i of head hr with the four tokens
-      // {2j, 2j+1, 2j+8, 2j+9}, exact in 64-bit integers (the centring keeps
-      // the two score terms small, so their binary32 rounding stays small)
-      long long dt[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int nt = e >> 1, c = e & 1;
-        int l3, l2, l1, l0;
-        if (GP == 8) {
-          l3 = ci[0][nt][c];
-          l2 = ci[0][nt][2 + c];
-          l1 = ci[C::NQT - 1][nt][c];
-          l0 = ci[C::NQT - 1][nt][2 + c];
-        } else {
-          // lanes r < 4 hold the (l3, l1) rows, lanes r + 4 the (l2, l0) rows
-          const int o0 = __shfl_xor_sync(0xffffffffu, ci[0][nt][c], 16);
-          const int o2 = __shfl_xor_sync(0xffffffffu, ci[0][nt][2 + c], 16);
-          l3 = lo_row ? o0 : ci[0][nt][c];
-          l2 = lo_row ? ci[0][nt][c] : o0;
-          l1 = lo_row ? o2 : ci[0][nt][2 + c];
-          l0 = lo_row ? ci[0][nt][2 + c] : o2;
-        }
-        dt[e] = (((long long)l3 * 256ll + l2) * 256ll + l1) * 256ll + l0 - 8ll * qsum;
-      }
-      const uint2 kp01 = kpar[8 * tt + j];      // tokens 16tt + 2j, 2j+1
-      const uint2 kp89 = kpar[8 * tt + 4 + j];  // tokens 16tt + 2j+8, 2j+9
-      const uint32_t kp[4] = {kp01.x, kp01.y, kp89.x, kp89.y};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 sm = __half22float2(u32_as_h2(kp[e]));  // (scale, min)
-        const int tok = pidx * P + 16 * tt + 2 * j + (e & 1) + 8 * (e >> 1);
-        const double sd = (double)sm.x, md = (double)sm.y;
-        const double sc = zk * (sd * (double)dt[e] + (md + 8.0 * sd) * (double)qsum);
-        z[tt][e] = (page_ok && tok < L) ? sc : -INFINITY;
+    const bool page_ok = page >= 0 && page < a.NP && !dead;
+    if (!(page >= 0 && page < a.NP) && lane == 0) raise_flag(a.err, KVQ_ERRF_PAGE);
+    const int sidx = i % C::NST;
+    if (page_ok) {
+      const bool ok = mbar_wait(&bars[sidx], (parity >> sidx) & 1u);
+      parity ^= 1u << sidx;
+      pending &= ~(1u << sidx);
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) raise_flag(a.err, KVQ_ERRF_TIMEOUT);
+        dead = true;
+        break;
       }
     }
+    const uint8_t* st = ring + sidx * C::STAGE_B;
+    // pages whose every token is cached skip all per-token masking
+    const bool full = page_ok && (pidx + 1) * P <= L;
 
-    // ---- online softmax update for head hr (max over the 4 lanes j)
-    double mloc = -INFINITY;
+    auto body = [&](auto masked_tag) {
+      constexpr bool MASKED = decltype(masked_tag)::value;
+      double z[C::TILES][NE];
 #pragma unroll
-    for (int tt = 0; tt < C::TILES; ++tt)
+      for (int tt = 0; tt < C::TILES; ++tt) {
+        int ci[C::NQT][2][4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) mloc = fmax(mloc, z[tt][e]);
-    mloc = fmax(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
-    mloc = fmax(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
-    const double Mn = fmax(M, mloc);
-    const float alpha = (Mn == -INFINITY) ? 1.f : fast_exp2((float)(M - Mn));
-    M = Mn;
-    Lp *= alpha;
-    Op *= alpha;
-    // rescale the output accumulators: lane (r, j) holds columns of heads
-    // c0 = 2(j & (GP/2 - 1)), c0 + 1 -> their alpha from lanes r = c0, c0 + 1
-    if (__any_sync(0xffffffffu, alpha != 1.f)) {  // warp-uniform: skip when no max moved
-      const int c0 = (GP == 8) ? 2 * j : 2 * (j & 1);
-      const float a0 = __shfl_sync(0xffffffffu, alpha, 4 * c0);
-      const float a1 = __shfl_sync(0xffffffffu, alpha, 4 * c0 + 4);
+        for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
-      for (int mt = 0; mt < C::NMT; ++mt)
+          for (int t = 0; t < C::NQT; ++t)
 #pragma unroll
-        for (int n = 0; n < C::NPV; ++n) {
-          acc[mt][n][0] *= a0; acc[mt][n][1] *= a1;
-          acc[mt][n][2] *= a0; acc[mt][n][3] *= a1;
-        }
-    }
-
-    // ---- PV per tile
+            for (int e = 0; e < 4; ++e) ci[t][nt][e] = 0;
+          uint32_t w[D / 32];
 #pragma unroll
-    for (int tt = 0; tt < C::TILES; ++tt) {
-      const uint2 vp01 = vpar[8 * tt + j];
-      const uint2 vp89 = vpar[8 * tt + 4 + j];
-      const uint32_t vp[4] = {vp01.x, vp01.y, vp89.x, vp89.y};
-      float pv[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        // masked tokens may sit on stale or never-written shared memory:
-        // their terms are forced to exact zeros rather than p * (params)
-        const bool live = z[tt][e] != -INFINITY;
-        const float2 sm = __half22float2(u32_as_h2(vp[e]));
-        const float p = live ? fast_exp2((float)(z[tt][e] - M)) : 0.f;
-        Lp += p;
-        Op += live ? p * (sm.y + 8.f * sm.x) : 0.f;
-        pv[e] = live ? p * sm.x : 0.f;
-      }
-      // p * s as f16 hi + lo pairs (packed conversions): hi = RN16(x),
-      // lo = RN16(x - hi), for tokens (2j, 2j+1) and (2j+8, 2j+9)
-      const __half2 h01 = __floats2half2_rn(pv[0], pv[1]);
-      const __half2 h89 = __floats2half2_rn(pv[2], pv[3]);
-      const float2 f01 = __half22float2(h01), f89 = __half22float2(h89);
-      const uint32_t hi01 = h2_as_u32(h01), hi89 = h2_as_u32(h89);
-      const uint32_t lo01 = h2_as_u32(__floats2half2_rn(pv[0] - f01.x, pv[1] - f01.y));
-      const uint32_t lo89 = h2_as_u32(__floats2half2_rn(pv[2] - f89.x, pv[3] - f89.y));
-      // B operand columns: GP = 8: n-tile 0 = hi, 1 = lo (col r = head r);
-      // GP = 4: col r < 4 = hi of head r, r >= 4 = lo of head r - 4
-      uint32_t pb[C::NPV][2];
-      if (GP == 8) {
-        pb[0][0] = hi01;
-        pb[0][1] = hi89;
-        pb[C::NPV - 1][0] = lo01;
-        pb[C::NPV - 1][1] = lo89;
-      } else {
-        pb[0][0] = lo_row ? lo01 : hi01;
-        pb[0][1] = lo_row ? lo89 : hi89;
-      }
-      if (!head_ok) {
-#pragma unroll
-        for (int n = 0; n < C::NPV; ++n) pb[n][0] = pb[n][1] = 0u;
-      }
-      // A operand: V codes of tokens {2j, 2j+1} and {2j+8, 2j+9}, channels of
-      // lane row r: [r*D/8, (r+1)*D/8)
-      constexpr int WPT = D / 64;  // 32-bit words per token per lane
-      uint32_t vw[4][WPT];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int tok = 16 * tt + 2 * j + (e & 1) + 8 * (e >> 1);
-        if (D == 128) {
-          const uint2 v2 = *reinterpret_cast<const uint2*>(vbuf + v_unit_off<D>(tok, r >> 1) + 8 * (r & 1));
-          vw[e][0] = v2.x; vw[e][1] = v2.y;
-        } else {
-          const uint4 v4 = *reinterpret_cast<const uint4*>(vbuf + v_unit_off<D>(tok, r));
-          vw[e][0] = v4.x; vw[e][1] = v4.y; vw[e][2] = v4.z; vw[e][3] = v4.w;
-        }
-      }
-      // m-tile mt: group gq = mt / 8 (words 2gq, 2gq+1), nibble e = mt % 8;
-      // row slot r <- word 2gq, slot r+8 <- word 2gq+1
-#pragma unroll
-      for (int gq = 0; gq < WPT / 2; ++gq) {
-        uint32_t pr[2][2][2];  // [token pair][word in group][lo/hi bytes]
-#pragma unroll
-        for (int tp = 0; tp < 2; ++tp)
-#pragma unroll
-          for (int wi = 0; wi < 2; ++wi) {
-            const int wd = 2 * gq + wi;
-            const uint32_t X = vw[2 * tp][wd], Y = vw[2 * tp + 1][wd];
-            pr[tp][wi][0] = __byte_perm(X, Y, 0x5410);
-            pr[tp][wi][1] = __byte_perm(X, Y, 0x7632);
+          for (int u = 0; u < D / 128; ++u) {
+            const uint4 v4 = *reinterpret_cast<const uint4*>(st + k_ld[nt] + 16 * tt * C::ROWB + 16 * u);
+            w[4 * u] = v4.x; w[4 * u + 1] = v4.y; w[4 * u + 2] = v4.z; w[4 * u + 3] = v4.w;
           }
-        // nibbles of every (token pair, word, byte half): nb[tp][wi][bsel][k]
-        uint32_t nb[2][2][2][4];
 #pragma unroll
-        for (int tp = 0; tp < 2; ++tp)
+          for (int kk = 0; kk < C::NKS8; ++kk) {
+            const uint32_t b0 = w[kk] & 0x0F0F0F0Fu;         // even channels as bytes
+            const uint32_t b1 = (w[kk] >> 4) & 0x0F0F0F0Fu;  // odd channels
 #pragma unroll
-          for (int wi = 0; wi < 2; ++wi)
+            for (int t = 0; t < C::NQT; ++t) mma16832_s8u8(ci[t][nt], qa[t][kk], b0, b1);
+          }
+        }
+        // dot = sum_i c_i qint_i of head hr with each of the lane's tokens,
+        // exact: the limb dots combine as (l3*256 + l2) * 2^16 + (l1*256 + l0)
+        int hA[NE], hB[NE];  // l3*256 + l2 and l1*256 + l0 (|.| < 2^27)
+        if (GP == 8) {
 #pragma unroll
-            for (int bs = 0; bs < 2; ++bs) nib4(pr[tp][wi][bs], nb[tp][wi][bs]);
+          for (int e = 0; e < 4; ++e) {
+            const int nt = e >> 1, c = e & 1;
+            hA[e] = ci[0][nt][c] * 256 + ci[0][nt][2 + c];
+            hB[e] = ci[C::NQT - 1][nt][c] * 256 + ci[C::NQT - 1][nt][2 + c];
+          }
+        } else {
+          // lanes r < 4 hold the (l3, l1) rows, lanes r + 4 the (l2, l0)
+          // rows: each sends the rows of its partner's token half
 #pragma unroll
-        for (int e8 = 0; e8 < 8; ++e8) {
-          const int mt = gq * 8 + e8;
-          const int bsel = e8 >> 2, k = e8 & 3;
-          uint32_t av[4];
-          av[0] = nb[0][0][bsel][k];  // slot r,   tokens 2j, 2j+1
-          av[1] = nb[0][1][bsel][k];  // slot r+8, tokens 2j, 2j+1
-          av[2] = nb[1][0][bsel][k];  // slot r,   tokens 2j+8, 2j+9
-          av[3] = nb[1][1][bsel][k];  // slot r+8, tokens 2j+8, 2j+9
-          // each 16-token product starts from zero and joins the running sum
-          // through an IEEE round-to-nearest add: accumulating inside the
-          // tensor core would round toward zero against a large running sum
+          for (int c = 0; c < 2; ++c) {
+            const int r0 = __shfl_xor_sync(0xffffffffu, lo_row ? ci[0][0][c] : ci[0][1][c], 16);
+            const int r2 = __shfl_xor_sync(0xffffffffu, lo_row ? ci[0][0][2 + c] : ci[0][1][2 + c], 16);
+            const int m0 = lo_row ? ci[0][1][c] : ci[0][0][c];
+            const int m2 = lo_row ? ci[0][1][2 + c] : ci[0][0][2 + c];
+            hA[c] = lo_row ? r0 * 256 + m0 : m0 * 256 + r0;
+            hB[c] = lo_row ? r2 * 256 + m2 : m2 * 256 + r2;
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < NE; ++e) {
+          // exact int32 -> double through the biased exponent 2^52 + 2^31
+          constexpr double kBias = 4503601774854144.0;  // 2^52 + 2^31
+          const double dA = __hiloint2double(0x43300000, hA[e] ^ (int)0x80000000) - kBias;
+          const double dot = fma(dA, 65536.0, __hiloint2double(0x43300000, hB[e] ^ (int)0x80000000)) - kBias;
+          const uint32_t kpw = *reinterpret_cast<const uint32_t*>(st + kps[e] + 64 * tt);
+          const float2 sm = __half22float2(u32_as_h2(kpw));  // (scale, min)
+          // s * dot and m * qsum are exact in double (11 + 41 and 11 + 38 bits)
+          const double sc = zk * fma((double)sm.x, dot, (double)sm.y * qsum);
+          if (MASKED) {
+            const int tok = pidx * P + 16 * tt + tks[e];
+            z[tt][e] = (page_ok && tok < L) ? sc : -INFINITY;
+          } else {
+            z[tt][e] = sc;
+          }
+        }
+      }
+
+      // ---- online softmax update for head hr (max over the lanes sharing it)
+      float mloc = -INFINITY;
+#pragma unroll
+      for (int tt = 0; tt < C::TILES; ++tt)
+#pragma unroll
+        for (int e = 0; e < NE; ++e) mloc = fmaxf(mloc, (float)z[tt][e]);
+      mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
+      mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
+      if (GP == 4) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 16));
+      const float Mn = fmaxf(M, mloc);
+      const float alpha = (Mn == M) ? 1.f : fast_exp2(M - Mn);  // M = -inf: 0
+      M = Mn;
+      const double Md = (double)M;
+      Lp *= alpha;
+      Op *= alpha;
+      // rescale the output accumulators: lane (r, j) holds columns of heads
+      // c0 = 2(j & (GP/2 - 1)), c0 + 1 -> their alpha from lanes r = c0, c0 + 1
+      if (__any_sync(0xffffffffu, alpha != 1.f)) {  // warp-uniform: skip when no max moved
+        const int c0 = (GP == 8) ? 2 * j : 2 * (j & 1);
+        const float a0 = __shfl_sync(0xffffffffu, alpha, 4 * c0);
+        const float a1 = __shfl_sync(0xffffffffu, alpha, 4 * c0 + 4);
+#pragma unroll
+        for (int mt = 0; mt < C::NMT; ++mt)
 #pragma unroll
           for (int n = 0; n < C::NPV; ++n) {
-            float t4[4] = {0.f, 0.f, 0.f, 0.f};
-            mma16816(t4, av, pb[n][0], pb[n][1]);
+            acc[mt][n][0] *= a0; acc[mt][n][1] *= a1;
+            acc[mt][n][2] *= a0; acc[mt][n][3] *= a1;
+          }
+      }
+
+      // ---- PV per tile
 #pragma unroll
-            for (int e = 0; e < 4; ++e) acc[mt][n][e] = __fadd_rn(acc[mt][n][e], t4[e]);
+      for (int tt = 0; tt < C::TILES; ++tt) {
+        float pv[NE];
+#pragma unroll
+        for (int e = 0; e < NE; ++e) {
+          const uint32_t vpw = *reinterpret_cast<const uint32_t*>(st + kps[e] + P * 4 + 64 * tt);
+          const float2 sm = __half22float2(u32_as_h2(vpw));  // (scale, min)
+          if (MASKED) {
+            // masked tokens may sit on stale or never-written shared memory:
+            // their terms are forced to exact zeros rather than p * (params)
+            const bool live = z[tt][e] != -INFINITY;
+            const float p = live ? fast_exp2((float)(z[tt][e] - Md)) : 0.f;
+            Lp += p;
+            Op += live ? p * (sm.y + 8.f * sm.x) : 0.f;
+            pv[e] = live ? p * sm.x : 0.f;
+          } else {
+            const float p = fast_exp2((float)(z[tt][e] - Md));
+            Lp += p;
+            Op = fmaf(p, sm.y + 8.f * sm.x, Op);
+            pv[e] = p * sm.x;
+          }
+        }
+        // p * s as binary16 hi + lo pairs (packed conversions): hi = RN16(x),
+        // lo = RN16(x - hi)
+        uint32_t pb[C::NPV][2];
+        if (GP == 8) {
+          // n-tile 0 = hi, 1 = lo; column r = head r; k slots (0, 1), (2, 3)
+          const __half2 h01 = __floats2half2_rn(pv[0], pv[1]);
+          const __half2 h89 = __floats2half2_rn(pv[NE - 2], pv[NE - 1]);
+          const float2 f01 = __half22float2(h01), f89 = __half22float2(h89);
+          pb[0][0] = h2_as_u32(h01);
+          pb[0][1] = h2_as_u32(h89);
+          pb[C::NPV - 1][0] = h2_as_u32(__floats2half2_rn(pv[0] - f01.x, pv[1] - f01.y));
+          pb[C::NPV - 1][1] = h2_as_u32(__floats2half2_rn(pv[NE - 2] - f89.x, pv[NE - 1] - f89.y));
+        } else {
+          // column r < 4 = hi of head r, r >= 4 = lo of head r - 4: lane r
+          // keeps hi (or lo) of its own token half and takes the other
+          // half's from its partner r ^ 4
+          const __half2 ho = __floats2half2_rn(pv[0], pv[1]);
+          const float2 fo = __half22float2(ho);
+          const uint32_t hi_own = h2_as_u32(ho);
+          const uint32_t lo_own = h2_as_u32(__floats2half2_rn(pv[0] - fo.x, pv[1] - fo.y));
+          const uint32_t got = __shfl_xor_sync(0xffffffffu, lo_row ? hi_own : lo_own, 16);
+          pb[0][0] = lo_row ? got : hi_own;  // slots 0, 1
+          pb[0][1] = lo_row ? lo_own : got;  // slots 2, 3
+        }
+        if (!head_ok) {
+#pragma unroll
+          for (int n = 0; n < C::NPV; ++n) pb[n][0] = pb[n][1] = 0u;
+        }
+        // A operand: V codes of the slots' tokens, channels of lane row r:
+        // [r*D/8, (r+1)*D/8)
+        constexpr int WPT = D / 64;  // 32-bit words per token per lane
+        uint32_t vw[4][WPT];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint8_t* src = st + v_ld[e] + 16 * tt * C::ROWB;
+          if (D == 128) {
+            const uint2 v2 = *reinterpret_cast<const uint2*>(src);
+            vw[e][0] = v2.x; vw[e][1] = v2.y;
+          } else {
+            const uint4 v4 = *reinterpret_cast<const uint4*>(src);
+            vw[e][0] = v4.x; vw[e][1] = v4.y; vw[e][2] = v4.z; vw[e][3] = v4.w;
+          }
+        }
+        // m-tile mt: group gq = mt / 8 (words 2gq, 2gq+1), nibble e = mt % 8;
+        // row slot r <- word 2gq, slot r+8 <- word 2gq+1
+#pragma unroll
+        for (int gq = 0; gq < WPT / 2; ++gq) {
+          uint32_t pr[2][2][2];  // [slot pair][word in group][lo/hi bytes]
+#pragma unroll
+          for (int tp = 0; tp < 2; ++tp)
+#pragma unroll
+            for (int wi = 0; wi < 2; ++wi) {
+              const int wd = 2 * gq + wi;
+              const uint32_t X = vw[2 * tp][wd], Y = vw[2 * tp + 1][wd];
+              pr[tp][wi][0] = __byte_perm(X, Y, 0x5410);
+              pr[tp][wi][1] = __byte_perm(X, Y, 0x7632);
+            }
+          // nibbles of every (slot pair, word, byte half): nb[tp][wi][bsel][k]
+          uint32_t nb[2][2][2][4];
+#pragma unroll
+          for (int tp = 0; tp < 2; ++tp)
+#pragma unroll
+            for (int wi = 0; wi < 2; ++wi)
+#pragma unroll
+              for (int bs = 0; bs < 2; ++bs) nib4(pr[tp][wi][bs], nb[tp][wi][bs]);
+#pragma unroll
+          for (int e8 = 0; e8 < 8; ++e8) {
+            const int mt = gq * 8 + e8;
+            const int bsel = e8 >> 2, k = e8 & 3;
+            uint32_t av[4];
+            av[0] = nb[0][0][bsel][k];  // row slot r,   k slots 0, 1
+            av[1] = nb[0][1][bsel][k];  // row slot r+8, k slots 0, 1
+            av[2] = nb[1][0][bsel][k];  // row slot r,   k slots 2, 3
+            av[3] = nb[1][1][bsel][k];  // row slot r+8, k slots 2, 3
+            // each 16-token product starts from zero and joins the running
+            // sum through an IEEE round-to-nearest add: accumulating inside
+            // the tensor core would round toward zero against a large sum
+#pragma unroll
+            for (int n = 0; n < C::NPV; ++n) {
+              float t4[4] = {0.f, 0.f, 0.f, 0.f};
+              mma16816(t4, av, pb[n][0], pb[n][1]);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) acc[mt][n][e] = __fadd_rn(acc[mt][n][e], t4[e]);
+            }
           }
         }
       }
-    }
-    __syncwarp();  // stage i % C::NST is refilled by the next issue
+    };
+    if (full)
+      body(std::false_type{});
+    else
+      body(std::true_type{});
+    __syncwarp();  // every lane is done with stage i % C::NST before it is refilled
   }
-  cp_async_wait<0>();
+  if (dead) {
+    // let the copies already in flight land (bounded) before leaving the ring
+#pragma unroll 1
+    for (int b = 0; b < C::NST; ++b)
+      if ((pending >> b) & 1u) mbar_wait(&bars[b], (parity >> b) & 1u);
+  }
 
   // ---- partial results: (acc + sum p (m + 8 s)) per channel, M, sum p
   Lp += __shfl_xor_sync(0xffffffffu, Lp, 1);
   Lp += __shfl_xor_sync(0xffffffffu, Lp, 2);
   Op += __shfl_xor_sync(0xffffffffu, Op, 1);
   Op += __shfl_xor_sync(0xffffffffu, Op, 2);
+  if (GP == 4) {  // the two token halves of head hr
+    Lp += __shfl_xor_sync(0xffffffffu, Lp, 16);
+    Op += __shfl_xor_sync(0xffffffffu, Op, 16);
+  }
   if (GP == 4) {
     // fold the lo columns (lanes j = 2, 3) onto the hi columns (j = 0, 1)
 #pragma unroll
@@ -574,33 +632,48 @@ __global__ void __launch_bounds__(kDecWarps * kWarp) decode_split_kernel(const D
   if (!last) return;
   __threadfence();
   const bool owner = head_ok && !lo_row;
+  // lanes of head hr: quarter j of the channels; for GP = 4 the partner
+  // lanes r + 4 take the odd splits and the two halves are added at the end
+  const int sub = (GP == 4) ? own : 0, nsub = (GP == 4) ? 2 : 1;
   float x[C::QW];
 #pragma unroll
   for (int c = 0; c < C::QW; ++c) x[c] = 0.f;
-  if (owner) {
+  float Ls = 0.f;
+  if (head_ok) {
     const float* src = a.part + ((int64_t)s * a.Hq + g) * a.splits * (D + 4);
     double Mx = -INFINITY;
+#pragma unroll 4
     for (int i = 0; i < a.splits; ++i)
       Mx = fmax(Mx, __ldcg(reinterpret_cast<const double*>(src + (int64_t)i * (D + 4) + D)));
-    float Ls = 0.f;
     if (Mx != -INFINITY) {
-      for (int i = 0; i < a.splits; ++i) {
+#pragma unroll 2
+      for (int i = sub; i < a.splits; i += nsub) {
         const float* pi = src + (int64_t)i * (D + 4);
         const double Mi = __ldcg(reinterpret_cast<const double*>(pi + D));
-        if (Mi == -INFINITY) continue;
-        const float wgt = fast_exp2((float)(Mi - Mx));
-        Ls += wgt * __ldcg(pi + D + 2);
+        const float li = __ldcg(pi + D + 2);
         const float4* v4 = reinterpret_cast<const float4*>(pi + j * C::QW);
+        float4 f[C::QW / 4];
+#pragma unroll
+        for (int c = 0; c < C::QW / 4; ++c) f[c] = __ldcg(v4 + c);
+        // an empty split (max -inf) has a zero row and a zero sum: weight 0
+        const float wgt = Mi == -INFINITY ? 0.f : fast_exp2((float)(Mi - Mx));
+        Ls += wgt * li;
 #pragma unroll
         for (int c = 0; c < C::QW / 4; ++c) {
-          const float4 f = __ldcg(v4 + c);
-          x[4 * c] += wgt * f.x;
-          x[4 * c + 1] += wgt * f.y;
-          x[4 * c + 2] += wgt * f.z;
-          x[4 * c + 3] += wgt * f.w;
+          x[4 * c] += wgt * f[c].x;
+          x[4 * c + 1] += wgt * f[c].y;
+          x[4 * c + 2] += wgt * f[c].z;
+          x[4 * c + 3] += wgt * f[c].w;
         }
       }
     }
+  }
+  if (GP == 4) {
+    Ls += __shfl_xor_sync(0xffffffffu, Ls, 16);
+#pragma unroll
+    for (int c = 0; c < C::QW; ++c) x[c] += __shfl_xor_sync(0xffffffffu, x[c], 16);
+  }
+  {
     const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
 #pragma unroll
     for (int c = 0; c < C::QW; ++c) x[c] *= inv;
