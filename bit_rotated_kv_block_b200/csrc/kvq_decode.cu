@@ -77,12 +77,14 @@ struct DecCfg {
   static constexpr int QW = D / 4;             // query channels per lane
   static constexpr int ROWB = D / 2;           // code bytes per token
   static constexpr int CODE_B = P * ROWB;      // code bytes per (page, head)
-  static constexpr int STAGE_B = 2 * CODE_B + 8 * P;
+  static constexpr int PAGE_B = 2 * CODE_B + 8 * P;  // K codes, V codes, K and V params
+  static constexpr int PG = P == 16 ? 2 : 1;         // pages per pipeline stage
+  static constexpr int TPG = TILES * PG;             // 16-token tiles per stage
+  static constexpr int STAGE_B = PG * PAGE_B;
   // pipeline depth: about 8-13 KB of pages in flight per warp
   static constexpr int NST = STAGE_B <= 2304 ? 4 : (STAGE_B <= 4608 ? 3 : 2);
   static constexpr int IDS_B = kMaxPagesPerSplit * 4;
-  static constexpr int BAR_OFF = NST * STAGE_B + IDS_B;  // NST mbarriers
-  static constexpr int WARP_B = (BAR_OFF + NST * 8 + 127) / 128 * 128;
+  static constexpr int WARP_B = (NST * STAGE_B + IDS_B + 127) / 128 * 128;
 };
 
 // Rotation of a query (or output) row held as quarters: lane j of a group
@@ -123,7 +125,8 @@ __device__ __forceinline__ void rotate_quarter(float (&x)[QW], int j, int rot_ki
 }
 
 template <int D, int P, int GP>
-__global__ void __launch_bounds__(kDecWarps * kWarp) decode_split_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kDecWarps * kWarp, (D == 128 && GP == 4) ? 4 : 1)
+    decode_split_kernel(const DecodeArgs a) {
   static_assert(D == 128 || D == 256, "decode attention supports head_dim 128 and 256");
   using C = DecCfg<D, P, GP>;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -161,35 +164,45 @@ __global__ void __launch_bounds__(kDecWarps * kWarp) decode_split_kernel(const D
   const bool lo_row = (GP == 4) && (r >= 4);
   const int g = h * a.G + hr;           // global query head
   const bool head_ok = hr < a.G;
-  // ---- page ring: one lane stages each (page, head) chunk with four bulk
-  // copies (K codes, V codes, K params, V params, all contiguous in the
-  // pools) that complete on the stage's mbarrier. Waits are bounded.
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + C::BAR_OFF);
-  if (lane == 0) {
+  // ---- page ring: the warp stages each (page, head) chunk (K codes, V
+  // codes, K params, V params, all contiguous in their pools) with 16-byte
+  // cp.async copies, linear in shared memory: 16-byte unit u of a page block
+  // is copied by lane u % 32. One commit group per stage of PG pages.
+  constexpr int KU = C::CODE_B / 16;  // units of codes per pool (a multiple of 32)
+  constexpr int PU = P / 4;           // units of params per pool (<= 16)
+  static_assert(KU % kWarp == 0 && 2 * PU <= kWarp, "page block does not tile the warp");
+  const int64_t cstride = (int64_t)a.H * C::CODE_B, pstride = (int64_t)a.H * P * 4;
+  const uint8_t* const kc_l = a.k_codes + (int64_t)h * C::CODE_B + lane * 16;
+  const uint8_t* const vc_l = a.v_codes + (int64_t)h * C::CODE_B + lane * 16;
+  const uint8_t* const par_l =
+      lane < PU ? reinterpret_cast<const uint8_t*>(a.k_params) + (int64_t)h * P * 4 + lane * 16
+                : reinterpret_cast<const uint8_t*>(a.v_params) + (int64_t)h * P * 4 + (lane - PU) * 16;
+  const int ngrp = (nmine + C::PG - 1) / C::PG;
+  auto page_valid = [&](int pi) {
+    if (pi >= nmine) return false;
+    const int pg = ids[pi];
+    return pg >= 0 && pg < a.NP;
+  };
+  // stage the pages of group gi (pages gi*PG .. gi*PG + PG - 1 of the item)
+  // into stage sidx; pages outside the pool or the item are not copied
+  // (their tokens are masked)
+  auto issue = [&](int gi, int sidx) {
+    if (gi < ngrp) {
 #pragma unroll
-    for (int b = 0; b < C::NST; ++b) mbar_init(&bars[b], 1);
-    mbar_fence_init();
-  }
-  __syncwarp();
-  auto page_of = [&](int i) { return i < nmine ? ids[i] : -1; };
-  uint32_t pending = 0;  // bit b: stage b has copies in flight (same in all lanes)
-  auto issue = [&](int i) {
-    const int page = page_of(i);
-    if (page < 0 || page >= a.NP) return;
-    const int sidx = i % C::NST;
-    pending |= 1u << sidx;
-    if (lane == 0) {
-      uint8_t* st = ring + sidx * C::STAGE_B;
-      const int64_t row = (int64_t)page * a.H + h;
-      // the stage was last read through ordinary loads: order those before
-      // the bulk copies that overwrite it
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_arrive_expect_tx(&bars[sidx], (uint32_t)C::STAGE_B);
-      bulk_g2s(st, a.k_codes + row * C::CODE_B, C::CODE_B, &bars[sidx]);
-      bulk_g2s(st + C::CODE_B, a.v_codes + row * C::CODE_B, C::CODE_B, &bars[sidx]);
-      bulk_g2s(st + 2 * C::CODE_B, a.k_params + row * P, P * 4, &bars[sidx]);
-      bulk_g2s(st + 2 * C::CODE_B + P * 4, a.v_params + row * P, P * 4, &bars[sidx]);
+      for (int q = 0; q < C::PG; ++q) {
+        const int pi = gi * C::PG + q;
+        if (!page_valid(pi)) continue;
+        const int64_t page = ids[pi];
+        const int64_t co = page * cstride;
+        uint8_t* dst = ring + sidx * C::STAGE_B + q * C::PAGE_B + lane * 16;
+#pragma unroll
+        for (int m = 0; m < KU / kWarp; ++m) cp_async16(dst + m * 512, kc_l + co + m * 512);
+#pragma unroll
+        for (int m = 0; m < KU / kWarp; ++m) cp_async16(dst + C::CODE_B + m * 512, vc_l + co + m * 512);
+        if (lane < 2 * PU) cp_async16(dst + 2 * C::CODE_B, par_l + page * pstride);
+      }
     }
+    cp_async_commit();
   };
 
   // Tokens of a 16-token tile are visited in the order
@@ -243,10 +256,9 @@ __global__ void __launch_bounds__(kDecWarps * kWarp) decode_split_kernel(const D
   // GP = 8: lane (r, j) scores head r with the tokens of slots e = 0..3;
   // GP = 4: lanes r and r + 4 share head r % 4 and split those slots,
   // {0, 1} for r < 4 and {2, 3} for r >= 4
-  uint32_t parity = 0;             // bit b: phase parity awaited on stage b
-  bool dead = false;               // a copy timed out: stop reading pages
 
-  for (int i = 0; i < C::NST - 1; ++i) issue(i);
+#pragma unroll
+  for (int i = 0; i < C::NST - 1; ++i) issue(i, i);
 
   // the first pages are in flight while the query is prepared
   // The query as a 30-bit fixed point qint = qhat * 2^30 / amax (amax = the
@@ -256,7 +268,7 @@ __global__ void __launch_bounds__(kDecWarps * kWarp) decode_split_kernel(const D
   double zk;       // sm_scale * log2(e) * amax / 2^30
   // A fragments per k-step kk: the lane's 8 channels j*QW + 8kk + [0, 8),
   // even ones in a[0]/a[1], odd ones in a[2]/a[3]. Rows:
-  //   GP = 4: rows 0-3 l3, 4-7 l2, 8-11 l1, 12-15 l0 of heads 0-3;
+  //   GP = 4: rows 0-3 l3, 4-7 l1, 8-11 l2, 12-15 l0 of heads 0-3;
   //   GP = 8: tile 0 rows 0-7 l3, 8-15 l2; tile 1 rows 0-7 l1, 8-15 l0.
   uint32_t qa[C::NQT][C::NKS8][4];
   {
@@ -318,11 +330,11 @@ __global__ void __launch_bounds__(kDecWarps * kWarp) decode_split_kernel(const D
         qa[C::NQT - 1][kk][2] = pk4(1, 1);
         qa[C::NQT - 1][kk][3] = pk4(1, 0);
       } else {
-        // row r: l3 (r < 4) or l2 (r >= 4); row r + 8: l1 (r < 4) or l0
-        qa[0][kk][0] = lo_row ? pk4(0, 2) : pk4(0, 3);
-        qa[0][kk][2] = lo_row ? pk4(1, 2) : pk4(1, 3);
-        qa[0][kk][1] = lo_row ? pk4(0, 0) : pk4(0, 1);
-        qa[0][kk][3] = lo_row ? pk4(1, 0) : pk4(1, 1);
+        // row r: l3 (r < 4) or l1 (r >= 4); row r + 8: l2 (r < 4) or l0
+        qa[0][kk][0] = lo_row ? pk4(0, 1) : pk4(0, 3);
+        qa[0][kk][2] = lo_row ? pk4(1, 1) : pk4(1, 3);
+        qa[0][kk][1] = lo_row ? pk4(0, 0) : pk4(0, 2);
+        qa[0][kk][3] = lo_row ? pk4(1, 0) : pk4(1, 2);
       }
     }
     qs_l += __shfl_xor_sync(0xffffffffu, qs_l, 1);
@@ -331,32 +343,36 @@ __global__ void __launch_bounds__(kDecWarps * kWarp) decode_split_kernel(const D
   }
 
 
-  for (int i = 0; i < nmine; ++i) {
-    if (!dead) issue(i + C::NST - 1);
-    const int pidx = pbeg + i;
-    const int page = ids[i];
-    const bool page_ok = page >= 0 && page < a.NP && !dead;
-    if (!(page >= 0 && page < a.NP) && lane == 0) raise_flag(a.err, KVQ_ERRF_PAGE);
-    const int sidx = i % C::NST;
-    if (page_ok) {
-      const bool ok = mbar_wait(&bars[sidx], (parity >> sidx) & 1u);
-      parity ^= 1u << sidx;
-      pending &= ~(1u << sidx);
-      if (!__all_sync(0xffffffffu, ok)) {
-        if (lane == 0) raise_flag(a.err, KVQ_ERRF_TIMEOUT);
-        dead = true;
-        break;
-      }
+  int sidx = 0;             // stage of group gi
+  int sissue = C::NST - 1;  // stage of group gi + NST - 1
+  for (int gi = 0; gi < ngrp; ++gi) {
+    issue(gi + C::NST - 1, sissue);
+    sissue = sissue + 1 == C::NST ? 0 : sissue + 1;
+    bool pgok[C::PG];  // page q of the group is in the item and in the pool
+    bool all_ok = true;
+#pragma unroll
+    for (int q = 0; q < C::PG; ++q) {
+      const int pi = gi * C::PG + q;
+      pgok[q] = page_valid(pi);
+      all_ok = all_ok && pgok[q];
+      if (pi < nmine && !pgok[q] && lane == 0) raise_flag(a.err, KVQ_ERRF_PAGE);
     }
+    cp_async_wait<C::NST - 1>();  // this lane's copies of group gi have landed
+    __syncwarp();                 // ... and every other lane's
     const uint8_t* st = ring + sidx * C::STAGE_B;
-    // pages whose every token is cached skip all per-token masking
-    const bool full = page_ok && (pidx + 1) * P <= L;
+    sidx = sidx + 1 == C::NST ? 0 : sidx + 1;
+    const int tok0 = (pbeg + gi * C::PG) * P;  // first token of the group
+    // groups whose every token is cached skip all per-token masking
+    const bool full = all_ok && tok0 + C::PG * P <= L;
 
     auto body = [&](auto masked_tag) {
       constexpr bool MASKED = decltype(masked_tag)::value;
-      double z[C::TILES][NE];
+      double z[C::TPG][NE];
 #pragma unroll
-      for (int tt = 0; tt < C::TILES; ++tt) {
+      for (int tt = 0; tt < C::TPG; ++tt) {
+        // tile tt of the group: page tt / TILES, 16-token tile tt % TILES
+        const int cofs = (tt / C::TILES) * C::PAGE_B + (tt % C::TILES) * 16 * C::ROWB;
+        const int pofs = (tt / C::TILES) * C::PAGE_B + (tt % C::TILES) * 64;
         int ci[C::NQT][2][4];
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
@@ -367,7 +383,7 @@ __global__ void __launch_bounds__(kDecWarps * kWarp) decode_split_kernel(const D
           uint32_t w[D / 32];
 #pragma unroll
           for (int u = 0; u < D / 128; ++u) {
-            const uint4 v4 = *reinterpret_cast<const uint4*>(st + k_ld[nt] + 16 * tt * C::ROWB + 16 * u);
+            const uint4 v4 = *reinterpret_cast<const uint4*>(st + k_ld[nt] + cofs + 16 * u);
             w[4 * u] = v4.x; w[4 * u + 1] = v4.y; w[4 * u + 2] = v4.z; w[4 * u + 3] = v4.w;
           }
 #pragma unroll
@@ -389,16 +405,17 @@ __global__ void __launch_bounds__(kDecWarps * kWarp) decode_split_kernel(const D
             hB[e] = ci[C::NQT - 1][nt][c] * 256 + ci[C::NQT - 1][nt][2 + c];
           }
         } else {
-          // lanes r < 4 hold the (l3, l1) rows, lanes r + 4 the (l2, l0)
-          // rows: each sends the rows of its partner's token half
+          // lanes r < 4 hold the (l3, l2) rows and form l3*256 + l2, lanes
+          // r + 4 the (l1, l0) rows and form l1*256 + l0, for both token
+          // halves; each sends its partner the half that partner scores
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
-            const int r0 = __shfl_xor_sync(0xffffffffu, lo_row ? ci[0][0][c] : ci[0][1][c], 16);
-            const int r2 = __shfl_xor_sync(0xffffffffu, lo_row ? ci[0][0][2 + c] : ci[0][1][2 + c], 16);
-            const int m0 = lo_row ? ci[0][1][c] : ci[0][0][c];
-            const int m2 = lo_row ? ci[0][1][2 + c] : ci[0][0][2 + c];
-            hA[c] = lo_row ? r0 * 256 + m0 : m0 * 256 + r0;
-            hB[c] = lo_row ? r2 * 256 + m2 : m2 * 256 + r2;
+            const int loc0 = ci[0][0][c] * 256 + ci[0][0][2 + c];
+            const int loc1 = ci[0][1][c] * 256 + ci[0][1][2 + c];
+            const int got = __shfl_xor_sync(0xffffffffu, lo_row ? loc0 : loc1, 16);
+            const int mine = lo_row ? loc1 : loc0;
+            hA[c] = lo_row ? got : mine;
+            hB[c] = lo_row ? mine : got;
           }
         }
 #pragma unroll
@@ -407,13 +424,13 @@ __global__ void __launch_bounds__(kDecWarps * kWarp) decode_split_kernel(const D
           constexpr double kBias = 4503601774854144.0;  // 2^52 + 2^31
           const double dA = __hiloint2double(0x43300000, hA[e] ^ (int)0x80000000) - kBias;
           const double dot = fma(dA, 65536.0, __hiloint2double(0x43300000, hB[e] ^ (int)0x80000000)) - kBias;
-          const uint32_t kpw = *reinterpret_cast<const uint32_t*>(st + kps[e] + 64 * tt);
+          const uint32_t kpw = *reinterpret_cast<const uint32_t*>(st + kps[e] + pofs);
           const float2 sm = __half22float2(u32_as_h2(kpw));  // (scale, min)
           // s * dot and m * qsum are exact in double (11 + 41 and 11 + 38 bits)
           const double sc = zk * fma((double)sm.x, dot, (double)sm.y * qsum);
           if (MASKED) {
-            const int tok = pidx * P + 16 * tt + tks[e];
-            z[tt][e] = (page_ok && tok < L) ? sc : -INFINITY;
+            const int tok = tok0 + (tt / C::TILES) * P + (tt % C::TILES) * 16 + tks[e];
+            z[tt][e] = (pgok[tt / C::TILES] && tok < L) ? sc : -INFINITY;
           } else {
             z[tt][e] = sc;
           }
@@ -423,7 +440,7 @@ __global__ void __launch_bounds__(kDecWarps * kWarp) decode_split_kernel(const D
       // ---- online softmax update for head hr (max over the lanes sharing it)
       float mloc = -INFINITY;
 #pragma unroll
-      for (int tt = 0; tt < C::TILES; ++tt)
+      for (int tt = 0; tt < C::TPG; ++tt)
 #pragma unroll
         for (int e = 0; e < NE; ++e) mloc = fmaxf(mloc, (float)z[tt][e]);
       mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
@@ -452,11 +469,13 @@ __global__ void __launch_bounds__(kDecWarps * kWarp) decode_split_kernel(const D
 
       // ---- PV per tile
 #pragma unroll
-      for (int tt = 0; tt < C::TILES; ++tt) {
+      for (int tt = 0; tt < C::TPG; ++tt) {
+        const int cofs = (tt / C::TILES) * C::PAGE_B + (tt % C::TILES) * 16 * C::ROWB;
+        const int pofs = (tt / C::TILES) * C::PAGE_B + (tt % C::TILES) * 64;
         float pv[NE];
 #pragma unroll
         for (int e = 0; e < NE; ++e) {
-          const uint32_t vpw = *reinterpret_cast<const uint32_t*>(st + kps[e] + P * 4 + 64 * tt);
+          const uint32_t vpw = *reinterpret_cast<const uint32_t*>(st + kps[e] + P * 4 + pofs);
           const float2 sm = __half22float2(u32_as_h2(vpw));  // (scale, min)
           if (MASKED) {
             // masked tokens may sit on stale or never-written shared memory:
@@ -507,7 +526,7 @@ __global__ void __launch_bounds__(kDecWarps * kWarp) decode_split_kernel(const D
         uint32_t vw[4][WPT];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const uint8_t* src = st + v_ld[e] + 16 * tt * C::ROWB;
+          const uint8_t* src = st + v_ld[e] + cofs;
           if (D == 128) {
             const uint2 v2 = *reinterpret_cast<const uint2*>(src);
             vw[e][0] = v2.x; vw[e][1] = v2.y;
@@ -567,12 +586,7 @@ __global__ void __launch_bounds__(kDecWarps * kWarp) decode_split_kernel(const D
       body(std::true_type{});
     __syncwarp();  // every lane is done with stage i % C::NST before it is refilled
   }
-  if (dead) {
-    // let the copies already in flight land (bounded) before leaving the ring
-#pragma unroll 1
-    for (int b = 0; b < C::NST; ++b)
-      if ((pending >> b) & 1u) mbar_wait(&bars[b], (parity >> b) & 1u);
-  }
+  cp_async_wait<0>();
 
   // ---- partial results: (acc + sum p (m + 8 s)) per channel, M, sum p
   Lp += __shfl_xor_sync(0xffffffffu, Lp, 1);
@@ -624,13 +638,21 @@ __global__ void __launch_bounds__(kDecWarps * kWarp) decode_split_kernel(const D
   }
 
   // ---- the last warp of this (sequence, KV head) merges the splits
-  __threadfence();
+  // The warp's partial writes are ordered before lane 0's counter update by
+  // the warp barrier; the update is a release (publishes them) and an
+  // acquire (the last arriver then sees every split's writes).
   __syncwarp();
   int last = 0;
-  if (lane == 0) last = atomicAdd(a.counter + (int64_t)s * a.H + h, 1) == a.splits - 1;
+  if (lane == 0) {
+    int prev;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;"
+                 : "=r"(prev)
+                 : "l"(a.counter + (int64_t)s * a.H + h)
+                 : "memory");
+    last = prev == a.splits - 1;
+  }
   last = __shfl_sync(0xffffffffu, last, 0);
   if (!last) return;
-  __threadfence();
   const bool owner = head_ok && !lo_row;
   // lanes of head hr: quarter j of the channels; for GP = 4 the partner
   // lanes r + 4 take the odd splits and the two halves are added at the end
@@ -639,12 +661,31 @@ __global__ void __launch_bounds__(kDecWarps * kWarp) decode_split_kernel(const D
 #pragma unroll
   for (int c = 0; c < C::QW; ++c) x[c] = 0.f;
   float Ls = 0.f;
+  // lanes of a head without a query head (G < GP) load nothing; the
+  // shuffles below run in every lane and stay within one head's lanes
+  const float* src = a.part + ((int64_t)s * a.Hq + g) * a.splits * (D + 4);
+  double Mx = -INFINITY;
+  {
+    // the splits' maxima: the NL lanes of the head load interleaved splits,
+    // four rounds at a time, then reduce
+    constexpr int NL = GP == 4 ? 8 : 4;
+    const int li0 = GP == 4 ? 4 * own + j : j;
+    const int nsp = head_ok ? a.splits : 0;
+    for (int i0 = 0; i0 < nsp; i0 += 4 * NL) {
+      double mv[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int i = i0 + li0 + NL * m;
+        mv[m] = i < nsp ? __ldcg(reinterpret_cast<const double*>(src + (int64_t)i * (D + 4) + D))
+                        : -INFINITY;
+      }
+      Mx = fmax(Mx, fmax(fmax(mv[0], mv[1]), fmax(mv[2], mv[3])));
+    }
+  }
+  Mx = fmax(Mx, __shfl_xor_sync(0xffffffffu, Mx, 1));
+  Mx = fmax(Mx, __shfl_xor_sync(0xffffffffu, Mx, 2));
+  if (GP == 4) Mx = fmax(Mx, __shfl_xor_sync(0xffffffffu, Mx, 16));
   if (head_ok) {
-    const float* src = a.part + ((int64_t)s * a.Hq + g) * a.splits * (D + 4);
-    double Mx = -INFINITY;
-#pragma unroll 4
-    for (int i = 0; i < a.splits; ++i)
-      Mx = fmax(Mx, __ldcg(reinterpret_cast<const double*>(src + (int64_t)i * (D + 4) + D)));
     if (Mx != -INFINITY) {
 #pragma unroll 2
       for (int i = sub; i < a.splits; i += nsub) {
