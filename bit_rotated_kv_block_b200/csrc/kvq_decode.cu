@@ -125,7 +125,7 @@ __device__ __forceinline__ void rotate_quarter(float (&x)[QW], int j, int rot_ki
 }
 
 template <int D, int P, int GP>
-__global__ void __launch_bounds__(kDecWarps * kWarp, (D == 128 && GP == 4) ? 4 : 1)
+__global__ void __launch_bounds__(kDecWarps * kWarp, (D == 128 && GP == 4) ? 4 : 2)
     decode_split_kernel(const DecodeArgs a) {
   static_assert(D == 128 || D == 256, "decode attention supports head_dim 128 and 256");
   using C = DecCfg<D, P, GP>;
@@ -140,30 +140,41 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, (D == 128 && GP == 4) ? 4 :
   const int split = item % a.splits;
   uint8_t* ring = smem + warp * C::WARP_B;
 
-  // ---- sequence length and page range of this work item
+  // ---- independent loads first: the sequence length, the block-table
+  // entries of the split's page range and the query rows are fetched in one
+  // round trip (the entries past the sequence's end are never used)
+  const int hr = (GP == 8) ? r : (r & 3);
+  const bool lo_row = (GP == 4) && (r >= 4);
+  const int g = h * a.G + hr;           // global query head
+  const bool head_ok = hr < a.G;
   int L = a.seq_lens[s];
+  const int pbeg = split * a.pages_per_split;
+  int32_t* ids = reinterpret_cast<int32_t*>(ring + C::NST * C::STAGE_B);
+  {
+    int nload = a.bt_stride - pbeg;
+    nload = nload < a.pages_per_split ? nload : a.pages_per_split;
+    for (int c = lane; c < nload; c += kWarp) ids[c] = a.block_table[(int64_t)s * a.bt_stride + pbeg + c];
+  }
+  uint4 qraw[C::QW / 8];
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(a.q + ((int64_t)s * a.Hq + g) * D + j * C::QW);
+#pragma unroll
+    for (int c = 0; c < C::QW / 8; ++c) qraw[c] = head_ok ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+  }
+  // ---- page range of this work item
   bool len_ok = L >= 0 && L <= a.max_seq_len && (L + a.P - 1) / a.P <= a.bt_stride;
   if (!len_ok) {
     if (lane == 0 && h == 0 && split == 0) raise_flag(a.err, KVQ_ERRF_LEN);
     L = 0;
   }
   const int npages = (L + P - 1) / P;
-  const int pbeg = split * a.pages_per_split;
   int pend = pbeg + a.pages_per_split;
   if (pend > npages) pend = npages;
   const int nmine = pend > pbeg ? pend - pbeg : 0;
-
-  // block-table entries of the item's pages, loaded once (independent loads)
-  int32_t* ids = reinterpret_cast<int32_t*>(ring + C::NST * C::STAGE_B);
-  for (int c = lane; c < nmine; c += kWarp) ids[c] = a.block_table[(int64_t)s * a.bt_stride + pbeg + c];
   __syncwarp();
 
   // ---- query fragments: rows = [hi ; lo] of the GP heads of this KV head
   // lane (r, j) handles query head hr and channels [j*QW, (j+1)*QW)
-  const int hr = (GP == 8) ? r : (r & 3);
-  const bool lo_row = (GP == 4) && (r >= 4);
-  const int g = h * a.G + hr;           // global query head
-  const bool head_ok = hr < a.G;
   // ---- page ring: the warp stages each (page, head) chunk (K codes, V
   // codes, K params, V params, all contiguous in their pools) with 16-byte
   // cp.async copies, linear in shared memory: 16-byte unit u of a page block
@@ -274,10 +285,9 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, (D == 128 && GP == 4) ? 4 :
   {
     float x[C::QW];
     {
-      const uint4* src = reinterpret_cast<const uint4*>(a.q + ((int64_t)s * a.Hq + g) * D + j * C::QW);
 #pragma unroll
       for (int c = 0; c < C::QW / 8; ++c) {
-        const uint4 u = head_ok ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+        const uint4 u = qraw[c];
         const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -656,21 +666,20 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, (D == 128 && GP == 4) ? 4 :
   const bool owner = head_ok && !lo_row;
   // lanes of head hr: quarter j of the channels; for GP = 4 the partner
   // lanes r + 4 take the odd splits and the two halves are added at the end
-  const int sub = (GP == 4) ? own : 0, nsub = (GP == 4) ? 2 : 1;
-  float x[C::QW];
-#pragma unroll
-  for (int c = 0; c < C::QW; ++c) x[c] = 0.f;
-  float Ls = 0.f;
-  // lanes of a head without a query head (G < GP) load nothing; the
-  // shuffles below run in every lane and stay within one head's lanes
+  // Channels of the merge: GP = 4: lane (j, own) of a head takes
+  // j*QW + own*QW/2 + [0, QW/2) (the 8 lanes of a head cover it); GP = 8:
+  // lane j takes the quarter j*QW + [0, QW). Loads go out in rounds of RB
+  // splits, the first round together with the splits' maxima.
+  constexpr int CW = GP == 4 ? C::QW / 2 : C::QW;
+  constexpr int RB = CW <= 16 ? 4 : (CW <= 32 ? 2 : 1);  // float4 loads per lane per round <= 16
+  const int coff = j * C::QW + (GP == 4 ? own * (C::QW / 2) : 0);
   const float* src = a.part + ((int64_t)s * a.Hq + g) * a.splits * (D + 4);
+  const int nsp = head_ok ? a.splits : 0;
   double Mx = -INFINITY;
   {
-    // the splits' maxima: the NL lanes of the head load interleaved splits,
-    // four rounds at a time, then reduce
+    // the splits' maxima: the NL lanes of the head load interleaved splits
     constexpr int NL = GP == 4 ? 8 : 4;
     const int li0 = GP == 4 ? 4 * own + j : j;
-    const int nsp = head_ok ? a.splits : 0;
     for (int i0 = 0; i0 < nsp; i0 += 4 * NL) {
       double mv[4];
 #pragma unroll
@@ -682,37 +691,56 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, (D == 128 && GP == 4) ? 4 :
       Mx = fmax(Mx, fmax(fmax(mv[0], mv[1]), fmax(mv[2], mv[3])));
     }
   }
-  Mx = fmax(Mx, __shfl_xor_sync(0xffffffffu, Mx, 1));
-  Mx = fmax(Mx, __shfl_xor_sync(0xffffffffu, Mx, 2));
-  if (GP == 4) Mx = fmax(Mx, __shfl_xor_sync(0xffffffffu, Mx, 16));
-  if (head_ok) {
-    if (Mx != -INFINITY) {
-#pragma unroll 2
-      for (int i = sub; i < a.splits; i += nsub) {
-        const float* pi = src + (int64_t)i * (D + 4);
-        const double Mi = __ldcg(reinterpret_cast<const double*>(pi + D));
-        const float li = __ldcg(pi + D + 2);
-        const float4* v4 = reinterpret_cast<const float4*>(pi + j * C::QW);
-        float4 f[C::QW / 4];
+  float xm[CW];
 #pragma unroll
-        for (int c = 0; c < C::QW / 4; ++c) f[c] = __ldcg(v4 + c);
-        // an empty split (max -inf) has a zero row and a zero sum: weight 0
-        const float wgt = Mi == -INFINITY ? 0.f : fast_exp2((float)(Mi - Mx));
-        Ls += wgt * li;
+  for (int c = 0; c < CW; ++c) xm[c] = 0.f;
+  float Ls = 0.f;
+  for (int i0 = 0; i0 < (nsp > 0 ? nsp : 1); i0 += RB) {
+    float4 f[RB][CW / 4];
+    double Mi[RB];
+    float li[RB];
 #pragma unroll
-        for (int c = 0; c < C::QW / 4; ++c) {
-          x[4 * c] += wgt * f[c].x;
-          x[4 * c + 1] += wgt * f[c].y;
-          x[4 * c + 2] += wgt * f[c].z;
-          x[4 * c + 3] += wgt * f[c].w;
-        }
+    for (int rb = 0; rb < RB; ++rb) {
+      const int i = i0 + rb;
+      const float* pi = src + (int64_t)i * (D + 4);
+      const bool in = i < nsp;
+      Mi[rb] = in ? __ldcg(reinterpret_cast<const double*>(pi + D)) : -INFINITY;
+      li[rb] = in ? __ldcg(pi + D + 2) : 0.f;
+#pragma unroll
+      for (int c = 0; c < CW / 4; ++c)
+        f[rb][c] = in ? __ldcg(reinterpret_cast<const float4*>(pi + coff) + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    if (i0 == 0) {  // every lane of a head ends with the head's maximum
+      Mx = fmax(Mx, __shfl_xor_sync(0xffffffffu, Mx, 1));
+      Mx = fmax(Mx, __shfl_xor_sync(0xffffffffu, Mx, 2));
+      if (GP == 4) Mx = fmax(Mx, __shfl_xor_sync(0xffffffffu, Mx, 16));
+    }
+#pragma unroll
+    for (int rb = 0; rb < RB; ++rb) {
+      // an empty split (max -inf) has a zero row and a zero sum: weight 0
+      const float wgt = Mi[rb] == -INFINITY ? 0.f : fast_exp2((float)(Mi[rb] - Mx));
+      Ls += wgt * li[rb];
+#pragma unroll
+      for (int c = 0; c < CW / 4; ++c) {
+        xm[4 * c] += wgt * f[rb][c].x;
+        xm[4 * c + 1] += wgt * f[rb][c].y;
+        xm[4 * c + 2] += wgt * f[rb][c].z;
+        xm[4 * c + 3] += wgt * f[rb][c].w;
       }
     }
   }
+  // the whole quarter in every lane of the head (GP = 4: swap halves)
+  float x[C::QW];
   if (GP == 4) {
-    Ls += __shfl_xor_sync(0xffffffffu, Ls, 16);
 #pragma unroll
-    for (int c = 0; c < C::QW; ++c) x[c] += __shfl_xor_sync(0xffffffffu, x[c], 16);
+    for (int c = 0; c < CW; ++c) {
+      const float o = __shfl_xor_sync(0xffffffffu, xm[c], 16);
+      x[c] = own ? o : xm[c];
+      x[CW + c] = own ? xm[c] : o;
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < C::QW; ++c) x[c] = xm[c % CW];
   }
   {
     const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
