@@ -40,4 +40,12 @@ int decode_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, const void* q,
                   float* out, void* workspace, size_t workspace_bytes, int32_t* err,
                   cudaStream_t st);
 
+// Baseline decode attention over a binary16 paged cache.
+DecodePlan decode_fp16_plan(const kvq_cache_desc& d, int32_t S, int32_t Hq, int32_t max_seq_len);
+int decode_fp16_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, const void* q,
+                       const int32_t* seq_lens, int32_t max_seq_len, const int32_t* block_table,
+                       int32_t bt_stride, float sm_scale, const void* k_pages,
+                       const void* v_pages, float* out, void* workspace, size_t workspace_bytes,
+                       int32_t* err, cudaStream_t st);
+
 }  // namespace kvq

@@ -32,6 +32,9 @@ SIGNATURES = {
                                             _P, _P]),
     "kvq_paged_decode_attn_noalloc": (ctypes.c_int, [_P, _I32, _I32, _P, _P, _I32, _P, _I32, _F32,
                                                      _P, _P, _P, _P, _P, _P, _P]),
+    "kvq_decode_fp16_workspace_bytes": (_SZ, [_P, _I32, _I32, _I32]),
+    "kvq_paged_decode_attn_fp16": (ctypes.c_int, [_P, _I32, _I32, _P, _P, _I32, _P, _I32, _F32,
+                                                  _P, _P, _P, _P, _SZ, _P, _P]),
     "kvq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "kvq_version": (ctypes.c_char_p, []),
 }
@@ -154,6 +157,35 @@ def paged_decode_attn(cache, q, seq_lens, max_seq_len, block_table, k_codes, k_p
                                      _ptr(workspace), workspace.numel() * workspace.element_size(),
                                      _ptr(err), _stream(stream))
     _check("kvq_paged_decode_attn", st)
+    return out
+
+
+def decode_fp16_workspace_bytes(cache, num_seqs, num_q_heads, max_seq_len):
+    return int(lib().kvq_decode_fp16_workspace_bytes(ctypes.byref(cache.desc), num_seqs,
+                                                     num_q_heads, max_seq_len))
+
+
+def paged_decode_attn_fp16(cache, q, seq_lens, max_seq_len, block_table, k_pages, v_pages,
+                           out=None, workspace=None, sm_scale=None, err=None, stream=None):
+    """Full-precision baseline over a binary16 paged cache ``k_pages``,
+    ``v_pages`` (float16 CUDA [NP][H][P][d], unrotated); q float16 [S][Hq][d];
+    returns float32 [S][Hq][d]. Workspace as for ``paged_decode_attn``."""
+    S, Hq, d = q.shape
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((S, Hq, d), dtype=torch.float32, device=q.device)
+    need = decode_fp16_workspace_bytes(cache, S, Hq, max_seq_len)
+    if workspace is None:
+        workspace = torch.zeros(max(need, 16), dtype=torch.uint8, device=q.device)
+    st = lib().kvq_paged_decode_attn_fp16(ctypes.byref(cache.desc), S, Hq, _ptr(q),
+                                          _ptr(seq_lens), int(max_seq_len), _ptr(block_table),
+                                          int(block_table.shape[1]), float(sm_scale),
+                                          _ptr(k_pages), _ptr(v_pages), _ptr(out),
+                                          _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(),
+                                          _ptr(err), _stream(stream))
+    _check("kvq_paged_decode_attn_fp16", st)
     return out
 
 

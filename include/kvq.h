@@ -187,6 +187,36 @@ int kvq_dequantize_pages(const kvq_cache_desc* desc, int32_t num_seqs,
                          const void* params, int32_t unrotate, int32_t out_fp32, void* out,
                          int32_t* err_flags, void* stream);
 
+/*
+ * Full-precision baseline: decode attention over an UNQUANTIZED binary16
+ * paged cache, without rotation. The INT4 cache is measured against it (page
+ * "SAW-INT4: System-Aware 4-Bit KV-Cache Quantization for Real-World LLM
+ * Serving", Summary and Key takeaways: INT4 against full-precision KV caches).
+ *
+ *  k_pages, v_pages  device binary16 [num_pages][num_kv_heads][page_size]
+ *                    [head_dim], 16-byte aligned, filled by the caller with the
+ *                    plain K and V rows of each cached token.
+ *  desc              geometry as for the INT4 cache; rot_kind, rot_block and
+ *                    quat are ignored (nothing is rotated).
+ *  q, seq_lens, max_seq_len, block_table, bt_stride, sm_scale, out
+ *                    as for kvq_paged_decode_attn; out is float32 [S][Hq][d]
+ *                    = softmax(sm_scale q K^T) V per query head.
+ *  workspace         >= kvq_decode_fp16_workspace_bytes(...) bytes, 16-byte
+ *                    aligned, zero-filled before its first use (the counters
+ *                    are left at zero by every call).
+ * Supported: head_dim 128 with page_size 16, 32 or 64 and GQA group <= 8;
+ * head_dim 256 with page_size 16 or 32 and group <= 4 (else
+ * KVQ_ERR_UNSUPPORTED). Errors and flags as for kvq_paged_decode_attn.
+ */
+size_t kvq_decode_fp16_workspace_bytes(const kvq_cache_desc* desc, int32_t num_seqs,
+                                       int32_t num_q_heads, int32_t max_seq_len);
+int kvq_paged_decode_attn_fp16(const kvq_cache_desc* desc, int32_t num_seqs,
+                               int32_t num_q_heads, const void* q, const int32_t* seq_lens,
+                               int32_t max_seq_len, const int32_t* block_table,
+                               int32_t bt_stride, float sm_scale, const void* k_pages,
+                               const void* v_pages, float* out, void* workspace,
+                               size_t workspace_bytes, int32_t* err_flags, void* stream);
+
 /* Size of the fixed scratch array behind kvq_paged_decode_attn_noalloc. */
 #define KVQ_NOALLOC_SCRATCH_BYTES (16u << 20)
 
