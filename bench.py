@@ -54,6 +54,10 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
+    ap.add_argument("--compare", action="store_true",
+                    help="print one JSON line with the baseline comparisons (long-context INT4 with "
+                         "and without rotation vs the binary16 cache; prefill append per Hadamard "
+                         "block with reconstruction MSE) and exit")
     ap.add_argument("--profile-case", choices=["append", "decode"], default=None,
                     help="run a short fixed case for an ncu capture (4 launches) and exit")
     return ap.parse_args()
@@ -454,8 +458,114 @@ def profile_case(which):
     print(f"profile case {which} done")
 
 
+def _device_time_us(fn, n=20):
+    """Median over 5 rounds of n back-to-back launches, CUDA events, in us."""
+    for i in range(3):
+        fn(i)
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(5):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(n):
+            fn(i)
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1) / n)
+    return float(np.median(ts)) * 1e3
+
+
+def compare():
+    """Baselines on one GPU: the long-context 70B-shaped decode (8 x 32768
+    tokens, GQA 8, page 32) over INT4 pages with Hadamard b 128, over INT4
+    pages without rotation, and over binary16 pages; then the bulk prefill
+    append of one layer (65536 tokens x 8 heads) per Hadamard block size with
+    the reconstruction MSE of the INT4 cache (GPU dequantization, un-rotated,
+    against the fp16 input). Two replicas of every cache alternate (> L2)."""
+    from bit_rotated_kv_block_b200 import kvq, workloads
+    torch.cuda.set_device(0)
+    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
+    res = {"workload_decode": "8 seqs x 32768 tokens, 8 KV heads, 64 q heads, d 128, page 32",
+           "workload_append": "65536 tokens x 8 KV heads x d 128 per layer, page 16"}
+    peak, _ = measured_peaks()
+    w = workloads.long70b()
+    k, v, ts, tp = w.prefill_tokens()
+    K, V, TS, TP, BT = dev(k), dev(v), dev(ts), dev(tp), dev(w.block_table)
+    q, lens, L = dev(w.queries()), dev(w.seq_lens), int(w.seq_lens.max())
+    out = torch.empty((w.S, w.Hq, w.d), dtype=torch.float32, device="cuda")
+    n_th = int(w.seq_lens.sum()) * w.H
+    for rot, blk in ((workloads.ROT_HADAMARD, 128), (workloads.ROT_NONE, 0)):
+        reps = []
+        for _ in range(2):
+            c = kvq.Cache(w.d, w.H, w.P, w.NP, rot, blk)
+            kc, kp = c.new_pools(fill=0)
+            vc, vp = c.new_pools(fill=0)
+            kvq.quantize_append(c, K, V, TS, TP, BT, kc, kp, vc, vp)
+            reps.append((c, kc, kp, vc, vp))
+        ws = torch.zeros(kvq.decode_workspace_bytes(reps[0][0], w.S, w.Hq, L), dtype=torch.uint8,
+                         device="cuda")
+        t = _device_time_us(lambda i: kvq.paged_decode_attn(
+            reps[i % 2][0], q, lens, L, BT, *reps[i % 2][1:], out=out, workspace=ws))
+        gbs = n_th * 136 / t / 1e3
+        res["decode_int4_" + ("hadamard128" if blk else "no_rotation")] = {
+            "us": t, "gbs": gbs, "frac": gbs / peak, "bytes": n_th * 136}
+        del reps, ws
+    page = BT[TS.long(), (TP // w.P).long()].long()
+    slot = (TP % w.P).long()
+    reps = []
+    for _ in range(2):
+        kp16 = torch.zeros((w.NP, w.H, w.P, w.d), dtype=torch.float16, device="cuda")
+        vp16 = torch.zeros_like(kp16)
+        kp16[page, :, slot, :] = K
+        vp16[page, :, slot, :] = V
+        reps.append((kp16, vp16))
+    c16 = kvq.Cache(w.d, w.H, w.P, w.NP, workloads.ROT_NONE, 0)
+    ws = torch.zeros(kvq.decode_fp16_workspace_bytes(c16, w.S, w.Hq, L), dtype=torch.uint8,
+                     device="cuda")
+    t = _device_time_us(lambda i: kvq.paged_decode_attn_fp16(
+        c16, q, lens, L, BT, reps[i % 2][0], reps[i % 2][1], out=out, workspace=ws))
+    gbs = n_th * 512 / t / 1e3
+    res["decode_fp16_baseline"] = {"us": t, "gbs": gbs, "frac": gbs / peak, "bytes": n_th * 512}
+    res["rotation_overhead_decode"] = (res["decode_int4_hadamard128"]["us"] /
+                                       res["decode_int4_no_rotation"]["us"] - 1)
+    del reps, ws, K, V, page, slot
+    torch.cuda.empty_cache()
+
+    sweep = {}
+    for blk in (16, 32, 64, 128, 0):
+        w = workloads.prefill(rot_block=blk)
+        k, v, ts, tp = w.prefill_tokens()
+        K, V, TS, TP, BT = dev(k), dev(v), dev(ts), dev(tp), dev(w.block_table)
+        c = kvq.Cache(w.d, w.H, w.P, w.NP, w.rot_kind, w.rot_block)
+        kc, kp = c.new_pools(fill=0)
+        vc, vp = c.new_pools(fill=0)
+        t = _device_time_us(lambda i: kvq.quantize_append(c, K, V, TS, TP, BT, kc, kp, vc, vp),
+                            n=10)
+        byts = len(ts) * w.H * APPEND_BYTES_PER_TOKEN_HEAD
+        lens = dev(np.full(w.S, int(w.seq_lens[0]), np.int32))
+        Lmax = int(w.seq_lens[0])
+        mse = 0.0
+        for codes, params, src in ((kc, kp, K), (vc, vp, V)):
+            xh = kvq.dequantize_pages(c, lens, Lmax, BT, codes, params, unrotate=True)
+            x = src.view(w.S, Lmax, w.H, w.d).double()
+            mse += float(((xh.double() - x) ** 2).mean()) / 2
+            del xh, x
+        sweep["hadamard%d" % blk if blk else "no_rotation"] = {
+            "us": t, "gbs": byts / t / 1e3, "frac": byts / t / 1e3 / peak, "mse": mse}
+        del K, V, kc, kp, vc, vp
+        torch.cuda.empty_cache()
+    res["append_prefill_sweep"] = sweep
+    res["rotation_overhead_append_b128"] = sweep["hadamard128"]["us"] / sweep["no_rotation"]["us"] - 1
+    res["peak_gbs"] = peak
+    print(json.dumps({"mode": "compare", **res}), flush=True)
+
+
 def main():
     args = parse()
+    if args.compare:
+        compare()
+        return
     if args.profile_case:
         profile_case(args.profile_case)
         return
