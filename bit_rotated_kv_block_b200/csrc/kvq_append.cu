@@ -287,6 +287,193 @@ __global__ void __launch_bounds__(kAppendThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Small batches (a decode step appends one token per sequence): one row of
+// K or V per 32 lanes (16 for d = 64), each lane owning CPL = max(4, d/32)
+// consecutive channels. The same arithmetic as append_kernel in the same
+// order: butterfly stages below CPL in registers, the wider ones across
+// lanes (the lower-channel lane adds, the upper one subtracts the lower
+// element minus its own), then the scale, the statistics, the parameters
+// and the codes. Latency rather than bandwidth decides these launches: the
+// work of a row is spread over a warp instead of one thread.
+// ---------------------------------------------------------------------------
+
+struct AppendRowsArgs {
+  int T, H, P, lg_page, NP, num_seqs, bt_stride;
+  int64_t tok_stride;
+  const __half* k;
+  const __half* v;
+  const int32_t* token_seq;
+  const int32_t* token_pos;
+  const int32_t* block_table;
+  uint8_t* k_codes;
+  uint8_t* v_codes;
+  uint32_t* k_params;
+  uint32_t* v_params;
+  const float* quat;
+  int32_t* err;
+};
+
+constexpr int kRowsWarps = 4;
+
+template <int D, int ROT, int LGB>
+__global__ void __launch_bounds__(kRowsWarps * kWarp) append_rows_kernel(const AppendRowsArgs a) {
+  constexpr int CPL = D / 32 < 4 ? 4 : D / 32;  // channels per lane
+  constexpr int LPR = D / CPL;                  // lanes per row (16 or 32)
+  constexpr int RPW = kWarp / LPR;              // rows per warp
+  constexpr int B = 1 << LGB;
+  const int lane = threadIdx.x % kWarp;
+  const int rl = lane % LPR;
+  const int row = (blockIdx.x * kRowsWarps + threadIdx.x / kWarp) * RPW + lane / LPR;
+  const int nrows = a.T * a.H * 2;
+  const bool active = row < nrows;
+  // row = ((t * H) + h) * 2 + kv
+  const int kv = row & 1;
+  const int h = (row >> 1) % a.H;
+  const int t = active ? (row >> 1) / a.H : 0;
+
+  // destination first: its dependent loads (token -> sequence and position
+  // -> block-table entry) overlap the arithmetic below
+  const int seq = active ? a.token_seq[t] : -1;
+  const int pos = active ? a.token_pos[t] : 0;
+  const bool seq_ok = seq >= 0 && seq < a.num_seqs;
+  const bool pos_ok = pos >= 0 && (pos >> a.lg_page) < a.bt_stride;
+  const int page = (seq_ok && pos_ok) ? a.block_table[(int64_t)seq * a.bt_stride + (pos >> a.lg_page)] : -1;
+
+  float x[CPL];
+  {
+    const __half* src = (kv ? a.v : a.k) + (int64_t)t * a.tok_stride + (int64_t)h * D + rl * CPL;
+    if (CPL == 4) {
+      const uint2 u = active ? *reinterpret_cast<const uint2*>(src) : make_uint2(0u, 0u);
+      const float2 f0 = __half22float2(u32_as_h2(u.x)), f1 = __half22float2(u32_as_h2(u.y));
+      x[0] = f0.x; x[1] = f0.y; x[2] = f1.x; x[3] = f1.y;
+    } else {
+#pragma unroll
+      for (int c = 0; c < CPL / 8; ++c) {
+        const uint4 u = active ? reinterpret_cast<const uint4*>(src)[c] : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __half22float2(u32_as_h2(w4[e]));
+          x[8 * c + 2 * e] = f.x;
+          x[8 * c + 2 * e + 1] = f.y;
+        }
+      }
+    }
+  }
+
+  if (ROT == KVQ_ROT_HADAMARD) {
+    // stages h = 1, 2, 4, ... < B in ascending order
+#pragma unroll
+    for (int dd = 1; dd < CPL && dd < B; dd <<= 1) {
+#pragma unroll
+      for (int i = 0; i < CPL; ++i) {
+        if ((i & dd) == 0) {
+          const float p = x[i], q = x[i + dd];
+          x[i] = __fadd_rn(p, q);
+          x[i + dd] = __fsub_rn(p, q);
+        }
+      }
+    }
+#pragma unroll
+    for (int m = 1; m * CPL < B; m <<= 1) {
+      const bool lower = (rl & m) == 0;
+#pragma unroll
+      for (int i = 0; i < CPL; ++i) {
+        const float o = __shfl_xor_sync(0xffffffffu, x[i], m);
+        x[i] = lower ? __fadd_rn(x[i], o) : __fsub_rn(o, x[i]);
+      }
+    }
+    const float cb = hadamard_scale(LGB);
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) x[i] = __fmul_rn(x[i], cb);
+  } else if (ROT == KVQ_ROT_QUAT) {
+    quat_regs<CPL>(x, a.quat, rl * CPL);
+  }
+
+  // row statistics over the LPR lanes of the row
+  float mn = x[0], mx = x[0];
+#pragma unroll
+  for (int i = 1; i < CPL; ++i) {
+    mn = fminf(mn, x[i]);
+    mx = fmaxf(mx, x[i]);
+  }
+#pragma unroll
+  for (int m = 1; m < LPR; m <<= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, m));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
+  }
+  mn = __fadd_rn(mn, 0.0f);
+  mx = __fadd_rn(mx, 0.0f);
+  const __half m16 = __float2half_rd(mn);
+  const float m = __half2float(m16);
+  const float s32 = __fdiv_ru(__fsub_ru(mx, m), 15.0f);
+  const __half s16 = __float2half_ru(s32);
+  const float s = __half2float(s16);
+  uint32_t packed = 0;
+  if (s != 0.0f) {
+    const float inv = __frcp_rn(s);
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) {
+      // nearest integer (ties to even) of the exact product: one fused
+      // multiply-add with 1.5 * 2^23 leaves it in the low mantissa bits
+      const uint32_t c = __float_as_uint(__fmaf_rn(__fsub_rn(x[i], m), inv, 12582912.0f)) & 0xFu;
+      packed |= c << (4 * i);
+    }
+  }
+
+  if (!active || seq < 0) return;
+  const bool lead = kv == 0 && h == 0 && rl == 0;
+  if (!seq_ok) {
+    if (lead) raise_flag(a.err, KVQ_ERRF_SEQ);
+    return;
+  }
+  if (!pos_ok) {
+    if (lead) raise_flag(a.err, KVQ_ERRF_POS);
+    return;
+  }
+  if (page < 0 || page >= a.NP) {
+    if (lead) raise_flag(a.err, KVQ_ERRF_PAGE);
+    return;
+  }
+  const int64_t dst = (((int64_t)page * a.H + h) << a.lg_page) + (pos & ((1 << a.lg_page) - 1));
+  uint8_t* codes = (kv ? a.v_codes : a.k_codes) + dst * (D / 2) + rl * (CPL / 2);
+  if (CPL == 4)
+    *reinterpret_cast<uint16_t*>(codes) = (uint16_t)packed;
+  else
+    *reinterpret_cast<uint32_t*>(codes) = packed;
+  if (rl == 0)
+    (kv ? a.v_params : a.k_params)[dst] =
+        (uint32_t)__half_as_ushort(s16) | ((uint32_t)__half_as_ushort(m16) << 16);
+}
+
+template <int D, int ROT, int LGB>
+static cudaError_t launch_rows(const AppendRowsArgs& a, cudaStream_t st) {
+  constexpr int CPL = D / 32 < 4 ? 4 : D / 32;
+  constexpr int RPW = kWarp / (D / CPL);
+  const int warps = (a.T * a.H * 2 + RPW - 1) / RPW;
+  append_rows_kernel<D, ROT, LGB><<<(warps + kRowsWarps - 1) / kRowsWarps, kRowsWarps * kWarp, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t dispatch_rows(const AppendRowsArgs& a, int rot, int lgb, cudaStream_t st) {
+  if (rot == KVQ_ROT_NONE) return launch_rows<D, KVQ_ROT_NONE, 0>(a, st);
+  if (rot == KVQ_ROT_QUAT) return launch_rows<D, KVQ_ROT_QUAT, 0>(a, st);
+  switch (lgb) {
+    case 4: return launch_rows<D, KVQ_ROT_HADAMARD, 4>(a, st);
+    case 5: return launch_rows<D, KVQ_ROT_HADAMARD, 5>(a, st);
+    case 6: return launch_rows<D, KVQ_ROT_HADAMARD, 6>(a, st);
+    case 7:
+      if (D >= 128) return launch_rows<D, KVQ_ROT_HADAMARD, (D >= 128 ? 7 : 6)>(a, st);
+      break;
+    case 8:
+      if (D >= 256) return launch_rows<D, KVQ_ROT_HADAMARD, (D >= 256 ? 8 : 6)>(a, st);
+      break;
+  }
+  return cudaErrorInvalidValue;
+}
+
 // Driver entry point for tensor-map encoding (no link-time libcuda needed).
 static PFN_cuTensorMapEncodeTiled encode_fn() {
   static PFN_cuTensorMapEncodeTiled fn = nullptr;
@@ -363,6 +550,31 @@ int append_launch(const kvq_cache_desc& d, int32_t T, const void* k, const void*
   if (tok_max < 1 || d.num_kv_heads > 256) return KVQ_ERR_UNSUPPORTED;
   const int sms = device_sm_count();
   if (sms <= 0) return KVQ_ERR_CUDA;
+  int lgb = 0;
+  while ((1 << lgb) < d.rot_block) ++lgb;
+  // small batches (up to 8192 rows of K and V): a warp per row
+  if ((int64_t)T * d.num_kv_heads * 2 <= 8192) {
+    AppendRowsArgs r;
+    r.T = T; r.H = d.num_kv_heads; r.P = d.page_size;
+    r.lg_page = 0;
+    while ((1 << r.lg_page) < d.page_size) ++r.lg_page;
+    r.NP = d.num_pages; r.num_seqs = num_seqs; r.bt_stride = bt_stride;
+    r.tok_stride = tok_stride;
+    r.k = static_cast<const __half*>(k); r.v = static_cast<const __half*>(v);
+    r.token_seq = token_seq; r.token_pos = token_pos; r.block_table = block_table;
+    r.k_codes = k_codes; r.v_codes = v_codes;
+    r.k_params = static_cast<uint32_t*>(k_params); r.v_params = static_cast<uint32_t*>(v_params);
+    r.quat = d.quat; r.err = err;
+    cudaError_t e;
+    switch (D) {
+      case 64: e = dispatch_rows<64>(r, d.rot_kind, lgb, st); break;
+      case 128: e = dispatch_rows<128>(r, d.rot_kind, lgb, st); break;
+      case 256: e = dispatch_rows<256>(r, d.rot_kind, lgb, st); break;
+      default: return KVQ_ERR_UNSUPPORTED;
+    }
+    if (e == cudaErrorInvalidValue) return KVQ_ERR_UNSUPPORTED;
+    return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+  }
   // small batches: fewer tokens per tile so more SMs share the work
   int tok = (T + sms - 1) / sms;
   if (tok > tok_max) tok = tok_max;
@@ -393,8 +605,6 @@ int append_launch(const kvq_cache_desc& d, int32_t T, const void* k, const void*
       !encode_rows(&tv, v, D, a.H, T, tok_stride, tok))
     return KVQ_ERR_CUDA;
   const int grid = a.num_tiles < sms ? a.num_tiles : sms;
-  int lgb = 0;
-  while ((1 << lgb) < d.rot_block) ++lgb;
   cudaError_t e;
   switch (D) {
     case 64: e = dispatch_rot<64>(a, tk, tv, d.rot_kind, lgb, grid, st); break;
