@@ -59,7 +59,7 @@ struct DecodeArgs {
   const uint32_t* v_params;
   float* out;        // [S][Hq][D]
   float* part;       // [S][Hq][splits][D + 4]: acc[D], max (double), sum, pad
-  int32_t* counter;  // [S][H], zero between calls
+  int32_t* counter;  // [S][H] split arrivals, zero between calls
   int32_t* err;
 };
 
@@ -148,30 +148,25 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, (D == 128 && GP == 4) ? 4 :
   const int g = h * a.G + hr;           // global query head
   const bool head_ok = hr < a.G;
   int L = a.seq_lens[s];
-  const int pbeg = split * a.pages_per_split;
-  int32_t* ids = reinterpret_cast<int32_t*>(ring + C::NST * C::STAGE_B);
-  {
-    int nload = a.bt_stride - pbeg;
-    nload = nload < a.pages_per_split ? nload : a.pages_per_split;
-    for (int c = lane; c < nload; c += kWarp) ids[c] = a.block_table[(int64_t)s * a.bt_stride + pbeg + c];
-  }
   uint4 qraw[C::QW / 8];
   {
     const uint4* src = reinterpret_cast<const uint4*>(a.q + ((int64_t)s * a.Hq + g) * D + j * C::QW);
 #pragma unroll
     for (int c = 0; c < C::QW / 8; ++c) qraw[c] = head_ok ? src[c] : make_uint4(0u, 0u, 0u, 0u);
   }
-  // ---- page range of this work item
   bool len_ok = L >= 0 && L <= a.max_seq_len && (L + a.P - 1) / a.P <= a.bt_stride;
   if (!len_ok) {
     if (lane == 0 && h == 0 && split == 0) raise_flag(a.err, KVQ_ERRF_LEN);
     L = 0;
   }
   const int npages = (L + P - 1) / P;
-  int pend = pbeg + a.pages_per_split;
-  if (pend > npages) pend = npages;
-  const int nmine = pend > pbeg ? pend - pbeg : 0;
-  __syncwarp();
+  const int ngrp = (npages + C::PG - 1) / C::PG;  // stage groups of the (sequence, KV head)
+  const int32_t* const bt_row = a.block_table + (int64_t)s * a.bt_stride;
+  // block-table entry of page q (lane q < PG) of group gi; -1: no such page
+  auto group_ids = [&](int gi) {
+    const int pi = gi * C::PG + lane;
+    return (lane < C::PG && gi < ngrp && pi < npages) ? bt_row[pi] : -1;
+  };
 
   // ---- query fragments: rows = [hi ; lo] of the GP heads of this KV head
   // lane (r, j) handles query head hr and channels [j*QW, (j+1)*QW)
@@ -188,22 +183,21 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, (D == 128 && GP == 4) ? 4 :
   const uint8_t* const par_l =
       lane < PU ? reinterpret_cast<const uint8_t*>(a.k_params) + (int64_t)h * P * 4 + lane * 16
                 : reinterpret_cast<const uint8_t*>(a.v_params) + (int64_t)h * P * 4 + (lane - PU) * 16;
-  const int ngrp = (nmine + C::PG - 1) / C::PG;
-  auto page_valid = [&](int pi) {
-    if (pi >= nmine) return false;
-    const int pg = ids[pi];
-    return pg >= 0 && pg < a.NP;
-  };
-  // stage the pages of group gi (pages gi*PG .. gi*PG + PG - 1 of the item)
-  // into stage sidx; pages outside the pool or the item are not copied
-  // (their tokens are masked)
-  auto issue = [&](int gi, int sidx) {
-    if (gi < ngrp) {
+  // The (sequence, KV head)'s page groups are dealt out to its `splits`
+  // warps in turn: warp `split` takes groups split, split + splits, ... (a
+  // short sequence still keeps every warp of the pair busy). Each group's
+  // block-table entries are loaded one step before its copies are issued.
+  int32_t* const meta = reinterpret_cast<int32_t*>(ring + C::NST * C::STAGE_B);  // [stage][4]
+  // copy group gi (page ids in lanes q < PG) into stage sidx and record it
+  auto issue = [&](int gi, int idl, int sidx) {
+    const bool any = gi < ngrp;
+    if (lane == 0) meta[sidx * 4] = any ? gi : -1;
+    if (lane < C::PG) meta[sidx * 4 + 1 + lane] = idl;
+    if (any) {
 #pragma unroll
       for (int q = 0; q < C::PG; ++q) {
-        const int pi = gi * C::PG + q;
-        if (!page_valid(pi)) continue;
-        const int64_t page = ids[pi];
+        const int64_t page = __shfl_sync(0xffffffffu, idl, q);
+        if (page < 0 || page >= a.NP) continue;  // beyond the sequence or out of the pool
         const int64_t co = page * cstride;
         uint8_t* dst = ring + sidx * C::STAGE_B + q * C::PAGE_B + lane * 16;
 #pragma unroll
@@ -268,8 +262,15 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, (D == 128 && GP == 4) ? 4 :
   // GP = 4: lanes r and r + 4 share head r % 4 and split those slots,
   // {0, 1} for r < 4 and {2, 3} for r >= 4
 
+  // groups split + k * splits (k < NST): the first NST - 1 are copied now,
+  // the last waits in the "entries loaded" slot of the pipeline
+  int idk[C::NST];
 #pragma unroll
-  for (int i = 0; i < C::NST - 1; ++i) issue(i, i);
+  for (int k = 0; k < C::NST; ++k) idk[k] = group_ids(split + k * a.splits);
+#pragma unroll
+  for (int k = 0; k < C::NST - 1; ++k) issue(split + k * a.splits, idk[k], k);
+  int gB = split + (C::NST - 1) * a.splits;  // group whose entries are loaded
+  int idB = idk[C::NST - 1];
 
   // the first pages are in flight while the query is prepared
   // The query as a 30-bit fixed point qint = qhat * 2^30 / amax (amax = the
@@ -353,25 +354,30 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, (D == 128 && GP == 4) ? 4 :
   }
 
 
-  int sidx = 0;             // stage of group gi
-  int sissue = C::NST - 1;  // stage of group gi + NST - 1
-  for (int gi = 0; gi < ngrp; ++gi) {
-    issue(gi + C::NST - 1, sissue);
+  int sidx = 0;             // stage consumed this step
+  int sissue = C::NST - 1;  // stage refilled this step
+  for (;;) {
+    issue(gB, idB, sissue);
     sissue = sissue + 1 == C::NST ? 0 : sissue + 1;
-    bool pgok[C::PG];  // page q of the group is in the item and in the pool
+    gB += a.splits;
+    idB = group_ids(gB);
+    cp_async_wait<C::NST - 1>();  // this lane's copies of the stage have landed
+    __syncwarp();                 // ... and every other lane's, and the stage's record
+    const int gi = meta[sidx * 4];
+    if (gi < 0) break;            // no group left for this warp
+    bool pgok[C::PG];             // page q of the group is cached and in the pool
     bool all_ok = true;
 #pragma unroll
     for (int q = 0; q < C::PG; ++q) {
-      const int pi = gi * C::PG + q;
-      pgok[q] = page_valid(pi);
+      const int pid = meta[sidx * 4 + 1 + q];
+      const bool cached = gi * C::PG + q < npages;
+      pgok[q] = cached && pid >= 0 && pid < a.NP;
       all_ok = all_ok && pgok[q];
-      if (pi < nmine && !pgok[q] && lane == 0) raise_flag(a.err, KVQ_ERRF_PAGE);
+      if (cached && !pgok[q] && lane == 0) raise_flag(a.err, KVQ_ERRF_PAGE);
     }
-    cp_async_wait<C::NST - 1>();  // this lane's copies of group gi have landed
-    __syncwarp();                 // ... and every other lane's
     const uint8_t* st = ring + sidx * C::STAGE_B;
     sidx = sidx + 1 == C::NST ? 0 : sidx + 1;
-    const int tok0 = (pbeg + gi * C::PG) * P;  // first token of the group
+    const int tok0 = gi * C::PG * P;  // first token of the group
     // groups whose every token is cached skip all per-token masking
     const bool full = all_ok && tok0 + C::PG * P <= L;
 
