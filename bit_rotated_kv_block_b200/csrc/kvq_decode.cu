@@ -43,10 +43,9 @@
 namespace kvq {
 
 constexpr int kDecWarps = 4;
-constexpr int kMaxPagesPerSplit = 256;  // page ids of one work item live in shared memory
 
 struct DecodeArgs {
-  int S, Hq, H, G, P, NP, bt_stride, max_seq_len, splits, pages_per_split;
+  int S, Hq, H, G, P, NP, bt_stride, max_seq_len, splits;
   int rot_kind, lgb;
   double scale2;  // sm_scale * log2(e), in double
   const __half* q;  // [S][Hq][D]
@@ -83,8 +82,8 @@ struct DecCfg {
   static constexpr int STAGE_B = PG * PAGE_B;
   // pipeline depth: about 8-13 KB of pages in flight per warp
   static constexpr int NST = STAGE_B <= 2304 ? 4 : (STAGE_B <= 4608 ? 3 : 2);
-  static constexpr int IDS_B = kMaxPagesPerSplit * 4;
-  static constexpr int WARP_B = (NST * STAGE_B + IDS_B + 127) / 128 * 128;
+  static constexpr int META_B = NST * 16;  // per stage: group index and page ids
+  static constexpr int WARP_B = (NST * STAGE_B + META_B + 127) / 128 * 128;
 };
 
 // Rotation of a query (or output) row held as quarters: lane j of a group
@@ -812,7 +811,10 @@ DecodePlan decode_plan(const kvq_cache_desc& d, int32_t S, int32_t Hq, int32_t m
   const int target = resident_warps(d.head_dim, P, GP);
   const int pairs = S * d.num_kv_heads;
   int splits = target / (pairs > 0 ? pairs : 1);
-  const int min_splits = (pl.pages_max + kMaxPagesPerSplit - 1) / kMaxPagesPerSplit;
+  // long contexts get at least one split per 256 pages: with lengths that
+  // vary across the batch this puts more warps on the long sequences' pairs
+  // (short pairs' warps leave the GPU early and the next CTAs take their place)
+  const int min_splits = (pl.pages_max + 255) / 256;
   if (splits < min_splits) splits = min_splits;
   if (splits < 1) splits = 1;
   if (splits > pl.pages_max) splits = pl.pages_max;
@@ -862,7 +864,6 @@ int decode_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, const void* q,
   DecodeArgs a;
   a.S = S; a.Hq = Hq; a.H = d.num_kv_heads; a.G = G; a.P = d.page_size; a.NP = d.num_pages;
   a.bt_stride = bt_stride; a.max_seq_len = max_seq_len; a.splits = pl.splits;
-  a.pages_per_split = pl.pages_per_split;
   a.rot_kind = d.rot_kind; a.lgb = lgb;
   a.scale2 = (double)sm_scale * 1.4426950408889634074;
   a.q = static_cast<const __half*>(q); a.quat = d.quat;

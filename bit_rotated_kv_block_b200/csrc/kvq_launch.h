@@ -28,7 +28,7 @@ int dequant_launch(const kvq_cache_desc& d, int32_t S, const int32_t* seq_lens,
 struct DecodePlan {
   int pages_max;        // ceil(max_seq_len / P)
   int splits;           // work items per (sequence, KV head)
-  int pages_per_split;  // pages one work item walks
+  int pages_per_split;  // pages per split (contiguous ranges; an even share for interleaved groups)
   size_t workspace;     // bytes of partial results
 };
 DecodePlan decode_plan(const kvq_cache_desc& d, int32_t S, int32_t Hq, int32_t max_seq_len);
