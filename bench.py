@@ -4,7 +4,8 @@ One step = one pass of the whole path over one batch of the Llama-3-8B-shaped
 decode layer (32 sequences x 4096 cached tokens, 8 KV heads, 32 query heads,
 head_dim 128, Hadamard block 64, page 16, shuffled block table): append one
 new token per sequence (fused rotate -> INT4 -> pack -> page scatter), then
-paged decode attention over the 4097 cached INT4 tokens. Inputs are seeded
+paged decode attention over the 4097 cached INT4 tokens -- both in one
+kvq_decode_step launch. Inputs are seeded
 synthetic draws of that shape (no dataset exists for this).
 
 The device-timed region covers exactly --steps steps between a barrier and a
@@ -228,12 +229,11 @@ def run_ours(args, world, rank, local):
     ws = torch.zeros(kvq.decode_workspace_bytes(c0, S, Hq, L), dtype=torch.uint8, device=device)
     err = torch.zeros(1, dtype=torch.int32, device=device)
     stream = torch.cuda.current_stream()
-    launches_per_step = 2  # one append kernel + one decode kernel
+    launches_per_step = 1  # kvq_decode_step: new-token append and attention in one kernel
 
     def step(i):
         c, kc, kp, vc, vp = caches[i % 2]
-        kvq.quantize_append(c, SK, SV, STS, STP, BT, kc, kp, vc, vp, err=err)
-        kvq.paged_decode_attn(c, Q, LENS, L, BT, kc, kp, vc, vp, out=out, workspace=ws, err=err)
+        kvq.decode_step(c, Q, SK, SV, LENS, L, BT, kc, kp, vc, vp, out=out, workspace=ws, err=err)
 
     for i in range(args.warmup):
         step(i)
@@ -251,9 +251,8 @@ def run_ours(args, world, rank, local):
     t0.record(stream)
     for i in range(steps):
         c, kc, kp, vc, vp = caches[i % 2]
-        kvq.quantize_append(c, SK, SV, STS, STP, BT, kc, kp, vc, vp, err=err)
         dec0[i].record(stream)
-        kvq.paged_decode_attn(c, Q, LENS, L, BT, kc, kp, vc, vp, out=out, workspace=ws, err=err)
+        kvq.decode_step(c, Q, SK, SV, LENS, L, BT, kc, kp, vc, vp, out=out, workspace=ws, err=err)
         dec1[i].record(stream)
     t1.record(stream)
     torch.cuda.synchronize()
@@ -289,8 +288,7 @@ def run_ours(args, world, rank, local):
     def e2e_step(i):
         c, kc, kp, vc, vp = caches[i % 2]
         din.copy_(hin, non_blocking=True)
-        kvq.quantize_append(c, SK, SV, STS, STP, BT, kc, kp, vc, vp, err=err)
-        kvq.paged_decode_attn(c, Q, LENS, L, BT, kc, kp, vc, vp, out=out, workspace=ws, err=err)
+        kvq.decode_step(c, Q, SK, SV, LENS, L, BT, kc, kp, vc, vp, out=out, workspace=ws, err=err)
         hout.copy_(out, non_blocking=True)
 
     for i in range(3):

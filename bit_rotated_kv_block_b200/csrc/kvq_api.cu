@@ -118,6 +118,36 @@ int kvq_paged_decode_attn(const kvq_cache_desc* desc, int32_t num_seqs, int32_t 
                        workspace_bytes, err_flags, static_cast<cudaStream_t>(stream));
 }
 
+int kvq_decode_step(const kvq_cache_desc* desc, int32_t num_seqs, int32_t num_q_heads,
+                    const void* q, const void* k_new, const void* v_new, int64_t new_stride,
+                    const int32_t* seq_lens, int32_t max_seq_len, const int32_t* block_table,
+                    int32_t bt_stride, float sm_scale, uint8_t* k_codes, void* k_params,
+                    uint8_t* v_codes, void* v_params, float* out, void* workspace,
+                    size_t workspace_bytes, int32_t* err_flags, void* stream) {
+  int st = check_desc(desc);
+  if (st != KVQ_OK) return st;
+  if (num_seqs < 1 || num_q_heads < 1 || max_seq_len < 0 || bt_stride < 1 ||
+      !std::isfinite(sm_scale))
+    return KVQ_ERR_INVALID_ARG;
+  if (num_q_heads % desc->num_kv_heads != 0) return KVQ_ERR_INVALID_ARG;
+  const int G = num_q_heads / desc->num_kv_heads;
+  if (desc->head_dim == 64 || G > 8 || (desc->head_dim == 256 && G > 4)) return KVQ_ERR_UNSUPPORTED;
+  if (!q || !k_new || !v_new || !seq_lens || !block_table || !k_codes || !k_params || !v_codes ||
+      !v_params || !out)
+    return KVQ_ERR_INVALID_ARG;
+  if (new_stride < (int64_t)desc->num_kv_heads * desc->head_dim) return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(k_new) || !aligned16(v_new) ||
+      new_stride % 8 != 0 || !aligned16(k_codes) || !aligned16(v_codes) || !aligned16(k_params) ||
+      !aligned16(v_params) || !aligned4(seq_lens) || !aligned4(block_table) ||
+      (err_flags && !aligned4(err_flags)))
+    return KVQ_ERR_MISALIGNED;
+  if (workspace && !aligned16(workspace)) return KVQ_ERR_MISALIGNED;
+  const DecodeStepRows rows{k_new, v_new, new_stride};
+  return decode_launch(*desc, num_seqs, num_q_heads, q, seq_lens, max_seq_len, block_table,
+                       bt_stride, sm_scale, k_codes, k_params, v_codes, v_params, out, workspace,
+                       workspace_bytes, err_flags, static_cast<cudaStream_t>(stream), &rows);
+}
+
 size_t kvq_decode_fp16_workspace_bytes(const kvq_cache_desc* desc, int32_t num_seqs,
                                        int32_t num_q_heads, int32_t max_seq_len) {
   if (check_desc(desc) != KVQ_OK || num_seqs < 1 || num_q_heads < 1 || max_seq_len < 0 ||

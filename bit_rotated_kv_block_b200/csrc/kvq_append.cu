@@ -40,6 +40,7 @@
 #include "kvq_device.cuh"
 #include "kvq_launch.h"
 #include "kvq_rotate.cuh"
+#include "kvq_rowquant.cuh"
 
 namespace kvq {
 
@@ -318,10 +319,9 @@ constexpr int kRowsWarps = 4;
 
 template <int D, int ROT, int LGB>
 __global__ void __launch_bounds__(kRowsWarps * kWarp) append_rows_kernel(const AppendRowsArgs a) {
-  constexpr int CPL = D / 32 < 4 ? 4 : D / 32;  // channels per lane
-  constexpr int LPR = D / CPL;                  // lanes per row (16 or 32)
-  constexpr int RPW = kWarp / LPR;              // rows per warp
-  constexpr int B = 1 << LGB;
+  constexpr int CPL = RowQuantShape<D>::CPL;  // channels per lane
+  constexpr int LPR = RowQuantShape<D>::LPR;  // lanes per row (16 or 32)
+  constexpr int RPW = kWarp / LPR;            // rows per warp
   const int lane = threadIdx.x % kWarp;
   const int rl = lane % LPR;
   const int row = (blockIdx.x * kRowsWarps + threadIdx.x / kWarp) * RPW + lane / LPR;
@@ -341,86 +341,9 @@ __global__ void __launch_bounds__(kRowsWarps * kWarp) append_rows_kernel(const A
   const int page = (seq_ok && pos_ok) ? a.block_table[(int64_t)seq * a.bt_stride + (pos >> a.lg_page)] : -1;
 
   float x[CPL];
-  {
-    const __half* src = (kv ? a.v : a.k) + (int64_t)t * a.tok_stride + (int64_t)h * D + rl * CPL;
-    if (CPL == 4) {
-      const uint2 u = active ? *reinterpret_cast<const uint2*>(src) : make_uint2(0u, 0u);
-      const float2 f0 = __half22float2(u32_as_h2(u.x)), f1 = __half22float2(u32_as_h2(u.y));
-      x[0] = f0.x; x[1] = f0.y; x[2] = f1.x; x[3] = f1.y;
-    } else {
-#pragma unroll
-      for (int c = 0; c < CPL / 8; ++c) {
-        const uint4 u = active ? reinterpret_cast<const uint4*>(src)[c] : make_uint4(0u, 0u, 0u, 0u);
-        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __half22float2(u32_as_h2(w4[e]));
-          x[8 * c + 2 * e] = f.x;
-          x[8 * c + 2 * e + 1] = f.y;
-        }
-      }
-    }
-  }
-
-  if (ROT == KVQ_ROT_HADAMARD) {
-    // stages h = 1, 2, 4, ... < B in ascending order
-#pragma unroll
-    for (int dd = 1; dd < CPL && dd < B; dd <<= 1) {
-#pragma unroll
-      for (int i = 0; i < CPL; ++i) {
-        if ((i & dd) == 0) {
-          const float p = x[i], q = x[i + dd];
-          x[i] = __fadd_rn(p, q);
-          x[i + dd] = __fsub_rn(p, q);
-        }
-      }
-    }
-#pragma unroll
-    for (int m = 1; m * CPL < B; m <<= 1) {
-      const bool lower = (rl & m) == 0;
-#pragma unroll
-      for (int i = 0; i < CPL; ++i) {
-        const float o = __shfl_xor_sync(0xffffffffu, x[i], m);
-        x[i] = lower ? __fadd_rn(x[i], o) : __fsub_rn(o, x[i]);
-      }
-    }
-    const float cb = hadamard_scale(LGB);
-#pragma unroll
-    for (int i = 0; i < CPL; ++i) x[i] = __fmul_rn(x[i], cb);
-  } else if (ROT == KVQ_ROT_QUAT) {
-    quat_regs<CPL>(x, a.quat, rl * CPL);
-  }
-
-  // row statistics over the LPR lanes of the row
-  float mn = x[0], mx = x[0];
-#pragma unroll
-  for (int i = 1; i < CPL; ++i) {
-    mn = fminf(mn, x[i]);
-    mx = fmaxf(mx, x[i]);
-  }
-#pragma unroll
-  for (int m = 1; m < LPR; m <<= 1) {
-    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, m));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
-  }
-  mn = __fadd_rn(mn, 0.0f);
-  mx = __fadd_rn(mx, 0.0f);
-  const __half m16 = __float2half_rd(mn);
-  const float m = __half2float(m16);
-  const float s32 = __fdiv_ru(__fsub_ru(mx, m), 15.0f);
-  const __half s16 = __float2half_ru(s32);
-  const float s = __half2float(s16);
-  uint32_t packed = 0;
-  if (s != 0.0f) {
-    const float inv = __frcp_rn(s);
-#pragma unroll
-    for (int i = 0; i < CPL; ++i) {
-      // nearest integer (ties to even) of the exact product: one fused
-      // multiply-add with 1.5 * 2^23 leaves it in the low mantissa bits
-      const uint32_t c = __float_as_uint(__fmaf_rn(__fsub_rn(x[i], m), inv, 12582912.0f)) & 0xFu;
-      packed |= c << (4 * i);
-    }
-  }
+  row_load<D>(x, (kv ? a.v : a.k) + (int64_t)t * a.tok_stride + (int64_t)h * D + rl * CPL, active);
+  __half s16, m16;
+  const uint32_t packed = row_quantize<D, ROT, LGB>(x, rl, a.quat, s16, m16);
 
   if (!active || seq < 0) return;
   const bool lead = kv == 0 && h == 0 && rl == 0;
@@ -437,11 +360,7 @@ __global__ void __launch_bounds__(kRowsWarps * kWarp) append_rows_kernel(const A
     return;
   }
   const int64_t dst = (((int64_t)page * a.H + h) << a.lg_page) + (pos & ((1 << a.lg_page) - 1));
-  uint8_t* codes = (kv ? a.v_codes : a.k_codes) + dst * (D / 2) + rl * (CPL / 2);
-  if (CPL == 4)
-    *reinterpret_cast<uint16_t*>(codes) = (uint16_t)packed;
-  else
-    *reinterpret_cast<uint32_t*>(codes) = packed;
+  row_store_codes<D>((kv ? a.v_codes : a.k_codes) + dst * (D / 2) + rl * (CPL / 2), packed);
   if (rl == 0)
     (kv ? a.v_params : a.k_params)[dst] =
         (uint32_t)__half_as_ushort(s16) | ((uint32_t)__half_as_ushort(m16) << 16);

@@ -39,6 +39,7 @@
 #include "kvq_device.cuh"
 #include "kvq_launch.h"
 #include "kvq_rotate.cuh"
+#include "kvq_rowquant.cuh"
 
 namespace kvq {
 
@@ -60,7 +61,59 @@ struct DecodeArgs {
   float* part;       // [S][Hq][splits][D + 4]: acc[D], max (double), sum, pad
   int32_t* counter;  // [S][H] split arrivals, zero between calls
   int32_t* err;
+  // fused decode step (kvq_decode_step): the new token of each sequence, K
+  // and V rows [S][H][D] binary16 (row (s, h) at s * new_stride + h * D),
+  // quantized into the pools at position seq_lens[s] - 1 before attention;
+  // nullptr for plain decode attention
+  const __half* k_new;
+  const __half* v_new;
+  int64_t new_stride;
+  uint8_t* k_codes_w;
+  uint32_t* k_params_w;
+  uint8_t* v_codes_w;
+  uint32_t* v_params_w;
 };
+
+// The new token of one (sequence, KV head) (position L - 1) quantized and
+// written by one warp, exactly as kvq_quantize_append would write it.
+struct StepRowArgs {
+  const __half* k_row;  // this (sequence, KV head)'s new K row
+  const __half* v_row;
+  const float* quat;
+  uint8_t* k_codes;     // this row's destination slot in each pool
+  uint8_t* v_codes;
+  uint32_t* k_param;
+  uint32_t* v_param;
+};
+
+template <int D, int ROT, int LGB>
+__device__ __forceinline__ void step_rows(const StepRowArgs& r, int lane) {
+  constexpr int CPL = RowQuantShape<D>::CPL;
+#pragma unroll 1
+  for (int kv = 0; kv < 2; ++kv) {
+    float x[CPL];
+    row_load<D>(x, (kv ? r.v_row : r.k_row) + lane * CPL, true);
+    __half s16, m16;
+    const uint32_t packed = row_quantize<D, ROT, LGB>(x, lane, r.quat, s16, m16);
+    row_store_codes<D>((kv ? r.v_codes : r.k_codes) + lane * (CPL / 2), packed);
+    if (lane == 0)
+      *(kv ? r.v_param : r.k_param) =
+          (uint32_t)__half_as_ushort(s16) | ((uint32_t)__half_as_ushort(m16) << 16);
+  }
+}
+
+template <int D>
+__device__ __noinline__ void append_step_token(StepRowArgs r, int rot_kind, int lgb, int lane) {
+  if (rot_kind == KVQ_ROT_NONE) return step_rows<D, KVQ_ROT_NONE, 0>(r, lane);
+  if (rot_kind == KVQ_ROT_QUAT) return step_rows<D, KVQ_ROT_QUAT, 0>(r, lane);
+  switch (lgb) {
+    case 4: return step_rows<D, KVQ_ROT_HADAMARD, 4>(r, lane);
+    case 5: return step_rows<D, KVQ_ROT_HADAMARD, 5>(r, lane);
+    case 6: return step_rows<D, KVQ_ROT_HADAMARD, 6>(r, lane);
+    case 7: return step_rows<D, KVQ_ROT_HADAMARD, 7>(r, lane);
+    default: return step_rows<D, KVQ_ROT_HADAMARD, (D >= 256 ? 8 : 7)>(r, lane);
+  }
+}
 
 // ---------------------------------------------------------------------------
 // 2. split kernel
@@ -161,6 +214,23 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, (D == 128 && GP == 4) ? 4 :
   const int npages = (L + P - 1) / P;
   const int ngrp = (npages + C::PG - 1) / C::PG;  // stage groups of the (sequence, KV head)
   const int32_t* const bt_row = a.block_table + (int64_t)s * a.bt_stride;
+  // fused step: the warp that owns the page group of position L - 1 writes
+  // the sequence's new token of this KV head before any of its copies start
+  if (a.k_new != nullptr && L >= 1 && ((L - 1) / P / C::PG) % a.splits == split) {
+    const int pos = L - 1;
+    const int page = bt_row[pos / P];
+    if (page >= 0 && page < a.NP) {
+      const int64_t dst = ((int64_t)page * a.H + h) * P + pos % P;
+      const int64_t src = (int64_t)s * a.new_stride + (int64_t)h * D;
+      const StepRowArgs r{a.k_new + src, a.v_new + src, a.quat, a.k_codes_w + dst * (D / 2),
+                          a.v_codes_w + dst * (D / 2), a.k_params_w + dst, a.v_params_w + dst};
+      append_step_token<D>(r, a.rot_kind, a.lgb, lane);
+      __threadfence();  // visible to this warp's page copies below
+      __syncwarp();
+    } else if (lane == 0) {
+      raise_flag(a.err, KVQ_ERRF_PAGE);
+    }
+  }
   // block-table entry of page q (lane q < PG) of group gi; -1: no such page
   auto group_ids = [&](int gi) {
     const int pi = gi * C::PG + lane;
@@ -851,7 +921,7 @@ int decode_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, const void* q,
                   int32_t bt_stride, float sm_scale, const uint8_t* k_codes,
                   const void* k_params, const uint8_t* v_codes, const void* v_params,
                   float* out, void* workspace, size_t workspace_bytes, int32_t* err,
-                  cudaStream_t st) {
+                  cudaStream_t st, const DecodeStepRows* step) {
   const int D = d.head_dim;
   const int G = Hq / d.num_kv_heads;
   const int GP = G <= 4 ? 4 : 8;
@@ -875,6 +945,13 @@ int decode_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, const void* q,
   a.part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
                                     align256((size_t)S * d.num_kv_heads * sizeof(int32_t)));
   a.err = err;
+  a.k_new = step ? static_cast<const __half*>(step->k_new) : nullptr;
+  a.v_new = step ? static_cast<const __half*>(step->v_new) : nullptr;
+  a.new_stride = step ? step->new_stride : 0;
+  a.k_codes_w = const_cast<uint8_t*>(k_codes);
+  a.v_codes_w = const_cast<uint8_t*>(v_codes);
+  a.k_params_w = static_cast<uint32_t*>(const_cast<void*>(k_params));
+  a.v_params_w = static_cast<uint32_t*>(const_cast<void*>(v_params));
   const cudaError_t e = launch_split_any(a, D, GP, st);
   if (e == cudaErrorInvalidValue) return KVQ_ERR_UNSUPPORTED;
   return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;

@@ -33,12 +33,21 @@ struct DecodePlan {
 };
 DecodePlan decode_plan(const kvq_cache_desc& d, int32_t S, int32_t Hq, int32_t max_seq_len);
 
+// New-token rows of a fused decode step (kvq_decode_step).
+struct DecodeStepRows {
+  const void* k_new;   // binary16 [S][H][d] rows, row (s, h) at s * new_stride + h * d
+  const void* v_new;
+  int64_t new_stride;  // elements between consecutive sequences' rows
+};
+
+// step == nullptr: decode attention only; otherwise the new token of every
+// sequence is quantized into the pools (which the kernel then writes) first.
 int decode_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, const void* q,
                   const int32_t* seq_lens, int32_t max_seq_len, const int32_t* block_table,
                   int32_t bt_stride, float sm_scale, const uint8_t* k_codes,
                   const void* k_params, const uint8_t* v_codes, const void* v_params,
                   float* out, void* workspace, size_t workspace_bytes, int32_t* err,
-                  cudaStream_t st);
+                  cudaStream_t st, const DecodeStepRows* step = nullptr);
 
 // Baseline decode attention over a binary16 paged cache.
 DecodePlan decode_fp16_plan(const kvq_cache_desc& d, int32_t S, int32_t Hq, int32_t max_seq_len);

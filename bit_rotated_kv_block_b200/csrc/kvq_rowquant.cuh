@@ -1,0 +1,133 @@
+// One K or V row (one token, one KV head) rotated, quantized and packed by a
+// group of LPR consecutive lanes, each owning CPL = max(4, d/32) consecutive
+// channels (LPR = d / CPL: 32 lanes, or 16 at d = 64).
+//
+// Arithmetic and order are those of the tiled append kernel and of the
+// method's definition (see kvq.h): butterfly stages h = 1, 2, 4, ... in
+// ascending order, each one binary32 add or subtract (stages below CPL in
+// registers; wider stages across lanes, the lower-channel lane adding and
+// the upper one taking (lower - upper)), the binary32 scale nearest 1/sqrt(b),
+// min and max with -0 normalised to +0, m16 rounded down, the scale from the
+// upward-rounded binary32 subtraction and division by 15 rounded up to
+// binary16, and each code the nearest integer (ties to even) of the exact
+// product RN(x - m16) * RN(1/s16) from one fused multiply-add.
+#pragma once
+
+#include <cuda_fp16.h>
+
+#include "kvq.h"
+#include "kvq_device.cuh"
+#include "kvq_rotate.cuh"
+
+namespace kvq {
+
+template <int D>
+struct RowQuantShape {
+  static constexpr int CPL = D / 32 < 4 ? 4 : D / 32;  // channels per lane
+  static constexpr int LPR = D / CPL;                  // lanes per row
+};
+
+// x: this lane's CPL channels (binary16 values widened to binary32); rl: the
+// lane's index inside its row. Every lane of the warp must call it (the
+// shuffles span the warp; rows never mix because lane distances stay below
+// LPR). Returns the lane's codes, channel i of the lane in bits 4i..4i+3.
+template <int D, int ROT, int LGB>
+__device__ __forceinline__ uint32_t row_quantize(float (&x)[RowQuantShape<D>::CPL], int rl,
+                                                 const float* quat, __half& s16, __half& m16) {
+  constexpr int CPL = RowQuantShape<D>::CPL;
+  constexpr int LPR = RowQuantShape<D>::LPR;
+  constexpr int B = 1 << LGB;
+  if (ROT == KVQ_ROT_HADAMARD) {
+#pragma unroll
+    for (int dd = 1; dd < CPL && dd < B; dd <<= 1) {
+#pragma unroll
+      for (int i = 0; i < CPL; ++i) {
+        if ((i & dd) == 0) {
+          const float p = x[i], q = x[i + dd];
+          x[i] = __fadd_rn(p, q);
+          x[i + dd] = __fsub_rn(p, q);
+        }
+      }
+    }
+#pragma unroll
+    for (int m = 1; m * CPL < B; m <<= 1) {
+      const bool lower = (rl & m) == 0;
+#pragma unroll
+      for (int i = 0; i < CPL; ++i) {
+        const float o = __shfl_xor_sync(0xffffffffu, x[i], m);
+        x[i] = lower ? __fadd_rn(x[i], o) : __fsub_rn(o, x[i]);
+      }
+    }
+    const float cb = hadamard_scale(LGB);
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) x[i] = __fmul_rn(x[i], cb);
+  } else if (ROT == KVQ_ROT_QUAT) {
+    quat_regs<CPL>(x, quat, rl * CPL);
+  }
+
+  float mn = x[0], mx = x[0];
+#pragma unroll
+  for (int i = 1; i < CPL; ++i) {
+    mn = fminf(mn, x[i]);
+    mx = fmaxf(mx, x[i]);
+  }
+#pragma unroll
+  for (int m = 1; m < LPR; m <<= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, m));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
+  }
+  mn = __fadd_rn(mn, 0.0f);
+  mx = __fadd_rn(mx, 0.0f);
+  m16 = __float2half_rd(mn);
+  const float m = __half2float(m16);
+  const float s32 = __fdiv_ru(__fsub_ru(mx, m), 15.0f);
+  s16 = __float2half_ru(s32);
+  const float s = __half2float(s16);
+  uint32_t packed = 0;
+  if (s != 0.0f) {
+    const float inv = __frcp_rn(s);
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) {
+      // nearest integer (ties to even) of the exact product: one fused
+      // multiply-add with 1.5 * 2^23 leaves it in the low mantissa bits
+      const uint32_t c = __float_as_uint(__fmaf_rn(__fsub_rn(x[i], m), inv, 12582912.0f)) & 0xFu;
+      packed |= c << (4 * i);
+    }
+  }
+  return packed;
+}
+
+// Loads this lane's CPL channels of a binary16 row (zeros when !active).
+template <int D>
+__device__ __forceinline__ void row_load(float (&x)[RowQuantShape<D>::CPL], const __half* src,
+                                         bool active) {
+  constexpr int CPL = RowQuantShape<D>::CPL;
+  if (CPL == 4) {
+    const uint2 u = active ? *reinterpret_cast<const uint2*>(src) : make_uint2(0u, 0u);
+    const float2 f0 = __half22float2(u32_as_h2(u.x)), f1 = __half22float2(u32_as_h2(u.y));
+    x[0] = f0.x; x[1] = f0.y; x[2] = f1.x; x[3] = f1.y;
+  } else {
+#pragma unroll
+    for (int c = 0; c < CPL / 8; ++c) {
+      const uint4 u = active ? reinterpret_cast<const uint4*>(src)[c] : make_uint4(0u, 0u, 0u, 0u);
+      const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __half22float2(u32_as_h2(w4[e]));
+        x[8 * c + 2 * e] = f.x;
+        x[8 * c + 2 * e + 1] = f.y;
+      }
+    }
+  }
+}
+
+// Stores this lane's codes (CPL/2 bytes) at `codes` (the lane's slice).
+template <int D>
+__device__ __forceinline__ void row_store_codes(uint8_t* codes, uint32_t packed) {
+  if (RowQuantShape<D>::CPL == 4)
+    *reinterpret_cast<uint16_t*>(codes) = (uint16_t)packed;
+  else
+    *reinterpret_cast<uint32_t*>(codes) = packed;
+}
+
+}  // namespace kvq

@@ -32,6 +32,8 @@ SIGNATURES = {
                                             _P, _P]),
     "kvq_paged_decode_attn_noalloc": (ctypes.c_int, [_P, _I32, _I32, _P, _P, _I32, _P, _I32, _F32,
                                                      _P, _P, _P, _P, _P, _P, _P]),
+    "kvq_decode_step": (ctypes.c_int, [_P, _I32, _I32, _P, _P, _P, _I64, _P, _I32, _P, _I32, _F32,
+                                       _P, _P, _P, _P, _P, _P, _SZ, _P, _P]),
     "kvq_decode_fp16_workspace_bytes": (_SZ, [_P, _I32, _I32, _I32]),
     "kvq_paged_decode_attn_fp16": (ctypes.c_int, [_P, _I32, _I32, _P, _P, _I32, _P, _I32, _F32,
                                                   _P, _P, _P, _P, _SZ, _P, _P]),
@@ -157,6 +159,36 @@ def paged_decode_attn(cache, q, seq_lens, max_seq_len, block_table, k_codes, k_p
                                      _ptr(workspace), workspace.numel() * workspace.element_size(),
                                      _ptr(err), _stream(stream))
     _check("kvq_paged_decode_attn", st)
+    return out
+
+
+def decode_step(cache, q, k_new, v_new, seq_lens, max_seq_len, block_table, k_codes, k_params,
+                v_codes, v_params, out=None, workspace=None, sm_scale=None, err=None,
+                stream=None):
+    """One fused decode step: writes the new token of every sequence (k_new,
+    v_new float16 CUDA [S][H][d], or row-strided views with the same row
+    layout) at position seq_lens[s] - 1 and returns the attention output
+    float32 [S][Hq][d] over seq_lens[s] tokens (lengths include the new
+    token). Workspace as for ``paged_decode_attn``."""
+    S, Hq, d = q.shape
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((S, Hq, d), dtype=torch.float32, device=q.device)
+    need = decode_workspace_bytes(cache, S, Hq, max_seq_len)
+    if workspace is None:
+        workspace = torch.zeros(max(need, 16), dtype=torch.uint8, device=q.device)
+    new_stride = k_new.stride(0)
+    if v_new.stride(0) != new_stride:
+        raise ValueError("k_new and v_new must share the row stride")
+    st = lib().kvq_decode_step(ctypes.byref(cache.desc), S, Hq, _ptr(q), _ptr(k_new), _ptr(v_new),
+                               int(new_stride), _ptr(seq_lens), int(max_seq_len),
+                               _ptr(block_table), int(block_table.shape[1]), float(sm_scale),
+                               _ptr(k_codes), _ptr(k_params), _ptr(v_codes), _ptr(v_params),
+                               _ptr(out), _ptr(workspace),
+                               workspace.numel() * workspace.element_size(), _ptr(err),
+                               _stream(stream))
+    _check("kvq_decode_step", st)
     return out
 
 

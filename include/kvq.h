@@ -188,6 +188,36 @@ int kvq_dequantize_pages(const kvq_cache_desc* desc, int32_t num_seqs,
                          int32_t* err_flags, void* stream);
 
 /*
+ * kvq_decode_step -- one decode step in one launch: for every sequence s with
+ * seq_lens[s] >= 1, the new token's K and V rows are rotated, quantized and
+ * written at position seq_lens[s] - 1 exactly as kvq_quantize_append writes
+ * them (token_seq = s, token_pos = seq_lens[s] - 1), and decode attention then
+ * runs over positions [0, seq_lens[s]) as kvq_paged_decode_attn. The pools
+ * and the output equal those of the two calls in that order. The quantized
+ * write inside the paged cache follows the method (page "SAW-INT4:
+ * System-Aware 4-Bit KV-Cache Quantization for Real-World LLM Serving",
+ * Summary and Method); doing it inside the attention launch, by the warp that
+ * reads that page, is this library's own step (one launch per step, and the
+ * write overlaps the launch's start-up latency).
+ *
+ *  k_new, v_new  device binary16 rows of the new tokens: row (s, h) starts at
+ *                element s * new_stride + h * head_dim; 16-byte aligned,
+ *                new_stride a multiple of 8 elements and >= H * head_dim.
+ *  seq_lens      device int32 [S], lengths INCLUDING the new token.
+ *  k_codes, k_params, v_codes, v_params
+ *                the pools, written at the new tokens' slots and read.
+ *  all other arguments, the workspace, the return codes and the flags as for
+ *  kvq_paged_decode_attn; a block-table entry outside [0, num_pages) for a
+ *  new token's page skips that write and sets KVQ_ERRF_PAGE.
+ */
+int kvq_decode_step(const kvq_cache_desc* desc, int32_t num_seqs, int32_t num_q_heads,
+                    const void* q, const void* k_new, const void* v_new, int64_t new_stride,
+                    const int32_t* seq_lens, int32_t max_seq_len, const int32_t* block_table,
+                    int32_t bt_stride, float sm_scale, uint8_t* k_codes, void* k_params,
+                    uint8_t* v_codes, void* v_params, float* out, void* workspace,
+                    size_t workspace_bytes, int32_t* err_flags, void* stream);
+
+/*
  * Full-precision baseline: decode attention over an UNQUANTIZED binary16
  * paged cache, without rotation. The INT4 cache is measured against it (page
  * "SAW-INT4: System-Aware 4-Bit KV-Cache Quantization for Real-World LLM
