@@ -6,7 +6,7 @@ head_dim 128, Hadamard block 64, page 16, shuffled block table): append one
 new token per sequence (fused rotate -> INT4 -> pack -> page scatter), then
 paged decode attention over the 4097 cached INT4 tokens -- both in one
 kvq_decode_step launch. Inputs are seeded
-synthetic draws of that shape (no dataset exists for this).
+synthetic draws of that shape (no dataset exists for this workload).
 
 The device-timed region covers exactly --steps steps between a barrier and a
 synchronize on both sides; consecutive steps alternate between two cache
@@ -31,6 +31,7 @@ import math
 import os
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -111,7 +112,7 @@ class ClockSampler:
     def __init__(self, index):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        self.path = os.path.join(tempfile.gettempdir(), f"kvq_clocks_rank{index}.csv")
 
     def start(self):
         try:

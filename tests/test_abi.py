@@ -75,3 +75,34 @@ def test_host_validation_codes(L):
     desc = _desc()
     assert L.kvq_decode_workspace_bytes(ctypes.byref(desc), 0, 32, 100) == 0
     assert L.kvq_decode_workspace_bytes(ctypes.byref(desc), 2, 30, 100) == 0   # Hq % H != 0
+
+
+def test_host_validation_of_step_and_baseline(L):
+    """kvq_decode_step and kvq_paged_decode_attn_fp16 reject bad arguments on
+    the host before touching any device memory (fake pointers, no launch)."""
+    OK, INV, UNS, MIS = 0, 1, 2, 3
+    desc = _desc()
+    P = ctypes.c_void_p
+    good = 1 << 20  # a 16-byte aligned fake address
+
+    def step(q=good, k=good, v=good, stride=4096, lens=good, Hq=32, ws=good):
+        return L.kvq_decode_step(ctypes.byref(desc), 2, Hq, P(q), P(k), P(v), stride, P(lens), 100,
+                                 P(good), 8, 0.1, P(good), P(good), P(good), P(good), P(good),
+                                 P(ws), 0, None, None)
+
+    assert step(Hq=30) == INV            # query heads not a multiple of KV heads
+    assert step(Hq=8 * 16) == UNS        # GQA group above 8
+    assert step(k=0) == INV              # null new-token rows
+    assert step(stride=100) == INV       # row stride below H * d
+    assert step(stride=1028 + 4096) == MIS  # stride not a multiple of 8
+    assert step(v=good + 8) == MIS       # misaligned rows
+    assert step(q=good + 4) == MIS
+    d16 = _desc()
+    assert L.kvq_paged_decode_attn_fp16(ctypes.byref(d16), 2, 30, P(good), P(good), 100, P(good),
+                                        8, 0.1, P(good), P(good), P(good), P(good), 0, None,
+                                        None) == INV
+    assert L.kvq_paged_decode_attn_fp16(ctypes.byref(d16), 2, 32, P(good), P(good), 100, P(good),
+                                        8, 0.1, P(good + 8), P(good), P(good), P(good), 0, None,
+                                        None) == MIS
+    assert L.kvq_decode_fp16_workspace_bytes(ctypes.byref(d16), 0, 32, 100) == 0
+
