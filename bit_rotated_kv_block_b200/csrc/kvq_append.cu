@@ -65,6 +65,8 @@ template <int D, int ROT, int LGB>
 __global__ void __launch_bounds__(kAppendThreads, 1)
     append_kernel(const AppendArgs a, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv) {
+  pdl_wait();     // K/V and the metadata may come from the previous kernel
+  pdl_trigger();
   constexpr int E = D < 128 ? D : 128;   // channels per thread
   constexpr int TPR = D / E;             // threads per row
   constexpr int NH = D / 64;             // 64-channel boxes per row
@@ -319,6 +321,8 @@ constexpr int kRowsWarps = 4;
 
 template <int D, int ROT, int LGB>
 __global__ void __launch_bounds__(kRowsWarps * kWarp) append_rows_kernel(const AppendRowsArgs a) {
+  pdl_wait();     // K/V and the metadata may come from the previous kernel
+  pdl_trigger();
   constexpr int CPL = RowQuantShape<D>::CPL;  // channels per lane
   constexpr int LPR = RowQuantShape<D>::LPR;  // lanes per row (16 or 32)
   constexpr int RPW = kWarp / LPR;            // rows per warp
@@ -371,7 +375,9 @@ static cudaError_t launch_rows(const AppendRowsArgs& a, cudaStream_t st) {
   constexpr int CPL = D / 32 < 4 ? 4 : D / 32;
   constexpr int RPW = kWarp / (D / CPL);
   const int warps = (a.T * a.H * 2 + RPW - 1) / RPW;
-  append_rows_kernel<D, ROT, LGB><<<(warps + kRowsWarps - 1) / kRowsWarps, kRowsWarps * kWarp, 0, st>>>(a);
+  const cudaError_t e = launch_pdl(append_rows_kernel<D, ROT, LGB>, (warps + kRowsWarps - 1) / kRowsWarps,
+                                   kRowsWarps * kWarp, 0, st, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -434,7 +440,8 @@ static cudaError_t launch_append(const AppendArgs& a, const CUtensorMap& tk, con
   auto kern = append_kernel<D, ROT, LGB>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kAppendThreads, smem, st>>>(a, tk, tv);
+  e = launch_pdl(kern, grid, kAppendThreads, smem, st, a, tk, tv);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

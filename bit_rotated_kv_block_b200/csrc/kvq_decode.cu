@@ -182,6 +182,10 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, (D == 128 && GP == 4) ? 4 :
   static_assert(D == 128 || D == 256, "decode attention supports head_dim 128 and 256");
   using C = DecCfg<D, P, GP>;
   extern __shared__ __align__(128) uint8_t smem[];
+  // inputs may come from the previous kernel of the stream: nothing is read
+  // before it has completed; the next launch may be scheduled right away
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
   const int r = lane >> 2, j = lane & 3;
   const int item = blockIdx.x * kDecWarps + warp;
@@ -904,7 +908,8 @@ static cudaError_t launch_split(const DecodeArgs& a, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   const int items = a.S * a.H * a.splits;
   const int grid = (items + kDecWarps - 1) / kDecWarps;
-  kern<<<grid, kDecWarps * kWarp, smem, st>>>(a);
+  e = launch_pdl(kern, grid, kDecWarps * kWarp, smem, st, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -122,6 +122,19 @@ __device__ __forceinline__ void cp_async_wait() {
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch. A kernel launched with programmatic stream
+// serialization may start while the previous kernel of the stream finishes;
+// pdl_wait() then blocks until that kernel has completed and its writes are
+// visible, so it must precede every read of memory another kernel may have
+// written (it is a no-op for an ordinary launch). pdl_trigger() lets the next
+// such launch be scheduled as soon as every CTA of this grid has started.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // Bulk (TMA) copies global -> shared completing on an mbarrier. No multicast.
 // Waits are bounded: after kMbarSpinLimit polls the caller gets `false` and
 // must raise KVQ_ERRF_TIMEOUT instead of hanging.

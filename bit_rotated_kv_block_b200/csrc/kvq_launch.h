@@ -25,6 +25,23 @@ int dequant_launch(const kvq_cache_desc& d, int32_t S, const int32_t* seq_lens,
                    void* out, int32_t* err, cudaStream_t st);
 
 // Split-K plan of the decode attention for these sizes.
+// Launches `kern` with programmatic stream serialization (see pdl_wait).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), int grid, int threads, size_t smem,
+                              cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+}
+
 struct DecodePlan {
   int pages_max;        // ceil(max_seq_len / P)
   int splits;           // work items per (sequence, KV head)
