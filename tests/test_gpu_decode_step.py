@@ -106,3 +106,27 @@ def test_new_token_page_outside_pool_is_flagged():
                     dev(table), p.kc, p.kp, p.vc, p.vp, err=p.err)
     torch.cuda.synchronize()
     assert int(p.err.item()) & kvq.ERRF_PAGE
+
+
+def test_llama8b_full_size_step_matches_two_calls():
+    # the bench's workload and launch configuration: 32 sequences x 4096
+    # cached tokens, one new token each; the fused step and the two-call path
+    # leave identical pools and outputs (the two-call path is checked against
+    # the oracle at this size in test_gpu_decode.py)
+    w = workloads.llama8b()
+    p, _ = fill_workload(w, oracle_too=False)
+    k_new, v_new, ts, tp = w.step_tokens(0)
+    lens = (w.seq_lens + 1).astype(np.int32)
+    L = int(lens.max())
+    q = dev(w.queries())
+    kc2, kp2, vc2, vp2 = p.kc.clone(), p.kp.clone(), p.vc.clone(), p.vp.clone()
+    bt = dev(w.block_table)
+    kvq.quantize_append(p.gpu, dev(k_new), dev(v_new), dev(ts), dev(tp), bt, kc2, kp2, vc2, vp2)
+    out2 = kvq.paged_decode_attn(p.gpu, q, dev(lens), L, bt, kc2, kp2, vc2, vp2)
+    out1 = kvq.decode_step(p.gpu, q, dev(k_new), dev(v_new), dev(lens), L, bt, p.kc, p.kp, p.vc,
+                           p.vp, err=p.err)
+    torch.cuda.synchronize()
+    assert int(p.err.item()) == 0
+    for a, b in ((p.kc, kc2), (p.kp, kp2), (p.vc, vc2), (p.vp, vp2)):
+        assert torch.equal(a, b)
+    assert torch.equal(out1, out2)
