@@ -44,7 +44,16 @@
 
 namespace kvq {
 
-constexpr int kAppendThreads = 384;
+// Channels per thread: 64 (two threads per d = 128 row, 256-thread CTAs, two
+// CTAs per SM), or 128 (384-thread CTAs, one per SM) where a Hadamard block of
+// 128 would need a cross-thread butterfly stage, for d = 256, and for Hadamard
+// blocks of 2..16, which measured faster with the wider thread.
+__host__ __device__ constexpr int append_e(int D, int rot, int lgb) {
+  return D <= 64 ? D
+                 : (D == 256 || (rot == KVQ_ROT_HADAMARD && (lgb >= 7 || lgb <= 4))) ? 128 : 64;
+}
+__host__ __device__ constexpr int append_threads(int E) { return E == 64 ? 256 : 384; }
+__host__ __device__ constexpr int append_ctas_per_sm(int E) { return E == 64 ? 2 : 1; }
 
 struct AppendArgs {
   int T, H, P, lg_page, NP, num_seqs, bt_stride, tok_per_tile, num_tiles;
@@ -62,12 +71,14 @@ struct AppendArgs {
 
 // D: head_dim, ROT: rotation kind, LGB: log2 of the Hadamard block.
 template <int D, int ROT, int LGB>
-__global__ void __launch_bounds__(kAppendThreads, 1)
+__global__ void __launch_bounds__(append_threads(append_e(D, ROT, LGB)),
+                                  append_ctas_per_sm(append_e(D, ROT, LGB)))
     append_kernel(const AppendArgs a, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv) {
   pdl_wait();     // K/V and the metadata may come from the previous kernel
   pdl_trigger();
-  constexpr int E = D < 128 ? D : 128;   // channels per thread
+  constexpr int E = append_e(D, ROT, LGB);    // channels per thread
+  constexpr int kAppendThreads = append_threads(E);
   constexpr int TPR = D / E;             // threads per row
   constexpr int NH = D / 64;             // 64-channel boxes per row
 
@@ -440,7 +451,7 @@ static cudaError_t launch_append(const AppendArgs& a, const CUtensorMap& tk, con
   auto kern = append_kernel<D, ROT, LGB>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  e = launch_pdl(kern, grid, kAppendThreads, smem, st, a, tk, tv);
+  e = launch_pdl(kern, grid, append_threads(append_e(D, ROT, LGB)), smem, st, a, tk, tv);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -470,9 +481,12 @@ int append_launch(const kvq_cache_desc& d, int32_t T, const void* k, const void*
                   uint8_t* k_codes, void* k_params, uint8_t* v_codes, void* v_params,
                   int32_t* err, cudaStream_t st) {
   const int D = d.head_dim;
-  const int E = D < 128 ? D : 128;
+  int lgb0 = 0;
+  while ((1 << lgb0) < d.rot_block) ++lgb0;
+  const int E = append_e(D, d.rot_kind, lgb0);
   const int TPR = D / E;
-  const int tok_max = kAppendThreads / (2 * d.num_kv_heads * TPR);
+  const int per_sm = append_ctas_per_sm(E);
+  const int tok_max = append_threads(E) / (2 * d.num_kv_heads * TPR);
   if (tok_max < 1 || d.num_kv_heads > 256) return KVQ_ERR_UNSUPPORTED;
   const int sms = device_sm_count();
   if (sms <= 0) return KVQ_ERR_CUDA;
@@ -502,7 +516,7 @@ int append_launch(const kvq_cache_desc& d, int32_t T, const void* k, const void*
     return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
   }
   // small batches: fewer tokens per tile so more SMs share the work
-  int tok = (T + sms - 1) / sms;
+  int tok = (T + per_sm * sms - 1) / (per_sm * sms);
   if (tok > tok_max) tok = tok_max;
   if (tok < 1) tok = 1;
   AppendArgs a;
@@ -530,7 +544,7 @@ int append_launch(const kvq_cache_desc& d, int32_t T, const void* k, const void*
   if (!encode_rows(&tk, k, D, a.H, T, tok_stride, tok) ||
       !encode_rows(&tv, v, D, a.H, T, tok_stride, tok))
     return KVQ_ERR_CUDA;
-  const int grid = a.num_tiles < sms ? a.num_tiles : sms;
+  const int grid = a.num_tiles < per_sm * sms ? a.num_tiles : per_sm * sms;
   cudaError_t e;
   switch (D) {
     case 64: e = dispatch_rot<64>(a, tk, tv, d.rot_kind, lgb, grid, st); break;
