@@ -102,6 +102,30 @@ def test_ragged_token_batch_and_edges(d, H, P, rot, b):
     p.assert_pools_equal()
 
 
+@pytest.mark.parametrize("T,b", [(520, 64), (1201, 128), (4999, 0), (9000, 32), (3000, 16)])
+def test_tiled_kernel_few_tiles_per_cta(T, b):
+    # batches just above the warp-per-row path (T * H * 2 > 8192 rows): the
+    # tiled kernel runs with one to a few tiles per CTA, fewer than its ring
+    # of tile buffers, and a partial last tile
+    g = np.random.default_rng(T + b)
+    d, H, P, S = 128, 8, 16, 3
+    bt_stride = (T + P - 1) // P + 2
+    NP = S * bt_stride + 5
+    table = g.permutation(NP)[:S * bt_stride].reshape(S, bt_stride).astype(np.int32)
+    token_seq = g.integers(0, S, size=T).astype(np.int32)
+    token_seq[::97] = -1                                    # skipped tokens
+    token_pos = np.zeros(T, np.int32)
+    for s in range(S):
+        idx = np.nonzero(token_seq == s)[0]
+        token_pos[idx] = g.permutation(bt_stride * P)[:len(idx)]
+    k = (g.standard_normal((T, H, d)) * g.uniform(0.05, 20, size=(T, H, 1))).astype(np.float16)
+    v = g.standard_normal((T, H, d)).astype(np.float16)
+    p = Pair(d, H, P, NP, 1 if b else 0, b)
+    e, oe = p.append(k, v, token_seq, token_pos, table)
+    assert e == 0 and oe == 0
+    p.assert_pools_equal()
+
+
 def test_strided_input_from_fused_qkv():
     # K and V are slices of a [T][(Hq + 2H) * d] projection output
     g = np.random.default_rng(3)
