@@ -102,13 +102,19 @@ def test_ragged_token_batch_and_edges(d, H, P, rot, b):
     p.assert_pools_equal()
 
 
-@pytest.mark.parametrize("T,b", [(520, 64), (1201, 128), (4999, 0), (9000, 32), (3000, 16)])
-def test_tiled_kernel_few_tiles_per_cta(T, b):
-    # batches just above the warp-per-row path (T * H * 2 > 8192 rows): the
-    # tiled kernel runs with one to a few tiles per CTA, fewer than its ring
-    # of tile buffers, and a partial last tile
-    g = np.random.default_rng(T + b)
-    d, H, P, S = 128, 8, 16, 3
+@pytest.mark.parametrize("T,d,H,rot,b,qkv", [
+    (520, 128, 8, 1, 64, False), (1201, 128, 8, 1, 128, False), (4999, 128, 8, 0, 0, False),
+    (9000, 128, 8, 1, 32, False), (3000, 128, 8, 1, 16, False), (2000, 64, 8, 1, 64, False),
+    (3001, 64, 3, 1, 32, False), (2500, 128, 5, 2, 0, False), (1700, 64, 4, 2, 0, False),
+    (1200, 128, 8, 1, 128, True), (1200, 128, 8, 1, 64, True)])
+def test_bulk_batches_ragged(T, d, H, rot, b, qkv):
+    # batches above the warp-per-row path (T * H * 2 > 8192 rows): a few
+    # work units per warp or CTA, a partial last unit, skipped tokens, an
+    # odd head count, both channel ownerships of the streaming kernel
+    # (b < d and b = d), quaternions, and rows read out of a fused
+    # [T][(Hq + 2H) d] projection
+    g = np.random.default_rng(T + d + H + b)
+    P, S = 16, 3
     bt_stride = (T + P - 1) // P + 2
     NP = S * bt_stride + 5
     table = g.permutation(NP)[:S * bt_stride].reshape(S, bt_stride).astype(np.int32)
@@ -118,10 +124,24 @@ def test_tiled_kernel_few_tiles_per_cta(T, b):
     for s in range(S):
         idx = np.nonzero(token_seq == s)[0]
         token_pos[idx] = g.permutation(bt_stride * P)[:len(idx)]
+    quat = workloads.random_quaternions(11, d) if rot == 2 else None
     k = (g.standard_normal((T, H, d)) * g.uniform(0.05, 20, size=(T, H, 1))).astype(np.float16)
     v = g.standard_normal((T, H, d)).astype(np.float16)
-    p = Pair(d, H, P, NP, 1 if b else 0, b)
-    e, oe = p.append(k, v, token_seq, token_pos, table)
+    k[1, 0] = 0.0                                           # degenerate rows
+    v[2, 0] = 1.5
+    p = Pair(d, H, P, NP, rot, b, quat)
+    if not qkv:
+        e, oe = p.append(k, v, token_seq, token_pos, table)
+    else:
+        Hq = 4 * H
+        stride = (Hq + 2 * H) * d
+        buf = g.standard_normal((T, stride)).astype(np.float16)
+        buf[:, Hq * d:(Hq + H) * d] = k.reshape(T, H * d)
+        buf[:, (Hq + H) * d:] = v.reshape(T, H * d)
+        flat = buf.reshape(-1)
+        bd = dev(buf).reshape(-1)
+        e, oe = p.append(flat[Hq * d:], flat[(Hq + H) * d:], token_seq, token_pos, table,
+                         tok_stride=stride, k_dev=bd[Hq * d:], v_dev=bd[(Hq + H) * d:])
     assert e == 0 and oe == 0
     p.assert_pools_equal()
 
