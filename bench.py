@@ -184,6 +184,10 @@ def run_ours(args, world, rank, local):
     from bit_rotated_kv_block_b200 import kvq, workloads
     from bit_rotated_kv_block_b200 import build as kbuild
 
+    if not torch.cuda.is_available():
+        # the measured path is the CUDA library; there is no CPU fallback
+        raise SystemExit("bench.py: the INT4 KV-cache path needs a CUDA GPU; "
+                         "--impl reference times the CPU oracle")
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     if rank == 0 or not os.path.exists(kbuild.LIB):
