@@ -19,9 +19,9 @@ module only marshals numpy arrays. Method sources, by page title and section:
   Compression" -- Abstract: T(v) = qL v conj(qR) per 4-D block.
 
 Every function here is pinned by ``tests/test_oracle_*.py`` against
-closed forms, textbook identities, library routines and brute force; the
-end-to-end numbers are "parity unpinned" by the pages, which print no value
-this path can reproduce.
+closed forms, textbook identities, library routines and brute force. The
+pages print no worked example or table that this path reproduces, so none of
+those pins is a number taken from them.
 """
 
 import ctypes
