@@ -170,46 +170,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
   return false;
 }
-// Variants on shared-window addresses (no generic -> shared conversions).
-__device__ __forceinline__ void mbar_arrive_expect_tx_s(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-// one test of the phase with the given parity (true once it has completed)
-__device__ __forceinline__ bool mbar_try_wait_s(uint32_t bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(done)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return done != 0;
-}
-// bounded wait: false after kMbarSpinLimit tests
-static __device__ __noinline__ bool mbar_wait_s(uint32_t bar, uint32_t parity) {
-  for (uint32_t it = 0; it < kMbarSpinLimit; ++it)
-    if (mbar_try_wait_s(bar, parity)) return true;
-  return false;
-}
-__device__ __forceinline__ void bulk_g2s_s(uint32_t dst, const void* src, uint32_t bytes,
-                                           uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(dst),
-      "l"(src), "r"(bytes), "r"(bar)
-      : "memory");
-}
-__device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, uint32_t bytes,
-                                         uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(smem_u32(smem_dst)),
-      "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-
 // Tiled TMA load of one 3-D box (coordinates in elements, innermost first)
 // into shared memory, completing on an mbarrier. No multicast.
 __device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* tmap, int x, int y, int z,
@@ -255,31 +215,11 @@ __device__ __forceinline__ void mma16832_s8u8(int (&c)[4], const uint32_t (&a)[4
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// Packs four signed 8-bit values (given as int) into one register, first in
-// the lowest byte.
-__device__ __forceinline__ uint32_t pack_s8x4(int v0, int v1, int v2, int v3) {
-  return (uint32_t)(v0 & 0xff) | ((uint32_t)(v1 & 0xff) << 8) | ((uint32_t)(v2 & 0xff) << 16) |
-         ((uint32_t)(v3 & 0xff) << 24);
-}
-
 __device__ __forceinline__ uint32_t h2_as_u32(__half2 h) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 __device__ __forceinline__ __half2 u32_as_h2(uint32_t u) {
   return *reinterpret_cast<__half2*>(&u);
-}
-
-// Four packed 4-bit codes -> two half2 holding (code - 8), exact.
-// From a 32-bit word w of 8 nibbles n0..n7 (n_i at bits 4i) and shift e*4,
-// returns half2(n_e - 8, n_{e+4} - 8): the nibble is placed in the mantissa
-// of 1024.0 (0x6400) and 1032 is subtracted.
-template <int E>
-__device__ __forceinline__ uint32_t nib_pair(uint32_t w) {
-  uint32_t t;
-  const uint32_t x = (E == 0) ? w : (w >> (4 * E));
-  asm("lop3.b32 %0, %1, %2, %3, 0xea;" : "=r"(t) : "r"(x), "r"(0x000F000Fu), "r"(0x64006400u));
-  const __half2 h = __hsub2(u32_as_h2(t), u32_as_h2(0x64086408u));  // 1032.0 = 0x6408
-  return h2_as_u32(h);
 }
 
 // The four nibbles of each 16-bit half of z as half2 (code - 8), exact:
@@ -300,12 +240,6 @@ __device__ __forceinline__ void nib4(uint32_t z, uint32_t (&out)[4]) {
   out[1] = h2_as_u32(__hfma2(u32_as_h2(t1), k16th, km72));
   out[2] = h2_as_u32(__hsub2(u32_as_h2(t2), k1032));
   out[3] = h2_as_u32(__hfma2(u32_as_h2(t3), k16th, km72));
-}
-
-// half2 (hi, lo) split of a binary32 value: hi = RN16(x), lo = RN16(x - hi).
-__device__ __forceinline__ void split_hl(float x, __half& hi, __half& lo) {
-  hi = __float2half_rn(x);
-  lo = __float2half_rn(x - __half2float(hi));
 }
 
 __device__ __forceinline__ float fast_exp2(float x) {
