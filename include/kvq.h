@@ -53,7 +53,7 @@ extern "C" {
 typedef enum {
   KVQ_OK = 0,
   KVQ_ERR_INVALID_ARG = 1, /* a size, index or pointer argument is invalid */
-  KVQ_ERR_UNSUPPORTED = 2, /* a valid geometry this build has no kernel for */
+  KVQ_ERR_UNSUPPORTED = 2, /* a valid geometry the library has no kernel for */
   KVQ_ERR_MISALIGNED = 3,  /* a pointer or stride is not 16-byte aligned   */
   KVQ_ERR_WORKSPACE = 4,   /* workspace missing or smaller than required   */
   KVQ_ERR_CUDA = 5         /* the CUDA runtime reported an error at launch  */
