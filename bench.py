@@ -64,6 +64,8 @@ def parse():
                     help="run a short fixed case for an ncu capture (4 launches) and exit")
     ap.add_argument("--profile-block", type=int, default=128,
                     help="Hadamard block size of the append profile case (0: no rotation)")
+    ap.add_argument("--profile-workload", choices=["llama8b", "long70b"], default="llama8b",
+                    help="workload of the decode profile case")
     return ap.parse_args()
 
 
@@ -442,16 +444,19 @@ def run_reference(args, world, rank):
     }
 
 
-def profile_case(which, block=128):
+def profile_case(which, block=128, workload="llama8b"):
     """Short cases for ncu captures, each well above L2 and well below a few GB:
     append = 4 bulk appends of one prefill layer (65536 tokens, Hadamard block
     `block`, 268 MB in, 71 MB out); decode = 4 decode calls of the
-    Llama-3-8B-shaped layer (143 MB of INT4 pages) after filling its cache with
-    one append."""
+    Llama-3-8B-shaped layer (143 MB of INT4 pages) or of the long-context
+    70B-shaped one (285 MB) after filling its cache with one append."""
     from bit_rotated_kv_block_b200 import kvq, workloads
     torch.cuda.set_device(0)
     dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
-    w = workloads.prefill(rot_block=block) if which == "append" else workloads.llama8b()
+    if which == "append":
+        w = workloads.prefill(rot_block=block)
+    else:
+        w = workloads.long70b() if workload == "long70b" else workloads.llama8b()
     k, v, ts, tp = w.prefill_tokens()
     c = kvq.Cache(w.d, w.H, w.P, w.NP, w.rot_kind, w.rot_block)
     kc, kp = c.new_pools(fill=0)
@@ -584,7 +589,7 @@ def main():
         compare()
         return
     if args.profile_case:
-        profile_case(args.profile_case, args.profile_block)
+        profile_case(args.profile_case, args.profile_block, args.profile_workload)
         return
     world, rank, local = dist_setup(args)
     try:
