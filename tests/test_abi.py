@@ -106,3 +106,48 @@ def test_host_validation_of_step_and_baseline(L):
                                         None) == MIS
     assert L.kvq_decode_fp16_workspace_bytes(ctypes.byref(d16), 0, 32, 100) == 0
 
+
+
+def _prototypes():
+    """name -> (return type, [parameter types]) parsed from include/kvq.h."""
+    text = open(os.path.join(ROOT, "include", "kvq.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    out = {}
+    for m in re.finditer(r"^\s*((?:const\s+)?[A-Za-z_]\w*\s*\**)\s*\b(kvq_\w+)\s*\(([^)]*)\)\s*;",
+                         text, flags=re.M):
+        ret, name, params = m.group(1).strip(), m.group(2), m.group(3).strip()
+        types = []
+        if params and params != "void":
+            for p in params.split(","):
+                p = " ".join(p.split())
+                ptr = p.count("*")
+                base = re.sub(r"\b(const)\b", "", p).replace("*", " ").split()
+                # drop the parameter name (the last identifier) when present
+                if len(base) > 1:
+                    base = base[:-1]
+                types.append((" ".join(base), ptr))
+        out[name] = (ret, types)
+    return out
+
+
+_CTYPE = {("int32_t", 0): ctypes.c_int32, ("int64_t", 0): ctypes.c_int64,
+          ("float", 0): ctypes.c_float, ("size_t", 0): ctypes.c_size_t, ("int", 0): ctypes.c_int}
+
+
+def test_binding_signatures_match_the_header():
+    protos = _prototypes()
+    assert set(protos) == set(declared_functions())
+    for name, (res, args) in kvq.SIGNATURES.items():
+        ret, params = protos[name]
+        assert len(params) == len(args), (name, len(params), len(args))
+        for i, ((base, ptr), a) in enumerate(zip(params, args)):
+            if ptr:
+                assert a in (ctypes.c_void_p, ctypes.c_char_p), (name, i, base, a)
+            else:
+                want = _CTYPE[(base, 0)]
+                assert ctypes.sizeof(a) == ctypes.sizeof(want), (name, i, base, a)
+                assert (a == ctypes.c_float) == (want == ctypes.c_float), (name, i, base, a)
+        if "*" in ret:
+            assert res in (ctypes.c_char_p, ctypes.c_void_p), name
+        else:
+            assert ctypes.sizeof(res) == ctypes.sizeof(_CTYPE[(ret.replace("const", "").strip(), 0)]), name
