@@ -151,3 +151,18 @@ def test_binding_signatures_match_the_header():
             assert res in (ctypes.c_char_p, ctypes.c_void_p), name
         else:
             assert ctypes.sizeof(res) == ctypes.sizeof(_CTYPE[(ret.replace("const", "").strip(), 0)]), name
+
+
+def test_cache_desc_mirrors_the_header_struct():
+    text = open(os.path.join(ROOT, "include", "kvq.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    body = re.search(r"typedef struct\s*\{(.*?)\}\s*kvq_cache_desc\s*;", text, flags=re.S).group(1)
+    fields = [f.split() for f in body.replace("*", " * ").split(";") if f.strip()]
+    names = [f[-1] for f in fields]
+    assert names == [n for n, _ in kvq.CacheDesc._fields_]
+    for f, (n, t) in zip(fields, kvq.CacheDesc._fields_):
+        if "*" in f:
+            assert t is ctypes.c_void_p, n
+        else:
+            assert f[-2] == "int32_t" and t is ctypes.c_int32, n
+    assert ctypes.sizeof(kvq.CacheDesc) == 32 and kvq.CacheDesc.quat.offset == 24
