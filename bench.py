@@ -29,6 +29,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import subprocess
 import sys
 import tempfile
@@ -166,18 +167,27 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+def source_code_hash(path):
+    """sha256 (16 hex digits) of a C/CUDA source with its comments, blank lines
+    and indentation removed: it changes with the code, not with its comments."""
+    text = open(path).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    code = "\n".join(" ".join(ln.split()) for ln in text.splitlines() if ln.strip())
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
+
+
 def kernel_traffic(kernel):
     """DRAM bytes per launch from the committed ncu summary, valid only while
-    the kernel's source is unchanged since the capture (else None)."""
+    the kernel's code is unchanged since the capture (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     d = json.load(open(path)).get(kernel)
     if not d:
         return None
-    src = os.path.join(ROOT, d["source"])
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    return float(d["bytes_per_launch"]) if h == d["source_sha256_16"] else None
+    h = source_code_hash(os.path.join(ROOT, d["source"]))
+    return float(d["bytes_per_launch"]) if h == d["source_code_sha256_16"] else None
 
 
 # ---------------------------------------------------------------- our arm

@@ -7,11 +7,17 @@
 // output is rotated back once per query head.
 //
 // One kernel, one warp per (sequence, KV head, split of the page range):
+//  0. For a fused decode step (kvq_decode_step) the warp that owns the page
+//     group of position seq_len - 1 first quantizes and writes that
+//     sequence's new K and V rows for its KV head, exactly as
+//     kvq_quantize_append would.
 //  1. The warp rotates its query heads in registers: lane (r, j) holds
 //     channels [j*d/4, (j+1)*d/4) of query head r (GP = 8) or r % 4 (GP = 4);
 //     butterfly stages inside a quarter run in registers, wider ones across
-//     lanes j by shuffles. Each rotated head is then held as a 30-bit fixed
-//     point qint = RN(qhat * 2^30 / amax), split into four signed 8-bit limbs.
+//     lanes j by shuffles. Each rotated head is then held as a fixed point
+//     qint = RN(qhat * 2^k), 2^k the power of two that brings the head's
+//     largest |qhat| just below 2^30 (so qhat * 2^k is exact in binary32),
+//     split into four signed 8-bit limbs.
 //  2. It streams its (page, KV head) chunks (codes + params of K and V,
 //     contiguous in the pool) into a 2-4 stage shared-memory ring with
 //     cp.async and runs both contractions on tensor cores (mma.sync):
@@ -19,14 +25,16 @@
 //             (head, limb)), B = the K codes as bytes (two lop3 per word,
 //             no unpacking to floats); the four limb dots recombine exactly
 //             into sum_i c_i qint_i, and the score
-//               z = sm_scale log2(e) (amax / 2^30) (s_k dot + m_k sum qint)
+//               z = sm_scale log2(e) 2^-k (s_k dot + m_k sum qint)
 //             is formed in double from exact integers;
 //       PV:   m16n8k16 f16 x f16 -> f32, A = V codes transposed (channels x
 //             tokens) as c - 8 (exact in binary16, built from nibbles with
 //             prmt/lop3), B = p * s_v split into binary16 hi + lo columns;
 //             each 16-token product joins the running sum through an IEEE
 //             round-to-nearest add, and sum p (m_v + 8 s_v) is added once at
-//             the end. Online softmax in base 2 (the running max in double).
+//             the end. Online softmax in base 2: the running max is binary32
+//             (only the exponent offset), each weight 2^(z - M) with the
+//             difference taken in double.
 //  3. It writes (acc, max, sum) per query head to the workspace, fences, and
 //     bumps a per-(sequence, KV head) counter; the warp that brings the
 //     counter to the number of splits merges all splits (log-sum-exp),

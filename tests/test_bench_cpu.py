@@ -48,3 +48,14 @@ def test_measured_arm_refuses_to_run_without_a_gpu():
     assert p.returncode != 0
     assert not [ln for ln in p.stdout.splitlines() if ln.startswith("{")]
     assert "needs a CUDA GPU" in p.stderr
+
+
+def test_traffic_hash_follows_code_not_comments(tmp_path):
+    import bench
+    a = tmp_path / "a.cu"
+    a.write_text("// header\nint f(int x) {\n  return x + 1;  // one\n}\n")
+    h = bench.source_code_hash(str(a))
+    a.write_text("/* another\n   header */\n\nint f(int x) {\n    return x + 1;\n}\n")
+    assert bench.source_code_hash(str(a)) == h         # comments and layout only
+    a.write_text("// header\nint f(int x) {\n  return x + 2;  // one\n}\n")
+    assert bench.source_code_hash(str(a)) != h         # a code change
