@@ -8,18 +8,23 @@
 // Rotations for LLM KV Cache Compression", Abstract (qL v conj(qR)).
 //
 // B200 design:
-//  * One thread owns E = min(d, 128) consecutive channels of one (token, head)
-//    row of K or V, so every butterfly stage of a block of up to 128 channels
-//    runs in registers without shuffles; d = 256 uses two threads per row and
-//    one xor-1 shuffle stage for b = 256.
-//  * A CTA of 384 threads owns a tile of TOK tokens x {K, V} x H heads. One
-//    elected thread fills the tile's shared-memory buffer with TMA tensor
-//    copies (cp.async.bulk.tensor.3d, boxes of 64 channels x H heads x TOK
-//    tokens, 128-byte swizzle so that every thread's 128-bit reads of its
-//    row are bank-conflict free) that complete on the buffer's mbarrier,
-//    while the previous tile is computed (two buffers). The grid is
-//    persistent: one CTA per SM walks the tiles. Waits on the mbarriers are
-//    bounded and end in KVQ_ERRF_TIMEOUT, never in a hang.
+//  * A thread owns E consecutive channels of one (token, head) row of K or V,
+//    E = 64 or 128 by configuration (append_e): 128 for Hadamard blocks of
+//    16 and 128 and for d = 256, 64 otherwise (two threads per d = 128 row,
+//    more warps per SM; one thread per row at d = 64). Every butterfly stage of a block that fits the
+//    thread runs in registers; only b = 256 at d = 256 crosses the thread
+//    pair, with one xor-1 shuffle stage.
+//  * A CTA (384 threads at E = 128, one per SM; 256 threads at E = 64, two
+//    per SM) owns a tile of TOK tokens x {K, V} x H heads. One elected thread
+//    fills the tile's shared-memory buffer with TMA tensor copies
+//    (cp.async.bulk.tensor.3d, boxes of 64 channels x H heads x TOK tokens,
+//    128-byte swizzle, so the 128-bit reads of consecutive rows spread over
+//    the banks) that complete on the buffer's mbarrier, while the previous
+//    tile is computed (two buffers). The grid is persistent and walks the
+//    tiles. Waits on the mbarriers are bounded and end in KVQ_ERRF_TIMEOUT,
+//    never in a hang.
+//  * Batches of at most 8192 rows (a decode step's one token per sequence)
+//    go to append_rows_kernel instead: a warp per row, the same arithmetic.
 //  * Threads are ordered token-major, head-minor, so a warp's rows are
 //    consecutive lines of the swizzled boxes, and the destination of each
 //    row (token -> sequence, position -> block table) is resolved one tile
