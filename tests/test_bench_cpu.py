@@ -59,3 +59,23 @@ def test_traffic_hash_follows_code_not_comments(tmp_path):
     assert bench.source_code_hash(str(a)) == h         # comments and layout only
     a.write_text("// header\nint f(int x) {\n  return x + 2;  // one\n}\n")
     assert bench.source_code_hash(str(a)) != h         # a code change
+
+
+def test_reference_arm_under_torchrun_prints_once():
+    # the driver launches every N > 1 arm through torch.distributed.run; on
+    # the host the ranks join over gloo, rank 0 alone runs the oracle and
+    # prints, the others leave without work, and every rank exits 0
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    p = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+                        "--nproc-per-node", "2", "--master-addr", "127.0.0.1", "--master-port",
+                        str(port), os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--gpus", "2", "--steps", "2", "--warmup", "3"],
+                       cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert p.returncode == 0, p.stderr[-2000:]
+    lines = [ln for ln in p.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
