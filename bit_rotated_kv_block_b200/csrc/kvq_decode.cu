@@ -750,6 +750,9 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, (D == 128 && GP == 4) ? 4 :
   }
   last = __shfl_sync(0xffffffffu, last, 0);
   if (!last) return;
+  // the shuffle carries no memory ordering: the warp barrier extends lane
+  // 0's acquire to every lane before they read the other splits' partials
+  __syncwarp();
   const bool owner = head_ok && !lo_row;
   // lanes of head hr: quarter j of the channels; for GP = 4 the partner
   // lanes r + 4 take the odd splits and the two halves are added at the end

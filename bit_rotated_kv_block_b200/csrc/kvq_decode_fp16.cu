@@ -330,6 +330,7 @@ __global__ void __launch_bounds__(kF16Warps * kWarp)
   }
   last = __shfl_sync(0xffffffffu, last, 0);
   if (!last) return;
+  __syncwarp();  // extends lane 0's acquire to the lanes that read the partials
   // lane l: query head l / (32 / GP) of the group, channels of its share
   constexpr int LPH = kWarp / GP;  // lanes per head (8 or 4)
   constexpr int CW = D / LPH;      // channels per lane

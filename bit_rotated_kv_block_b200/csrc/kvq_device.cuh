@@ -222,6 +222,13 @@ __device__ __forceinline__ __half2 u32_as_h2(uint32_t u) {
   return *reinterpret_cast<__half2*>(&u);
 }
 
+// INT4 -> binary16 by the exponent-bias ("magic number") method published for
+// weight-only INT4 GEMM kernels (Kim et al., "Who Says Elephants Can't Run:
+// Bringing Large Scale MoE Models into Cloud Scale Production", 2022): OR-ing
+// a nibble into the mantissa of the binary16 value 1024 (0x6400) with one
+// three-input logic operation gives 1024 + c exactly, and one subtraction or
+// fused multiply-add removes the bias. The constants follow from the binary16
+// format.
 // The four nibbles of each 16-bit half of z as half2 (code - 8), exact:
 // out[k] = half2(nibble k of the low half, nibble k of the high half). Nibbles
 // 0 and 2 land at 1024 + c (mantissa bits 0-3) and lose 1032; nibbles 1 and 3

@@ -10,6 +10,7 @@
 // into the library: every GPU that loads libkvq holds kNoallocScratchBytes of
 // it until the process exits, and no call allocates or frees anything.
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -27,22 +28,60 @@ static_assert(kNoallocScratchBytes % 256 == 0, "scratch size must keep 256-byte 
 // The scratch itself: zero at module load, shared by every call on a device.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoallocScratchBytes];
 
-// Device address of the array per device, looked up once with that device
-// current (in host code the array's name is only a host-side stand-in).
-static void* g_scratch_addr[64] = {nullptr};
+// In host code the array's name is only a host-side stand-in: its device
+// address is looked up (cudaGetSymbolAddress) with the device current and
+// remembered per device together with the unique id of the CUDA context it
+// belongs to. A device reset, or a caller running in another context of the
+// same device, gives a new id, and the address is looked up again instead of
+// reusing one from a context that no longer holds the array.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+static void* driver_entry(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return p;
+}
+
+// Unique id of the calling thread's current context; false if there is none
+// yet (the runtime creates it on its first use) or the driver lacks the call.
+static bool current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_ctx = reinterpret_cast<CtxGetCurrentFn>(driver_entry("cuCtxGetCurrent"));
+  static CtxGetIdFn get_id = reinterpret_cast<CtxGetIdFn>(driver_entry("cuCtxGetId"));
+  if (get_ctx == nullptr || get_id == nullptr) return false;
+  CUcontext ctx = nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+constexpr int kMaxDevices = 64;
+struct ScratchSlot {
+  unsigned long long ctx_id;  // context the address belongs to
+  bool known;                 // ctx_id is valid
+  void* addr;
+};
+static ScratchSlot g_scratch[kMaxDevices] = {};
 static std::mutex g_scratch_mu;
 
 static int scratch_address(void** out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return KVQ_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KVQ_ERR_CUDA;
+  unsigned long long id = 0;
+  const bool have_id = current_context_id(&id);
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
+  ScratchSlot& sl = g_scratch[dev];
+  if (sl.addr == nullptr || !have_id || !sl.known || sl.ctx_id != id) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
       return KVQ_ERR_CUDA;
-    g_scratch_addr[dev] = p;
+    sl.addr = p;
+    // the lookup made the runtime's context current if there was none
+    sl.known = current_context_id(&sl.ctx_id);
   }
-  *out = g_scratch_addr[dev];
+  *out = sl.addr;
   return KVQ_OK;
 }
 

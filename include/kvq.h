@@ -70,8 +70,12 @@ typedef enum {
 #define KVQ_ERRF_POS 2  /* position < 0 or position/page_size >= bt_stride       */
 #define KVQ_ERRF_SEQ 4  /* token's sequence index >= num_seqs                    */
 #define KVQ_ERRF_LEN 8  /* seq_lens[s] < 0, > max_seq_len, or past the table      */
-#define KVQ_ERRF_TIMEOUT 16 /* a bounded wait for an asynchronous copy expired; the
-                               affected tile was skipped (never expected)          */
+#define KVQ_ERRF_TIMEOUT 16 /* a bounded wait for an asynchronous copy expired (never
+                               expected). Copies of that launch may still have been in
+                               flight when its blocks returned: every output of the
+                               launch is then undefined and the caller should discard
+                               the whole batch (pool bytes outside the batch's slots
+                               are still untouched).                               */
 
 /* Geometry of one paged cache (both pools share it).
  *  head_dim     d: 64, 128 or 256.
@@ -269,8 +273,11 @@ int kvq_paged_decode_attn_fp16(const kvq_cache_desc* desc, int32_t num_seqs,
  *    KVQ_NOALLOC_SCRATCH_BYTES are rejected with KVQ_ERR_WORKSPACE before
  *    anything is launched.
  *  - The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress, once per device, with that device current); make
- *    that first call before any stream capture on the device.
+ *    (cudaGetSymbolAddress, with that device current) and keeps it for that
+ *    device's current CUDA context; a call in a context not seen before
+ *    (after a device reset, or from a non-primary context) looks it up
+ *    again. Make the first call on each device and context before any
+ *    stream capture there.
  *  - All calls on a device share the one array and it keeps the last call's
  *    contents: calls that overlap on the GPU (different streams, or
  *    different host threads without ordering) race and give wrong results.

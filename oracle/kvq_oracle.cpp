@@ -316,9 +316,12 @@ void orc_quantize_append(int d, int H, int P, int NP, int rot_kind, int rot_bloc
                          const int32_t* block_table, int bt_stride, uint8_t* k_codes,
                          uint16_t* k_params, uint8_t* v_codes, uint16_t* v_params,
                          int32_t* err) {
+  // Tokens are independent (each writes only its own slot), so they are
+  // spread over threads; the arithmetic of every row is unchanged.
   int32_t flags = 0;
-  std::vector<float> row(d);
+#pragma omp parallel for schedule(static) reduction(| : flags)
   for (int t = 0; t < T; ++t) {
+    std::vector<float> row(d);
     const int seq = token_seq[t];
     if (seq < 0) continue;
     if (seq >= num_seqs) { flags |= ORC_ERR_SEQ; continue; }

@@ -83,3 +83,24 @@ def fill_workload(w, seqs=None, layer=0, oracle_too=True, fill=0xAA):
     e, oe = p.append(k, v, ts, tp, w.block_table, oracle_too=oracle_too)
     assert e == 0 and oe == 0
     return p, (k, v, ts, tp)
+
+
+def fused_step_vs_oracle(p, k_new, v_new, lens, table, q, sm_scale):
+    """kvq_decode_step on p's GPU pools; the oracle's append of the same new
+    tokens (token_seq = s, token_pos = lens[s] - 1; sequences with lens 0 skip)
+    followed by its attention on p's oracle pools. Returns (GPU out, oracle
+    out, GPU flags, oracle flags); the caller compares pools and outputs."""
+    L = int(lens.max())
+    S = len(lens)
+    keep = lens >= 1
+    ts = np.where(keep, np.arange(S, dtype=np.int32), -1).astype(np.int32)
+    tp = np.maximum(lens - 1, 0).astype(np.int32)
+    p.err.zero_()
+    out = kvq.decode_step(p.gpu, dev(q), dev(k_new), dev(v_new), dev(lens.astype(np.int32)), L,
+                          dev(table.astype(np.int32)), p.kc, p.kp, p.vc, p.vp, sm_scale=sm_scale,
+                          err=p.err)
+    torch.cuda.synchronize()
+    oe = oracle.quantize_append(p.orc, k_new.view(np.uint16), v_new.view(np.uint16), ts, tp, table,
+                                p.okc, p.okp.reshape(p.orc.NP, p.orc.H, p.orc.P, 2), p.ovc, p.ovp)
+    ref, oe2 = p.oracle_attention(q, lens, L, table, sm_scale)
+    return out.cpu().numpy().astype(np.float64), ref, int(p.err.item()), oe | oe2

@@ -53,7 +53,7 @@ def test_golden_rows_on_gpu():
     # head_dim 64 (tiling keeps the row minimum and maximum)
     g = read_golden("quant_rows_hand.txt")
     for row, kind, b in (("row1", kvq.ROT_NONE, 0), ("row2", kvq.ROT_HADAMARD, 16),
-                         ("row3", kvq.ROT_NONE, 0)):
+                         ("row3", kvq.ROT_NONE, 0), ("row4", kvq.ROT_HADAMARD, 16)):
         x = np.array([float(t) for t in g[row + "_x"].split()], np.float16)
         k = np.tile(x, 4).reshape(1, 1, 64)
         p = Pair(64, 1, 16, 2, kind, b)

@@ -10,7 +10,7 @@ import pytest
 import torch
 
 from bit_rotated_kv_block_b200 import kvq, workloads
-from gpu_helpers import Pair, fill_workload
+from gpu_helpers import Pair, fill_workload, fused_step_vs_oracle
 
 pytestmark = pytest.mark.gpu
 
@@ -46,20 +46,29 @@ def test_llama8b_full_step():
 
 
 @pytest.mark.parametrize("rot", [workloads.ROT_HADAMARD, workloads.ROT_NONE])
-def test_long70b_sampled(rot):
-    # full 8 x 32768 cache on the GPU (pools checked bit-exact); the oracle
-    # attends for two of the sequences
+def test_long70b_full(rot):
+    # the full 8 x 32768 cache (pools checked bit-exact); every sequence and
+    # query head of the one decode launch against the oracle
     w = workloads.long70b(rot_kind=rot)
     p, _ = fill_workload(w)
     p.assert_pools_equal()
-    q = w.queries()
-    out, e = p.gpu_attention(q, w.seq_lens, int(w.seq_lens.max()), w.block_table,
-                             1 / math.sqrt(w.d))
-    assert e == 0
-    for s in (0, 5):
-        ref, _ = p.oracle_attention(q[s:s + 1], w.seq_lens[s:s + 1], int(w.seq_lens.max()),
-                                    w.block_table[s:s + 1], 1 / math.sqrt(w.d))
-        assert np.max(np.abs(out[s] - ref[0])) <= TOL
+    check(p, w.queries(), w.seq_lens, int(w.seq_lens.max()), w.block_table,
+          1 / math.sqrt(w.d))
+
+
+def test_long70b_full_fused_step():
+    # 8 x 32767 cached tokens, then one fused step writes token 32768 of every
+    # sequence (the last slot of its last page) and attends over 32768
+    w = workloads.long70b(ctx=32767)
+    p, _ = fill_workload(w)
+    k_new, v_new, _, _ = w.step_tokens(0)
+    lens = (w.seq_lens + 1).astype(np.int32)
+    assert int(lens.max()) == 32768
+    out, ref, e, oe = fused_step_vs_oracle(p, k_new, v_new, lens, w.block_table, w.queries(),
+                                           1 / math.sqrt(w.d))
+    assert e == 0 and oe == 0
+    p.assert_pools_equal()
+    assert np.max(np.abs(out - ref)) <= TOL
 
 
 @pytest.mark.parametrize("rot", [workloads.ROT_HADAMARD, workloads.ROT_QUAT])

@@ -10,7 +10,7 @@ import pytest
 import torch
 
 from bit_rotated_kv_block_b200 import kvq, workloads
-from gpu_helpers import Pair, dev, fill_workload
+from gpu_helpers import Pair, dev, fill_workload, fused_step_vs_oracle
 
 pytestmark = pytest.mark.gpu
 
@@ -108,13 +108,12 @@ def test_new_token_page_outside_pool_is_flagged():
     assert int(p.err.item()) & kvq.ERRF_PAGE
 
 
-def test_llama8b_full_size_step_matches_two_calls():
+def test_llama8b_full_size_step_matches_two_calls_and_oracle():
     # the bench's workload and launch configuration: 32 sequences x 4096
     # cached tokens, one new token each; the fused step and the two-call path
-    # leave identical pools and outputs (the two-call path is checked against
-    # the oracle at this size in test_gpu_decode.py)
+    # leave identical pools and outputs, and both equal the oracle's
     w = workloads.llama8b()
-    p, _ = fill_workload(w, oracle_too=False)
+    p, _ = fill_workload(w)
     k_new, v_new, ts, tp = w.step_tokens(0)
     lens = (w.seq_lens + 1).astype(np.int32)
     L = int(lens.max())
@@ -123,10 +122,11 @@ def test_llama8b_full_size_step_matches_two_calls():
     bt = dev(w.block_table)
     kvq.quantize_append(p.gpu, dev(k_new), dev(v_new), dev(ts), dev(tp), bt, kc2, kp2, vc2, vp2)
     out2 = kvq.paged_decode_attn(p.gpu, q, dev(lens), L, bt, kc2, kp2, vc2, vp2)
-    out1 = kvq.decode_step(p.gpu, q, dev(k_new), dev(v_new), dev(lens), L, bt, p.kc, p.kp, p.vc,
-                           p.vp, err=p.err)
-    torch.cuda.synchronize()
-    assert int(p.err.item()) == 0
+    out1, ref, e, oe = fused_step_vs_oracle(p, k_new, v_new, lens, w.block_table, w.queries(),
+                                            1 / math.sqrt(w.d))
+    assert e == 0 and oe == 0
     for a, b in ((p.kc, kc2), (p.kp, kp2), (p.vc, vc2), (p.vp, vp2)):
         assert torch.equal(a, b)
-    assert torch.equal(out1, out2)
+    assert np.array_equal(out1, out2.cpu().numpy().astype(np.float64))
+    p.assert_pools_equal()
+    assert np.max(np.abs(out1 - ref)) <= TOL

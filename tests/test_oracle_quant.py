@@ -2,7 +2,7 @@
 placement ("SAW-INT4" Summary/Method: token-wise INT4 fused into paged
 KV-cache layouts).
 
-Pins: two hand-worked rows (golden fixture, worked in exact rationals), a
+Pins: four hand-worked rows (golden fixture, worked in exact rationals), a
 constant row, the nearest-level property by brute force over all 16 levels,
 the range guarantee x in [m16, m16 + 15 s16], the error bound
 |x - xhat| <= s16 (1/2 + 64 * 2^-24), argmin -> 0 and argmax -> 15, the
@@ -22,7 +22,7 @@ def _hex_bytes(s):
     return np.array([int(t, 16) for t in s.split()], np.uint8)
 
 
-@pytest.mark.parametrize("row", ["row1", "row2", "row3"])
+@pytest.mark.parametrize("row", ["row1", "row2", "row3", "row4"])
 def test_hand_worked_rows(row):
     g = read_golden("quant_rows_hand.txt")
     x = np.array([float(t) for t in g[row + "_x"].split()], np.float32)
