@@ -46,6 +46,7 @@ METRIC = "INT4 paged decode-attn tokens/s (append + decode step, one layer)"
 UNIT = "tokens/s"
 BYTES_PER_TOKEN_HEAD = 136  # decode: 2 * (64 code bytes + 4 param bytes), head_dim 128
 APPEND_BYTES_PER_TOKEN_HEAD = 648  # append: 2 * 256 B read + 2 * 68 B written
+NOMINAL_HBM_GBS = 8000.0  # the B200's nominal HBM bandwidth, for the second set of fractions
 
 
 def parse():
@@ -56,6 +57,9 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the per-workload records (long-context decode, prefill sweep, "
+                         "ragged head_dim-256 step) that a one-GPU run adds to the line")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
     ap.add_argument("--compare", action="store_true",
                     help="print one JSON line with the baseline comparisons (long-context INT4 with "
@@ -342,8 +346,10 @@ def run_ours(args, world, rank, local):
                    "l2": "steps alternate between 2 cache replicas (2 x 143 MB > 126 MB L2)"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic, "kernel": "decode attention",
-                     "bytes_per_launch": dec_bytes, "peak_source": peak_kind},
+                     "bytes_per_launch": dec_bytes, "peak_source": peak_kind,
+                     "frac_nominal": achieved / NOMINAL_HBM_GBS},
         "append_prefill": {"gbs": app_bytes / t_app / 1e9, "frac": app_bytes / t_app / 1e9 / peak,
+                           "frac_nominal": app_bytes / t_app / 1e9 / NOMINAL_HBM_GBS,
                            "us": t_app * 1e6, "bytes": app_bytes, "tokens": len(ts)},
         "decode": {"us": t_dec * 1e6, "kv_tokens_per_s": S * L / t_dec,
                    "gbs": achieved},
@@ -352,6 +358,11 @@ def run_ours(args, world, rank, local):
         "gpu_launches": launches_per_step * steps,
         "clocks": clk,
     }
+    if world == 1 and not args.no_workloads:
+        # outside the timed region: the other workloads' kernels, each timed alone
+        del caches, ws
+        torch.cuda.empty_cache()
+        line["workloads"] = workload_records(device, args.seed)
     return line, w
 
 
@@ -398,22 +409,53 @@ def oracle_step_sample(w, n_heads_budget, seed_rank=0):
     return run, nh / w.Hq
 
 
+def cpu_model():
+    """The host CPU's model name (lscpu, else /proc/cpuinfo)."""
+    try:
+        out = subprocess.run(["lscpu"], capture_output=True, text=True, timeout=10).stdout
+        for line in out.splitlines():
+            if line.startswith("Model name:"):
+                return line.split(":", 1)[1].strip()
+    except (OSError, subprocess.SubprocessError):
+        pass
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 def cpu_baseline(w, budget_s):
+    """The oracle timed on the host cores on a bounded sample, with OpenMP on
+    every core and again on one thread."""
     import oracle
     run, frac = oracle_step_sample(w, w.Hq)
-    t = time.perf_counter()
-    run()
-    one = time.perf_counter() - t
-    reps = max(1, int(budget_s / max(one, 1e-3)))
-    t = time.perf_counter()
-    for _ in range(reps):
+
+    def timed(budget):
+        t = time.perf_counter()
         run()
-    el = time.perf_counter() - t
-    return {"value": reps * frac / el, "unit": UNIT, "cores": oracle.num_threads(),
+        one = time.perf_counter() - t
+        reps = max(1, int(budget / max(one, 1e-3)))
+        t = time.perf_counter()
+        for _ in range(reps):
+            run()
+        return reps, time.perf_counter() - t
+
+    cores = oracle.num_threads()
+    reps, el = timed(budget_s)
+    oracle.set_num_threads(1)
+    try:
+        reps1, el1 = timed(budget_s / 2)
+    finally:
+        oracle.set_num_threads(cores)
+    return {"value": reps * frac / el, "unit": UNIT, "cores": cores,
+            "value_1thread": reps1 * frac / el1, "cpu_model": cpu_model(),
             "kind": "oracle",
-            "sample": f"{reps} x (append of 1 token + decode attention of 1 sequence x "
-                      f"{int(frac * w.Hq)} query heads over {int(w.seq_lens[0]) + 1} INT4 "
-                      f"tokens), fp64 attention, OpenMP over heads"}
+            "sample": f"{reps} (all cores) and {reps1} (1 thread) x (append of 1 token + decode "
+                      f"attention of 1 sequence x {int(frac * w.Hq)} query heads over "
+                      f"{int(w.seq_lens[0]) + 1} INT4 tokens), fp64 attention, OpenMP over heads"}
 
 
 def run_reference(args, world, rank):
@@ -508,73 +550,118 @@ def _device_time_us(fn, n=20):
     return float(np.median(ts)) * 1e3
 
 
-def compare():
-    """Baselines on one GPU: the long-context 70B-shaped decode (8 x 32768
-    tokens, GQA 8, page 32) over INT4 pages with Hadamard b 128, over INT4
-    pages without rotation, and over binary16 pages; then the bulk prefill
-    append of one layer (65536 tokens x 8 heads) per Hadamard block size with
-    the reconstruction MSE of the INT4 cache (GPU dequantization, un-rotated,
-    against the fp16 input). Two replicas of every cache alternate (> L2)."""
+def _device_kv(w, T, gen, device):
+    """K and V [T][H][d] binary16 of a workload's shape and value structure
+    (N(0,1) draws times its per-(head, channel) multipliers), drawn on the
+    device so that the large workloads need no host-side generation. Timing
+    only: the parity tests use the seeded host draws."""
+    mult = (torch.ones((w.H, w.d)) if w.channel_mult is None
+            else torch.from_numpy(w.channel_mult)).to(device)
+    out = []
+    for _ in range(2):
+        x = torch.empty((T, w.H, w.d), dtype=torch.float16, device=device)
+        for t0 in range(0, T, 1 << 16):
+            t1 = min(T, t0 + (1 << 16))
+            x[t0:t1] = (torch.randn((t1 - t0, w.H, w.d), generator=gen, device=device)
+                        * mult).half()
+        out.append(x)
+    return out
+
+
+def _all_tokens(w):
+    """(token_seq, token_pos) of every cached token, sequence-major."""
+    lens = w.seq_lens.astype(np.int64)
+    ts = np.repeat(np.arange(w.S, dtype=np.int32), lens)
+    tp = np.concatenate([np.arange(n, dtype=np.int32) for n in lens])
+    return ts, tp
+
+
+def _rate(nbytes, us, peak):
+    gbs = nbytes / us / 1e3
+    return {"us": us, "gbs": gbs, "frac": gbs / peak, "frac_nominal": gbs / NOMINAL_HBM_GBS,
+            "bytes": int(nbytes)}
+
+
+def workload_records(device, seed=0):
+    """The other workloads on one GPU, each timed by CUDA events (median of 5
+    rounds of back-to-back launches; every launch reads more than the 126 MB
+    L2, or alternates between two cache replicas that together do):
+
+    * long-context 70B-shaped decode (8 x 32768 tokens, GQA 8, page 32) over
+      INT4 pages with Hadamard b 128, over INT4 pages without rotation, and
+      over binary16 pages (the full-precision baseline);
+    * the bulk prefill append of one layer (65536 tokens x 8 KV heads) per
+      Hadamard block size and without rotation, with the reconstruction MSE
+      of the INT4 cache (GPU dequantization, un-rotated, against the input);
+    * the ragged head_dim-256 workload (128 sequences, lengths 512-16384):
+      one fused decode step (append + attention) with Hadamard b 256 and with
+      the quaternion rotation.
+    """
     from bit_rotated_kv_block_b200 import kvq, workloads
-    torch.cuda.set_device(0)
-    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
-    res = {"workload_decode": "8 seqs x 32768 tokens, 8 KV heads, 64 q heads, d 128, page 32",
-           "workload_append": "65536 tokens x 8 KV heads x d 128 per layer, page 16"}
+    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(device)
     peak, _ = measured_peaks()
-    w = workloads.long70b()
-    k, v, ts, tp = w.prefill_tokens()
-    K, V, TS, TP, BT = dev(k), dev(v), dev(ts), dev(tp), dev(w.block_table)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    res = {}
+
+    # ---- long-context 70B-shaped decode
+    w = workloads.long70b(seed=seed)
+    ts, tp = _all_tokens(w)
+    K, V = _device_kv(w, len(ts), gen, device)
+    TS, TP, BT = dev(ts), dev(tp), dev(w.block_table)
     q, lens, L = dev(w.queries()), dev(w.seq_lens), int(w.seq_lens.max())
-    out = torch.empty((w.S, w.Hq, w.d), dtype=torch.float32, device="cuda")
+    out = torch.empty((w.S, w.Hq, w.d), dtype=torch.float32, device=device)
     n_th = int(w.seq_lens.sum()) * w.H
-    for rot, blk in ((workloads.ROT_HADAMARD, 128), (workloads.ROT_NONE, 0)):
+    rec = {"workload": "8 seqs x 32768 tokens, 8 KV heads, 64 q heads, d 128, page 32"}
+    for rot, blk, name in ((workloads.ROT_HADAMARD, 128, "int4_hadamard128"),
+                           (workloads.ROT_NONE, 0, "int4_no_rotation")):
         reps = []
         for _ in range(2):
-            c = kvq.Cache(w.d, w.H, w.P, w.NP, rot, blk)
-            kc, kp = c.new_pools(fill=0)
-            vc, vp = c.new_pools(fill=0)
+            c = kvq.Cache(w.d, w.H, w.P, w.NP, rot, blk, device=device)
+            kc, kp = c.new_pools(device=device, fill=0)
+            vc, vp = c.new_pools(device=device, fill=0)
             kvq.quantize_append(c, K, V, TS, TP, BT, kc, kp, vc, vp)
             reps.append((c, kc, kp, vc, vp))
         ws = torch.zeros(kvq.decode_workspace_bytes(reps[0][0], w.S, w.Hq, L), dtype=torch.uint8,
-                         device="cuda")
+                         device=device)
         t = _device_time_us(lambda i: kvq.paged_decode_attn(
             reps[i % 2][0], q, lens, L, BT, *reps[i % 2][1:], out=out, workspace=ws))
-        gbs = n_th * 136 / t / 1e3
-        res["decode_int4_" + ("hadamard128" if blk else "no_rotation")] = {
-            "us": t, "gbs": gbs, "frac": gbs / peak, "bytes": n_th * 136}
+        rec[name] = _rate(n_th * BYTES_PER_TOKEN_HEAD, t, peak)
         del reps, ws
     page = BT[TS.long(), (TP // w.P).long()].long()
     slot = (TP % w.P).long()
     reps = []
     for _ in range(2):
-        kp16 = torch.zeros((w.NP, w.H, w.P, w.d), dtype=torch.float16, device="cuda")
+        kp16 = torch.zeros((w.NP, w.H, w.P, w.d), dtype=torch.float16, device=device)
         vp16 = torch.zeros_like(kp16)
         kp16[page, :, slot, :] = K
         vp16[page, :, slot, :] = V
         reps.append((kp16, vp16))
-    c16 = kvq.Cache(w.d, w.H, w.P, w.NP, workloads.ROT_NONE, 0)
+    c16 = kvq.Cache(w.d, w.H, w.P, w.NP, workloads.ROT_NONE, 0, device=device)
     ws = torch.zeros(kvq.decode_fp16_workspace_bytes(c16, w.S, w.Hq, L), dtype=torch.uint8,
-                     device="cuda")
+                     device=device)
     t = _device_time_us(lambda i: kvq.paged_decode_attn_fp16(
         c16, q, lens, L, BT, reps[i % 2][0], reps[i % 2][1], out=out, workspace=ws))
-    gbs = n_th * 512 / t / 1e3
-    res["decode_fp16_baseline"] = {"us": t, "gbs": gbs, "frac": gbs / peak, "bytes": n_th * 512}
-    res["rotation_overhead_decode"] = (res["decode_int4_hadamard128"]["us"] /
-                                       res["decode_int4_no_rotation"]["us"] - 1)
-    del reps, ws, K, V, page, slot
+    rec["fp16_baseline"] = _rate(n_th * 512, t, peak)
+    rec["rotation_overhead"] = rec["int4_hadamard128"]["us"] / rec["int4_no_rotation"]["us"] - 1
+    rec["speedup_vs_fp16"] = rec["fp16_baseline"]["us"] / rec["int4_hadamard128"]["us"]
+    res["long70b_decode"] = rec
+    del reps, ws, K, V, page, slot, TS, TP
     torch.cuda.empty_cache()
 
-    sweep = {}
+    # ---- prefill sweep: one layer per Hadamard block size
+    sweep = {"workload": "65536 tokens x 8 KV heads x d 128 per layer, page 16"}
     for blk in (16, 32, 64, 128, 0):
-        w = workloads.prefill(rot_block=blk)
-        k, v, ts, tp = w.prefill_tokens()
-        K, V, TS, TP, BT = dev(k), dev(v), dev(ts), dev(tp), dev(w.block_table)
-        c = kvq.Cache(w.d, w.H, w.P, w.NP, w.rot_kind, w.rot_block)
-        kc, kp = c.new_pools(fill=0)
-        vc, vp = c.new_pools(fill=0)
+        w = workloads.prefill(seed=seed, rot_block=blk)
+        ts, tp = _all_tokens(w)
+        K, V = _device_kv(w, len(ts), gen, device)
+        TS, TP, BT = dev(ts), dev(tp), dev(w.block_table)
+        c = kvq.Cache(w.d, w.H, w.P, w.NP, w.rot_kind, w.rot_block, device=device)
+        kc, kp = c.new_pools(device=device, fill=0)
+        vc, vp = c.new_pools(device=device, fill=0)
         t = _device_time_us(lambda i: kvq.quantize_append(c, K, V, TS, TP, BT, kc, kp, vc, vp),
                             n=10)
-        byts = len(ts) * w.H * APPEND_BYTES_PER_TOKEN_HEAD
+        r = _rate(len(ts) * w.H * APPEND_BYTES_PER_TOKEN_HEAD, t, peak)
         lens = dev(np.full(w.S, int(w.seq_lens[0]), np.int32))
         Lmax = int(w.seq_lens[0])
         mse = 0.0
@@ -583,14 +670,51 @@ def compare():
             x = src.view(w.S, Lmax, w.H, w.d).double()
             mse += float(((xh.double() - x) ** 2).mean()) / 2
             del xh, x
-        sweep["hadamard%d" % blk if blk else "no_rotation"] = {
-            "us": t, "gbs": byts / t / 1e3, "frac": byts / t / 1e3 / peak, "mse": mse}
+        r["mse"] = mse
+        sweep["hadamard%d" % blk if blk else "no_rotation"] = r
         del K, V, kc, kp, vc, vp
         torch.cuda.empty_cache()
-    res["append_prefill_sweep"] = sweep
-    res["rotation_overhead_append_b128"] = sweep["hadamard128"]["us"] / sweep["no_rotation"]["us"] - 1
+    for blk in (16, 32, 64, 128):
+        sweep["hadamard%d" % blk]["rotation_overhead"] = (
+            sweep["hadamard%d" % blk]["us"] / sweep["no_rotation"]["us"] - 1)
+    res["prefill_append_sweep"] = sweep
+
+    # ---- ragged head_dim 256: one fused decode step over the whole batch
+    rec = {"workload": "128 seqs, lengths U[512, 16384], 4 KV heads, 16 q heads, d 256, page 16"}
+    for rot, name in ((workloads.ROT_HADAMARD, "hadamard256"), (workloads.ROT_QUAT, "quaternion")):
+        w = workloads.ragged256(seed=seed, rot_kind=rot)
+        ts, tp = _all_tokens(w)
+        K, V = _device_kv(w, len(ts), gen, device)
+        c = kvq.Cache(w.d, w.H, w.P, w.NP, w.rot_kind, w.rot_block, w.quat, device=device)
+        kc, kp = c.new_pools(device=device, fill=0)
+        vc, vp = c.new_pools(device=device, fill=0)
+        BT = dev(w.block_table)
+        kvq.quantize_append(c, K, V, dev(ts), dev(tp), BT, kc, kp, vc, vp)
+        del K, V
+        kn = torch.randn((w.S, w.H, w.d), generator=gen, device=device).half()
+        vn = torch.randn((w.S, w.H, w.d), generator=gen, device=device).half()
+        lens_np = (w.seq_lens + 1).astype(np.int32)
+        lens, L = dev(lens_np), int(lens_np.max())
+        q = dev(w.queries())
+        out = torch.empty((w.S, w.Hq, w.d), dtype=torch.float32, device=device)
+        ws = torch.zeros(kvq.decode_workspace_bytes(c, w.S, w.Hq, L), dtype=torch.uint8,
+                         device=device)
+        t = _device_time_us(lambda i: kvq.decode_step(c, q, kn, vn, lens, L, BT, kc, kp, vc, vp,
+                                                      out=out, workspace=ws))
+        n_tok = int(lens_np.sum())
+        r = _rate(n_tok * w.H * (w.d + 8), t, peak)
+        r["kv_tokens"] = n_tok
+        rec["step_" + name] = r
+        del kc, kp, vc, vp, ws
+        torch.cuda.empty_cache()
+    res["ragged256_step"] = rec
     res["peak_gbs"] = peak
-    print(json.dumps({"mode": "compare", **res}), flush=True)
+    res["nominal_gbs"] = NOMINAL_HBM_GBS
+    return res
+
+
+def compare():
+    print(json.dumps({"mode": "compare", **workload_records(torch.device("cuda", 0))}), flush=True)
 
 
 def main():

@@ -8,33 +8,34 @@
 //
 // One kernel, one warp per (sequence, KV head, split of the page range):
 //  0. For a fused decode step (kvq_decode_step) the warp that owns the page
-//     group of position seq_len - 1 first quantizes and writes that
-//     sequence's new K and V rows for its KV head, exactly as
-//     kvq_quantize_append would.
+//     of position seq_len - 1 first quantizes and writes that sequence's new
+//     K and V rows for its KV head, exactly as kvq_quantize_append would.
 //  1. The warp rotates its query heads in registers: lane (r, j) holds
 //     channels [j*d/4, (j+1)*d/4) of query head r (GP = 8) or r % 4 (GP = 4);
 //     butterfly stages inside a quarter run in registers, wider ones across
 //     lanes j by shuffles. Each rotated head is then held as a fixed point
 //     qint = RN(qhat * 2^k), 2^k the power of two that brings the head's
-//     largest |qhat| just below 2^30 (so qhat * 2^k is exact in binary32),
-//     split into four signed 8-bit limbs.
-//  2. It streams its (page, KV head) chunks (codes + params of K and V,
-//     contiguous in the pool) into a 2-4 stage shared-memory ring with
-//     cp.async and runs both contractions on tensor cores (mma.sync):
+//     largest |qhat| just below 2^26 (so qhat * 2^k is exact in binary32),
+//     split into four signed 8-bit limbs (even channels as 16 qint).
+//  2. The sequence's pages are dealt out to its splits as contiguous ranges
+//     of near-equal size. The warp streams its (page, KV head) chunks (codes
+//     + params of K and V, contiguous in the pool) into a 2-4 stage
+//     shared-memory ring with cp.async and runs both contractions on tensor
+//     cores (mma.sync):
 //       QK^T: m16n8k32 s8 x u8 -> s32, A = the query limbs (one row per
-//             (head, limb)), B = the K codes as bytes (two lop3 per word,
-//             no unpacking to floats); the four limb dots recombine exactly
-//             into sum_i c_i qint_i, and the score
+//             (head, limb)), B = the K codes as bytes (even channels c, odd
+//             channels 16 c, one AND per word each); the limb dots
+//             recombine exactly into 16 sum_i c_i qint_i, and the score
 //               z = sm_scale log2(e) 2^-k (s_k dot + m_k sum qint)
-//             is formed in double from exact integers;
+//             is formed in binary32;
 //       PV:   m16n8k16 f16 x f16 -> f32, A = V codes transposed (channels x
-//             tokens) as c - 8 (exact in binary16, built from nibbles with
-//             prmt/lop3), B = p * s_v split into binary16 hi + lo columns;
-//             each 16-token product joins the running sum through an IEEE
-//             round-to-nearest add, and sum p (m_v + 8 s_v) is added once at
-//             the end. Online softmax in base 2: the running max is binary32
-//             (only the exponent offset), each weight 2^(z - M) with the
-//             difference taken in double.
+//             tokens) as c - 8, exact in binary16 (a logic operation and a
+//             half2 subtract per pair of codes after a byte interleave),
+//             B = p * s_v split into binary16 hi + lo; each 16-token product
+//             joins the running sum through a round-to-nearest add, and
+//             sum p (m_v + 8 s_v) is kept aside. Online softmax in base 2
+//             against a per-head reference maximum that moves only when a
+//             score exceeds it by more than 8.
 //  3. It writes (acc, max, sum) per query head to the workspace, fences, and
 //     bumps a per-(sequence, KV head) counter; the warp that brings the
 //     counter to the number of splits merges all splits (log-sum-exp),
@@ -56,7 +57,7 @@ constexpr int kDecWarps = 4;
 struct DecodeArgs {
   int S, Hq, H, G, P, NP, bt_stride, max_seq_len, splits;
   int rot_kind, lgb;
-  double scale2;  // sm_scale * log2(e), in double
+  float scale2;   // sm_scale * log2(e)
   const __half* q;  // [S][Hq][D]
   const float* quat;
   const int32_t* seq_lens;
@@ -66,7 +67,7 @@ struct DecodeArgs {
   const uint8_t* v_codes;
   const uint32_t* v_params;
   float* out;        // [S][Hq][D]
-  float* part;       // [S][Hq][splits][D + 4]: acc[D], max (double), sum, pad
+  float* part;       // [S][Hq][splits][D + 4]: acc[D], reference max, sum p, pad
   int32_t* counter;  // [S][H] split arrivals, zero between calls
   int32_t* err;
   // fused decode step (kvq_decode_step): the new token of each sequence, K
@@ -133,7 +134,7 @@ struct DecCfg {
   static constexpr int NQT = GP == 8 ? 2 : 1;  // 16-row tiles of query limbs
   static constexpr int NMT = D / 16;           // PV m-tiles over channels
   static constexpr int TILES = P / 16;         // 16-token tiles per page
-  static constexpr int NPV = GP == 8 ? 2 : 1;  // PV n-tiles (hi / lo columns)
+  static constexpr int NE = GP == 8 ? 4 : 2;   // scores per lane per tile
   static constexpr int QW = D / 4;             // query channels per lane
   static constexpr int ROWB = D / 2;           // code bytes per token
   static constexpr int CODE_B = P * ROWB;      // code bytes per (page, head)
@@ -143,15 +144,8 @@ struct DecCfg {
   static constexpr int STAGE_B = PG * PAGE_B;
   // pipeline depth: about 8-13 KB of pages in flight per warp
   static constexpr int NST = STAGE_B <= 2304 ? 4 : (STAGE_B <= 4608 ? 3 : 2);
-  static constexpr int META_B = NST * 16;  // per stage: group index and page ids
-  static constexpr int WARP_B = (NST * STAGE_B + META_B + 127) / 128 * 128;
+  static constexpr int WARP_B = (NST * STAGE_B + 127) / 128 * 128;
 };
-
-// Rotation of a query (or output) row held as quarters: lane j of a group
-// of four consecutive lanes owns channels [j*QW, (j+1)*QW). Butterfly
-// stages with distance < QW run in registers, wider ones across the lanes
-// (distance QW: lane ^ 1, 2*QW: lane ^ 2); the lower-channel lane adds and
-// the upper one subtracts. All 32 lanes must call it. Binary32, not part of
 // the bit-exact quantize path.
 template <int QW>
 __device__ __forceinline__ void rotate_quarter(float (&x)[QW], int j, int rot_kind, int lgb,
@@ -184,11 +178,19 @@ __device__ __forceinline__ void rotate_quarter(float (&x)[QW], int j, int rot_ki
   }
 }
 
+
+// Online-softmax slack in base-2 logit units: a head's reference maximum M
+// moves only when a score exceeds it by more than this, so every weight
+// 2^(z - M) stays below 2^8 (binary16 weights and binary32 sums have room to
+// spare) and most page groups skip the cross-lane maximum and the rescale.
+constexpr float kMaxSlack = 8.f;
+
 template <int D, int P, int GP>
-__global__ void __launch_bounds__(kDecWarps * kWarp, (D == 128 && GP == 4) ? 4 : 2)
+__global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : (GP == 8 ? 3 : 4))
     decode_split_kernel(const DecodeArgs a) {
   static_assert(D == 128 || D == 256, "decode attention supports head_dim 128 and 256");
   using C = DecCfg<D, P, GP>;
+  constexpr int NE = C::NE;
   extern __shared__ __align__(128) uint8_t smem[];
   // inputs may come from the previous kernel of the stream: nothing is read
   // before it has completed; the next launch may be scheduled right away
@@ -204,9 +206,7 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, (D == 128 && GP == 4) ? 4 :
   const int split = item % a.splits;
   uint8_t* ring = smem + warp * C::WARP_B;
 
-  // ---- independent loads first: the sequence length, the block-table
-  // entries of the split's page range and the query rows are fetched in one
-  // round trip (the entries past the sequence's end are never used)
+  // ---- independent loads first: the sequence length and the query rows
   const int hr = (GP == 8) ? r : (r & 3);
   const bool lo_row = (GP == 4) && (r >= 4);
   const int g = h * a.G + hr;           // global query head
@@ -224,33 +224,47 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, (D == 128 && GP == 4) ? 4 :
     L = 0;
   }
   const int npages = (L + P - 1) / P;
-  const int ngrp = (npages + C::PG - 1) / C::PG;  // stage groups of the (sequence, KV head)
+  // this warp's pages: a contiguous range; the sequence's pages are dealt
+  // out evenly over its splits (range sizes differ by at most one page)
+  const int pg_lo = (int)(((int64_t)split * npages) / a.splits);
+  const int pg_hi = (int)(((int64_t)(split + 1) * npages) / a.splits);
+  const int ngrp = (pg_hi - pg_lo + C::PG - 1) / C::PG;  // stage groups
   const int32_t* const bt_row = a.block_table + (int64_t)s * a.bt_stride;
-  // fused step: the warp that owns the page group of position L - 1 writes
-  // the sequence's new token of this KV head before any of its copies start
-  if (a.k_new != nullptr && L >= 1 && ((L - 1) / P / C::PG) % a.splits == split) {
+  // fused step: the warp that owns the page of position L - 1 writes the
+  // sequence's new token of this KV head before any of its copies start
+  if (a.k_new != nullptr && L >= 1 && (L - 1) / P >= pg_lo && (L - 1) / P < pg_hi) {
     const int pos = L - 1;
     const int page = bt_row[pos / P];
     if (page >= 0 && page < a.NP) {
       const int64_t dst = ((int64_t)page * a.H + h) * P + pos % P;
       const int64_t src = (int64_t)s * a.new_stride + (int64_t)h * D;
-      const StepRowArgs r{a.k_new + src, a.v_new + src, a.quat, a.k_codes_w + dst * (D / 2),
-                          a.v_codes_w + dst * (D / 2), a.k_params_w + dst, a.v_params_w + dst};
-      append_step_token<D>(r, a.rot_kind, a.lgb, lane);
+      const StepRowArgs rw{a.k_new + src, a.v_new + src, a.quat, a.k_codes_w + dst * (D / 2),
+                           a.v_codes_w + dst * (D / 2), a.k_params_w + dst, a.v_params_w + dst};
+      append_step_token<D>(rw, a.rot_kind, a.lgb, lane);
       __threadfence();  // visible to this warp's page copies below
       __syncwarp();
     } else if (lane == 0) {
       raise_flag(a.err, KVQ_ERRF_PAGE);
     }
   }
-  // block-table entry of page q (lane q < PG) of group gi; -1: no such page
-  auto group_ids = [&](int gi) {
-    const int pi = gi * C::PG + lane;
-    return (lane < C::PG && gi < ngrp && pi < npages) ? bt_row[pi] : -1;
+  // The warp's block-table entries sit in lane registers, 32 pages at a
+  // time: lane i holds the entry of page pg_lo + 32 c + i of chunk c. An
+  // entry outside [0, NP) raises KVQ_ERRF_PAGE when it is loaded and its page
+  // is skipped; -1 marks a skipped page or one past the range.
+  const int npg = pg_hi - pg_lo;  // pages of this warp
+  auto load_ids = [&](int c) {
+    const int pi = 32 * c + lane;
+    int id = -1;
+    if (pi < npg) {
+      id = bt_row[pg_lo + pi];
+      if (id < 0 || id >= a.NP) {
+        raise_flag(a.err, KVQ_ERRF_PAGE);
+        id = -1;
+      }
+    }
+    return id;
   };
 
-  // ---- query fragments: rows = [hi ; lo] of the GP heads of this KV head
-  // lane (r, j) handles query head hr and channels [j*QW, (j+1)*QW)
   // ---- page ring: the warp stages each (page, head) chunk (K codes, V
   // codes, K params, V params, all contiguous in their pools) with 16-byte
   // cp.async copies, linear in shared memory: 16-byte unit u of a page block
@@ -264,29 +278,32 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, (D == 128 && GP == 4) ? 4 :
   const uint8_t* const par_l =
       lane < PU ? reinterpret_cast<const uint8_t*>(a.k_params) + (int64_t)h * P * 4 + lane * 16
                 : reinterpret_cast<const uint8_t*>(a.v_params) + (int64_t)h * P * 4 + (lane - PU) * 16;
-  // The (sequence, KV head)'s page groups are dealt out to its `splits`
-  // warps in turn: warp `split` takes groups split, split + splits, ... (a
-  // short sequence still keeps every warp of the pair busy). Each group's
-  // block-table entries are loaded one step before its copies are issued.
-  int32_t* const meta = reinterpret_cast<int32_t*>(ring + C::NST * C::STAGE_B);  // [stage][4]
-  // copy group gi (page ids in lanes q < PG) into stage sidx and record it
-  auto issue = [&](int gi, int idl, int sidx) {
-    const bool any = gi < ngrp;
-    if (lane == 0) meta[sidx * 4] = any ? gi : -1;
-    if (lane < C::PG) meta[sidx * 4 + 1 + lane] = idl;
-    if (any) {
+  // ids_a holds chunk cidx of the entries, ids_b the next chunk (loaded 32
+  // pages ahead of its use); okbits bit (slot * PG + q): page q of the group
+  // in ring slot `slot` was copied
+  int cidx = 0;
+  int ids_a = load_ids(0), ids_b = load_ids(1);
+  uint32_t okbits = 0;
+  // copy group gn into ring slot `slot` (one commit group per call)
+  auto issue = [&](int gn, int slot) {
+    if ((gn * C::PG) >> 5 != cidx) {  // the group starts the next chunk
+      ids_a = ids_b;
+      ++cidx;
+      ids_b = load_ids(cidx + 1);
+    }
+    okbits &= ~(((1u << C::PG) - 1) << (slot * C::PG));
 #pragma unroll
-      for (int q = 0; q < C::PG; ++q) {
-        const int64_t page = __shfl_sync(0xffffffffu, idl, q);
-        if (page < 0 || page >= a.NP) continue;  // beyond the sequence or out of the pool
-        const int64_t co = page * cstride;
-        uint8_t* dst = ring + sidx * C::STAGE_B + q * C::PAGE_B + lane * 16;
+    for (int q = 0; q < C::PG; ++q) {
+      const int id = __shfl_sync(0xffffffffu, ids_a, (gn * C::PG + q) & 31);
+      if (id < 0) continue;  // past the range or skipped
+      okbits |= 1u << (slot * C::PG + q);
+      const int64_t co = (int64_t)id * cstride;
+      uint8_t* dst = ring + slot * C::STAGE_B + q * C::PAGE_B + lane * 16;
 #pragma unroll
-        for (int m = 0; m < KU / kWarp; ++m) cp_async16(dst + m * 512, kc_l + co + m * 512);
+      for (int m = 0; m < KU / kWarp; ++m) cp_async16(dst + m * 512, kc_l + co + m * 512);
 #pragma unroll
-        for (int m = 0; m < KU / kWarp; ++m) cp_async16(dst + C::CODE_B + m * 512, vc_l + co + m * 512);
-        if (lane < 2 * PU) cp_async16(dst + 2 * C::CODE_B, par_l + page * pstride);
-      }
+      for (int m = 0; m < KU / kWarp; ++m) cp_async16(dst + C::CODE_B + m * 512, vc_l + co + m * 512);
+      if (lane < 2 * PU) cp_async16(dst + 2 * C::CODE_B, par_l + (int64_t)id * pstride);
     }
     cp_async_commit();
   };
@@ -312,8 +329,6 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, (D == 128 && GP == 4) ? 4 :
     v_ld[e] = C::CODE_B + tk_e[e] * C::ROWB + r * VB;
     kp_ld[e] = 2 * C::CODE_B + tk_e[e] * 4;
   }
-
-  constexpr int NE = GP == 8 ? 4 : 2;
   const int own = lo_row ? 1 : 0;  // GP = 4: token half of this lane
   int kps[NE], tks[NE];            // K-param offset and token of score e
 #pragma unroll
@@ -322,43 +337,44 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, (D == 128 && GP == 4) ? 4 :
     tks[e] = GP == 8 ? tk_e[e] : (own ? tk_e[2 + e] : tk_e[e]);
   }
 
-  // ---- state
-  float acc[C::NMT][C::NPV][4];
+  // ---- state: PV accumulators (rows = channels, columns = query heads;
+  // GP = 4 keeps the hi and lo weight columns apart until the end), the
+  // head's reference maximum and this lane's shares of the sums
+  float acc[C::NMT][4];
 #pragma unroll
   for (int mt = 0; mt < C::NMT; ++mt)
 #pragma unroll
-    for (int n = 0; n < C::NPV; ++n)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[mt][n][e] = 0.f;
-  // Scores are formed in double from exact integers: with a dominant (sink)
-  // token the base-2 logits reach ~100, where a binary32 rounding would
-  // already move the other tokens' weights visibly. The running maximum only
-  // serves as the exponent offset, so it is kept in binary32 (a value within
-  // half an ulp of the true maximum) and every weight is 2^(z - M) with the
-  // difference taken in double.
-  float M = -INFINITY;  // running max (base-2 scaled scores) of head hr
+    for (int e = 0; e < 4; ++e) acc[mt][e] = 0.f;
+  float M = -INFINITY;  // reference maximum (base-2 scaled scores) of head hr
   float Lp = 0.f;       // this lane's share of sum p
   float Op = 0.f;       // this lane's share of sum p (m_v + 8 s_v)
   // GP = 8: lane (r, j) scores head r with the tokens of slots e = 0..3;
   // GP = 4: lanes r and r + 4 share head r % 4 and split those slots,
   // {0, 1} for r < 4 and {2, 3} for r >= 4
 
-  // groups split + k * splits (k < NST): the first NST - 1 are copied now,
-  // the last waits in the "entries loaded" slot of the pipeline
-  int idk[C::NST];
+  // the first NST - 1 groups are copied now
 #pragma unroll
-  for (int k = 0; k < C::NST; ++k) idk[k] = group_ids(split + k * a.splits);
-#pragma unroll
-  for (int k = 0; k < C::NST - 1; ++k) issue(split + k * a.splits, idk[k], k);
-  int gB = split + (C::NST - 1) * a.splits;  // group whose entries are loaded
-  int idB = idk[C::NST - 1];
+  for (int k = 0; k < C::NST - 1; ++k) {
+    if (k < ngrp)
+      issue(k, k);
+    else
+      cp_async_commit();
+  }
 
-  // the first pages are in flight while the query is prepared
-  // The query as a 30-bit fixed point qint = qhat * 2^30 / amax (amax = the
-  // head's largest |qhat|), split into four signed 8-bit limbs
-  // qint = l3*2^24 + l2*2^16 + l1*2^8 + l0 for the int8 tensor cores.
-  double qsum;     // sum of qint over the head's channels (exact)
-  double zk;       // sm_scale * log2(e) * amax / 2^30
+  // ---- the query, while the first pages are in flight: rotated, then held
+  // as a 26-bit fixed point qint = RN(qhat * 2^k) (2^k the power of two that
+  // brings the head's largest |qhat| just below 2^26, so qhat * 2^k is exact
+  // in binary32) and split into four signed 8-bit limbs for the int8 tensor
+  // cores. Even channels enter as 16 qint: the K codes of odd channels are
+  // then used in place as 16 c (the high nibble of each byte masked, never
+  // shifted), and the contraction gives 16 sum_i c_i qint_i exactly.
+  // score z = (s_k zs) dot_c + (m_k + 8 s_k) zq in base-2 logit units, with
+  // dot_c = 16 sum_i (c_i - 8) qint_i = dot' - 128 qsum: centred codes keep
+  // both terms near the score's own size instead of two large ones that
+  // cancel. 128 qsum = QA * 2^16 + QB (0 <= QB < 2^16) comes off the limb
+  // halves before they are combined.
+  float zs, zq;
+  int QA, QB;
   // A fragments per k-step kk: the lane's 8 channels j*QW + 8kk + [0, 8),
   // even ones in a[0]/a[1], odd ones in a[2]/a[3]. Rows:
   //   GP = 4: rows 0-3 l3, 4-7 l1, 8-11 l2, 12-15 l0 of heads 0-3;
@@ -366,17 +382,15 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, (D == 128 && GP == 4) ? 4 :
   uint32_t qa[C::NQT][C::NKS8][4];
   {
     float x[C::QW];
-    {
 #pragma unroll
-      for (int c = 0; c < C::QW / 8; ++c) {
-        const uint4 u = qraw[c];
-        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+    for (int c = 0; c < C::QW / 8; ++c) {
+      const uint4 u = qraw[c];
+      const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __half22float2(u32_as_h2(w4[e]));
-          x[8 * c + 2 * e] = f.x;
-          x[8 * c + 2 * e + 1] = f.y;
-        }
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __half22float2(u32_as_h2(w4[e]));
+        x[8 * c + 2 * e] = f.x;
+        x[8 * c + 2 * e + 1] = f.y;
       }
     }
     rotate_quarter<C::QW>(x, j, a.rot_kind, a.lgb, a.quat, false);
@@ -385,26 +399,25 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, (D == 128 && GP == 4) ? 4 :
     for (int i = 0; i < C::QW; ++i) amax = fmaxf(amax, fabsf(x[i]));
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-    // scale 2^k with amax * 2^k < 2^30: a power of two, so qhat * 2^k is
-    // exact in binary32 and the conversion only drops bits below 2^-k
     const int ebits = (__float_as_int(amax) >> 23) & 0xFF;  // amax < 2^(ebits - 126)
-    int k = 30 - (ebits - 126);
+    int k = 26 - (ebits - 126);
     k = k > 126 ? 126 : k;
     const float mulf = amax > 0.f ? __int_as_float((k + 127) << 23) : 0.f;
-    zk = a.scale2 * __hiloint2double((1023 - k) << 20, 0);  // sm_scale log2(e) 2^-k
+    const float zk = a.scale2 * __int_as_float((127 - k) << 23);  // sm_scale log2(e) 2^-k
     long long qs_l = 0;
 #pragma unroll
     for (int kk = 0; kk < C::NKS8; ++kk) {
       // limbs of the lane's 8 channels: with t = q + 0x808080 (128 added to
       // each of the three low bytes), q = sum_k (T_k - 128 [k < 3]) 256^k for
       // the bytes T_k of t, so the signed limbs are the bytes of
-      // t ^ 0x00808080, byte k = limb k (|q| < 2^30 keeps the top limb in s8)
+      // t ^ 0x00808080, byte k = limb k (|q| <= 2^30 keeps the top limb in s8)
       uint32_t u[8];
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         const int q = __float2int_rn(x[8 * kk + c] * mulf);
         qs_l += q;
-        u[c] = (uint32_t)(q + 0x808080) ^ 0x00808080u;
+        const int qe = (c & 1) ? q : q * 16;
+        u[c] = (uint32_t)(qe + 0x808080) ^ 0x00808080u;
       }
       // limb `lb` (0 = lowest) of channels {o, o+2, o+4, o+6} as one s8x4 word
       auto pk4 = [&](int o, int lb) {
@@ -431,42 +444,47 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, (D == 128 && GP == 4) ? 4 :
     }
     qs_l += __shfl_xor_sync(0xffffffffu, qs_l, 1);
     qs_l += __shfl_xor_sync(0xffffffffu, qs_l, 2);
-    qsum = (double)qs_l;  // |qsum| <= 2^30 * D: exact
+    zs = zk * 0.0625f;          // exact: the factor 16 of dot'
+    zq = zk * (float)qs_l;      // sum of qint over the head's channels
+    const long long q128 = qs_l * 128;  // |qsum| < 2^26 d: no overflow
+    QA = (int)(q128 >> 16);             // floor division
+    QB = (int)(q128 - ((long long)QA << 16));
   }
 
-
-  int sidx = 0;             // stage consumed this step
-  int sissue = C::NST - 1;  // stage refilled this step
-  for (;;) {
-    issue(gB, idB, sissue);
-    sissue = sissue + 1 == C::NST ? 0 : sissue + 1;
-    gB += a.splits;
-    idB = group_ids(gB);
-    cp_async_wait<C::NST - 1>();  // this lane's copies of the stage have landed
-    __syncwarp();                 // ... and every other lane's, and the stage's record
-    const int gi = meta[sidx * 4];
-    if (gi < 0) break;            // no group left for this warp
-    bool pgok[C::PG];             // page q of the group is cached and in the pool
+  int slot = 0;               // ring slot of group gi
+  int slot_n = C::NST - 1;    // ring slot of group gi + NST - 1
+  for (int gi = 0; gi < ngrp; ++gi) {
+    if (gi + C::NST - 1 < ngrp)
+      issue(gi + C::NST - 1, slot_n);
+    else
+      cp_async_commit();
+    slot_n = slot_n + 1 == C::NST ? 0 : slot_n + 1;
+    cp_async_wait<C::NST - 1>();  // this lane's copies of group gi have landed
+    __syncwarp();                 // ... and every other lane's
+    bool pgok[C::PG];             // page q of the group was copied
     bool all_ok = true;
 #pragma unroll
     for (int q = 0; q < C::PG; ++q) {
-      const int pid = meta[sidx * 4 + 1 + q];
-      const bool cached = gi * C::PG + q < npages;
-      pgok[q] = cached && pid >= 0 && pid < a.NP;
+      pgok[q] = (okbits >> (slot * C::PG + q)) & 1u;
       all_ok = all_ok && pgok[q];
-      if (cached && !pgok[q] && lane == 0) raise_flag(a.err, KVQ_ERRF_PAGE);
     }
-    const uint8_t* st = ring + sidx * C::STAGE_B;
-    sidx = sidx + 1 == C::NST ? 0 : sidx + 1;
-    const int tok0 = gi * C::PG * P;  // first token of the group
+    const uint8_t* st = ring + slot * C::STAGE_B;
+    slot = slot + 1 == C::NST ? 0 : slot + 1;
+    const int tok0 = (pg_lo + gi * C::PG) * P;  // first token of the group
     // groups whose every token is cached skip all per-token masking
     const bool full = all_ok && tok0 + C::PG * P <= L;
 
     auto body = [&](auto masked_tag) {
       constexpr bool MASKED = decltype(masked_tag)::value;
-      double z[C::TPG][NE];
+      // ---- QK and scores of every tile (tiles of a skipped page: -inf)
+      float z[C::TPG][NE];
 #pragma unroll
       for (int tt = 0; tt < C::TPG; ++tt) {
+        if (MASKED && !pgok[tt / C::TILES]) {
+#pragma unroll
+          for (int e = 0; e < NE; ++e) z[tt][e] = -INFINITY;
+          continue;
+        }
         // tile tt of the group: page tt / TILES, 16-token tile tt % TILES
         const int cofs = (tt / C::TILES) * C::PAGE_B + (tt % C::TILES) * 16 * C::ROWB;
         const int pofs = (tt / C::TILES) * C::PAGE_B + (tt % C::TILES) * 64;
@@ -485,30 +503,32 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, (D == 128 && GP == 4) ? 4 :
           }
 #pragma unroll
           for (int kk = 0; kk < C::NKS8; ++kk) {
-            const uint32_t b0 = w[kk] & 0x0F0F0F0Fu;         // even channels as bytes
-            const uint32_t b1 = (w[kk] >> 4) & 0x0F0F0F0Fu;  // odd channels
+            const uint32_t b0 = w[kk] & 0x0F0F0F0Fu;  // even channels: c
+            const uint32_t b1 = w[kk] & 0xF0F0F0F0u;  // odd channels: 16 c
 #pragma unroll
             for (int t = 0; t < C::NQT; ++t) mma16832_s8u8(ci[t][nt], qa[t][kk], b0, b1);
           }
         }
-        // dot = sum_i c_i qint_i of head hr with each of the lane's tokens,
-        // exact: the limb dots combine as (l3*256 + l2) * 2^16 + (l1*256 + l0)
-        int hA[NE], hB[NE];  // l3*256 + l2 and l1*256 + l0 (|.| < 2^27)
+        // dot' = 16 sum_i c_i qint_i of head hr with each of the lane's
+        // tokens: the limb dots combine as (l3*256 + l2) * 2^16 + (l1*256 + l0)
+        // halves of dot_c: l3*256 + l2 - QA and l1*256 + l0 - QB (|.| < 2^31)
+        int hA[NE], hB[NE];
         if (GP == 8) {
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int nt = e >> 1, c = e & 1;
-            hA[e] = ci[0][nt][c] * 256 + ci[0][nt][2 + c];
-            hB[e] = ci[C::NQT - 1][nt][c] * 256 + ci[C::NQT - 1][nt][2 + c];
+            hA[e] = ci[0][nt][c] * 256 + (ci[0][nt][2 + c] - QA);
+            hB[e] = ci[C::NQT - 1][nt][c] * 256 + (ci[C::NQT - 1][nt][2 + c] - QB);
           }
         } else {
-          // lanes r < 4 hold the (l3, l2) rows and form l3*256 + l2, lanes
-          // r + 4 the (l1, l0) rows and form l1*256 + l0, for both token
-          // halves; each sends its partner the half that partner scores
+          // lanes r < 4 hold the (l3, l2) rows and form l3*256 + l2 - QA,
+          // lanes r + 4 the (l1, l0) rows and form l1*256 + l0 - QB, for both
+          // token halves; each sends its partner the half that partner scores
+          const int Qh = lo_row ? QB : QA;
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
-            const int loc0 = ci[0][0][c] * 256 + ci[0][0][2 + c];
-            const int loc1 = ci[0][1][c] * 256 + ci[0][1][2 + c];
+            const int loc0 = ci[0][0][c] * 256 + (ci[0][0][2 + c] - Qh);
+            const int loc1 = ci[0][1][c] * 256 + (ci[0][1][2 + c] - Qh);
             const int got = __shfl_xor_sync(0xffffffffu, lo_row ? loc0 : loc1, 16);
             const int mine = lo_row ? loc1 : loc0;
             hA[c] = lo_row ? got : mine;
@@ -517,106 +537,91 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, (D == 128 && GP == 4) ? 4 :
         }
 #pragma unroll
         for (int e = 0; e < NE; ++e) {
-          // exact int32 -> double through the biased exponent 2^52 + 2^31
-          constexpr double kBias = 4503601774854144.0;  // 2^52 + 2^31
-          const double dA = __hiloint2double(0x43300000, hA[e] ^ (int)0x80000000) - kBias;
-          const double dot = fma(dA, 65536.0, __hiloint2double(0x43300000, hB[e] ^ (int)0x80000000)) - kBias;
+          const float dotf = fmaf((float)hA[e], 65536.f, (float)hB[e]);
           const uint32_t kpw = *reinterpret_cast<const uint32_t*>(st + kps[e] + pofs);
           const float2 sm = __half22float2(u32_as_h2(kpw));  // (scale, min)
-          // s * dot and m * qsum are exact in double (11 + 41 and 11 + 38 bits)
-          const double sc = zk * fma((double)sm.x, dot, (double)sm.y * qsum);
+          const float sc = fmaf(sm.x * zs, dotf, fmaf(8.f, sm.x, sm.y) * zq);
           if (MASKED) {
             const int tok = tok0 + (tt / C::TILES) * P + (tt % C::TILES) * 16 + tks[e];
-            z[tt][e] = (pgok[tt / C::TILES] && tok < L) ? sc : -INFINITY;
+            z[tt][e] = tok < L ? sc : -INFINITY;
           } else {
             z[tt][e] = sc;
           }
         }
       }
 
-      // ---- online softmax update for head hr (max over the lanes sharing it)
+      // ---- online softmax: move head hr's reference maximum only when a
+      // score of the group exceeds it by more than kMaxSlack (warp-uniform)
       float mloc = -INFINITY;
 #pragma unroll
       for (int tt = 0; tt < C::TPG; ++tt)
 #pragma unroll
-        for (int e = 0; e < NE; ++e) mloc = fmaxf(mloc, (float)z[tt][e]);
-      mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
-      mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
-      if (GP == 4) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 16));
-      const float Mn = fmaxf(M, mloc);
-      const float alpha = (Mn == M) ? 1.f : fast_exp2(M - Mn);  // M = -inf: 0
-      M = Mn;
-      const double Md = (double)M;
-      Lp *= alpha;
-      Op *= alpha;
-      // rescale the output accumulators: lane (r, j) holds columns of heads
-      // c0 = 2(j & (GP/2 - 1)), c0 + 1 -> their alpha from lanes r = c0, c0 + 1
-      if (__any_sync(0xffffffffu, alpha != 1.f)) {  // warp-uniform: skip when no max moved
+        for (int e = 0; e < NE; ++e) mloc = fmaxf(mloc, z[tt][e]);
+      if (__any_sync(0xffffffffu, mloc > M + kMaxSlack)) {
+        mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
+        mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
+        if (GP == 4) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 16));
+        const float Mn = fmaxf(M, mloc);
+        const float alpha = (Mn == M) ? 1.f : fast_exp2(M - Mn);  // M = -inf: 0
+        M = Mn;
+        Lp *= alpha;
+        Op *= alpha;
+        // lane (r, j) holds columns of heads c0 = 2(j & (GP/2 - 1)), c0 + 1:
+        // their factors from lanes r = c0, c0 + 1
         const int c0 = (GP == 8) ? 2 * j : 2 * (j & 1);
         const float a0 = __shfl_sync(0xffffffffu, alpha, 4 * c0);
         const float a1 = __shfl_sync(0xffffffffu, alpha, 4 * c0 + 4);
 #pragma unroll
-        for (int mt = 0; mt < C::NMT; ++mt)
-#pragma unroll
-          for (int n = 0; n < C::NPV; ++n) {
-            acc[mt][n][0] *= a0; acc[mt][n][1] *= a1;
-            acc[mt][n][2] *= a0; acc[mt][n][3] *= a1;
-          }
+        for (int mt = 0; mt < C::NMT; ++mt) {
+          acc[mt][0] *= a0; acc[mt][1] *= a1;
+          acc[mt][2] *= a0; acc[mt][3] *= a1;
+        }
       }
 
       // ---- PV per tile
 #pragma unroll
       for (int tt = 0; tt < C::TPG; ++tt) {
+        if (MASKED && !pgok[tt / C::TILES]) continue;
         const int cofs = (tt / C::TILES) * C::PAGE_B + (tt % C::TILES) * 16 * C::ROWB;
         const int pofs = (tt / C::TILES) * C::PAGE_B + (tt % C::TILES) * 64;
-        float pv[NE];
+        float wv[NE];
 #pragma unroll
         for (int e = 0; e < NE; ++e) {
           const uint32_t vpw = *reinterpret_cast<const uint32_t*>(st + kps[e] + P * 4 + pofs);
           const float2 sm = __half22float2(u32_as_h2(vpw));  // (scale, min)
-          if (MASKED) {
-            // masked tokens may sit on stale or never-written shared memory:
-            // their terms are forced to exact zeros rather than p * (params)
-            const bool live = z[tt][e] != -INFINITY;
-            const float p = live ? fast_exp2((float)(z[tt][e] - Md)) : 0.f;
-            Lp += p;
-            Op += live ? p * (sm.y + 8.f * sm.x) : 0.f;
-            pv[e] = live ? p * sm.x : 0.f;
-          } else {
-            const float p = fast_exp2((float)(z[tt][e] - Md));
-            Lp += p;
-            Op = fmaf(p, sm.y + 8.f * sm.x, Op);
-            pv[e] = p * sm.x;
-          }
+          // masked tokens may sit on stale or never-written shared memory:
+          // their terms are forced to exact zeros rather than p * (params)
+          const bool live = !MASKED || z[tt][e] != -INFINITY;
+          const float p = live ? fast_exp2(z[tt][e] - M) : 0.f;
+          Lp += p;
+          Op = live ? fmaf(p, fmaf(8.f, sm.x, sm.y), Op) : Op;  // p (m_v + 8 s_v)
+          wv[e] = live ? p * sm.x : 0.f;
         }
-        // p * s as binary16 hi + lo pairs (packed conversions): hi = RN16(x),
-        // lo = RN16(x - hi)
-        uint32_t pb[C::NPV][2];
+        // weights p * s as binary16 hi + lo pairs: hi = RN16(w), lo = RN16(w - hi)
+        uint32_t bh[2], bl[2];
         if (GP == 8) {
-          // n-tile 0 = hi, 1 = lo; column r = head r; k slots (0, 1), (2, 3)
-          const __half2 h01 = __floats2half2_rn(pv[0], pv[1]);
-          const __half2 h89 = __floats2half2_rn(pv[NE - 2], pv[NE - 1]);
-          const float2 f01 = __half22float2(h01), f89 = __half22float2(h89);
-          pb[0][0] = h2_as_u32(h01);
-          pb[0][1] = h2_as_u32(h89);
-          pb[C::NPV - 1][0] = h2_as_u32(__floats2half2_rn(pv[0] - f01.x, pv[1] - f01.y));
-          pb[C::NPV - 1][1] = h2_as_u32(__floats2half2_rn(pv[NE - 2] - f89.x, pv[NE - 1] - f89.y));
+          const __half2 h01 = __floats2half2_rn(wv[0], wv[1]);
+          const __half2 h23 = __floats2half2_rn(wv[NE - 2], wv[NE - 1]);
+          const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+          bh[0] = h2_as_u32(h01);
+          bh[1] = h2_as_u32(h23);
+          bl[0] = h2_as_u32(__floats2half2_rn(wv[0] - f01.x, wv[1] - f01.y));
+          bl[1] = h2_as_u32(__floats2half2_rn(wv[NE - 2] - f23.x, wv[NE - 1] - f23.y));
         } else {
           // column r < 4 = hi of head r, r >= 4 = lo of head r - 4: lane r
           // keeps hi (or lo) of its own token half and takes the other
           // half's from its partner r ^ 4
-          const __half2 ho = __floats2half2_rn(pv[0], pv[1]);
+          const __half2 ho = __floats2half2_rn(wv[0], wv[1]);
           const float2 fo = __half22float2(ho);
           const uint32_t hi_own = h2_as_u32(ho);
-          const uint32_t lo_own = h2_as_u32(__floats2half2_rn(pv[0] - fo.x, pv[1] - fo.y));
+          const uint32_t lo_own = h2_as_u32(__floats2half2_rn(wv[0] - fo.x, wv[1] - fo.y));
           const uint32_t got = __shfl_xor_sync(0xffffffffu, lo_row ? hi_own : lo_own, 16);
-          pb[0][0] = lo_row ? got : hi_own;  // slots 0, 1
-          pb[0][1] = lo_row ? lo_own : got;  // slots 2, 3
+          bh[0] = lo_row ? got : hi_own;  // slots 0, 1
+          bh[1] = lo_row ? lo_own : got;  // slots 2, 3
+          bl[0] = bl[1] = 0u;
         }
-        if (!head_ok) {
-#pragma unroll
-          for (int n = 0; n < C::NPV; ++n) pb[n][0] = pb[n][1] = 0u;
-        }
+        // (columns of padding heads, hr >= G, carry weights of a zero query;
+        // they never mix with other columns and are never written)
         // A operand: V codes of the slots' tokens, channels of lane row r:
         // [r*D/8, (r+1)*D/8)
         constexpr int WPT = D / 64;  // 32-bit words per token per lane
@@ -632,47 +637,53 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, (D == 128 && GP == 4) ? 4 :
             vw[e][0] = v4.x; vw[e][1] = v4.y; vw[e][2] = v4.z; vw[e][3] = v4.w;
           }
         }
-        // m-tile mt: group gq = mt / 8 (words 2gq, 2gq+1), nibble e = mt % 8;
-        // row slot r <- word 2gq, slot r+8 <- word 2gq+1
+        // Each code enters the f16 tensor core as c - 8, exact in binary16:
+        // the nibble is OR-ed into the mantissa of 1024 (one three-input
+        // logic operation on a masked word; nibbles in bits 4-7 land at
+        // 1024 + 16 c) and the bias comes off with one half2 subtract
+        // (1024 + c - 1032) or fused multiply-add ((1024 + 16 c) / 16 - 72).
+        // (Subnormal operands without a bias would save that operation, but
+        // the tensor core does not keep their products exact.) Token pairs
+        // are interleaved first (bytes of tokens 2j and 2j+1 side by side),
+        // so one operation yields the half2 of a channel for both tokens of
+        // a k pair. m-tile mt: group gq = mt / 8 (words 2gq, 2gq+1), channel
+        // e8 = mt % 8 of the word's 8 (byte e8 / 2, nibble e8 % 2); row slot
+        // r <- word 2gq, slot r+8 <- word 2gq+1.
 #pragma unroll
-        for (int gq = 0; gq < WPT / 2; ++gq) {
-          uint32_t pr[2][2][2];  // [slot pair][word in group][lo/hi bytes]
+        for (int gq = 0; gq < WPT / 2; ++gq)
+#pragma unroll
+          for (int bsel = 0; bsel < 2; ++bsel) {
+          // bytes 2 bsel, 2 bsel + 1 of the group's words, token pairs interleaved
+          uint32_t pr[2][2][2];  // [slot pair][word in group][shifted]
 #pragma unroll
           for (int tp = 0; tp < 2; ++tp)
 #pragma unroll
             for (int wi = 0; wi < 2; ++wi) {
               const int wd = 2 * gq + wi;
               const uint32_t X = vw[2 * tp][wd], Y = vw[2 * tp + 1][wd];
-              pr[tp][wi][0] = __byte_perm(X, Y, 0x5410);
-              pr[tp][wi][1] = __byte_perm(X, Y, 0x7632);
+              pr[tp][wi][0] = __byte_perm(X, Y, bsel ? 0x7632 : 0x5410);
+              pr[tp][wi][1] = pr[tp][wi][0] >> 8;
             }
-          // nibbles of every (slot pair, word, byte half): nb[tp][wi][bsel][k]
-          uint32_t nb[2][2][2][4];
 #pragma unroll
-          for (int tp = 0; tp < 2; ++tp)
-#pragma unroll
-            for (int wi = 0; wi < 2; ++wi)
-#pragma unroll
-              for (int bs = 0; bs < 2; ++bs) nib4(pr[tp][wi][bs], nb[tp][wi][bs]);
-#pragma unroll
-          for (int e8 = 0; e8 < 8; ++e8) {
+          for (int e4 = 0; e4 < 4; ++e4) {
+            const int e8 = 4 * bsel + e4;
             const int mt = gq * 8 + e8;
-            const int bsel = e8 >> 2, k = e8 & 3;
+            const int sh = (e8 >> 1) & 1;
+            const uint32_t mask = (e8 & 1) ? 0x00F000F0u : 0x000F000Fu;
             uint32_t av[4];
-            av[0] = nb[0][0][bsel][k];  // row slot r,   k slots 0, 1
-            av[1] = nb[0][1][bsel][k];  // row slot r+8, k slots 0, 1
-            av[2] = nb[1][0][bsel][k];  // row slot r,   k slots 2, 3
-            av[3] = nb[1][1][bsel][k];  // row slot r+8, k slots 2, 3
+            av[0] = nib_c8(pr[0][0][sh], mask, e8 & 1);  // row slot r,   k slots 0, 1
+            av[1] = nib_c8(pr[0][1][sh], mask, e8 & 1);  // row slot r+8, k slots 0, 1
+            av[2] = nib_c8(pr[1][0][sh], mask, e8 & 1);  // row slot r,   k slots 2, 3
+            av[3] = nib_c8(pr[1][1][sh], mask, e8 & 1);  // row slot r+8, k slots 2, 3
             // each 16-token product starts from zero and joins the running
-            // sum through an IEEE round-to-nearest add: accumulating inside
-            // the tensor core would round toward zero against a large sum
+            // sum through a round-to-nearest add: the tensor core truncates
+            // every product against its accumulator, which, fed the running
+            // sum of non-negative terms, would bias the sum low
+            float t4[4] = {0.f, 0.f, 0.f, 0.f};
+            mma16816(t4, av, bh[0], bh[1]);
+            if (GP == 8) mma16816(t4, av, bl[0], bl[1]);
 #pragma unroll
-            for (int n = 0; n < C::NPV; ++n) {
-              float t4[4] = {0.f, 0.f, 0.f, 0.f};
-              mma16816(t4, av, pb[n][0], pb[n][1]);
-#pragma unroll
-              for (int e = 0; e < 4; ++e) acc[mt][n][e] = __fadd_rn(acc[mt][n][e], t4[e]);
-            }
+            for (int e = 0; e < 4; ++e) acc[mt][e] += t4[e];
           }
         }
       }
@@ -681,11 +692,12 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, (D == 128 && GP == 4) ? 4 :
       body(std::false_type{});
     else
       body(std::true_type{});
-    __syncwarp();  // every lane is done with stage i % C::NST before it is refilled
+    __syncwarp();  // every lane is done with the stage before it is refilled
   }
   cp_async_wait<0>();
 
-  // ---- partial results: (acc + sum p (m + 8 s)) per channel, M, sum p
+  // ---- partial results: per channel acc + sum p (m + 8 s), the reference
+  // maximum M and sum p
   Lp += __shfl_xor_sync(0xffffffffu, Lp, 1);
   Lp += __shfl_xor_sync(0xffffffffu, Lp, 2);
   Op += __shfl_xor_sync(0xffffffffu, Op, 1);
@@ -693,13 +705,11 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, (D == 128 && GP == 4) ? 4 :
   if (GP == 4) {  // the two token halves of head hr
     Lp += __shfl_xor_sync(0xffffffffu, Lp, 16);
     Op += __shfl_xor_sync(0xffffffffu, Op, 16);
-  }
-  if (GP == 4) {
     // fold the lo columns (lanes j = 2, 3) onto the hi columns (j = 0, 1)
 #pragma unroll
     for (int mt = 0; mt < C::NMT; ++mt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) acc[mt][0][e] += __shfl_xor_sync(0xffffffffu, acc[mt][0][e], 2);
+      for (int e = 0; e < 4; ++e) acc[mt][e] += __shfl_xor_sync(0xffffffffu, acc[mt][e], 2);
   }
   const int c0 = (GP == 8) ? 2 * j : 2 * (j & 1);  // heads of this lane's columns
   const float o0 = __shfl_sync(0xffffffffu, Op, 4 * c0);
@@ -717,21 +727,15 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, (D == 128 && GP == 4) ? 4 :
       // m-tile mt, row slot r <- channel r*D/8 + 16*(mt/8) + mt%8,
       // row slot r+8 <- that channel + 8
       const int ch0 = r * (D / 8) + 16 * (mt / 8) + (mt % 8);
-      float v0 = 0.f, v1 = 0.f;
-#pragma unroll
-      for (int n = 0; n < C::NPV; ++n) {
-        v0 += acc[mt][n][hc];
-        v1 += acc[mt][n][2 + hc];
-      }
-      dst[ch0] = v0 + ov;
-      dst[ch0 + 8] = v1 + ov;
+      dst[ch0] = acc[mt][hc] + ov;
+      dst[ch0 + 8] = acc[mt][2 + hc] + ov;
     }
   }
   // the lanes that own head hr's softmax state write it (one lane per head)
   if (j == 0 && !lo_row && head_ok) {
     float* dst = a.part + (base + (int64_t)hr * a.splits) * (D + 4);
-    *reinterpret_cast<double*>(dst + D) = M;  // 8-byte aligned: (D + 4) * 4 * k + 4 * D
-    dst[D + 2] = Lp;
+    dst[D] = M;
+    dst[D + 1] = Lp;
   }
 
   // ---- the last warp of this (sequence, KV head) merges the splits
@@ -765,20 +769,19 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, (D == 128 && GP == 4) ? 4 :
   const int coff = j * C::QW + (GP == 4 ? own * (C::QW / 2) : 0);
   const float* src = a.part + ((int64_t)s * a.Hq + g) * a.splits * (D + 4);
   const int nsp = head_ok ? a.splits : 0;
-  double Mx = -INFINITY;
+  float Mx = -INFINITY;
   {
     // the splits' maxima: the NL lanes of the head load interleaved splits
     constexpr int NL = GP == 4 ? 8 : 4;
     const int li0 = GP == 4 ? 4 * own + j : j;
     for (int i0 = 0; i0 < nsp; i0 += 4 * NL) {
-      double mv[4];
+      float mv[4];
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
         const int i = i0 + li0 + NL * m;
-        mv[m] = i < nsp ? __ldcg(reinterpret_cast<const double*>(src + (int64_t)i * (D + 4) + D))
-                        : -INFINITY;
+        mv[m] = i < nsp ? __ldcg(src + (int64_t)i * (D + 4) + D) : -INFINITY;
       }
-      Mx = fmax(Mx, fmax(fmax(mv[0], mv[1]), fmax(mv[2], mv[3])));
+      Mx = fmaxf(Mx, fmaxf(fmaxf(mv[0], mv[1]), fmaxf(mv[2], mv[3])));
     }
   }
   float xm[CW];
@@ -787,28 +790,28 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, (D == 128 && GP == 4) ? 4 :
   float Ls = 0.f;
   for (int i0 = 0; i0 < (nsp > 0 ? nsp : 1); i0 += RB) {
     float4 f[RB][CW / 4];
-    double Mi[RB];
+    float Mi[RB];
     float li[RB];
 #pragma unroll
     for (int rb = 0; rb < RB; ++rb) {
       const int i = i0 + rb;
       const float* pi = src + (int64_t)i * (D + 4);
       const bool in = i < nsp;
-      Mi[rb] = in ? __ldcg(reinterpret_cast<const double*>(pi + D)) : -INFINITY;
-      li[rb] = in ? __ldcg(pi + D + 2) : 0.f;
+      Mi[rb] = in ? __ldcg(pi + D) : -INFINITY;
+      li[rb] = in ? __ldcg(pi + D + 1) : 0.f;
 #pragma unroll
       for (int c = 0; c < CW / 4; ++c)
         f[rb][c] = in ? __ldcg(reinterpret_cast<const float4*>(pi + coff) + c) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     if (i0 == 0) {  // every lane of a head ends with the head's maximum
-      Mx = fmax(Mx, __shfl_xor_sync(0xffffffffu, Mx, 1));
-      Mx = fmax(Mx, __shfl_xor_sync(0xffffffffu, Mx, 2));
-      if (GP == 4) Mx = fmax(Mx, __shfl_xor_sync(0xffffffffu, Mx, 16));
+      Mx = fmaxf(Mx, __shfl_xor_sync(0xffffffffu, Mx, 1));
+      Mx = fmaxf(Mx, __shfl_xor_sync(0xffffffffu, Mx, 2));
+      if (GP == 4) Mx = fmaxf(Mx, __shfl_xor_sync(0xffffffffu, Mx, 16));
     }
 #pragma unroll
     for (int rb = 0; rb < RB; ++rb) {
       // an empty split (max -inf) has a zero row and a zero sum: weight 0
-      const float wgt = Mi[rb] == -INFINITY ? 0.f : fast_exp2((float)(Mi[rb] - Mx));
+      const float wgt = Mi[rb] == -INFINITY ? 0.f : fast_exp2(Mi[rb] - Mx);
       Ls += wgt * li[rb];
 #pragma unroll
       for (int c = 0; c < CW / 4; ++c) {
@@ -951,7 +954,7 @@ int decode_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, const void* q,
   a.S = S; a.Hq = Hq; a.H = d.num_kv_heads; a.G = G; a.P = d.page_size; a.NP = d.num_pages;
   a.bt_stride = bt_stride; a.max_seq_len = max_seq_len; a.splits = pl.splits;
   a.rot_kind = d.rot_kind; a.lgb = lgb;
-  a.scale2 = (double)sm_scale * 1.4426950408889634074;
+  a.scale2 = (float)((double)sm_scale * 1.4426950408889634074);
   a.q = static_cast<const __half*>(q); a.quat = d.quat;
   a.seq_lens = seq_lens; a.block_table = block_table;
   a.k_codes = k_codes; a.k_params = static_cast<const uint32_t*>(k_params);

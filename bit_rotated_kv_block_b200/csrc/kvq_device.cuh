@@ -229,24 +229,16 @@ __device__ __forceinline__ __half2 u32_as_h2(uint32_t u) {
 // three-input logic operation gives 1024 + c exactly, and one subtraction or
 // fused multiply-add removes the bias. The constants follow from the binary16
 // format.
-// The four nibbles of each 16-bit half of z as half2 (code - 8), exact:
-// out[k] = half2(nibble k of the low half, nibble k of the high half). Nibbles
-// 0 and 2 land at 1024 + c (mantissa bits 0-3) and lose 1032; nibbles 1 and 3
-// land at 1024 + 16c (bits 4-7) and are mapped by (.)/16 - 72 = c - 8.
-__device__ __forceinline__ void nib4(uint32_t z, uint32_t (&out)[4]) {
-  const __half2 k1032 = u32_as_h2(0x64086408u);                    // 1032
-  const __half2 k16th = u32_as_h2(0x2C002C00u);                    // 1/16
-  const __half2 km72 = u32_as_h2(0xD480D480u);                     // -72
-  const uint32_t z8 = z >> 8;
-  uint32_t t0, t1, t2, t3;
-  asm("lop3.b32 %0, %1, %2, %3, 0xea;" : "=r"(t0) : "r"(z), "r"(0x000F000Fu), "r"(0x64006400u));
-  asm("lop3.b32 %0, %1, %2, %3, 0xea;" : "=r"(t1) : "r"(z), "r"(0x00F000F0u), "r"(0x64006400u));
-  asm("lop3.b32 %0, %1, %2, %3, 0xea;" : "=r"(t2) : "r"(z8), "r"(0x000F000Fu), "r"(0x64006400u));
-  asm("lop3.b32 %0, %1, %2, %3, 0xea;" : "=r"(t3) : "r"(z8), "r"(0x00F000F0u), "r"(0x64006400u));
-  out[0] = h2_as_u32(__hsub2(u32_as_h2(t0), k1032));
-  out[1] = h2_as_u32(__hfma2(u32_as_h2(t1), k16th, km72));
-  out[2] = h2_as_u32(__hsub2(u32_as_h2(t2), k1032));
-  out[3] = h2_as_u32(__hfma2(u32_as_h2(t3), k16th, km72));
+// Two codes (one channel of a token pair, selected by `mask` at bits 0-3 and
+// 16-19, or at bits 4-7 and 20-23 when `high`) as the half2 (c - 8): they
+// read 1024 + c (or 1024 + 16 c), and one subtraction of 1032 (or a multiply
+// by 1/16 and an add of -72) leaves c - 8. Exact: every intermediate is an
+// integer below 2048 or a multiple of 1/16 below 128 in binary16.
+__device__ __forceinline__ uint32_t nib_c8(uint32_t z, uint32_t mask, int high) {
+  uint32_t t;
+  asm("lop3.b32 %0, %1, %2, %3, 0xea;" : "=r"(t) : "r"(z), "r"(mask), "r"(0x64006400u));
+  return high ? h2_as_u32(__hfma2(u32_as_h2(t), u32_as_h2(0x2C002C00u), u32_as_h2(0xD480D480u)))
+              : h2_as_u32(__hsub2(u32_as_h2(t), u32_as_h2(0x64086408u)));
 }
 
 __device__ __forceinline__ float fast_exp2(float x) {
