@@ -6,10 +6,14 @@
 // Hadamard (or quaternion) map as the keys, so q . k is unchanged, and the
 // output is rotated back once per query head.
 //
-// One kernel, one warp per (sequence, KV head, split of the page range):
-//  0. For a fused decode step (kvq_decode_step) the warp that owns the page
-//     of position seq_len - 1 first quantizes and writes that sequence's new
-//     K and V rows for its KV head, exactly as kvq_quantize_append would.
+// Two kernels on the caller's stream, the second launched with programmatic
+// serialization so that it is resident as the first drains.
+// Split kernel, one warp per (sequence, KV head, split of the page range):
+//  0. For a fused decode step (kvq_decode_step) the warp whose range holds
+//     the page of position seq_len - 1 quantizes that sequence's new K and V
+//     rows for its KV head exactly as kvq_quantize_append would, writes them
+//     to the pools and patches them into its staged copy of that page (so
+//     the attention reads them without a fence or a global round trip).
 //  1. The warp rotates its query heads in registers: lane (r, j) holds
 //     channels [j*d/4, (j+1)*d/4) of query head r (GP = 8) or r % 4 (GP = 4);
 //     butterfly stages inside a quarter run in registers, wider ones across
@@ -25,8 +29,8 @@
 //       QK^T: m16n8k32 s8 x u8 -> s32, A = the query limbs (one row per
 //             (head, limb)), B = the K codes as bytes (even channels c, odd
 //             channels 16 c, one AND per word each); the limb dots
-//             recombine exactly into 16 sum_i c_i qint_i, and the score
-//               z = sm_scale log2(e) 2^-k (s_k dot + m_k sum qint)
+//             recombine exactly into 16 sum_i (c_i - 8) qint_i, and the score
+//               z = sm_scale log2(e) 2^-k (s_k dot + (m_k + 8 s_k) sum qint)
 //             is formed in binary32;
 //       PV:   m16n8k16 f16 x f16 -> f32, A = V codes transposed (channels x
 //             tokens) as c - 8, exact in binary16 (a logic operation and a
@@ -36,11 +40,10 @@
 //             sum p (m_v + 8 s_v) is kept aside. Online softmax in base 2
 //             against a per-head reference maximum that moves only when a
 //             score exceeds it by more than 8.
-//  3. It writes (acc, max, sum) per query head to the workspace, fences, and
-//     bumps a per-(sequence, KV head) counter; the warp that brings the
-//     counter to the number of splits merges all splits (log-sum-exp),
-//     normalises, rotates back in registers, writes the float32 output and
-//     resets the counter to zero. No warp ever waits on another.
+//  3. It writes (acc, max, sum) per query head to the workspace.
+// Merge kernel, one warp per (sequence, query head): combines the splits
+// (log-sum-exp), normalises, rotates back in registers and writes the
+// float32 output. No warp ever waits on another.
 #include <cuda_runtime.h>
 
 #include <type_traits>
@@ -68,7 +71,6 @@ struct DecodeArgs {
   const uint32_t* v_params;
   float* out;        // [S][Hq][D]
   float* part;       // [S][Hq][splits][D + 4]: acc[D], reference max, sum p, pad
-  int32_t* counter;  // [S][H] split arrivals, zero between calls
   int32_t* err;
   // fused decode step (kvq_decode_step): the new token of each sequence, K
   // and V rows [S][H][D] binary16 (row (s, h) at s * new_stride + h * D),
@@ -83,45 +85,66 @@ struct DecodeArgs {
   uint32_t* v_params_w;
 };
 
-// The new token of one (sequence, KV head) (position L - 1) quantized and
-// written by one warp, exactly as kvq_quantize_append would write it.
-struct StepRowArgs {
-  const __half* k_row;  // this (sequence, KV head)'s new K row
-  const __half* v_row;
-  const float* quat;
-  uint8_t* k_codes;     // this row's destination slot in each pool
-  uint8_t* v_codes;
-  uint32_t* k_param;
-  uint32_t* v_param;
+// The new token of one (sequence, KV head) (position L - 1), quantized by
+// one warp exactly as kvq_quantize_append would: this lane's code bytes of
+// the K and V rows (CPL / 2 of them, little-endian in the word) and the
+// (scale, min) words of both rows.
+struct StepRow {
+  uint32_t kc, vc;
+  uint32_t kp, vp;
 };
 
 template <int D, int ROT, int LGB>
-__device__ __forceinline__ void step_rows(const StepRowArgs& r, int lane) {
+__device__ __forceinline__ StepRow step_rows(const __half* k_row, const __half* v_row,
+                                             const float* quat, int lane) {
   constexpr int CPL = RowQuantShape<D>::CPL;
+  StepRow o;
 #pragma unroll 1
   for (int kv = 0; kv < 2; ++kv) {
     float x[CPL];
-    row_load<D>(x, (kv ? r.v_row : r.k_row) + lane * CPL, true);
+    row_load<D>(x, (kv ? v_row : k_row) + lane * CPL, true);
     __half s16, m16;
-    const uint32_t packed = row_quantize<D, ROT, LGB>(x, lane, r.quat, s16, m16);
-    row_store_codes<D>((kv ? r.v_codes : r.k_codes) + lane * (CPL / 2), packed);
-    if (lane == 0)
-      *(kv ? r.v_param : r.k_param) =
-          (uint32_t)__half_as_ushort(s16) | ((uint32_t)__half_as_ushort(m16) << 16);
+    const uint32_t packed = row_quantize<D, ROT, LGB>(x, lane, quat, s16, m16);
+    const uint32_t word =
+        (uint32_t)__half_as_ushort(s16) | ((uint32_t)__half_as_ushort(m16) << 16);
+    if (kv) {
+      o.vc = packed;
+      o.vp = word;
+    } else {
+      o.kc = packed;
+      o.kp = word;
+    }
   }
+  return o;
 }
 
 template <int D>
-__device__ __noinline__ void append_step_token(StepRowArgs r, int rot_kind, int lgb, int lane) {
-  if (rot_kind == KVQ_ROT_NONE) return step_rows<D, KVQ_ROT_NONE, 0>(r, lane);
-  if (rot_kind == KVQ_ROT_QUAT) return step_rows<D, KVQ_ROT_QUAT, 0>(r, lane);
+__device__ __noinline__ StepRow quantize_step_token(const __half* k_row, const __half* v_row,
+                                                    const float* quat, int rot_kind, int lgb,
+                                                    int lane) {
+  if (rot_kind == KVQ_ROT_NONE) return step_rows<D, KVQ_ROT_NONE, 0>(k_row, v_row, quat, lane);
+  if (rot_kind == KVQ_ROT_QUAT) return step_rows<D, KVQ_ROT_QUAT, 0>(k_row, v_row, quat, lane);
   switch (lgb) {
-    case 4: return step_rows<D, KVQ_ROT_HADAMARD, 4>(r, lane);
-    case 5: return step_rows<D, KVQ_ROT_HADAMARD, 5>(r, lane);
-    case 6: return step_rows<D, KVQ_ROT_HADAMARD, 6>(r, lane);
-    case 7: return step_rows<D, KVQ_ROT_HADAMARD, 7>(r, lane);
-    default: return step_rows<D, KVQ_ROT_HADAMARD, (D >= 256 ? 8 : 7)>(r, lane);
+    case 4: return step_rows<D, KVQ_ROT_HADAMARD, 4>(k_row, v_row, quat, lane);
+    case 5: return step_rows<D, KVQ_ROT_HADAMARD, 5>(k_row, v_row, quat, lane);
+    case 6: return step_rows<D, KVQ_ROT_HADAMARD, 6>(k_row, v_row, quat, lane);
+    case 7: return step_rows<D, KVQ_ROT_HADAMARD, 7>(k_row, v_row, quat, lane);
+    default: return step_rows<D, KVQ_ROT_HADAMARD, (D >= 256 ? 8 : 7)>(k_row, v_row, quat, lane);
   }
+}
+
+// Stores / loads a lane's CPL / 2 code bytes (shared or global memory).
+template <int D>
+__device__ __forceinline__ void put_codes(uint8_t* p, uint32_t packed) {
+  if (RowQuantShape<D>::CPL == 4)
+    *reinterpret_cast<uint16_t*>(p) = (uint16_t)packed;
+  else
+    *reinterpret_cast<uint32_t*>(p) = packed;
+}
+template <int D>
+__device__ __forceinline__ uint32_t get_codes(const uint8_t* p) {
+  if (RowQuantShape<D>::CPL == 4) return *reinterpret_cast<const uint16_t*>(p);
+  return *reinterpret_cast<const uint32_t*>(p);
 }
 
 // ---------------------------------------------------------------------------
@@ -144,7 +167,10 @@ struct DecCfg {
   static constexpr int STAGE_B = PG * PAGE_B;
   // pipeline depth: about 8-13 KB of pages in flight per warp
   static constexpr int NST = STAGE_B <= 2304 ? 4 : (STAGE_B <= 4608 ? 3 : 2);
-  static constexpr int WARP_B = (NST * STAGE_B + 127) / 128 * 128;
+  // behind the ring: the new token's K and V code rows and parameter words
+  // of a fused decode step, kept until its page is staged
+  static constexpr int STEP_B = (2 * ROWB + 8 + 127) / 128 * 128;
+  static constexpr int WARP_B = (NST * STAGE_B + STEP_B + 127) / 128 * 128;
 };
 // the bit-exact quantize path.
 template <int QW>
@@ -230,23 +256,14 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : (GP == 8 ? 3
   const int pg_hi = (int)(((int64_t)(split + 1) * npages) / a.splits);
   const int ngrp = (pg_hi - pg_lo + C::PG - 1) / C::PG;  // stage groups
   const int32_t* const bt_row = a.block_table + (int64_t)s * a.bt_stride;
-  // fused step: the warp that owns the page of position L - 1 writes the
-  // sequence's new token of this KV head before any of its copies start
-  if (a.k_new != nullptr && L >= 1 && (L - 1) / P >= pg_lo && (L - 1) / P < pg_hi) {
-    const int pos = L - 1;
-    const int page = bt_row[pos / P];
-    if (page >= 0 && page < a.NP) {
-      const int64_t dst = ((int64_t)page * a.H + h) * P + pos % P;
-      const int64_t src = (int64_t)s * a.new_stride + (int64_t)h * D;
-      const StepRowArgs rw{a.k_new + src, a.v_new + src, a.quat, a.k_codes_w + dst * (D / 2),
-                           a.v_codes_w + dst * (D / 2), a.k_params_w + dst, a.v_params_w + dst};
-      append_step_token<D>(rw, a.rot_kind, a.lgb, lane);
-      __threadfence();  // visible to this warp's page copies below
-      __syncwarp();
-    } else if (lane == 0) {
-      raise_flag(a.err, KVQ_ERRF_PAGE);
-    }
-  }
+  // fused step: the warp whose range holds the page of position L - 1
+  // quantizes the sequence's new token for this KV head (after its first
+  // copies are in flight, below), writes it to the pools and patches it into
+  // the staged copy of that page, so no fence or global round trip stands
+  // between the write and the attention that reads it
+  const int new_pg = L >= 1 ? (L - 1) / P : -1;
+  const bool step_owner = a.k_new != nullptr && new_pg >= pg_lo && new_pg < pg_hi;
+  int new_grp = -1;  // group of the new token's page (-1: none to patch)
   // The warp's block-table entries sit in lane registers, 32 pages at a
   // time: lane i holds the entry of page pg_lo + 32 c + i of chunk c. An
   // entry outside [0, NP) raises KVQ_ERRF_PAGE when it is loaded and its page
@@ -360,6 +377,29 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : (GP == 8 ? 3
     else
       cp_async_commit();
   }
+  uint8_t* const stash = ring + C::NST * C::STAGE_B;  // [K row][V row][K, V params]
+  if (step_owner) {
+    const int page = bt_row[new_pg];
+    if (page >= 0 && page < a.NP) {
+      const int64_t src = (int64_t)s * a.new_stride + (int64_t)h * D;
+      const StepRow nr =
+          quantize_step_token<D>(a.k_new + src, a.v_new + src, a.quat, a.rot_kind, a.lgb, lane);
+      const int64_t row = ((int64_t)page * a.H + h) * P + (L - 1) % P;
+      constexpr int LB = RowQuantShape<D>::CPL / 2;  // code bytes per lane
+      put_codes<D>(a.k_codes_w + row * (D / 2) + lane * LB, nr.kc);
+      put_codes<D>(a.v_codes_w + row * (D / 2) + lane * LB, nr.vc);
+      put_codes<D>(stash + lane * LB, nr.kc);
+      put_codes<D>(stash + C::ROWB + lane * LB, nr.vc);
+      if (lane == 0) {
+        a.k_params_w[row] = nr.kp;
+        a.v_params_w[row] = nr.vp;
+        *reinterpret_cast<uint2*>(stash + 2 * C::ROWB) = make_uint2(nr.kp, nr.vp);
+      }
+      new_grp = (new_pg - pg_lo) / C::PG;
+    } else if (lane == 0) {
+      raise_flag(a.err, KVQ_ERRF_PAGE);
+    }
+  }
 
   // ---- the query, while the first pages are in flight: rotated, then held
   // as a 26-bit fixed point qint = RN(qhat * 2^k) (2^k the power of two that
@@ -468,8 +508,25 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : (GP == 8 ? 3
       pgok[q] = (okbits >> (slot * C::PG + q)) & 1u;
       all_ok = all_ok && pgok[q];
     }
-    const uint8_t* st = ring + slot * C::STAGE_B;
+    uint8_t* const st = ring + slot * C::STAGE_B;
     slot = slot + 1 == C::NST ? 0 : slot + 1;
+    if (gi == new_grp) {
+      // the staged page may predate this launch's write of the new token:
+      // its rows and parameters are replaced by the stashed values (each
+      // lane copies the bytes it stashed)
+      constexpr int LB = RowQuantShape<D>::CPL / 2;
+      uint8_t* const pb = st + ((new_pg - pg_lo) % C::PG) * C::PAGE_B;
+      const int sl = (L - 1) % P;
+      put_codes<D>(pb + sl * C::ROWB + lane * LB, get_codes<D>(stash + lane * LB));
+      put_codes<D>(pb + C::CODE_B + sl * C::ROWB + lane * LB,
+                   get_codes<D>(stash + C::ROWB + lane * LB));
+      if (lane == 0) {
+        const uint2 pw = *reinterpret_cast<const uint2*>(stash + 2 * C::ROWB);
+        *reinterpret_cast<uint32_t*>(pb + 2 * C::CODE_B + sl * 4) = pw.x;
+        *reinterpret_cast<uint32_t*>(pb + 2 * C::CODE_B + P * 4 + sl * 4) = pw.y;
+      }
+      __syncwarp();
+    }
     const int tok0 = (pg_lo + gi * C::PG) * P;  // first token of the group
     // groups whose every token is cached skip all per-token masking
     const bool full = all_ok && tok0 + C::PG * P <= L;
@@ -720,133 +777,144 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : (GP == 8 ? 3
   for (int hc = 0; hc < 2; ++hc) {
     const int gh = c0 + hc;
     if (!writer || gh >= a.G) continue;
-    float* dst = a.part + (base + (int64_t)gh * a.splits) * (D + 4);
+    // lane row r holds channels [r*D/8, (r+1)*D/8) of head gh: m-tile mt,
+    // row slot r <- channel r*D/8 + 16*(mt/8) + mt%8, row slot r+8 <- that
+    // channel + 8
+    float4* dst = reinterpret_cast<float4*>(a.part + (base + (int64_t)gh * a.splits) * (D + 4) +
+                                            r * (D / 8));
     const float ov = hc ? o1 : o0;
 #pragma unroll
-    for (int mt = 0; mt < C::NMT; ++mt) {
-      // m-tile mt, row slot r <- channel r*D/8 + 16*(mt/8) + mt%8,
-      // row slot r+8 <- that channel + 8
-      const int ch0 = r * (D / 8) + 16 * (mt / 8) + (mt % 8);
-      dst[ch0] = acc[mt][hc] + ov;
-      dst[ch0 + 8] = acc[mt][2 + hc] + ov;
-    }
+    for (int gq = 0; gq < D / 128; ++gq)
+#pragma unroll
+      for (int half = 0; half < 2; ++half)
+#pragma unroll
+        for (int q4 = 0; q4 < 2; ++q4) {
+          const int mt = 8 * gq + 4 * q4;
+          const int e = 2 * half + hc;
+          dst[4 * gq + 2 * half + q4] = make_float4(acc[mt][e] + ov, acc[mt + 1][e] + ov,
+                                                    acc[mt + 2][e] + ov, acc[mt + 3][e] + ov);
+        }
   }
   // the lanes that own head hr's softmax state write it (one lane per head)
   if (j == 0 && !lo_row && head_ok) {
     float* dst = a.part + (base + (int64_t)hr * a.splits) * (D + 4);
-    dst[D] = M;
-    dst[D + 1] = Lp;
+    *reinterpret_cast<float2*>(dst + D) = make_float2(M, Lp);
   }
+}
 
-  // ---- the last warp of this (sequence, KV head) merges the splits
-  // The warp's partial writes are ordered before lane 0's counter update by
-  // the warp barrier; the update is a release (publishes them) and an
-  // acquire (the last arriver then sees every split's writes).
-  __syncwarp();
-  int last = 0;
-  if (lane == 0) {
-    int prev;
-    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;"
-                 : "=r"(prev)
-                 : "l"(a.counter + (int64_t)s * a.H + h)
-                 : "memory");
-    last = prev == a.splits - 1;
-  }
-  last = __shfl_sync(0xffffffffu, last, 0);
-  if (!last) return;
-  // the shuffle carries no memory ordering: the warp barrier extends lane
-  // 0's acquire to every lane before they read the other splits' partials
-  __syncwarp();
-  const bool owner = head_ok && !lo_row;
-  // lanes of head hr: quarter j of the channels; for GP = 4 the partner
-  // lanes r + 4 take the odd splits and the two halves are added at the end
-  // Channels of the merge: GP = 4: lane (j, own) of a head takes
-  // j*QW + own*QW/2 + [0, QW/2) (the 8 lanes of a head cover it); GP = 8:
-  // lane j takes the quarter j*QW + [0, QW). Loads go out in rounds of RB
-  // splits, the first round together with the splits' maxima.
-  constexpr int CW = GP == 4 ? C::QW / 2 : C::QW;
-  constexpr int RB = CW <= 16 ? 4 : (CW <= 32 ? 2 : 1);  // float4 loads per lane per round <= 16
-  const int coff = j * C::QW + (GP == 4 ? own * (C::QW / 2) : 0);
-  const float* src = a.part + ((int64_t)s * a.Hq + g) * a.splits * (D + 4);
-  const int nsp = head_ok ? a.splits : 0;
-  float Mx = -INFINITY;
-  {
-    // the splits' maxima: the NL lanes of the head load interleaved splits
-    constexpr int NL = GP == 4 ? 8 : 4;
-    const int li0 = GP == 4 ? 4 * own + j : j;
-    for (int i0 = 0; i0 < nsp; i0 += 4 * NL) {
-      float mv[4];
+// ---------------------------------------------------------------------------
+// 3. merge kernel: one warp per (sequence, query head), launched after the
+// split kernel with programmatic serialization (its blocks wait for every
+// split's partial result). Lane l owns channels [l*CPL, (l+1)*CPL). The
+// splits' (acc, M, L) are combined in rounds of RB with a running maximum
+// (log-sum-exp), normalised by the total weight, rotated back by R^-1 and
+// written as the float32 output.
+// ---------------------------------------------------------------------------
+
+struct MergeArgs {
+  int S, Hq, splits, rot_kind, lgb;
+  const float* quat;
+  const float* part;  // [S][Hq][splits][D + 4]
+  float* out;         // [S][Hq][D]
+};
+
+// R^-1 of a row held as CPL consecutive channels per lane over the 32 lanes
+// (the inverse of the block Hadamard rotation is the rotation itself; the
+// quaternion map is inverted block by block). Binary32, not part of the
+// bit-exact quantize path.
+template <int CPL>
+__device__ __forceinline__ void row_unrotate(float (&x)[CPL], int lane, int rot_kind, int lgb,
+                                             const float* quat) {
+  if (rot_kind == KVQ_ROT_HADAMARD) {
+    const int b = 1 << lgb;
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const int i = i0 + li0 + NL * m;
-        mv[m] = i < nsp ? __ldcg(src + (int64_t)i * (D + 4) + D) : -INFINITY;
+    for (int dd = 1; dd < CPL; dd <<= 1) {
+      if (dd >= b) break;
+#pragma unroll
+      for (int i = 0; i < CPL; ++i) {
+        if ((i & dd) == 0) {
+          const float p = x[i], q = x[i + dd];
+          x[i] = p + q;
+          x[i + dd] = p - q;
+        }
       }
-      Mx = fmaxf(Mx, fmaxf(fmaxf(mv[0], mv[1]), fmaxf(mv[2], mv[3])));
     }
-  }
-  float xm[CW];
+    for (int m = 1; m * CPL < b; m <<= 1) {
+      const bool lower = (lane & m) == 0;
 #pragma unroll
-  for (int c = 0; c < CW; ++c) xm[c] = 0.f;
-  float Ls = 0.f;
-  for (int i0 = 0; i0 < (nsp > 0 ? nsp : 1); i0 += RB) {
-    float4 f[RB][CW / 4];
-    float Mi[RB];
-    float li[RB];
+      for (int i = 0; i < CPL; ++i) {
+        const float o = __shfl_xor_sync(0xffffffffu, x[i], m);
+        x[i] = lower ? x[i] + o : o - x[i];
+      }
+    }
+    const float cb = hadamard_scale(lgb);
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) x[i] *= cb;
+  } else if (rot_kind == KVQ_ROT_QUAT) {
+    quat_inv_regs<CPL>(x, quat, lane * CPL);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kDecWarps * kWarp) decode_merge_kernel(const MergeArgs m) {
+  constexpr int CPL = D / 32;              // channels per lane
+  constexpr int RB = CPL == 4 ? 16 : 8;    // splits per round
+  pdl_wait();  // every partial result of the split kernel is written
+  pdl_trigger();
+  const int lane = threadIdx.x % kWarp;
+  const int gw = blockIdx.x * kDecWarps + threadIdx.x / kWarp;
+  if (gw >= m.S * m.Hq) return;
+  const float* src = m.part + (int64_t)gw * m.splits * (D + 4);
+  float Mr = -INFINITY, Ls = 0.f;
+  float x[CPL];
+#pragma unroll
+  for (int c = 0; c < CPL; ++c) x[c] = 0.f;
+  for (int i0 = 0; i0 < m.splits; i0 += RB) {
+    float4 f[RB][CPL / 4];
+    float2 ml[RB];  // (M, L) of each split
 #pragma unroll
     for (int rb = 0; rb < RB; ++rb) {
       const int i = i0 + rb;
       const float* pi = src + (int64_t)i * (D + 4);
-      const bool in = i < nsp;
-      Mi[rb] = in ? __ldcg(pi + D) : -INFINITY;
-      li[rb] = in ? __ldcg(pi + D + 1) : 0.f;
+      const bool in = i < m.splits;
+      ml[rb] = in ? __ldcg(reinterpret_cast<const float2*>(pi + D)) : make_float2(-INFINITY, 0.f);
 #pragma unroll
-      for (int c = 0; c < CW / 4; ++c)
-        f[rb][c] = in ? __ldcg(reinterpret_cast<const float4*>(pi + coff) + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int c = 0; c < CPL / 4; ++c)
+        f[rb][c] = in ? __ldcg(reinterpret_cast<const float4*>(pi + lane * CPL) + c)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    if (i0 == 0) {  // every lane of a head ends with the head's maximum
-      Mx = fmaxf(Mx, __shfl_xor_sync(0xffffffffu, Mx, 1));
-      Mx = fmaxf(Mx, __shfl_xor_sync(0xffffffffu, Mx, 2));
-      if (GP == 4) Mx = fmaxf(Mx, __shfl_xor_sync(0xffffffffu, Mx, 16));
+    float Mc = Mr;
+#pragma unroll
+    for (int rb = 0; rb < RB; ++rb) Mc = fmaxf(Mc, ml[rb].x);
+    if (Mc != Mr) {  // rescale what is summed so far (Mr = -inf: nothing yet)
+      const float sc = Mr == -INFINITY ? 0.f : fast_exp2(Mr - Mc);
+      Ls *= sc;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) x[c] *= sc;
+      Mr = Mc;
     }
 #pragma unroll
     for (int rb = 0; rb < RB; ++rb) {
       // an empty split (max -inf) has a zero row and a zero sum: weight 0
-      const float wgt = Mi[rb] == -INFINITY ? 0.f : fast_exp2(Mi[rb] - Mx);
-      Ls += wgt * li[rb];
+      const float wgt = ml[rb].x == -INFINITY ? 0.f : fast_exp2(ml[rb].x - Mr);
+      Ls = fmaf(wgt, ml[rb].y, Ls);
 #pragma unroll
-      for (int c = 0; c < CW / 4; ++c) {
-        xm[4 * c] += wgt * f[rb][c].x;
-        xm[4 * c + 1] += wgt * f[rb][c].y;
-        xm[4 * c + 2] += wgt * f[rb][c].z;
-        xm[4 * c + 3] += wgt * f[rb][c].w;
+      for (int c = 0; c < CPL / 4; ++c) {
+        x[4 * c] = fmaf(wgt, f[rb][c].x, x[4 * c]);
+        x[4 * c + 1] = fmaf(wgt, f[rb][c].y, x[4 * c + 1]);
+        x[4 * c + 2] = fmaf(wgt, f[rb][c].z, x[4 * c + 2]);
+        x[4 * c + 3] = fmaf(wgt, f[rb][c].w, x[4 * c + 3]);
       }
     }
   }
-  // the whole quarter in every lane of the head (GP = 4: swap halves)
-  float x[C::QW];
-  if (GP == 4) {
+  const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
 #pragma unroll
-    for (int c = 0; c < CW; ++c) {
-      const float o = __shfl_xor_sync(0xffffffffu, xm[c], 16);
-      x[c] = own ? o : xm[c];
-      x[CW + c] = own ? xm[c] : o;
-    }
-  } else {
+  for (int c = 0; c < CPL; ++c) x[c] *= inv;
+  row_unrotate<CPL>(x, lane, m.rot_kind, m.lgb, m.quat);
+  float4* dst = reinterpret_cast<float4*>(m.out + (int64_t)gw * D + lane * CPL);
 #pragma unroll
-    for (int c = 0; c < C::QW; ++c) x[c] = xm[c % CW];
-  }
-  {
-    const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
-#pragma unroll
-    for (int c = 0; c < C::QW; ++c) x[c] *= inv;
-  }
-  rotate_quarter<C::QW>(x, j, a.rot_kind, a.lgb, a.quat, true);  // R^-1 (R^-1 = R for Hadamard)
-  if (owner) {
-    float4* dst = reinterpret_cast<float4*>(a.out + ((int64_t)s * a.Hq + g) * D + j * C::QW);
-#pragma unroll
-    for (int c = 0; c < C::QW / 4; ++c) dst[c] = make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]);
-  }
-  if (lane == 0) a.counter[(int64_t)s * a.H + h] = 0;
+  for (int c = 0; c < CPL / 4; ++c)
+    dst[c] = make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]);
 }
 
 // ---------------------------------------------------------------------------
@@ -887,8 +955,6 @@ static int resident_warps(int D, int P, int GP) {
   return 148 * 8;
 }
 
-static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
-
 DecodePlan decode_plan(const kvq_cache_desc& d, int32_t S, int32_t Hq, int32_t max_seq_len) {
   DecodePlan pl{};
   const int P = d.page_size;
@@ -908,9 +974,7 @@ DecodePlan decode_plan(const kvq_cache_desc& d, int32_t S, int32_t Hq, int32_t m
   if (splits > pl.pages_max) splits = pl.pages_max;
   pl.pages_per_split = (pl.pages_max + splits - 1) / splits;
   pl.splits = (pl.pages_max + pl.pages_per_split - 1) / pl.pages_per_split;
-  const size_t counters = (size_t)S * d.num_kv_heads * sizeof(int32_t);
-  const size_t parts = (size_t)S * Hq * pl.splits * (d.head_dim + 4) * sizeof(float);
-  pl.workspace = align256(counters) + parts;
+  pl.workspace = (size_t)S * Hq * pl.splits * (d.head_dim + 4) * sizeof(float);
   return pl;
 }
 
@@ -960,9 +1024,7 @@ int decode_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, const void* q,
   a.k_codes = k_codes; a.k_params = static_cast<const uint32_t*>(k_params);
   a.v_codes = v_codes; a.v_params = static_cast<const uint32_t*>(v_params);
   a.out = out;
-  a.counter = static_cast<int32_t*>(workspace);
-  a.part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                    align256((size_t)S * d.num_kv_heads * sizeof(int32_t)));
+  a.part = static_cast<float*>(workspace);
   a.err = err;
   a.k_new = step ? static_cast<const __half*>(step->k_new) : nullptr;
   a.v_new = step ? static_cast<const __half*>(step->v_new) : nullptr;
@@ -971,8 +1033,16 @@ int decode_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, const void* q,
   a.v_codes_w = const_cast<uint8_t*>(v_codes);
   a.k_params_w = static_cast<uint32_t*>(const_cast<void*>(k_params));
   a.v_params_w = static_cast<uint32_t*>(const_cast<void*>(v_params));
-  const cudaError_t e = launch_split_any(a, D, GP, st);
+  cudaError_t e = launch_split_any(a, D, GP, st);
   if (e == cudaErrorInvalidValue) return KVQ_ERR_UNSUPPORTED;
+  if (e != cudaSuccess) return KVQ_ERR_CUDA;
+  MergeArgs mg;
+  mg.S = S; mg.Hq = Hq; mg.splits = pl.splits; mg.rot_kind = d.rot_kind; mg.lgb = lgb;
+  mg.quat = d.quat; mg.part = a.part; mg.out = out;
+  const int mgrid = (S * Hq + kDecWarps - 1) / kDecWarps;
+  e = D == 128 ? launch_pdl(decode_merge_kernel<128>, mgrid, kDecWarps * kWarp, 0, st, mg)
+               : launch_pdl(decode_merge_kernel<256>, mgrid, kDecWarps * kWarp, 0, st, mg);
+  if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 

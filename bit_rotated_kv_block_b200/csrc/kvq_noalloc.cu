@@ -105,12 +105,9 @@ extern "C" int kvq_paged_decode_attn_noalloc(
   void* scratch = nullptr;
   const int st = scratch_address(&scratch);
   if (st != KVQ_OK) return st;
-  // the per-(sequence, KV head) counters at the start of the scratch must be
-  // zero when the kernel starts; the previous call normally leaves them so,
-  // but a call that failed part-way might not: clear them on the stream
-  const size_t counters = (size_t)num_seqs * desc->num_kv_heads * sizeof(int32_t);
-  if (cudaMemsetAsync(scratch, 0, counters, static_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return KVQ_ERR_CUDA;
+  // every byte the decode kernels read from the scratch is written by the
+  // same call first (the partial result of each split), so nothing left by
+  // an earlier call needs clearing
   return kvq_paged_decode_attn(desc, num_seqs, num_q_heads, q, seq_lens, max_seq_len,
                                block_table, bt_stride, sm_scale, k_codes, k_params, v_codes,
                                v_params, out, scratch, kNoallocScratchBytes, err_flags, stream);

@@ -141,9 +141,9 @@ def decode_workspace_bytes(cache, num_seqs, num_q_heads, max_seq_len):
 
 def paged_decode_attn(cache, q, seq_lens, max_seq_len, block_table, k_codes, k_params, v_codes,
                       v_params, out=None, workspace=None, sm_scale=None, err=None, stream=None):
-    """q: float16 CUDA [S][Hq][d]; returns float32 [S][Hq][d]. A given
-    workspace must have been zero-filled before its first use (the calls keep
-    its counters at zero); without one, a zeroed one is allocated."""
+    """q: float16 CUDA [S][Hq][d]; returns float32 [S][Hq][d]. The workspace
+    (``decode_workspace_bytes``) needs no initialisation; without one, one is
+    allocated for the call."""
     S, Hq, d = q.shape
     if sm_scale is None:
         sm_scale = 1.0 / math.sqrt(d)
@@ -151,7 +151,7 @@ def paged_decode_attn(cache, q, seq_lens, max_seq_len, block_table, k_codes, k_p
         out = torch.empty((S, Hq, d), dtype=torch.float32, device=q.device)
     need = decode_workspace_bytes(cache, S, Hq, max_seq_len)
     if workspace is None:
-        workspace = torch.zeros(max(need, 16), dtype=torch.uint8, device=q.device)
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     st = lib().kvq_paged_decode_attn(ctypes.byref(cache.desc), S, Hq, _ptr(q), _ptr(seq_lens),
                                      int(max_seq_len), _ptr(block_table),
                                      int(block_table.shape[1]), float(sm_scale), _ptr(k_codes),
@@ -177,7 +177,7 @@ def decode_step(cache, q, k_new, v_new, seq_lens, max_seq_len, block_table, k_co
         out = torch.empty((S, Hq, d), dtype=torch.float32, device=q.device)
     need = decode_workspace_bytes(cache, S, Hq, max_seq_len)
     if workspace is None:
-        workspace = torch.zeros(max(need, 16), dtype=torch.uint8, device=q.device)
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     new_stride = k_new.stride(0)
     if v_new.stride(0) != new_stride:
         raise ValueError("k_new and v_new must share the row stride")

@@ -139,11 +139,10 @@ int kvq_quantize_append(const kvq_cache_desc* desc, int32_t num_tokens, const vo
 /*
  * kvq_decode_workspace_bytes -- bytes of device workspace that
  * kvq_paged_decode_attn needs for these sizes (0 on invalid arguments). The
- * workspace holds one counter per (sequence, KV head) followed by per-split
- * partial results. It must be zero-filled before its first use; every call
- * that returns KVQ_OK leaves the counters at zero again, so one zeroed
- * workspace serves any number of later calls on the same stream. Calls that
- * share a workspace must not overlap in time.
+ * workspace holds the per-split partial results (float32, written and then
+ * read by each call); it needs no initialisation, and one workspace serves
+ * any number of later calls on the same stream. Calls that share a
+ * workspace must not overlap in time.
  */
 size_t kvq_decode_workspace_bytes(const kvq_cache_desc* desc, int32_t num_seqs,
                                   int32_t num_q_heads, int32_t max_seq_len);
@@ -159,8 +158,8 @@ size_t kvq_decode_workspace_bytes(const kvq_cache_desc* desc, int32_t num_seqs,
  *  max_seq_len  upper bound of seq_lens (sizes the split-K work).
  *  sm_scale     softmax scale (typically 1/sqrt(d)).
  *  out          float32 [S][Hq][d], in the original (un-rotated) basis.
- *  workspace    >= kvq_decode_workspace_bytes(...) bytes, 16-byte aligned,
- *               zero-filled before its first use (see above).
+ *  workspace    >= kvq_decode_workspace_bytes(...) bytes, 16-byte aligned
+ *               (see above).
  *
  * For query head g (KV head h = g / (Hq/H)): qhat = R q_g;
  * z_j = sm_scale * qhat . khat_j; p = softmax(z); out = R^-1 sum_j p_j vhat_j,
@@ -192,7 +191,7 @@ int kvq_dequantize_pages(const kvq_cache_desc* desc, int32_t num_seqs,
                          int32_t* err_flags, void* stream);
 
 /*
- * kvq_decode_step -- one decode step in one launch: for every sequence s with
+ * kvq_decode_step -- one decode step in one call: for every sequence s with
  * seq_lens[s] >= 1, the new token's K and V rows are rotated, quantized and
  * written at position seq_lens[s] - 1 exactly as kvq_quantize_append writes
  * them (token_seq = s, token_pos = seq_lens[s] - 1), and decode attention then
@@ -200,9 +199,9 @@ int kvq_dequantize_pages(const kvq_cache_desc* desc, int32_t num_seqs,
  * and the output equal those of the two calls in that order. The quantized
  * write inside the paged cache follows the method (page "SAW-INT4:
  * System-Aware 4-Bit KV-Cache Quantization for Real-World LLM Serving",
- * Summary and Method); doing it inside the attention launch, by the warp that
- * reads that page, is this library's own step (one launch per step, and the
- * write overlaps the launch's start-up latency).
+ * Summary and Method); doing it inside the attention kernel, by the warp
+ * that reads that page, is this library's own step (the write needs no
+ * launch of its own and overlaps the attention's start-up latency).
  *
  *  k_new, v_new  device binary16 rows of the new tokens: row (s, h) starts at
  *                element s * new_stride + h * head_dim; 16-byte aligned,
@@ -267,8 +266,8 @@ int kvq_paged_decode_attn_fp16(const kvq_cache_desc* desc, int32_t num_seqs,
  * `workspace` / `workspace_bytes`. The scratch is a 16 MiB array compiled
  * into the library (KVQ_NOALLOC_SCRATCH_BYTES): every GPU that loads libkvq
  * holds it until the process exits. The call allocates and frees nothing;
- * it enqueues one cudaMemsetAsync (clearing the split counters at the start
- * of the scratch) and the decode kernel on `stream`.
+ * it enqueues the decode kernels on `stream`. Nothing in the scratch needs
+ * clearing between calls: each call writes every byte it reads there.
  *  - Sizes whose workspace (kvq_decode_workspace_bytes) exceeds
  *    KVQ_NOALLOC_SCRATCH_BYTES are rejected with KVQ_ERR_WORKSPACE before
  *    anything is launched.
