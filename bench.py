@@ -252,7 +252,9 @@ def run_ours(args, world, rank, local):
     ws = torch.zeros(kvq.decode_workspace_bytes(c0, S, Hq, L), dtype=torch.uint8, device=device)
     err = torch.zeros(1, dtype=torch.int32, device=device)
     stream = torch.cuda.current_stream()
-    launches_per_step = 1  # kvq_decode_step: new-token append and attention in one kernel
+    # kvq_decode_step: the split kernel (new-token append and attention over
+    # page ranges) and the merge kernel of the splits
+    launches_per_step = 2
 
     def step(i):
         c, kc, kp, vc, vp = caches[i % 2]
@@ -270,10 +272,11 @@ def run_ours(args, world, rank, local):
     barrier(world)
     torch.cuda.synchronize()
     t0.record(stream)
-    # the timed region holds nothing but the step kernels (one per step,
-    # launched with programmatic serialization so each starts while the
-    # previous one drains); its duration per step is the kernel's launch
-    # duration used for the roofline
+    # the timed region holds nothing but the step kernels (a split and a merge
+    # kernel per step, launched with programmatic serialization so each starts
+    # while the previous one drains); its duration per step bounds the split
+    # kernel's launch duration from above, so the roofline figure derived
+    # from it is conservative
     for i in range(steps):
         c, kc, kp, vc, vp = caches[i % 2]
         kvq.decode_step(c, Q, SK, SV, LENS, L, BT, kc, kp, vc, vp, out=out, workspace=ws, err=err)
@@ -345,7 +348,8 @@ def run_ours(args, world, rank, local):
                    "global_batch": S * world, "seq_len": L, "parallelism": f"replicas x{world}",
                    "l2": "steps alternate between 2 cache replicas (2 x 143 MB > 126 MB L2)"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": traffic, "kernel": "decode attention",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "kernel": "decode step (split kernel; per-step time incl. the merge kernel)",
                      "bytes_per_launch": dec_bytes, "peak_source": peak_kind,
                      "frac_nominal": achieved / NOMINAL_HBM_GBS},
         "append_prefill": {"gbs": app_bytes / t_app / 1e9, "frac": app_bytes / t_app / 1e9 / peak,
@@ -649,14 +653,25 @@ def workload_records(device, seed=0):
     del reps, ws, K, V, page, slot, TS, TP
     torch.cuda.empty_cache()
 
-    # ---- prefill sweep: one layer per Hadamard block size
+    # ---- prefill sweep: one layer per Hadamard block size, then the other
+    # rotation kinds (quaternion full and fast maps, randomised-sign b 64)
     sweep = {"workload": "65536 tokens x 8 KV heads x d 128 per layer, page 16"}
-    for blk in (16, 32, 64, 128, 0):
+    variants = [(workloads.ROT_HADAMARD, b, "hadamard%d" % b) for b in (16, 32, 64, 128)]
+    variants += [(workloads.ROT_NONE, 0, "no_rotation"),
+                 (workloads.ROT_QUAT, 0, "quaternion"),
+                 (workloads.ROT_QUAT_FAST, 0, "quaternion_fast"),
+                 (workloads.ROT_HADAMARD_SIGNED, 64, "hadamard64_signed")]
+    for kind, blk, name in variants:
         w = workloads.prefill(seed=seed, rot_block=blk)
         ts, tp = _all_tokens(w)
         K, V = _device_kv(w, len(ts), gen, device)
         TS, TP, BT = dev(ts), dev(tp), dev(w.block_table)
-        c = kvq.Cache(w.d, w.H, w.P, w.NP, w.rot_kind, w.rot_block, device=device)
+        table = None
+        if kind in (workloads.ROT_QUAT, workloads.ROT_QUAT_FAST):
+            table = workloads.random_quaternions(seed, w.d)
+        elif kind == workloads.ROT_HADAMARD_SIGNED:
+            table = workloads.random_signs(seed, w.d)
+        c = kvq.Cache(w.d, w.H, w.P, w.NP, kind, blk, table, device=device)
         kc, kp = c.new_pools(device=device, fill=0)
         vc, vp = c.new_pools(device=device, fill=0)
         t = _device_time_us(lambda i: kvq.quantize_append(c, K, V, TS, TP, BT, kc, kp, vc, vp),
@@ -671,12 +686,12 @@ def workload_records(device, seed=0):
             mse += float(((xh.double() - x) ** 2).mean()) / 2
             del xh, x
         r["mse"] = mse
-        sweep["hadamard%d" % blk if blk else "no_rotation"] = r
+        sweep[name] = r
         del K, V, kc, kp, vc, vp
         torch.cuda.empty_cache()
-    for blk in (16, 32, 64, 128):
-        sweep["hadamard%d" % blk]["rotation_overhead"] = (
-            sweep["hadamard%d" % blk]["us"] / sweep["no_rotation"]["us"] - 1)
+    for name in sweep:
+        if name not in ("workload", "no_rotation"):
+            sweep[name]["rotation_overhead"] = sweep[name]["us"] / sweep["no_rotation"]["us"] - 1
     res["prefill_append_sweep"] = sweep
 
     # ---- ragged head_dim 256: one fused decode step over the whole batch

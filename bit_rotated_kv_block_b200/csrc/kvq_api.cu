@@ -38,15 +38,25 @@ static int check_desc(const kvq_cache_desc* d) {
     case KVQ_ROT_NONE:
       break;
     case KVQ_ROT_HADAMARD:
+    case KVQ_ROT_HADAMARD_SIGNED:
       if (!pow2(d->rot_block) || d->rot_block > d->head_dim) return KVQ_ERR_INVALID_ARG;
       if (d->rot_block < 16 || d->rot_block > 256) return KVQ_ERR_UNSUPPORTED;
+      if (d->rot_kind == KVQ_ROT_HADAMARD_SIGNED) {
+        if (d->quat == nullptr) return KVQ_ERR_INVALID_ARG;
+        if (!aligned16(d->quat)) return KVQ_ERR_MISALIGNED;
+      }
       break;
     case KVQ_ROT_QUAT:
+    case KVQ_ROT_QUAT_FAST:
       if (d->quat == nullptr) return KVQ_ERR_INVALID_ARG;
       if (!aligned16(d->quat)) return KVQ_ERR_MISALIGNED;
       break;
     default:
       return KVQ_ERR_INVALID_ARG;
+  }
+  if (d->rope != nullptr) {
+    if (d->rope_max_pos < 1) return KVQ_ERR_INVALID_ARG;
+    if (!aligned16(d->rope)) return KVQ_ERR_MISALIGNED;
   }
   return KVQ_OK;
 }

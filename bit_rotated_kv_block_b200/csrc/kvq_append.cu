@@ -29,6 +29,8 @@
 //    consecutive lines of the swizzled boxes, and the destination of each
 //    row (token -> sequence, position -> block table) is resolved one tile
 //    ahead of its use.
+//  * An optional RoPE table turns every key row before the rotation
+//    (binary32, products and sums rounded separately).
 //  * Arithmetic is bit-exact with the published definition (see kvq.h):
 //    binary32 butterflies in ascending stage order (packed f32x2 lanes for
 //    stages >= 2), directed roundings through __fsub_ru / __fdiv_ru /
@@ -60,6 +62,133 @@ __host__ __device__ constexpr int append_e(int D, int rot, int lgb) {
 __host__ __device__ constexpr int append_threads(int E) { return E == 64 ? 256 : 384; }
 __host__ __device__ constexpr int append_ctas_per_sm(int E) { return E == 64 ? 2 : 1; }
 
+// One thread's part of one row: E channels of a (token, head) row of K or
+// V, read from the row's line of the 128-byte swizzled TMA boxes (channel
+// block c of the row sits in box my_part * E/64 + c/8, 16-byte chunk c % 8 at
+// position (c % 8) ^ (line & 7)); rotated, quantized and stored at row
+// dst_cur of the pools (no store when dst_cur < 0). The two threads of a row
+// with E < D are lanes 2i, 2i+1 of one warp.
+// With a RoPE table row cs (key rows; NULL otherwise) the row's channel
+// pairs are turned before the rotation.
+// For ROT == KVQ_ROT_HADAMARD a non-NULL qtbl is the sign table of the
+// randomised-sign Hadamard (channels flipped before the butterflies).
+// PRE: the kernel turns rows (RoPE) or flips signs before the rotation; without
+// it the first butterfly stage is taken straight from binary16.
+template <int D, int ROT, int LGB, bool PRE>
+__device__ __forceinline__ void quantize_row_part(const uint8_t* boxes, int box_stride,
+                                                  int my_line, int my_part, const float* qtbl,
+                                                  const float* cs, int64_t dst_cur,
+                                                  uint8_t* codes, uint32_t* params) {
+  constexpr bool fused1 = ROT == KVQ_ROT_HADAMARD && !PRE;
+  constexpr int E = append_e(D, ROT, LGB);  // channels per thread
+  constexpr int TPR = D / E;                // threads per row
+  float x[E];
+#pragma unroll
+  for (int c = 0; c < E / 8; ++c) {
+    // channel block c of this thread: box (part*E/64 + c/8), 16-byte
+    // chunk c%8 of line my_line, at its 128B-swizzled position
+    const uint8_t* box = boxes + (my_part * (E / 64) + c / 8) * box_stride;
+    const uint4 u = *reinterpret_cast<const uint4*>(
+        box + my_line * 128 + (((c % 8) ^ (my_line & 7)) << 4));
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const __half2 h2 = u32_as_h2(w[q]);
+      if (fused1) {
+        // first butterfly stage straight from binary16: widening is
+        // exact, so (x_i + x_{i+1}, x_i - x_{i+1}) round as in binary32
+        const float b = __high2float(h2);
+        x[8 * c + 2 * q] = add_h_f(__low2half(h2), b);
+        x[8 * c + 2 * q + 1] = sub_h_f(__low2half(h2), b);
+      } else {
+        const float2 f = __half22float2(h2);
+        x[8 * c + 2 * q] = f.x;
+        x[8 * c + 2 * q + 1] = f.y;
+      }
+    }
+  }
+
+  // the two threads of a d = 256 row are lanes 2i, 2i+1 of one warp
+  const unsigned pair_mask = 3u << ((threadIdx.x % kWarp) & ~1);
+  if (PRE && cs != nullptr) rope_regs<E>(x, cs + my_part * E);
+  if (ROT == KVQ_ROT_HADAMARD) {
+    if (fused1) {
+      hadamard_regs<E, LGB, true>(x, my_part, pair_mask);  // first stage done on load
+    } else {
+      if (PRE && qtbl != nullptr) sign_regs<E>(x, qtbl + my_part * E);
+      hadamard_regs<E, LGB, false>(x, my_part, pair_mask);
+    }
+  } else if (ROT == KVQ_ROT_QUAT_FAST) {
+    quat_fast_regs<E>(x, qtbl, my_part * E);
+  } else if (ROT == KVQ_ROT_QUAT) {
+    quat_regs<E>(x, qtbl, my_part * E);
+  }
+
+  // row statistics
+  float mn0 = fminf(x[0], x[1]), mx0 = fmaxf(x[0], x[1]);
+  float mn1 = fminf(x[2], x[3]), mx1 = fmaxf(x[2], x[3]);
+#pragma unroll
+  for (int i = 4; i < E; i += 4) {
+    mn0 = min3(mn0, x[i], x[i + 1]);
+    mn1 = min3(mn1, x[i + 2], x[i + 3]);
+    mx0 = max3(mx0, x[i], x[i + 1]);
+    mx1 = max3(mx1, x[i + 2], x[i + 3]);
+  }
+  float mn = fminf(mn0, mn1);
+  float mx = fmaxf(mx0, mx1);
+  if (TPR == 2) {
+    mn = fminf(mn, __shfl_xor_sync(pair_mask, mn, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(pair_mask, mx, 1));
+  }
+  mn = __fadd_rn(mn, 0.0f);
+  mx = __fadd_rn(mx, 0.0f);
+  const __half m16 = __float2half_rd(mn);
+  const float m = __half2float(m16);
+  const float s32 = __fdiv_ru(__fsub_ru(mx, m), 15.0f);
+  const __half s16 = __float2half_ru(s32);
+  const float s = __half2float(s16);
+
+  uint32_t packed[E / 8];
+  if (s != 0.0f) {
+    const float inv = __frcp_rn(s);
+    const uint64_t m2 = pk(m, m), inv2 = pk(inv, inv);
+    const uint64_t magic2 = pk(12582912.0f, 12582912.0f);  // 1.5 * 2^23
+#pragma unroll
+    for (int c = 0; c < E / 8; ++c) {
+      uint32_t b[8];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        // code = nearest integer (ties to even) of the exact product
+        // t * inv: one fused multiply-add with 1.5 * 2^23 rounds it
+        // once, leaving the integer in the low mantissa bits
+        const uint64_t t = sub2(pk(x[8 * c + 2 * q], x[8 * c + 2 * q + 1]), m2);
+        const float2 r = upk(fma2(t, inv2, magic2));
+        b[2 * q] = __float_as_uint(r.x);
+        b[2 * q + 1] = __float_as_uint(r.y);
+      }
+      // low byte of each pair = c_even | c_odd << 4 (no carry: both <= 15)
+      const uint32_t p0 = b[0] + (b[1] << 4), p1 = b[2] + (b[3] << 4);
+      const uint32_t p2 = b[4] + (b[5] << 4), p3 = b[6] + (b[7] << 4);
+      packed[c] = __byte_perm(__byte_perm(p0, p1, 0x0040), __byte_perm(p2, p3, 0x0040),
+                              0x5410);
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < E / 8; ++c) packed[c] = 0u;
+  }
+
+  if (dst_cur >= 0) {
+    uint4* dst = reinterpret_cast<uint4*>(codes + dst_cur * (D / 2) + my_part * (E / 2));
+#pragma unroll
+    for (int c = 0; c < E / 32; ++c)
+      dst[c] = make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+    if (my_part == 0) {
+      params[dst_cur] =
+          (uint32_t)__half_as_ushort(s16) | ((uint32_t)__half_as_ushort(m16) << 16);
+    }
+  }
+}
+
 struct AppendArgs {
   int T, H, P, lg_page, NP, num_seqs, bt_stride, tok_per_tile, num_tiles;
   int box_stride;  // bytes between TMA boxes in a tile buffer (multiple of 1024)
@@ -71,11 +200,14 @@ struct AppendArgs {
   uint32_t* k_params;
   uint32_t* v_params;
   const float* quat;
+  const float* rope;  // RoPE table [rope_max_pos][D] or NULL
+  int rope_max_pos;
   int32_t* err;
 };
 
-// D: head_dim, ROT: rotation kind, LGB: log2 of the Hadamard block.
-template <int D, int ROT, int LGB>
+// D: head_dim, ROT: rotation kind, LGB: log2 of the Hadamard block, PRE: a
+// RoPE table or a sign table acts before the rotation.
+template <int D, int ROT, int LGB, bool PRE>
 __global__ void __launch_bounds__(append_threads(append_e(D, ROT, LGB)),
                                   append_ctas_per_sm(append_e(D, ROT, LGB)))
     append_kernel(const AppendArgs a, const __grid_constant__ CUtensorMap tmk,
@@ -105,9 +237,14 @@ __global__ void __launch_bounds__(append_threads(append_e(D, ROT, LGB)),
     mbar_init(&bars[1], 1);
     mbar_fence_init();
   }
-  if (ROT == KVQ_ROT_QUAT) {
+  // the rotation's table in shared memory: quaternions (2 D floats) or signs (D)
+  if (ROT == KVQ_ROT_QUAT || ROT == KVQ_ROT_QUAT_FAST) {
     for (int i = tid; i < D * 2; i += kAppendThreads) qtbl[i] = a.quat[i];
+  } else if (ROT == KVQ_ROT_HADAMARD && a.quat != nullptr) {
+    for (int i = tid; i < D; i += kAppendThreads) qtbl[i] = a.quat[i];
   }
+  const float* const rtbl =
+      (ROT == KVQ_ROT_HADAMARD && a.quat == nullptr) || ROT == KVQ_ROT_NONE ? nullptr : qtbl;
 
   // this thread's role, fixed for all tiles (token-major):
   // thread row = ((kv*TOK + t)*H + h)*TPR + part
@@ -158,7 +295,7 @@ __global__ void __launch_bounds__(append_threads(append_e(D, ROT, LGB)),
       if (lead) raise_flag(a.err, KVQ_ERRF_SEQ);
       return -1;
     }
-    if (pos < 0 || (pos >> lgP) >= a.bt_stride) {
+    if (pos < 0 || (pos >> lgP) >= a.bt_stride || (a.rope != nullptr && pos >= a.rope_max_pos)) {
       if (lead) raise_flag(a.err, KVQ_ERRF_POS);
       return -1;
     }
@@ -176,6 +313,7 @@ __global__ void __launch_bounds__(append_threads(append_e(D, ROT, LGB)),
   int seq_n, pos_n;
   meta_load(tile, seq_n, pos_n);
   int64_t dst_cur = resolve(seq_n, pos_n);
+  int pos_cur = pos_n;
   uint32_t parity = 0;  // bit b: phase parity to wait for on buffer b
 
   for (int it = 0; tile < a.num_tiles; ++it, tile += gridDim.x) {
@@ -199,109 +337,15 @@ __global__ void __launch_bounds__(append_threads(append_e(D, ROT, LGB)),
     // computes (the two threads of a d = 256 row always agree) and stores
     // only if its destination resolved
     if (active && tok < a.T) {
-      {
-        float x[E];
-#pragma unroll
-        for (int c = 0; c < E / 8; ++c) {
-          // channel block c of this thread: box (part*E/64 + c/8), 16-byte
-          // chunk c%8 of line my_line, at its 128B-swizzled position
-          const uint8_t* box = cur + (my_kv * NH + my_part * (E / 64) + c / 8) * a.box_stride;
-          const uint4 u = *reinterpret_cast<const uint4*>(
-              box + my_line * 128 + (((c % 8) ^ (my_line & 7)) << 4));
-          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const __half2 h2 = u32_as_h2(w[q]);
-            if (ROT == KVQ_ROT_HADAMARD) {
-              // first butterfly stage straight from binary16: widening is
-              // exact, so (x_i + x_{i+1}, x_i - x_{i+1}) round as in binary32
-              const float b = __high2float(h2);
-              x[8 * c + 2 * q] = add_h_f(__low2half(h2), b);
-              x[8 * c + 2 * q + 1] = sub_h_f(__low2half(h2), b);
-            } else {
-              const float2 f = __half22float2(h2);
-              x[8 * c + 2 * q] = f.x;
-              x[8 * c + 2 * q + 1] = f.y;
-            }
-          }
-        }
-
-        // the two threads of a d = 256 row are lanes 2i, 2i+1 of one warp
-        const unsigned pair_mask = 3u << ((tid % kWarp) & ~1);
-        if (ROT == KVQ_ROT_HADAMARD) {
-          hadamard_regs<E, LGB, true>(x, my_part, pair_mask);
-        } else if (ROT == KVQ_ROT_QUAT) {
-          quat_regs<E>(x, qtbl, my_part * E);
-        }
-
-        // row statistics
-        float mn0 = fminf(x[0], x[1]), mx0 = fmaxf(x[0], x[1]);
-        float mn1 = fminf(x[2], x[3]), mx1 = fmaxf(x[2], x[3]);
-#pragma unroll
-        for (int i = 4; i < E; i += 4) {
-          mn0 = min3(mn0, x[i], x[i + 1]);
-          mn1 = min3(mn1, x[i + 2], x[i + 3]);
-          mx0 = max3(mx0, x[i], x[i + 1]);
-          mx1 = max3(mx1, x[i + 2], x[i + 3]);
-        }
-        float mn = fminf(mn0, mn1);
-        float mx = fmaxf(mx0, mx1);
-        if (TPR == 2) {
-          mn = fminf(mn, __shfl_xor_sync(pair_mask, mn, 1));
-          mx = fmaxf(mx, __shfl_xor_sync(pair_mask, mx, 1));
-        }
-        mn = __fadd_rn(mn, 0.0f);
-        mx = __fadd_rn(mx, 0.0f);
-        const __half m16 = __float2half_rd(mn);
-        const float m = __half2float(m16);
-        const float s32 = __fdiv_ru(__fsub_ru(mx, m), 15.0f);
-        const __half s16 = __float2half_ru(s32);
-        const float s = __half2float(s16);
-
-        uint32_t packed[E / 8];
-        if (s != 0.0f) {
-          const float inv = __frcp_rn(s);
-          const uint64_t m2 = pk(m, m), inv2 = pk(inv, inv);
-          const uint64_t magic2 = pk(12582912.0f, 12582912.0f);  // 1.5 * 2^23
-#pragma unroll
-          for (int c = 0; c < E / 8; ++c) {
-            uint32_t b[8];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              // code = nearest integer (ties to even) of the exact product
-              // t * inv: one fused multiply-add with 1.5 * 2^23 rounds it
-              // once, leaving the integer in the low mantissa bits
-              const uint64_t t = sub2(pk(x[8 * c + 2 * q], x[8 * c + 2 * q + 1]), m2);
-              const float2 r = upk(fma2(t, inv2, magic2));
-              b[2 * q] = __float_as_uint(r.x);
-              b[2 * q + 1] = __float_as_uint(r.y);
-            }
-            // low byte of each pair = c_even | c_odd << 4 (no carry: both <= 15)
-            const uint32_t p0 = b[0] + (b[1] << 4), p1 = b[2] + (b[3] << 4);
-            const uint32_t p2 = b[4] + (b[5] << 4), p3 = b[6] + (b[7] << 4);
-            packed[c] = __byte_perm(__byte_perm(p0, p1, 0x0040), __byte_perm(p2, p3, 0x0040),
-                                    0x5410);
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < E / 8; ++c) packed[c] = 0u;
-        }
-
-        if (dst_cur >= 0) {
-          uint8_t* codes = my_kv ? a.v_codes : a.k_codes;
-          uint32_t* params = my_kv ? a.v_params : a.k_params;
-          uint4* dst = reinterpret_cast<uint4*>(codes + dst_cur * (D / 2) + my_part * (E / 2));
-#pragma unroll
-          for (int c = 0; c < E / 32; ++c)
-            dst[c] = make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
-          if (my_part == 0) {
-            params[dst_cur] =
-                (uint32_t)__half_as_ushort(s16) | ((uint32_t)__half_as_ushort(m16) << 16);
-          }
-        }
-      }
+      const float* cs = (PRE && a.rope != nullptr && my_kv == 0 && dst_cur >= 0)
+                            ? a.rope + (int64_t)pos_cur * D : nullptr;
+      quantize_row_part<D, ROT, LGB, PRE>(cur + my_kv * NH * a.box_stride, a.box_stride, my_line,
+                                          my_part, rtbl, cs, dst_cur,
+                                          my_kv ? a.v_codes : a.k_codes,
+                                          my_kv ? a.v_params : a.k_params);
     }
     dst_cur = resolve(seq_n, pos_n);  // next tile's destination (its loads were in flight)
+    pos_cur = pos_n;
     __syncthreads();  // buffer `cur` is refilled by the next iteration's issue
   }
 }
@@ -330,6 +374,8 @@ struct AppendRowsArgs {
   uint32_t* k_params;
   uint32_t* v_params;
   const float* quat;
+  const float* rope;  // RoPE table [rope_max_pos][D] or NULL
+  int rope_max_pos;
   int32_t* err;
 };
 
@@ -357,11 +403,13 @@ __global__ void __launch_bounds__(kRowsWarps * kWarp) append_rows_kernel(const A
   const int seq = active ? a.token_seq[t] : -1;
   const int pos = active ? a.token_pos[t] : 0;
   const bool seq_ok = seq >= 0 && seq < a.num_seqs;
-  const bool pos_ok = pos >= 0 && (pos >> a.lg_page) < a.bt_stride;
+  const bool pos_ok = pos >= 0 && (pos >> a.lg_page) < a.bt_stride &&
+                      (a.rope == nullptr || pos < a.rope_max_pos);
   const int page = (seq_ok && pos_ok) ? a.block_table[(int64_t)seq * a.bt_stride + (pos >> a.lg_page)] : -1;
 
   float x[CPL];
   row_load<D>(x, (kv ? a.v : a.k) + (int64_t)t * a.tok_stride + (int64_t)h * D + rl * CPL, active);
+  if (a.rope != nullptr && kv == 0 && pos_ok) rope_regs<CPL>(x, a.rope + (int64_t)pos * D + rl * CPL);
   __half s16, m16;
   const uint32_t packed = row_quantize<D, ROT, LGB>(x, rl, a.quat, s16, m16);
 
@@ -401,6 +449,7 @@ template <int D>
 static cudaError_t dispatch_rows(const AppendRowsArgs& a, int rot, int lgb, cudaStream_t st) {
   if (rot == KVQ_ROT_NONE) return launch_rows<D, KVQ_ROT_NONE, 0>(a, st);
   if (rot == KVQ_ROT_QUAT) return launch_rows<D, KVQ_ROT_QUAT, 0>(a, st);
+  if (rot == KVQ_ROT_QUAT_FAST) return launch_rows<D, KVQ_ROT_QUAT_FAST, 0>(a, st);
   switch (lgb) {
     case 4: return launch_rows<D, KVQ_ROT_HADAMARD, 4>(a, st);
     case 5: return launch_rows<D, KVQ_ROT_HADAMARD, 5>(a, st);
@@ -430,14 +479,14 @@ static PFN_cuTensorMapEncodeTiled encode_fn() {
 }
 
 // [T][H][D] binary16 rows with token stride tok_stride (elements) as a 3-D
-// tensor (D innermost); box (64 channels, H heads, TOK tokens), 128B swizzle.
+// tensor (D innermost); box (64 channels, HB heads, TOK tokens), 128B swizzle.
 static bool encode_rows(CUtensorMap* m, const void* base, int D, int H, int T,
-                        int64_t tok_stride, int TOK) {
+                        int64_t tok_stride, int HB, int TOK) {
   PFN_cuTensorMapEncodeTiled fn = encode_fn();
   if (fn == nullptr) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T};
   const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)tok_stride * 2};
-  const cuuint32_t box[3] = {64u, (cuuint32_t)H, (cuuint32_t)TOK};
+  const cuuint32_t box[3] = {64u, (cuuint32_t)HB, (cuuint32_t)TOK};
   const cuuint32_t estr[3] = {1u, 1u, 1u};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -453,7 +502,8 @@ template <int D, int ROT, int LGB>
 static cudaError_t launch_append(const AppendArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
                                  int grid, cudaStream_t st) {
   const size_t smem = append_smem(D, a.box_stride);
-  auto kern = append_kernel<D, ROT, LGB>;
+  const bool pre = a.rope != nullptr || (ROT == KVQ_ROT_HADAMARD && a.quat != nullptr);
+  auto kern = pre ? append_kernel<D, ROT, LGB, true> : append_kernel<D, ROT, LGB, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   e = launch_pdl(kern, grid, append_threads(append_e(D, ROT, LGB)), smem, st, a, tk, tv);
@@ -466,6 +516,7 @@ static cudaError_t dispatch_rot(const AppendArgs& a, const CUtensorMap& tk, cons
                                 int rot, int lgb, int grid, cudaStream_t st) {
   if (rot == KVQ_ROT_NONE) return launch_append<D, KVQ_ROT_NONE, 0>(a, tk, tv, grid, st);
   if (rot == KVQ_ROT_QUAT) return launch_append<D, KVQ_ROT_QUAT, 0>(a, tk, tv, grid, st);
+  if (rot == KVQ_ROT_QUAT_FAST) return launch_append<D, KVQ_ROT_QUAT_FAST, 0>(a, tk, tv, grid, st);
   switch (lgb) {
     case 4: return launch_append<D, KVQ_ROT_HADAMARD, 4>(a, tk, tv, grid, st);
     case 5: return launch_append<D, KVQ_ROT_HADAMARD, 5>(a, tk, tv, grid, st);
@@ -480,6 +531,16 @@ static cudaError_t dispatch_rot(const AppendArgs& a, const CUtensorMap& tk, cons
   return cudaErrorInvalidValue;
 }
 
+// The kernels' rotation template: the randomised-sign Hadamard runs as the
+// Hadamard kernels given its sign table; the table a kernel receives (NULL
+// for the plain Hadamard and for no rotation).
+static int rot_template(const kvq_cache_desc& d) {
+  return d.rot_kind == KVQ_ROT_HADAMARD_SIGNED ? KVQ_ROT_HADAMARD : d.rot_kind;
+}
+static const float* rot_table(const kvq_cache_desc& d) {
+  return (d.rot_kind == KVQ_ROT_NONE || d.rot_kind == KVQ_ROT_HADAMARD) ? nullptr : d.quat;
+}
+
 int append_launch(const kvq_cache_desc& d, int32_t T, const void* k, const void* v,
                   int64_t tok_stride, const int32_t* token_seq, const int32_t* token_pos,
                   int32_t num_seqs, const int32_t* block_table, int32_t bt_stride,
@@ -488,7 +549,7 @@ int append_launch(const kvq_cache_desc& d, int32_t T, const void* k, const void*
   const int D = d.head_dim;
   int lgb0 = 0;
   while ((1 << lgb0) < d.rot_block) ++lgb0;
-  const int E = append_e(D, d.rot_kind, lgb0);
+  const int E = append_e(D, rot_template(d), lgb0);
   const int TPR = D / E;
   const int per_sm = append_ctas_per_sm(E);
   const int tok_max = append_threads(E) / (2 * d.num_kv_heads * TPR);
@@ -509,12 +570,12 @@ int append_launch(const kvq_cache_desc& d, int32_t T, const void* k, const void*
     r.token_seq = token_seq; r.token_pos = token_pos; r.block_table = block_table;
     r.k_codes = k_codes; r.v_codes = v_codes;
     r.k_params = static_cast<uint32_t*>(k_params); r.v_params = static_cast<uint32_t*>(v_params);
-    r.quat = d.quat; r.err = err;
+    r.quat = rot_table(d); r.rope = d.rope; r.rope_max_pos = d.rope_max_pos; r.err = err;
     cudaError_t e;
     switch (D) {
-      case 64: e = dispatch_rows<64>(r, d.rot_kind, lgb, st); break;
-      case 128: e = dispatch_rows<128>(r, d.rot_kind, lgb, st); break;
-      case 256: e = dispatch_rows<256>(r, d.rot_kind, lgb, st); break;
+      case 64: e = dispatch_rows<64>(r, rot_template(d), lgb, st); break;
+      case 128: e = dispatch_rows<128>(r, rot_template(d), lgb, st); break;
+      case 256: e = dispatch_rows<256>(r, rot_template(d), lgb, st); break;
       default: return KVQ_ERR_UNSUPPORTED;
     }
     if (e == cudaErrorInvalidValue) return KVQ_ERR_UNSUPPORTED;
@@ -543,18 +604,20 @@ int append_launch(const kvq_cache_desc& d, int32_t T, const void* k, const void*
   a.v_codes = v_codes;
   a.k_params = static_cast<uint32_t*>(k_params);
   a.v_params = static_cast<uint32_t*>(v_params);
-  a.quat = d.quat;
+  a.quat = rot_table(d);
+  a.rope = d.rope;
+  a.rope_max_pos = d.rope_max_pos;
   a.err = err;
   CUtensorMap tk, tv;
-  if (!encode_rows(&tk, k, D, a.H, T, tok_stride, tok) ||
-      !encode_rows(&tv, v, D, a.H, T, tok_stride, tok))
+  if (!encode_rows(&tk, k, D, a.H, T, tok_stride, a.H, tok) ||
+      !encode_rows(&tv, v, D, a.H, T, tok_stride, a.H, tok))
     return KVQ_ERR_CUDA;
   const int grid = a.num_tiles < per_sm * sms ? a.num_tiles : per_sm * sms;
   cudaError_t e;
   switch (D) {
-    case 64: e = dispatch_rot<64>(a, tk, tv, d.rot_kind, lgb, grid, st); break;
-    case 128: e = dispatch_rot<128>(a, tk, tv, d.rot_kind, lgb, grid, st); break;
-    case 256: e = dispatch_rot<256>(a, tk, tv, d.rot_kind, lgb, grid, st); break;
+    case 64: e = dispatch_rot<64>(a, tk, tv, rot_template(d), lgb, grid, st); break;
+    case 128: e = dispatch_rot<128>(a, tk, tv, rot_template(d), lgb, grid, st); break;
+    case 256: e = dispatch_rot<256>(a, tk, tv, rot_template(d), lgb, grid, st); break;
     default: return KVQ_ERR_UNSUPPORTED;
   }
   if (e == cudaErrorInvalidValue) return KVQ_ERR_UNSUPPORTED;

@@ -63,6 +63,8 @@ struct DecodeArgs {
   float scale2;   // sm_scale * log2(e)
   const __half* q;  // [S][Hq][D]
   const float* quat;
+  const float* rope;  // RoPE table [rope_max_pos][D] or NULL
+  int rope_max_pos;
   const int32_t* seq_lens;
   const int32_t* block_table;
   const uint8_t* k_codes;
@@ -96,13 +98,14 @@ struct StepRow {
 
 template <int D, int ROT, int LGB>
 __device__ __forceinline__ StepRow step_rows(const __half* k_row, const __half* v_row,
-                                             const float* quat, int lane) {
+                                             const float* quat, const float* cs, int lane) {
   constexpr int CPL = RowQuantShape<D>::CPL;
   StepRow o;
 #pragma unroll 1
   for (int kv = 0; kv < 2; ++kv) {
     float x[CPL];
     row_load<D>(x, (kv ? v_row : k_row) + lane * CPL, true);
+    if (kv == 0 && cs != nullptr) rope_regs<CPL>(x, cs + lane * CPL);
     __half s16, m16;
     const uint32_t packed = row_quantize<D, ROT, LGB>(x, lane, quat, s16, m16);
     const uint32_t word =
@@ -118,18 +121,24 @@ __device__ __forceinline__ StepRow step_rows(const __half* k_row, const __half* 
   return o;
 }
 
+// cs: the RoPE table row of the token's position (NULL: no RoPE)
 template <int D>
 __device__ __noinline__ StepRow quantize_step_token(const __half* k_row, const __half* v_row,
-                                                    const float* quat, int rot_kind, int lgb,
-                                                    int lane) {
-  if (rot_kind == KVQ_ROT_NONE) return step_rows<D, KVQ_ROT_NONE, 0>(k_row, v_row, quat, lane);
-  if (rot_kind == KVQ_ROT_QUAT) return step_rows<D, KVQ_ROT_QUAT, 0>(k_row, v_row, quat, lane);
+                                                    const float* quat, const float* cs,
+                                                    int rot_kind, int lgb, int lane) {
+  if (rot_kind == KVQ_ROT_NONE) return step_rows<D, KVQ_ROT_NONE, 0>(k_row, v_row, quat, cs, lane);
+  if (rot_kind == KVQ_ROT_QUAT) return step_rows<D, KVQ_ROT_QUAT, 0>(k_row, v_row, quat, cs, lane);
+  if (rot_kind == KVQ_ROT_QUAT_FAST)
+    return step_rows<D, KVQ_ROT_QUAT_FAST, 0>(k_row, v_row, quat, cs, lane);
+  // the Hadamard rows take the sign table (randomised signs) or NULL
+  if (rot_kind == KVQ_ROT_HADAMARD) quat = nullptr;
   switch (lgb) {
-    case 4: return step_rows<D, KVQ_ROT_HADAMARD, 4>(k_row, v_row, quat, lane);
-    case 5: return step_rows<D, KVQ_ROT_HADAMARD, 5>(k_row, v_row, quat, lane);
-    case 6: return step_rows<D, KVQ_ROT_HADAMARD, 6>(k_row, v_row, quat, lane);
-    case 7: return step_rows<D, KVQ_ROT_HADAMARD, 7>(k_row, v_row, quat, lane);
-    default: return step_rows<D, KVQ_ROT_HADAMARD, (D >= 256 ? 8 : 7)>(k_row, v_row, quat, lane);
+    case 4: return step_rows<D, KVQ_ROT_HADAMARD, 4>(k_row, v_row, quat, cs, lane);
+    case 5: return step_rows<D, KVQ_ROT_HADAMARD, 5>(k_row, v_row, quat, cs, lane);
+    case 6: return step_rows<D, KVQ_ROT_HADAMARD, 6>(k_row, v_row, quat, cs, lane);
+    case 7: return step_rows<D, KVQ_ROT_HADAMARD, 7>(k_row, v_row, quat, cs, lane);
+    default:
+      return step_rows<D, KVQ_ROT_HADAMARD, (D >= 256 ? 8 : 7)>(k_row, v_row, quat, cs, lane);
   }
 }
 
@@ -172,11 +181,17 @@ struct DecCfg {
   static constexpr int STEP_B = (2 * ROWB + 8 + 127) / 128 * 128;
   static constexpr int WARP_B = (NST * STAGE_B + STEP_B + 127) / 128 * 128;
 };
-// the bit-exact quantize path.
+// Rotation of a query row held as quarters: lane j of a group of four
+// consecutive lanes owns channels [j*QW, (j+1)*QW). Butterfly stages with
+// distance < QW run in registers, wider ones across the lanes (distance QW:
+// lane ^ 1, 2*QW: lane ^ 2); the lower-channel lane adds and the upper one
+// subtracts. All 32 lanes must call it. Binary32, not part of the bit-exact
+// quantize path. `tbl` is the rotation's table (quaternions or signs).
 template <int QW>
 __device__ __forceinline__ void rotate_quarter(float (&x)[QW], int j, int rot_kind, int lgb,
-                                               const float* quat, bool inverse) {
-  if (rot_kind == KVQ_ROT_HADAMARD) {
+                                               const float* tbl) {
+  if (rot_kind == KVQ_ROT_HADAMARD || rot_kind == KVQ_ROT_HADAMARD_SIGNED) {
+    if (rot_kind == KVQ_ROT_HADAMARD_SIGNED) sign_regs<QW>(x, tbl + j * QW);
     constexpr int LQ = QW == 32 ? 5 : 6;
     const int lin = lgb < LQ ? lgb : LQ;
     switch (lin) {
@@ -197,10 +212,9 @@ __device__ __forceinline__ void rotate_quarter(float (&x)[QW], int j, int rot_ki
 #pragma unroll
     for (int i = 0; i < QW; ++i) x[i] *= cb;
   } else if (rot_kind == KVQ_ROT_QUAT) {
-    if (inverse)
-      quat_inv_regs<QW>(x, quat, j * QW);
-    else
-      quat_regs<QW>(x, quat, j * QW);
+    quat_regs<QW>(x, tbl, j * QW);
+  } else if (rot_kind == KVQ_ROT_QUAT_FAST) {
+    quat_fast_regs<QW>(x, tbl, j * QW);
   }
 }
 
@@ -244,7 +258,8 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : (GP == 8 ? 3
 #pragma unroll
     for (int c = 0; c < C::QW / 8; ++c) qraw[c] = head_ok ? src[c] : make_uint4(0u, 0u, 0u, 0u);
   }
-  bool len_ok = L >= 0 && L <= a.max_seq_len && (L + a.P - 1) / a.P <= a.bt_stride;
+  bool len_ok = L >= 0 && L <= a.max_seq_len && (L + a.P - 1) / a.P <= a.bt_stride &&
+                (a.rope == nullptr || L <= a.rope_max_pos);
   if (!len_ok) {
     if (lane == 0 && h == 0 && split == 0) raise_flag(a.err, KVQ_ERRF_LEN);
     L = 0;
@@ -382,8 +397,9 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : (GP == 8 ? 3
     const int page = bt_row[new_pg];
     if (page >= 0 && page < a.NP) {
       const int64_t src = (int64_t)s * a.new_stride + (int64_t)h * D;
-      const StepRow nr =
-          quantize_step_token<D>(a.k_new + src, a.v_new + src, a.quat, a.rot_kind, a.lgb, lane);
+      const StepRow nr = quantize_step_token<D>(
+          a.k_new + src, a.v_new + src, a.quat,
+          a.rope != nullptr ? a.rope + (int64_t)(L - 1) * D : nullptr, a.rot_kind, a.lgb, lane);
       const int64_t row = ((int64_t)page * a.H + h) * P + (L - 1) % P;
       constexpr int LB = RowQuantShape<D>::CPL / 2;  // code bytes per lane
       put_codes<D>(a.k_codes_w + row * (D / 2) + lane * LB, nr.kc);
@@ -433,7 +449,9 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : (GP == 8 ? 3
         x[8 * c + 2 * e + 1] = f.y;
       }
     }
-    rotate_quarter<C::QW>(x, j, a.rot_kind, a.lgb, a.quat, false);
+    // the query's RoPE at its own position L - 1, in front of the rotation
+    if (a.rope != nullptr && L >= 1) rope_regs<C::QW>(x, a.rope + (int64_t)(L - 1) * D + j * C::QW);
+    rotate_quarter<C::QW>(x, j, a.rot_kind, a.lgb, a.quat);
     float amax = 0.f;
 #pragma unroll
     for (int i = 0; i < C::QW; ++i) amax = fmaxf(amax, fabsf(x[i]));
@@ -819,13 +837,14 @@ struct MergeArgs {
 };
 
 // R^-1 of a row held as CPL consecutive channels per lane over the 32 lanes
-// (the inverse of the block Hadamard rotation is the rotation itself; the
-// quaternion map is inverted block by block). Binary32, not part of the
+// (the inverse of the block Hadamard rotation is the rotation itself, after
+// it the sign flip when there is one; the quaternion maps are inverted block
+// by block). Binary32, not part of the
 // bit-exact quantize path.
 template <int CPL>
 __device__ __forceinline__ void row_unrotate(float (&x)[CPL], int lane, int rot_kind, int lgb,
                                              const float* quat) {
-  if (rot_kind == KVQ_ROT_HADAMARD) {
+  if (rot_kind == KVQ_ROT_HADAMARD || rot_kind == KVQ_ROT_HADAMARD_SIGNED) {
     const int b = 1 << lgb;
 #pragma unroll
     for (int dd = 1; dd < CPL; dd <<= 1) {
@@ -850,8 +869,12 @@ __device__ __forceinline__ void row_unrotate(float (&x)[CPL], int lane, int rot_
     const float cb = hadamard_scale(lgb);
 #pragma unroll
     for (int i = 0; i < CPL; ++i) x[i] *= cb;
+    // R = H S with the sign diagonal S: R^-1 = S H
+    if (rot_kind == KVQ_ROT_HADAMARD_SIGNED) sign_regs<CPL>(x, quat + lane * CPL);
   } else if (rot_kind == KVQ_ROT_QUAT) {
     quat_inv_regs<CPL>(x, quat, lane * CPL);
+  } else if (rot_kind == KVQ_ROT_QUAT_FAST) {
+    quat_fast_inv_regs<CPL>(x, quat, lane * CPL);
   }
 }
 
@@ -1020,6 +1043,7 @@ int decode_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, const void* q,
   a.rot_kind = d.rot_kind; a.lgb = lgb;
   a.scale2 = (float)((double)sm_scale * 1.4426950408889634074);
   a.q = static_cast<const __half*>(q); a.quat = d.quat;
+  a.rope = d.rope; a.rope_max_pos = d.rope_max_pos;
   a.seq_lens = seq_lens; a.block_table = block_table;
   a.k_codes = k_codes; a.k_params = static_cast<const uint32_t*>(k_params);
   a.v_codes = v_codes; a.v_params = static_cast<const uint32_t*>(v_params);

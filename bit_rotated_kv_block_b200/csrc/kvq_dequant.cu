@@ -2,8 +2,9 @@
 //
 // The dequantization rule is the one of the token-wise asymmetric INT4 format
 // ("SAW-INT4: System-Aware 4-Bit KV-Cache Quantization for Real-World LLM
-// Serving", Summary); the inverse rotation is R (Hadamard, R R = I) or
-// conj(qL) w qR (quaternion, "IsoQuant ...", Abstract).
+// Serving", Summary); the inverse rotation is R (Hadamard, R R = I; with the
+// sign diagonal S in front, S R), conj(qL) w qR (quaternion, "IsoQuant ...",
+// Abstract) or conj(qL) w (its one-factor variant).
 //
 // One thread owns E = min(d, 128) channels of one (sequence, position, head)
 // row; c * s16 is exact in binary32 (4-bit times 11-bit), so the rotated-basis
@@ -23,7 +24,8 @@ struct DequantArgs {
   const int32_t* block_table;
   const uint8_t* codes;
   const uint32_t* params;
-  const float* quat;
+  const float* quat;   // quaternion table (QUAT kinds)
+  const float* signs;  // sign table of the randomised-sign Hadamard, or NULL
   void* out;
   int32_t* err;
 };
@@ -68,8 +70,12 @@ __global__ void __launch_bounds__(128) dequant_kernel(const DequantArgs a, int u
   }
   if (unrotate) {
     const unsigned pair_mask = 3u << ((threadIdx.x % kWarp) & ~1);
-    if (ROT == KVQ_ROT_HADAMARD) hadamard_regs<E, LGB>(x, part, pair_mask);
+    if (ROT == KVQ_ROT_HADAMARD) {
+      hadamard_regs<E, LGB>(x, part, pair_mask);
+      if (a.signs != nullptr) sign_regs<E>(x, a.signs + part * E);  // R^-1 = S H
+    }
     if (ROT == KVQ_ROT_QUAT) quat_inv_regs<E>(x, a.quat, part * E);
+    if (ROT == KVQ_ROT_QUAT_FAST) quat_fast_inv_regs<E>(x, a.quat, part * E);
   }
   const int64_t o = (((int64_t)s * a.L + j) * a.H + h) * D + part * E;
   if (F32) {
@@ -106,6 +112,7 @@ static cudaError_t dq_rot(const DequantArgs& a, int rot, int lgb, int unrotate, 
                           cudaStream_t st) {
   if (rot == KVQ_ROT_NONE || !unrotate) return launch_dq<D, KVQ_ROT_NONE, 0>(a, 0, f32, st);
   if (rot == KVQ_ROT_QUAT) return launch_dq<D, KVQ_ROT_QUAT, 0>(a, 1, f32, st);
+  if (rot == KVQ_ROT_QUAT_FAST) return launch_dq<D, KVQ_ROT_QUAT_FAST, 0>(a, 1, f32, st);
   switch (lgb) {
     case 4: return launch_dq<D, KVQ_ROT_HADAMARD, 4>(a, 1, f32, st);
     case 5: return launch_dq<D, KVQ_ROT_HADAMARD, 5>(a, 1, f32, st);
@@ -124,6 +131,7 @@ int dequant_launch(const kvq_cache_desc& d, int32_t S, const int32_t* seq_lens,
   a.S = S; a.L = max_seq_len; a.H = d.num_kv_heads; a.P = d.page_size; a.NP = d.num_pages;
   a.bt_stride = bt_stride; a.seq_lens = seq_lens; a.block_table = block_table;
   a.codes = codes; a.params = static_cast<const uint32_t*>(params); a.quat = d.quat;
+  a.signs = d.rot_kind == KVQ_ROT_HADAMARD_SIGNED ? d.quat : nullptr;
   a.out = out; a.err = err;
   int lgb = 0;
   while ((1 << lgb) < d.rot_block) ++lgb;

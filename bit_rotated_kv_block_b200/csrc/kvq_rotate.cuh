@@ -131,4 +131,63 @@ __device__ __forceinline__ void quat_inv_regs(float (&x)[E], const float* tbl, i
   }
 }
 
+// IsoQuant-Fast: per 4-channel block v -> qL v (one Hamilton product, the
+// same fused multiply-add order as the full map); qL[j] from the table of
+// the full map (qR unused). Exact inverse for a unit qL: w -> conj(qL) w.
+template <int E>
+__device__ __forceinline__ void quat_fast_regs(float (&x)[E], const float* tbl, int ch0) {
+#pragma unroll
+  for (int k = 0; k < E / 4; ++k) {
+    const float* q = tbl + (ch0 / 4 + k) * 8;
+    const float qL[4] = {q[0], q[1], q[2], q[3]};
+    const float v[4] = {x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3]};
+    float y[4];
+    hamilton(qL, v, y);
+    x[4 * k] = y[0];
+    x[4 * k + 1] = y[1];
+    x[4 * k + 2] = y[2];
+    x[4 * k + 3] = y[3];
+  }
+}
+template <int E>
+__device__ __forceinline__ void quat_fast_inv_regs(float (&x)[E], const float* tbl, int ch0) {
+#pragma unroll
+  for (int k = 0; k < E / 4; ++k) {
+    const float* q = tbl + (ch0 / 4 + k) * 8;
+    const float qLc[4] = {q[0], -q[1], -q[2], -q[3]};
+    const float w[4] = {x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3]};
+    float y[4];
+    hamilton(qLc, w, y);
+    x[4 * k] = y[0];
+    x[4 * k + 1] = y[1];
+    x[4 * k + 2] = y[2];
+    x[4 * k + 3] = y[3];
+  }
+}
+
+// Randomised-sign Hadamard: each channel times its fixed sign (+1 or -1,
+// exact); `signs` offset to the thread's first channel.
+template <int E>
+__device__ __forceinline__ void sign_regs(float (&x)[E], const float* signs) {
+#pragma unroll
+  for (int i = 0; i < E; ++i) x[i] = __fmul_rn(x[i], signs[i]);
+}
+
+// Rotary position embedding in front of the rotation: channel pairs
+// (2i, 2i+1) of a thread's E consecutive channels (starting at an even
+// channel) turned by (cos, sin) read from cs (the table row of the position,
+// offset to the thread's first channel; 8-byte aligned). Binary32, each
+// product and the difference / sum rounded on its own:
+//   x'_2i = RN(RN(x_2i c) - RN(x_2i+1 s)), x'_2i+1 = RN(RN(x_2i s) + RN(x_2i+1 c)).
+template <int E>
+__device__ __forceinline__ void rope_regs(float (&x)[E], const float* cs) {
+#pragma unroll
+  for (int i = 0; i < E; i += 2) {
+    const float2 t = *reinterpret_cast<const float2*>(cs + i);
+    const float a = x[i], b = x[i + 1];
+    x[i] = __fsub_rn(__fmul_rn(a, t.x), __fmul_rn(b, t.y));
+    x[i + 1] = __fadd_rn(__fmul_rn(a, t.y), __fmul_rn(b, t.x));
+  }
+}
+
 }  // namespace kvq

@@ -28,7 +28,8 @@ struct RowQuantShape {
 };
 
 // x: this lane's CPL channels (binary16 values widened to binary32); rl: the
-// lane's index inside its row. Every lane of the warp must call it (the
+// lane's index inside its row; quat: the quaternion table (QUAT kinds), the
+// sign table (HADAMARD with signs) or NULL. Every lane of the warp must call it (the
 // shuffles span the warp; rows never mix because lane distances stay below
 // LPR). Returns the lane's codes, channel i of the lane in bits 4i..4i+3.
 template <int D, int ROT, int LGB>
@@ -38,6 +39,8 @@ __device__ __forceinline__ uint32_t row_quantize(float (&x)[RowQuantShape<D>::CP
   constexpr int LPR = RowQuantShape<D>::LPR;
   constexpr int B = 1 << LGB;
   if (ROT == KVQ_ROT_HADAMARD) {
+    // randomised-sign Hadamard: `quat` is then the sign table (else NULL)
+    if (quat != nullptr) sign_regs<CPL>(x, quat + rl * CPL);
 #pragma unroll
     for (int dd = 1; dd < CPL && dd < B; dd <<= 1) {
 #pragma unroll
@@ -63,6 +66,8 @@ __device__ __forceinline__ uint32_t row_quantize(float (&x)[RowQuantShape<D>::CP
     for (int i = 0; i < CPL; ++i) x[i] = __fmul_rn(x[i], cb);
   } else if (ROT == KVQ_ROT_QUAT) {
     quat_regs<CPL>(x, quat, rl * CPL);
+  } else if (ROT == KVQ_ROT_QUAT_FAST) {
+    quat_fast_regs<CPL>(x, quat, rl * CPL);
   }
 
   float mn = x[0], mx = x[0];

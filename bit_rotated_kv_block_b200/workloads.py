@@ -36,7 +36,7 @@ from typing import Optional
 
 import numpy as np
 
-ROT_NONE, ROT_HADAMARD, ROT_QUAT = 0, 1, 2
+ROT_NONE, ROT_HADAMARD, ROT_QUAT, ROT_QUAT_FAST, ROT_HADAMARD_SIGNED = 0, 1, 2, 3, 4
 
 WORKLOAD_IDS = {"tiny": 1, "llama8b": 2, "long70b": 3, "prefill": 4, "ragged256": 5}
 
@@ -244,3 +244,19 @@ def ragged256(seed: int = 0, S: int = 128, lo: int = 512, hi: int = 16384,
 def random_quaternions(seed: int, d: int) -> np.ndarray:
     """A seeded quaternion table for head_dim d (d/4 blocks)."""
     return unit_quaternions(np.random.default_rng([int(seed), 99, S_QUAT]), d // 4)
+
+
+def rope_table(max_pos: int, d: int, base: float = 10000.0) -> np.ndarray:
+    """Rotary-position table float32 [max_pos][d/2][2]: (cos, sin) of
+    pos * base^(-2i/d) for channel pair i = (2i, 2i+1), evaluated in float64
+    and rounded to float32 (the table a serving stack precomputes once and
+    hands to the cache; an input here, like the quaternion table)."""
+    inv = base ** (-np.arange(0, d, 2, dtype=np.float64) / d)
+    ang = np.arange(max_pos, dtype=np.float64)[:, None] * inv[None, :]
+    return np.stack([np.cos(ang), np.sin(ang)], axis=-1).astype(np.float32)
+
+
+def random_signs(seed: int, d: int) -> np.ndarray:
+    """A seeded sign table float32 [d] of +1 / -1 (randomised-sign Hadamard)."""
+    g = np.random.default_rng([int(seed), 98, S_QUAT])
+    return g.choice(np.array([-1.0, 1.0], np.float32), size=d).astype(np.float32)

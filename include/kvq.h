@@ -60,9 +60,14 @@ typedef enum {
 } kvq_status;
 
 typedef enum {
-  KVQ_ROT_NONE = 0,     /* identity: the rotation-free INT4 baseline       */
-  KVQ_ROT_HADAMARD = 1, /* block-diagonal Walsh-Hadamard, block rot_block   */
-  KVQ_ROT_QUAT = 2      /* per 4-channel block v -> qL v conj(qR)          */
+  KVQ_ROT_NONE = 0,            /* identity: the rotation-free INT4 baseline      */
+  KVQ_ROT_HADAMARD = 1,        /* block-diagonal Walsh-Hadamard, block rot_block  */
+  KVQ_ROT_QUAT = 2,            /* per 4-channel block v -> qL v conj(qR)
+                                  (IsoQuant-Full)                                */
+  KVQ_ROT_QUAT_FAST = 3,       /* per 4-channel block v -> qL v: one isoclinic
+                                  factor (IsoQuant-Fast)                         */
+  KVQ_ROT_HADAMARD_SIGNED = 4  /* channel i times a fixed sign s_i = +-1, then
+                                  the block Walsh-Hadamard rotation              */
 } kvq_rot_kind;
 
 /* Bits OR-ed into *err_flags by the kernels. */
@@ -83,11 +88,32 @@ typedef enum {
  *  page_size    P: tokens per page; 16, 32 or 64.
  *  num_pages    NP: pool capacity in pages (>= 1).
  *  rot_kind     a kvq_rot_kind.
- *  rot_block    b, for KVQ_ROT_HADAMARD: a power of two in [16, 256]
- *               dividing d (ignored otherwise).
- *  quat         for KVQ_ROT_QUAT: device float [d/4][2][4], per block j
- *               (qL[j], qR[j]) as (w, x, y, z); unit quaternions. NULL
- *               otherwise. Channels 4j..4j+3 form block j. */
+ *  rot_block    b, for KVQ_ROT_HADAMARD and KVQ_ROT_HADAMARD_SIGNED: a power
+ *               of two in [16, 256] dividing d (ignored otherwise).
+ *  quat         the rotation's table, a device pointer (NULL for
+ *               KVQ_ROT_NONE and KVQ_ROT_HADAMARD):
+ *               KVQ_ROT_QUAT, KVQ_ROT_QUAT_FAST: float [d/4][2][4], per block
+ *               j (qL[j], qR[j]) as (w, x, y, z); unit quaternions (the fast
+ *               map uses qL only). Channels 4j..4j+3 form block j.
+ *               KVQ_ROT_HADAMARD_SIGNED: float [d] of signs, each +1 or -1.
+ *               The quaternion maps' Hamilton components are fused
+ *               multiply-add chains in the term order of the quantize
+ *               definition below; the sign flip is exact.
+ *  rope         optional rotary position embedding in front of the rotation
+ *               (NULL: none): device float [rope_max_pos][d/2][2], row p
+ *               holding (cos, sin) of the angle of each channel pair
+ *               (2i, 2i+1) at position p, 16-byte aligned. Every key row is
+ *               turned by the row of its token's position before it is
+ *               rotated and quantized (values are not), and the query of a
+ *               decode by the row of position seq_len - 1:
+ *                 x'_2i = RN(RN(x_2i c) - RN(x_2i+1 s)),
+ *                 x'_2i+1 = RN(RN(x_2i s) + RN(x_2i+1 c))   (binary32).
+ *               The pages describe no RoPE; it is the step in front of the
+ *               method's path in a decode step, offered here so that the key
+ *               rows need not be turned by a separate kernel.
+ *  rope_max_pos rows of the rope table (>= 1 when rope is set); a position at
+ *               or past it is invalid (KVQ_ERRF_POS in an append, the row is
+ *               skipped; KVQ_ERRF_LEN in a decode, the output is zero). */
 typedef struct {
   int32_t head_dim;
   int32_t num_kv_heads;
@@ -96,6 +122,8 @@ typedef struct {
   int32_t rot_kind;
   int32_t rot_block;
   const float* quat;
+  const float* rope;
+  int32_t rope_max_pos;
 } kvq_cache_desc;
 
 /*

@@ -31,7 +31,7 @@ import numpy as np
 
 from . import build as _build
 
-ROT_NONE, ROT_HADAMARD, ROT_QUAT = 0, 1, 2
+ROT_NONE, ROT_HADAMARD, ROT_QUAT, ROT_QUAT_FAST, ROT_HADAMARD_SIGNED = 0, 1, 2, 3, 4
 RN, RD, RU = 0, 1, 2
 ERR_PAGE, ERR_POS, ERR_SEQ, ERR_LEN = 1, 2, 4, 8
 
@@ -61,11 +61,12 @@ def lib():
             "orc_fwht_unscaled": (None, [P, i32]),
             "orc_quantize_rows": (None, [P, i64, i32, P, P, P]),
             "orc_quantize_append": (None, [i32, i32, i32, i32, i32, i32, P, i32, P, P, i64,
-                                           P, P, i32, P, i32, P, P, P, P, P]),
+                                           P, P, i32, P, i32, P, P, P, P, P, i32, P]),
             "orc_dequantize_pages": (None, [i32, i32, i32, i32, i32, i32, P, i32, P, i32, P,
                                             i32, P, P, i32, i32, P, P]),
             "orc_paged_decode_attn": (None, [i32, i32, i32, i32, i32, i32, P, i32, i32, P, P,
-                                             i32, P, i32, dbl, P, P, P, P, P, P]),
+                                             i32, P, i32, dbl, P, P, P, P, P, i32, P, P]),
+            "orc_rope_row_f32": (None, [P, i32, P]),
             "orc_paged_decode_attn_fp16": (None, [i32, i32, i32, i32, i32, i32, P, P, i32, P,
                                                   i32, dbl, P, P, P, P]),
             "orc_num_threads": (i32, []),
@@ -113,6 +114,19 @@ def half_bits_to_double(h):
     out = np.empty(h.shape, np.float64)
     lib().orc_half_to_double_array(_p(h), h.size, _p(out))
     return out
+
+
+# --- rotary position embedding (optional, in front of the rotation) --------
+
+def rope_rows_f32(x, cs):
+    """Turns rows x (float32 [n][d]) by the RoPE table rows cs (float32
+    [n][d/2][2] of (cos, sin), one per row): binary32, products and the
+    difference / sum rounded separately."""
+    x = _c(x, np.float32).copy()
+    cs = _c(cs, np.float32).reshape(x.shape[0], -1)
+    for i in range(x.shape[0]):
+        lib().orc_rope_row_f32(x[i].ctypes.data, x.shape[1], cs[i].ctypes.data)
+    return x
 
 
 # --- rotation ---------------------------------------------------------------
@@ -210,10 +224,13 @@ class Cache:
     """Geometry of one paged INT4 cache (head_dim d, KV heads H, page size P,
     pool size NP, rotation kind / block / quaternion table)."""
 
-    def __init__(self, d, H, P, NP, rot_kind, rot_block=0, quat=None):
+    def __init__(self, d, H, P, NP, rot_kind, rot_block=0, quat=None, rope=None):
         self.d, self.H, self.P, self.NP = int(d), int(H), int(P), int(NP)
         self.rot_kind, self.rot_block = int(rot_kind), int(rot_block)
         self.quat = _quat(quat)
+        # optional RoPE table float32 [max_pos][d/2][2] of (cos, sin)
+        self.rope = None if rope is None else _c(rope, np.float32).reshape(-1, self.d)
+        self.rope_max_pos = 0 if rope is None else self.rope.shape[0]
 
     def alloc_pools(self, fill=0):
         codes = np.full((self.NP, self.H, self.P, self.d // 2), fill, np.uint8)
@@ -241,7 +258,8 @@ def quantize_append(cache, k, v, token_seq, token_pos, block_table, k_codes, k_p
     lib().orc_quantize_append(cache.d, cache.H, cache.P, cache.NP, cache.rot_kind,
                               cache.rot_block, _p(cache.quat), T, _p(k), _p(v), tok_stride,
                               _p(ts), _p(tp), num_seqs, _p(bt), bt.shape[1], _p(k_codes),
-                              _p(k_params), _p(v_codes), _p(v_params), _p(err))
+                              _p(k_params), _p(v_codes), _p(v_params), _p(cache.rope),
+                              cache.rope_max_pos, _p(err))
     return int(err[0])
 
 
@@ -277,7 +295,8 @@ def paged_decode_attn(cache, q, seq_lens, max_seq_len, block_table, sm_scale, k_
     lib().orc_paged_decode_attn(cache.d, cache.H, cache.P, cache.NP, cache.rot_kind,
                                 cache.rot_block, _p(cache.quat), S, Hq, _p(q), _p(lens),
                                 max_seq_len, _p(bt), bt.shape[1], float(sm_scale), _p(kc),
-                                _p(kp), _p(vc), _p(vp), _p(out), _p(err))
+                                _p(kp), _p(vc), _p(vp), _p(cache.rope), cache.rope_max_pos,
+                                _p(out), _p(err))
     return out, int(err[0])
 
 

@@ -201,12 +201,36 @@ void orc_rotate_quat_f32(float* x, int d, const float* quat) {
   }
 }
 
+// IsoQuant-Fast (IsoQuant Abstract: "keeps only one isoclinic factor"):
+// T(v) = qL v, one Hamilton product per 4-channel block (16 multiply-adds),
+// qL[j] from the same table layout as the full map (qR[j] unused).
+void orc_rotate_quat_fast_f32(float* x, int d, const float* quat) {
+  for (int j = 0; j < d / 4; ++j) {
+    float t[4];
+    orc_hamilton_f32(quat + j * 8, x + 4 * j, t);
+    for (int i = 0; i < 4; ++i) x[4 * j + i] = t[i];
+  }
+}
+
+// Randomised-sign Hadamard (a reading of the randomised Hadamard transform
+// the pages' rotation sources build on): every channel is first multiplied
+// by its sign s_i in {+1, -1} (exact), then the block Hadamard rotation
+// above; the signs are a caller-supplied binary32 table [d] shared by every
+// row, like the quaternion table.
+void orc_rotate_signed_hadamard_f32(float* x, int d, int b, const float* signs) {
+  for (int i = 0; i < d; ++i) x[i] = x[i] * signs[i];
+  orc_rotate_hadamard_f32(x, d, b);
+}
+
 // Rotation kinds (same numbering as the library's public enum, restated).
-enum { ORC_ROT_NONE = 0, ORC_ROT_HADAMARD = 1, ORC_ROT_QUAT = 2 };
+enum { ORC_ROT_NONE = 0, ORC_ROT_HADAMARD = 1, ORC_ROT_QUAT = 2, ORC_ROT_QUAT_FAST = 3,
+       ORC_ROT_HADAMARD_SIGNED = 4 };
 
 void orc_rotate_f32(float* x, int d, int kind, int b, const float* quat) {
   if (kind == ORC_ROT_HADAMARD) orc_rotate_hadamard_f32(x, d, b);
   else if (kind == ORC_ROT_QUAT) orc_rotate_quat_f32(x, d, quat);
+  else if (kind == ORC_ROT_QUAT_FAST) orc_rotate_quat_fast_f32(x, d, quat);
+  else if (kind == ORC_ROT_HADAMARD_SIGNED) orc_rotate_signed_hadamard_f32(x, d, b, quat);
 }
 
 // ---------------------------------------------------------------------------
@@ -297,6 +321,33 @@ void orc_unpack_row(const uint8_t* codes, int d, int* c) {
 }
 
 // ---------------------------------------------------------------------------
+// Rotary position embedding, optionally applied to each key row and to the
+// query in front of the block rotation (the step before the method's path in
+// a decode step; the pages do not describe it, so this is a reading).
+// Adjacent channel pairs (2i, 2i+1) turn by the angle of the pair at the
+// token's position, whose cosine and sine the caller supplies as one row of a
+// binary32 table: cs[2i] = cos, cs[2i+1] = sin. Binary32, every product and
+// the difference / sum rounded on its own (no fused multiply-add):
+//   x'_{2i} = RN(RN(x_{2i} c) - RN(x_{2i+1} s)),
+//   x'_{2i+1} = RN(RN(x_{2i} s) + RN(x_{2i+1} c)).
+void orc_rope_row_f32(float* x, int d, const float* cs) {
+  for (int i = 0; i < d / 2; ++i) {
+    const float a = x[2 * i], b = x[2 * i + 1], c = cs[2 * i], sn = cs[2 * i + 1];
+    const float ac = a * c, bs = b * sn, as = a * sn, bc = b * c;
+    x[2 * i] = ac - bs;
+    x[2 * i + 1] = as + bc;
+  }
+}
+
+// The same turn in double precision (the query side of attention).
+static void rope_row_f64(double* x, int d, const float* cs) {
+  for (int i = 0; i < d / 2; ++i) {
+    const double a = x[2 * i], b = x[2 * i + 1], c = cs[2 * i], sn = cs[2 * i + 1];
+    x[2 * i] = a * c - b * sn;
+    x[2 * i + 1] = a * sn + b * c;
+  }
+}
+
 // Paged placement (SAW-INT4 Summary: the quantizer writes straight into paged
 // KV-cache layouts). Reading: pools are [page][kv_head][slot][d/2] bytes of
 // codes and [page][kv_head][slot] pairs (s16, m16) of binary16 (scale first);
@@ -309,13 +360,16 @@ void orc_unpack_row(const uint8_t* codes, int d, int* c) {
 
 enum { ORC_ERR_PAGE = 1, ORC_ERR_POS = 2, ORC_ERR_SEQ = 4, ORC_ERR_LEN = 8 };
 
+// With a RoPE table (rope != NULL, rows [rope_max_pos][d]), every key row is
+// turned by the row of its position before the rotation; a token whose
+// position has no row in the table is skipped with flag 2.
 void orc_quantize_append(int d, int H, int P, int NP, int rot_kind, int rot_block,
                          const float* quat, int T, const uint16_t* k, const uint16_t* v,
                          int64_t tok_stride, const int32_t* token_seq,
                          const int32_t* token_pos, int num_seqs,
                          const int32_t* block_table, int bt_stride, uint8_t* k_codes,
                          uint16_t* k_params, uint8_t* v_codes, uint16_t* v_params,
-                         int32_t* err) {
+                         const float* rope, int rope_max_pos, int32_t* err) {
   // Tokens are independent (each writes only its own slot), so they are
   // spread over threads; the arithmetic of every row is unchanged.
   int32_t flags = 0;
@@ -327,6 +381,7 @@ void orc_quantize_append(int d, int H, int P, int NP, int rot_kind, int rot_bloc
     if (seq >= num_seqs) { flags |= ORC_ERR_SEQ; continue; }
     const int pos = token_pos[t];
     if (pos < 0 || pos / P >= bt_stride) { flags |= ORC_ERR_POS; continue; }
+    if (rope != nullptr && pos >= rope_max_pos) { flags |= ORC_ERR_POS; continue; }
     const int page = block_table[(int64_t)seq * bt_stride + pos / P];
     if (page < 0 || page >= NP) { flags |= ORC_ERR_PAGE; continue; }
     const int slot = pos % P;
@@ -337,6 +392,7 @@ void orc_quantize_append(int d, int H, int P, int NP, int rot_kind, int rot_bloc
       for (int h = 0; h < H; ++h) {
         const uint16_t* x = src + (int64_t)t * tok_stride + (int64_t)h * d;
         for (int i = 0; i < d; ++i) row[i] = orc_half_to_float(x[i]);
+        if (kv == 0 && rope != nullptr) orc_rope_row_f32(row.data(), d, rope + (int64_t)pos * d);
         orc_rotate_f32(row.data(), d, rot_kind, rot_block, quat);
         const int64_t r = ((int64_t)page * H + h) * P + slot;
         uint16_t s16, m16;
@@ -365,7 +421,17 @@ static void hamilton_f64(const double* a, const double* b, double* o) {
 }
 
 void orc_rotate_f64(double* x, int d, int kind, int b, const float* quat) {
-  if (kind == ORC_ROT_HADAMARD) {
+  if (kind == ORC_ROT_HADAMARD_SIGNED) {
+    for (int i = 0; i < d; ++i) x[i] *= (double)quat[i];
+    orc_rotate_f64(x, d, ORC_ROT_HADAMARD, b, quat);
+  } else if (kind == ORC_ROT_QUAT_FAST) {
+    for (int j = 0; j < d / 4; ++j) {
+      const double qL[4] = {quat[8 * j], quat[8 * j + 1], quat[8 * j + 2], quat[8 * j + 3]};
+      double t[4];
+      hamilton_f64(qL, x + 4 * j, t);
+      for (int i = 0; i < 4; ++i) x[4 * j + i] = t[i];
+    }
+  } else if (kind == ORC_ROT_HADAMARD) {
     const double cb = 1.0 / std::sqrt((double)b);
     std::vector<double> y(b);
     for (int t = 0; t < d; t += b) {
@@ -392,6 +458,19 @@ void orc_rotate_f64(double* x, int d, int kind, int b, const float* quat) {
 void orc_unrotate_f64(double* x, int d, int kind, int b, const float* quat) {
   if (kind == ORC_ROT_HADAMARD) {
     orc_rotate_f64(x, d, kind, b, quat);  // R^-1 = R
+  } else if (kind == ORC_ROT_HADAMARD_SIGNED) {
+    // R = H S with S the sign diagonal: R^-1 = S^-1 H^-1 = S H
+    orc_rotate_f64(x, d, ORC_ROT_HADAMARD, b, quat);
+    for (int i = 0; i < d; ++i) x[i] *= (double)quat[i];
+  } else if (kind == ORC_ROT_QUAT_FAST) {
+    for (int j = 0; j < d / 4; ++j) {
+      const double L[4] = {quat[8 * j], quat[8 * j + 1], quat[8 * j + 2], quat[8 * j + 3]};
+      const double nL = L[0] * L[0] + L[1] * L[1] + L[2] * L[2] + L[3] * L[3];
+      const double Linv[4] = {L[0] / nL, -L[1] / nL, -L[2] / nL, -L[3] / nL};
+      double t[4];
+      hamilton_f64(Linv, x + 4 * j, t);
+      for (int i = 0; i < 4; ++i) x[4 * j + i] = t[i];
+    }
   } else if (kind == ORC_ROT_QUAT) {
     for (int j = 0; j < d / 4; ++j) {
       const double L[4] = {quat[8 * j], quat[8 * j + 1], quat[8 * j + 2], quat[8 * j + 3]};
@@ -465,13 +544,17 @@ void orc_dequantize_pages(int d, int H, int P, int NP, int rot_kind, int rot_blo
 // and gives a zero output; a sequence with no token gives a zero output.
 // ---------------------------------------------------------------------------
 
+// With a RoPE table the query is turned by the row of its own position,
+// seq_len - 1 (the last cached token is the one being decoded), before the
+// rotation; a length whose last position has no row sets flag 8 and gives a
+// zero output.
 void orc_paged_decode_attn(int d, int H, int P, int NP, int rot_kind, int rot_block,
                            const float* quat, int S, int Hq, const uint16_t* q,
                            const int32_t* seq_lens, int max_seq_len,
                            const int32_t* block_table, int bt_stride, double sm_scale,
                            const uint8_t* k_codes, const uint16_t* k_params,
-                           const uint8_t* v_codes, const uint16_t* v_params, double* out,
-                           int32_t* err) {
+                           const uint8_t* v_codes, const uint16_t* v_params,
+                           const float* rope, int rope_max_pos, double* out, int32_t* err) {
   const int G = Hq / H;
   int32_t flags = 0;
 #pragma omp parallel for schedule(dynamic) reduction(| : flags)
@@ -481,9 +564,11 @@ void orc_paged_decode_attn(int d, int H, int P, int NP, int rot_kind, int rot_bl
     for (int i = 0; i < d; ++i) o[i] = 0.0;
     const int L = seq_lens[s];
     if (L < 0 || L > max_seq_len || (L + P - 1) / P > bt_stride) { flags |= ORC_ERR_LEN; continue; }
+    if (rope != nullptr && L > rope_max_pos) { flags |= ORC_ERR_LEN; continue; }
     std::vector<double> qh(d), kh(d), acc(d, 0.0);
     std::vector<int> c(d);
     for (int i = 0; i < d; ++i) qh[i] = orc_half_to_double(q[(int64_t)sg * d + i]);
+    if (rope != nullptr && L >= 1) rope_row_f64(qh.data(), d, rope + (int64_t)(L - 1) * d);
     orc_rotate_f64(qh.data(), d, rot_kind, rot_block, quat);
     std::vector<double> z;
     std::vector<int64_t> rows;
