@@ -96,15 +96,16 @@ struct StepRow {
   uint32_t kp, vp;
 };
 
+// raw: the new K row then the V row (binary16, staged in shared memory)
 template <int D, int ROT, int LGB>
-__device__ __forceinline__ StepRow step_rows(const __half* k_row, const __half* v_row,
-                                             const float* quat, const float* cs, int lane) {
+__device__ __forceinline__ StepRow step_rows(const __half* raw, const float* quat,
+                                             const float* cs, int lane) {
   constexpr int CPL = RowQuantShape<D>::CPL;
   StepRow o;
 #pragma unroll 1
   for (int kv = 0; kv < 2; ++kv) {
     float x[CPL];
-    row_load<D>(x, (kv ? v_row : k_row) + lane * CPL, true);
+    row_load<D>(x, raw + kv * D + lane * CPL, true);
     if (kv == 0 && cs != nullptr) rope_regs<CPL>(x, cs + lane * CPL);
     __half s16, m16;
     const uint32_t packed = row_quantize<D, ROT, LGB>(x, lane, quat, s16, m16);
@@ -123,22 +124,20 @@ __device__ __forceinline__ StepRow step_rows(const __half* k_row, const __half* 
 
 // cs: the RoPE table row of the token's position (NULL: no RoPE)
 template <int D>
-__device__ __noinline__ StepRow quantize_step_token(const __half* k_row, const __half* v_row,
-                                                    const float* quat, const float* cs,
-                                                    int rot_kind, int lgb, int lane) {
-  if (rot_kind == KVQ_ROT_NONE) return step_rows<D, KVQ_ROT_NONE, 0>(k_row, v_row, quat, cs, lane);
-  if (rot_kind == KVQ_ROT_QUAT) return step_rows<D, KVQ_ROT_QUAT, 0>(k_row, v_row, quat, cs, lane);
-  if (rot_kind == KVQ_ROT_QUAT_FAST)
-    return step_rows<D, KVQ_ROT_QUAT_FAST, 0>(k_row, v_row, quat, cs, lane);
+__device__ __noinline__ StepRow quantize_step_token(const __half* raw, const float* quat,
+                                                    const float* cs, int rot_kind, int lgb,
+                                                    int lane) {
+  if (rot_kind == KVQ_ROT_NONE) return step_rows<D, KVQ_ROT_NONE, 0>(raw, quat, cs, lane);
+  if (rot_kind == KVQ_ROT_QUAT) return step_rows<D, KVQ_ROT_QUAT, 0>(raw, quat, cs, lane);
+  if (rot_kind == KVQ_ROT_QUAT_FAST) return step_rows<D, KVQ_ROT_QUAT_FAST, 0>(raw, quat, cs, lane);
   // the Hadamard rows take the sign table (randomised signs) or NULL
   if (rot_kind == KVQ_ROT_HADAMARD) quat = nullptr;
   switch (lgb) {
-    case 4: return step_rows<D, KVQ_ROT_HADAMARD, 4>(k_row, v_row, quat, cs, lane);
-    case 5: return step_rows<D, KVQ_ROT_HADAMARD, 5>(k_row, v_row, quat, cs, lane);
-    case 6: return step_rows<D, KVQ_ROT_HADAMARD, 6>(k_row, v_row, quat, cs, lane);
-    case 7: return step_rows<D, KVQ_ROT_HADAMARD, 7>(k_row, v_row, quat, cs, lane);
-    default:
-      return step_rows<D, KVQ_ROT_HADAMARD, (D >= 256 ? 8 : 7)>(k_row, v_row, quat, cs, lane);
+    case 4: return step_rows<D, KVQ_ROT_HADAMARD, 4>(raw, quat, cs, lane);
+    case 5: return step_rows<D, KVQ_ROT_HADAMARD, 5>(raw, quat, cs, lane);
+    case 6: return step_rows<D, KVQ_ROT_HADAMARD, 6>(raw, quat, cs, lane);
+    case 7: return step_rows<D, KVQ_ROT_HADAMARD, 7>(raw, quat, cs, lane);
+    default: return step_rows<D, KVQ_ROT_HADAMARD, (D >= 256 ? 8 : 7)>(raw, quat, cs, lane);
   }
 }
 
@@ -176,9 +175,11 @@ struct DecCfg {
   static constexpr int STAGE_B = PG * PAGE_B;
   // pipeline depth: about 8-13 KB of pages in flight per warp
   static constexpr int NST = STAGE_B <= 2304 ? 4 : (STAGE_B <= 4608 ? 3 : 2);
-  // behind the ring: the new token's K and V code rows and parameter words
-  // of a fused decode step, kept until its page is staged
-  static constexpr int STEP_B = (2 * ROWB + 8 + 127) / 128 * 128;
+  // behind the ring, for a fused decode step: the new token's binary16 K and
+  // V rows as copied in, then its K and V code rows and parameter words,
+  // kept until its page is staged
+  static constexpr int RAW_B = 2 * D * 2;
+  static constexpr int STEP_B = (RAW_B + 2 * ROWB + 8 + 127) / 128 * 128;
   static constexpr int WARP_B = (NST * STAGE_B + STEP_B + 127) / 128 * 128;
 };
 // Rotation of a query row held as quarters: lane j of a group of four
@@ -279,6 +280,24 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : (GP == 8 ? 3
   const int new_pg = L >= 1 ? (L - 1) / P : -1;
   const bool step_owner = a.k_new != nullptr && new_pg >= pg_lo && new_pg < pg_hi;
   int new_grp = -1;  // group of the new token's page (-1: none to patch)
+  // its inputs go out before this warp's (and ahead of most warps') page
+  // copies, so they do not queue behind the page traffic: the two binary16
+  // rows by cp.async into the stash behind the ring (part of the first
+  // commit group), the block-table entry into a register
+  uint8_t* const stash = ring + C::NST * C::STAGE_B;  // [K, V raw rows][K, V codes][params]
+  int step_page = -1;
+  if (step_owner) {
+    step_page = bt_row[new_pg];
+    const int64_t src = (int64_t)s * a.new_stride + (int64_t)h * D;
+    constexpr int LB = D / 16;  // raw bytes per lane and row: 8 (d 128) or 16 (d 256)
+    if (LB == 16) {
+      cp_async16(stash + lane * 16, a.k_new + src + lane * 8);
+      cp_async16(stash + 2 * D + lane * 16, a.v_new + src + lane * 8);
+    } else {
+      cp_async8(stash + lane * 8, a.k_new + src + lane * 4);
+      cp_async8(stash + 2 * D + lane * 8, a.v_new + src + lane * 4);
+    }
+  }
   // The warp's block-table entries sit in lane registers, 32 pages at a
   // time: lane i holds the entry of page pg_lo + 32 c + i of chunk c. An
   // entry outside [0, NP) raises KVQ_ERRF_PAGE when it is loaded and its page
@@ -392,26 +411,30 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : (GP == 8 ? 3
     else
       cp_async_commit();
   }
-  uint8_t* const stash = ring + C::NST * C::STAGE_B;  // [K row][V row][K, V params]
   if (step_owner) {
-    const int page = bt_row[new_pg];
-    if (page >= 0 && page < a.NP) {
-      const int64_t src = (int64_t)s * a.new_stride + (int64_t)h * D;
+    // the new token's rows came in the first commit group: wait for that
+    // group alone, quantize the rows, write them to the pools and keep the
+    // codes for the patch of the staged page
+    cp_async_wait<C::NST - 2>();
+    __syncwarp();
+    if (step_page >= 0 && step_page < a.NP) {
       const StepRow nr = quantize_step_token<D>(
-          a.k_new + src, a.v_new + src, a.quat,
+          reinterpret_cast<const __half*>(stash), a.quat,
           a.rope != nullptr ? a.rope + (int64_t)(L - 1) * D : nullptr, a.rot_kind, a.lgb, lane);
-      const int64_t row = ((int64_t)page * a.H + h) * P + (L - 1) % P;
+      const int64_t row = ((int64_t)step_page * a.H + h) * P + (L - 1) % P;
       constexpr int LB = RowQuantShape<D>::CPL / 2;  // code bytes per lane
+      uint8_t* const cst = stash + C::RAW_B;
       put_codes<D>(a.k_codes_w + row * (D / 2) + lane * LB, nr.kc);
       put_codes<D>(a.v_codes_w + row * (D / 2) + lane * LB, nr.vc);
-      put_codes<D>(stash + lane * LB, nr.kc);
-      put_codes<D>(stash + C::ROWB + lane * LB, nr.vc);
+      put_codes<D>(cst + lane * LB, nr.kc);
+      put_codes<D>(cst + C::ROWB + lane * LB, nr.vc);
       if (lane == 0) {
         a.k_params_w[row] = nr.kp;
         a.v_params_w[row] = nr.vp;
-        *reinterpret_cast<uint2*>(stash + 2 * C::ROWB) = make_uint2(nr.kp, nr.vp);
+        *reinterpret_cast<uint2*>(cst + 2 * C::ROWB) = make_uint2(nr.kp, nr.vp);
       }
       new_grp = (new_pg - pg_lo) / C::PG;
+      __syncwarp();
     } else if (lane == 0) {
       raise_flag(a.err, KVQ_ERRF_PAGE);
     }
@@ -535,11 +558,11 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : (GP == 8 ? 3
       constexpr int LB = RowQuantShape<D>::CPL / 2;
       uint8_t* const pb = st + ((new_pg - pg_lo) % C::PG) * C::PAGE_B;
       const int sl = (L - 1) % P;
-      put_codes<D>(pb + sl * C::ROWB + lane * LB, get_codes<D>(stash + lane * LB));
-      put_codes<D>(pb + C::CODE_B + sl * C::ROWB + lane * LB,
-                   get_codes<D>(stash + C::ROWB + lane * LB));
+      const uint8_t* const cst = stash + C::RAW_B;
+      put_codes<D>(pb + sl * C::ROWB + lane * LB, get_codes<D>(cst + lane * LB));
+      put_codes<D>(pb + C::CODE_B + sl * C::ROWB + lane * LB, get_codes<D>(cst + C::ROWB + lane * LB));
       if (lane == 0) {
-        const uint2 pw = *reinterpret_cast<const uint2*>(stash + 2 * C::ROWB);
+        const uint2 pw = *reinterpret_cast<const uint2*>(cst + 2 * C::ROWB);
         *reinterpret_cast<uint32_t*>(pb + 2 * C::CODE_B + sl * 4) = pw.x;
         *reinterpret_cast<uint32_t*>(pb + 2 * C::CODE_B + P * 4 + sl * 4) = pw.y;
       }
