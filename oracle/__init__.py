@@ -31,7 +31,7 @@ import numpy as np
 
 from . import build as _build
 
-ROT_NONE, ROT_HADAMARD, ROT_QUAT, ROT_QUAT_FAST, ROT_HADAMARD_SIGNED = 0, 1, 2, 3, 4
+ROT_NONE, ROT_HADAMARD, ROT_QUAT, ROT_QUAT_FAST, ROT_HADAMARD_SIGNED, ROT_QUAT_MAT = 0, 1, 2, 3, 4, 5
 RN, RD, RU = 0, 1, 2
 ERR_PAGE, ERR_POS, ERR_SEQ, ERR_LEN = 1, 2, 4, 8
 
@@ -52,6 +52,7 @@ def lib():
             "orc_sub_ru": (ctypes.c_float, [ctypes.c_float, ctypes.c_float]),
             "orc_div_ru": (ctypes.c_float, [ctypes.c_float, ctypes.c_float]),
             "orc_hamilton_f32": (None, [P, P, P]),
+            "orc_quat_matrix_f32": (None, [P, P]),
             "orc_float_to_half_array": (None, [P, i64, i32, P]),
             "orc_double_to_half_array": (None, [P, i64, i32, P]),
             "orc_half_to_double_array": (None, [P, i64, P]),
@@ -157,6 +158,15 @@ def hamilton(a, b):
     out = np.empty(4, np.float32)
     lib().orc_hamilton_f32(_p(a), _p(b), _p(out))
     return out
+
+
+def quat_matrix(q8):
+    """The binary32 4x4 matrix of v -> qL v conj(qR) for one table entry
+    (qL, qR) as the matrix-form rotation builds it."""
+    q8 = _c(q8, np.float32).reshape(8)
+    out = np.empty(16, np.float32)
+    lib().orc_quat_matrix_f32(_p(q8), _p(out))
+    return out.reshape(4, 4)
 
 
 def rotate_f32(x, kind, block=0, quat=None):

@@ -222,15 +222,63 @@ void orc_rotate_signed_hadamard_f32(float* x, int d, int b, const float* signs) 
   orc_rotate_hadamard_f32(x, d, b);
 }
 
+// IsoQuant-Full folded into one 4x4 matrix per block (IsoQuant page,
+// Abstract: the map v -> qL v conj(qR) is linear in v, so it is a 4x4 real
+// matrix M = Rm(conj qR) Lm(qL), Lm(a) the matrix of v -> a v and Rm(b) the
+// matrix of t -> t b). Reading: M is built in binary32 from the table's
+// quaternions, each entry M[r][c] = sum over k of Rm[r][k] Lm[k][c] as
+// fma(t3, fma(t2, fma(t1, t0))) with t0 the plain product and k ascending;
+// the map is then y_r = fma(M[r][3] v3, fma(M[r][2] v2, fma(M[r][1] v1,
+// M[r][0] v0))): 16 multiply-adds per block instead of 32, with a rounding
+// that differs from the two Hamilton products'.
+//   Lm(a) rows: ( a.w, -a.x, -a.y, -a.z), ( a.x,  a.w, -a.z,  a.y),
+//               ( a.y,  a.z,  a.w, -a.x), ( a.z, -a.y,  a.x,  a.w)
+//   Rm(b) rows: ( b.w, -b.x, -b.y, -b.z), ( b.x,  b.w,  b.z, -b.y),
+//               ( b.y, -b.z,  b.w,  b.x), ( b.z,  b.y, -b.x,  b.w)
+void orc_quat_matrix_f32(const float* q8, float* M) {
+  const float* a = q8;
+  const float b[4] = {q8[4], -q8[5], -q8[6], -q8[7]};  // conj(qR)
+  const float Lm[4][4] = {{a[0], -a[1], -a[2], -a[3]},
+                          {a[1], a[0], -a[3], a[2]},
+                          {a[2], a[3], a[0], -a[1]},
+                          {a[3], -a[2], a[1], a[0]}};
+  const float Rm[4][4] = {{b[0], -b[1], -b[2], -b[3]},
+                          {b[1], b[0], b[3], -b[2]},
+                          {b[2], -b[3], b[0], b[1]},
+                          {b[3], b[2], -b[1], b[0]}};
+  for (int r = 0; r < 4; ++r)
+    for (int c = 0; c < 4; ++c) {
+      float m = Rm[r][0] * Lm[0][c];
+      for (int k = 1; k < 4; ++k) m = std::fma(Rm[r][k], Lm[k][c], m);
+      M[4 * r + c] = m;
+    }
+}
+
+void orc_rotate_quat_mat_f32(float* x, int d, const float* quat) {
+  for (int j = 0; j < d / 4; ++j) {
+    float M[16];
+    orc_quat_matrix_f32(quat + j * 8, M);
+    const float* v = x + 4 * j;
+    float y[4];
+    for (int r = 0; r < 4; ++r) {
+      float t = M[4 * r] * v[0];
+      for (int c = 1; c < 4; ++c) t = std::fma(M[4 * r + c], v[c], t);
+      y[r] = t;
+    }
+    for (int r = 0; r < 4; ++r) x[4 * j + r] = y[r];
+  }
+}
+
 // Rotation kinds (same numbering as the library's public enum, restated).
 enum { ORC_ROT_NONE = 0, ORC_ROT_HADAMARD = 1, ORC_ROT_QUAT = 2, ORC_ROT_QUAT_FAST = 3,
-       ORC_ROT_HADAMARD_SIGNED = 4 };
+       ORC_ROT_HADAMARD_SIGNED = 4, ORC_ROT_QUAT_MAT = 5 };
 
 void orc_rotate_f32(float* x, int d, int kind, int b, const float* quat) {
   if (kind == ORC_ROT_HADAMARD) orc_rotate_hadamard_f32(x, d, b);
   else if (kind == ORC_ROT_QUAT) orc_rotate_quat_f32(x, d, quat);
   else if (kind == ORC_ROT_QUAT_FAST) orc_rotate_quat_fast_f32(x, d, quat);
   else if (kind == ORC_ROT_HADAMARD_SIGNED) orc_rotate_signed_hadamard_f32(x, d, b, quat);
+  else if (kind == ORC_ROT_QUAT_MAT) orc_rotate_quat_mat_f32(x, d, quat);
 }
 
 // ---------------------------------------------------------------------------
@@ -421,7 +469,19 @@ static void hamilton_f64(const double* a, const double* b, double* o) {
 }
 
 void orc_rotate_f64(double* x, int d, int kind, int b, const float* quat) {
-  if (kind == ORC_ROT_HADAMARD_SIGNED) {
+  if (kind == ORC_ROT_QUAT_MAT) {
+    // the binary32 matrix M the cache was written with, applied exactly
+    for (int j = 0; j < d / 4; ++j) {
+      float M[16];
+      orc_quat_matrix_f32(quat + j * 8, M);
+      double y[4];
+      for (int r = 0; r < 4; ++r) {
+        y[r] = 0.0;
+        for (int c = 0; c < 4; ++c) y[r] += (double)M[4 * r + c] * x[4 * j + c];
+      }
+      for (int r = 0; r < 4; ++r) x[4 * j + r] = y[r];
+    }
+  } else if (kind == ORC_ROT_HADAMARD_SIGNED) {
     for (int i = 0; i < d; ++i) x[i] *= (double)quat[i];
     orc_rotate_f64(x, d, ORC_ROT_HADAMARD, b, quat);
   } else if (kind == ORC_ROT_QUAT_FAST) {
@@ -456,7 +516,20 @@ void orc_rotate_f64(double* x, int d, int kind, int b, const float* quat) {
 }
 
 void orc_unrotate_f64(double* x, int d, int kind, int b, const float* quat) {
-  if (kind == ORC_ROT_HADAMARD) {
+  if (kind == ORC_ROT_QUAT_MAT) {
+    // reading: the inverse of the (orthogonal up to binary32 rounding)
+    // matrix is taken as its transpose
+    for (int j = 0; j < d / 4; ++j) {
+      float M[16];
+      orc_quat_matrix_f32(quat + j * 8, M);
+      double y[4];
+      for (int c = 0; c < 4; ++c) {
+        y[c] = 0.0;
+        for (int r = 0; r < 4; ++r) y[c] += (double)M[4 * r + c] * x[4 * j + r];
+      }
+      for (int c = 0; c < 4; ++c) x[4 * j + c] = y[c];
+    }
+  } else if (kind == ORC_ROT_HADAMARD) {
     orc_rotate_f64(x, d, kind, b, quat);  // R^-1 = R
   } else if (kind == ORC_ROT_HADAMARD_SIGNED) {
     // R = H S with S the sign diagonal: R^-1 = S^-1 H^-1 = S H

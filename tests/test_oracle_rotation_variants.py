@@ -117,3 +117,84 @@ def test_signed_hadamard_against_the_matrix(b):
     back = oracle.unrotate_f64(oracle.rotate_f64(xd, oracle.ROT_HADAMARD_SIGNED, b, signs),
                                oracle.ROT_HADAMARD_SIGNED, b, signs)
     assert np.allclose(back, xd, rtol=0, atol=1e-12)
+
+
+# --- IsoQuant-Full as one 4x4 matrix per block ------------------------------
+# Pinned against the two multiplication matrices written out from the
+# quaternion unit table (i^2 = j^2 = k^2 = ijk = -1), exact Hurwitz cases,
+# the identity table, the two-product form to a few binary32 ulps, and
+# orthogonality.
+
+UNIT_PRODUCT = {  # (row unit) * (column unit) = sign, unit
+    (0, 0): (1, 0), (0, 1): (1, 1), (0, 2): (1, 2), (0, 3): (1, 3),
+    (1, 0): (1, 1), (1, 1): (-1, 0), (1, 2): (1, 3), (1, 3): (-1, 2),
+    (2, 0): (1, 2), (2, 1): (-1, 3), (2, 2): (-1, 0), (2, 3): (1, 1),
+    (3, 0): (1, 3), (3, 1): (1, 2), (3, 2): (-1, 1), (3, 3): (-1, 0),
+}
+
+
+def qmul(a, b):
+    """Quaternion product from the unit multiplication table (float64)."""
+    out = np.zeros(4)
+    for i in range(4):
+        for j in range(4):
+            sg, u = UNIT_PRODUCT[(i, j)]
+            out[u] += sg * a[i] * b[j]
+    return out
+
+
+def full_map_matrix(q8):
+    """Columns: T(e_c) = qL e_c conj(qR) in float64."""
+    qL = q8[:4].astype(np.float64)
+    qRc = np.array([q8[4], -q8[5], -q8[6], -q8[7]], np.float64)
+    return np.stack([qmul(qmul(qL, e), qRc) for e in np.eye(4)], axis=1)
+
+
+def test_matrix_entries_against_the_unit_table():
+    quat = workloads.random_quaternions(11, 128)
+    for j in range(32):
+        M = oracle.quat_matrix(quat[j])
+        ref = full_map_matrix(quat[j].reshape(8))
+        # four binary32 multiply-adds of terms at most 1 in size
+        assert np.max(np.abs(M.astype(np.float64) - ref)) <= 4 * 2.0 ** -24
+
+
+def test_matrix_hurwitz_exact_and_identity():
+    g = np.random.default_rng(4)
+    q = (0.5 * g.choice([-1.0, 1.0], size=(16, 8))).astype(np.float32)
+    for j in range(16):
+        assert np.array_equal(oracle.quat_matrix(q[j]).astype(np.float64), full_map_matrix(q[j]))
+    ident = np.tile(np.array([1, 0, 0, 0, 1, 0, 0, 0], np.float32), (16, 1))
+    assert np.array_equal(oracle.quat_matrix(ident[0]), np.eye(4, dtype=np.float32))
+    x = g.standard_normal((6, 64)).astype(np.float32)
+    assert np.array_equal(oracle.rotate_f32(x, oracle.ROT_QUAT_MAT, 0, ident.reshape(16, 2, 4)), x)
+    # Hurwitz table on small integers: every product and sum is exact
+    xi = g.integers(-50, 50, size=(6, 64)).astype(np.float32)
+    y = oracle.rotate_f32(xi, oracle.ROT_QUAT_MAT, 0, q.reshape(16, 2, 4))
+    ref = np.concatenate([xi[:, 4 * j:4 * j + 4].astype(np.float64) @ full_map_matrix(q[j]).T
+                          for j in range(16)], axis=1)
+    assert np.array_equal(y.astype(np.float64), ref)
+
+
+def test_matrix_form_close_to_two_products_and_orthogonal():
+    d = 128
+    g = np.random.default_rng(6)
+    quat = workloads.random_quaternions(2, d)
+    x = g.standard_normal((50, d)).astype(np.float32)
+    ym = oracle.rotate_f32(x, oracle.ROT_QUAT_MAT, 0, quat)
+    yq = oracle.rotate_f32(x, oracle.ROT_QUAT, 0, quat)
+    scale = np.abs(x).reshape(50, d // 4, 4).max(axis=2).repeat(4, axis=1)
+    assert np.all(np.abs(ym - yq) <= 16 * 2.0 ** -24 * scale)
+    assert np.any(ym != yq)  # a different rounding, not the same arithmetic
+    for j in range(d // 4):
+        M = oracle.quat_matrix(quat[j]).astype(np.float64)
+        assert np.allclose(M @ M.T, np.eye(4), rtol=0, atol=1e-6)
+    # the double-precision map is the binary32 matrix applied exactly; its
+    # transpose undoes it to the matrix's distance from orthogonality
+    xd = g.standard_normal((4, d))
+    fwd = oracle.rotate_f64(xd, oracle.ROT_QUAT_MAT, 0, quat)
+    for j in range(d // 4):
+        M = oracle.quat_matrix(quat[j]).astype(np.float64)
+        assert np.allclose(fwd[:, 4 * j:4 * j + 4], xd[:, 4 * j:4 * j + 4] @ M.T, rtol=0, atol=1e-13)
+    back = oracle.unrotate_f64(fwd, oracle.ROT_QUAT_MAT, 0, quat)
+    assert np.allclose(back, xd, rtol=0, atol=1e-5)
