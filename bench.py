@@ -654,12 +654,14 @@ def workload_records(device, seed=0):
     torch.cuda.empty_cache()
 
     # ---- prefill sweep: one layer per Hadamard block size, then the other
-    # rotation kinds (quaternion full and fast maps, randomised-sign b 64)
+    # rotation kinds (quaternion full, fast and matrix maps, randomised-sign
+    # b 64)
     sweep = {"workload": "65536 tokens x 8 KV heads x d 128 per layer, page 16"}
     variants = [(workloads.ROT_HADAMARD, b, "hadamard%d" % b) for b in (16, 32, 64, 128)]
     variants += [(workloads.ROT_NONE, 0, "no_rotation"),
                  (workloads.ROT_QUAT, 0, "quaternion"),
                  (workloads.ROT_QUAT_FAST, 0, "quaternion_fast"),
+                 (workloads.ROT_QUAT_MAT, 0, "quaternion_matrix"),
                  (workloads.ROT_HADAMARD_SIGNED, 64, "hadamard64_signed")]
     for kind, blk, name in variants:
         w = workloads.prefill(seed=seed, rot_block=blk)
@@ -667,7 +669,7 @@ def workload_records(device, seed=0):
         K, V = _device_kv(w, len(ts), gen, device)
         TS, TP, BT = dev(ts), dev(tp), dev(w.block_table)
         table = None
-        if kind in (workloads.ROT_QUAT, workloads.ROT_QUAT_FAST):
+        if kind in (workloads.ROT_QUAT, workloads.ROT_QUAT_FAST, workloads.ROT_QUAT_MAT):
             table = workloads.random_quaternions(seed, w.d)
         elif kind == workloads.ROT_HADAMARD_SIGNED:
             table = workloads.random_signs(seed, w.d)

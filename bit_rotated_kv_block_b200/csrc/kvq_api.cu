@@ -48,6 +48,7 @@ static int check_desc(const kvq_cache_desc* d) {
       break;
     case KVQ_ROT_QUAT:
     case KVQ_ROT_QUAT_FAST:
+    case KVQ_ROT_QUAT_MAT:
       if (d->quat == nullptr) return KVQ_ERR_INVALID_ARG;
       if (!aligned16(d->quat)) return KVQ_ERR_MISALIGNED;
       break;

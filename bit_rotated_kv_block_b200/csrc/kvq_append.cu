@@ -60,6 +60,11 @@ __host__ __device__ constexpr int append_e(int D, int rot, int lgb) {
                  : (D == 256 || (rot == KVQ_ROT_HADAMARD && (lgb >= 7 || lgb <= 4))) ? 128 : 64;
 }
 __host__ __device__ constexpr int append_threads(int E) { return E == 64 ? 256 : 384; }
+// bytes of the rotation table in shared memory: quaternion pairs (2 d
+// floats), signs (d), or the matrix form's 4x4 matrices (4 d floats)
+__host__ __device__ constexpr int append_table_bytes(int D, int rot) {
+  return rot == KVQ_ROT_QUAT_MAT ? D * 16 : D * 8;
+}
 __host__ __device__ constexpr int append_ctas_per_sm(int E) { return E == 64 ? 2 : 1; }
 
 // One thread's part of one row: E channels of a (token, head) row of K or
@@ -122,6 +127,8 @@ __device__ __forceinline__ void quantize_row_part(const uint8_t* boxes, int box_
     quat_fast_regs<E>(x, qtbl, my_part * E);
   } else if (ROT == KVQ_ROT_QUAT) {
     quat_regs<E>(x, qtbl, my_part * E);
+  } else if (ROT == KVQ_ROT_QUAT_MAT) {
+    quat_mat_regs<E>(x, qtbl, my_part * E);  // the CTA's matrices
   }
 
   // row statistics
@@ -227,7 +234,7 @@ __global__ void __launch_bounds__(append_threads(append_e(D, ROT, LGB)),
   uint8_t* const buf0 = smem;
   uint8_t* const buf1 = smem + bufb;
   float* qtbl = reinterpret_cast<float*>(smem + 2 * bufb);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * bufb + D * 8);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * bufb + append_table_bytes(D, ROT));
 
   const int tid = threadIdx.x;
   const int rows_per_tile = 2 * H * TOK * TPR;
@@ -238,7 +245,15 @@ __global__ void __launch_bounds__(append_threads(append_e(D, ROT, LGB)),
     mbar_fence_init();
   }
   // the rotation's table in shared memory: quaternions (2 D floats) or signs (D)
-  if (ROT == KVQ_ROT_QUAT || ROT == KVQ_ROT_QUAT_FAST) {
+  // or, for the matrix form, the 4x4 matrices built from the quaternions
+  if (ROT == KVQ_ROT_QUAT_MAT) {
+    for (int j = tid; j < D / 4; j += kAppendThreads) {
+      float M[16];
+      quat_matrix(a.quat + 8 * j, M);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) qtbl[16 * j + i] = M[i];
+    }
+  } else if (ROT == KVQ_ROT_QUAT || ROT == KVQ_ROT_QUAT_FAST) {
     for (int i = tid; i < D * 2; i += kAppendThreads) qtbl[i] = a.quat[i];
   } else if (ROT == KVQ_ROT_HADAMARD && a.quat != nullptr) {
     for (int i = tid; i < D; i += kAppendThreads) qtbl[i] = a.quat[i];
@@ -450,6 +465,7 @@ static cudaError_t dispatch_rows(const AppendRowsArgs& a, int rot, int lgb, cuda
   if (rot == KVQ_ROT_NONE) return launch_rows<D, KVQ_ROT_NONE, 0>(a, st);
   if (rot == KVQ_ROT_QUAT) return launch_rows<D, KVQ_ROT_QUAT, 0>(a, st);
   if (rot == KVQ_ROT_QUAT_FAST) return launch_rows<D, KVQ_ROT_QUAT_FAST, 0>(a, st);
+  if (rot == KVQ_ROT_QUAT_MAT) return launch_rows<D, KVQ_ROT_QUAT_MAT, 0>(a, st);
   switch (lgb) {
     case 4: return launch_rows<D, KVQ_ROT_HADAMARD, 4>(a, st);
     case 5: return launch_rows<D, KVQ_ROT_HADAMARD, 5>(a, st);
@@ -494,14 +510,15 @@ static bool encode_rows(CUtensorMap* m, const void* base, int D, int H, int T,
          CUDA_SUCCESS;
 }
 
-static size_t append_smem(int D, int box_stride) {
-  return 1024 + 2 * (size_t)(2 * (D / 64)) * box_stride + (size_t)D * 8 + 2 * sizeof(uint64_t);
+static size_t append_smem(int D, int rot, int box_stride) {
+  return 1024 + 2 * (size_t)(2 * (D / 64)) * box_stride + append_table_bytes(D, rot) +
+         2 * sizeof(uint64_t);
 }
 
 template <int D, int ROT, int LGB>
 static cudaError_t launch_append(const AppendArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
                                  int grid, cudaStream_t st) {
-  const size_t smem = append_smem(D, a.box_stride);
+  const size_t smem = append_smem(D, ROT, a.box_stride);
   const bool pre = a.rope != nullptr || (ROT == KVQ_ROT_HADAMARD && a.quat != nullptr);
   auto kern = pre ? append_kernel<D, ROT, LGB, true> : append_kernel<D, ROT, LGB, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -517,6 +534,7 @@ static cudaError_t dispatch_rot(const AppendArgs& a, const CUtensorMap& tk, cons
   if (rot == KVQ_ROT_NONE) return launch_append<D, KVQ_ROT_NONE, 0>(a, tk, tv, grid, st);
   if (rot == KVQ_ROT_QUAT) return launch_append<D, KVQ_ROT_QUAT, 0>(a, tk, tv, grid, st);
   if (rot == KVQ_ROT_QUAT_FAST) return launch_append<D, KVQ_ROT_QUAT_FAST, 0>(a, tk, tv, grid, st);
+  if (rot == KVQ_ROT_QUAT_MAT) return launch_append<D, KVQ_ROT_QUAT_MAT, 0>(a, tk, tv, grid, st);
   switch (lgb) {
     case 4: return launch_append<D, KVQ_ROT_HADAMARD, 4>(a, tk, tv, grid, st);
     case 5: return launch_append<D, KVQ_ROT_HADAMARD, 5>(a, tk, tv, grid, st);

@@ -130,6 +130,7 @@ __device__ __noinline__ StepRow quantize_step_token(const __half* raw, const flo
   if (rot_kind == KVQ_ROT_NONE) return step_rows<D, KVQ_ROT_NONE, 0>(raw, quat, cs, lane);
   if (rot_kind == KVQ_ROT_QUAT) return step_rows<D, KVQ_ROT_QUAT, 0>(raw, quat, cs, lane);
   if (rot_kind == KVQ_ROT_QUAT_FAST) return step_rows<D, KVQ_ROT_QUAT_FAST, 0>(raw, quat, cs, lane);
+  if (rot_kind == KVQ_ROT_QUAT_MAT) return step_rows<D, KVQ_ROT_QUAT_MAT, 0>(raw, quat, cs, lane);
   // the Hadamard rows take the sign table (randomised signs) or NULL
   if (rot_kind == KVQ_ROT_HADAMARD) quat = nullptr;
   switch (lgb) {
@@ -216,6 +217,8 @@ __device__ __forceinline__ void rotate_quarter(float (&x)[QW], int j, int rot_ki
     quat_regs<QW>(x, tbl, j * QW);
   } else if (rot_kind == KVQ_ROT_QUAT_FAST) {
     quat_fast_regs<QW>(x, tbl, j * QW);
+  } else if (rot_kind == KVQ_ROT_QUAT_MAT) {
+    quat_mat_fly_regs<QW>(x, tbl, j * QW);
   }
 }
 
@@ -898,6 +901,8 @@ __device__ __forceinline__ void row_unrotate(float (&x)[CPL], int lane, int rot_
     quat_inv_regs<CPL>(x, quat, lane * CPL);
   } else if (rot_kind == KVQ_ROT_QUAT_FAST) {
     quat_fast_inv_regs<CPL>(x, quat, lane * CPL);
+  } else if (rot_kind == KVQ_ROT_QUAT_MAT) {
+    quat_mat_fly_regs<CPL, true>(x, quat, lane * CPL);
   }
 }
 

@@ -76,6 +76,7 @@ __global__ void __launch_bounds__(128) dequant_kernel(const DequantArgs a, int u
     }
     if (ROT == KVQ_ROT_QUAT) quat_inv_regs<E>(x, a.quat, part * E);
     if (ROT == KVQ_ROT_QUAT_FAST) quat_fast_inv_regs<E>(x, a.quat, part * E);
+    if (ROT == KVQ_ROT_QUAT_MAT) quat_mat_fly_regs<E, true>(x, a.quat, part * E);
   }
   const int64_t o = (((int64_t)s * a.L + j) * a.H + h) * D + part * E;
   if (F32) {
@@ -113,6 +114,7 @@ static cudaError_t dq_rot(const DequantArgs& a, int rot, int lgb, int unrotate, 
   if (rot == KVQ_ROT_NONE || !unrotate) return launch_dq<D, KVQ_ROT_NONE, 0>(a, 0, f32, st);
   if (rot == KVQ_ROT_QUAT) return launch_dq<D, KVQ_ROT_QUAT, 0>(a, 1, f32, st);
   if (rot == KVQ_ROT_QUAT_FAST) return launch_dq<D, KVQ_ROT_QUAT_FAST, 0>(a, 1, f32, st);
+  if (rot == KVQ_ROT_QUAT_MAT) return launch_dq<D, KVQ_ROT_QUAT_MAT, 0>(a, 1, f32, st);
   switch (lgb) {
     case 4: return launch_dq<D, KVQ_ROT_HADAMARD, 4>(a, 1, f32, st);
     case 5: return launch_dq<D, KVQ_ROT_HADAMARD, 5>(a, 1, f32, st);

@@ -165,6 +165,66 @@ __device__ __forceinline__ void quat_fast_inv_regs(float (&x)[E], const float* t
   }
 }
 
+// IsoQuant-Full folded into one binary32 4x4 matrix per block: the map
+// v -> qL v conj(qR) is linear in v, M = Rm(conj qR) Lm(qL) with Lm(a) the
+// matrix of v -> a v and Rm(b) that of t -> t b. Entry (r, c) is the sum over
+// k of Rm[r][k] Lm[k][c], k ascending, as a chain of fused multiply-adds
+// from the plain first product; q = (qL, qR) as in the quaternion table.
+__device__ __forceinline__ void quat_matrix(const float* q, float (&M)[16]) {
+  const float aw = q[0], ax = q[1], ay = q[2], az = q[3];
+  const float bw = q[4], bx = -q[5], by = -q[6], bz = -q[7];  // conj(qR)
+  const float Lm[4][4] = {{aw, -ax, -ay, -az}, {ax, aw, -az, ay}, {ay, az, aw, -ax},
+                          {az, -ay, ax, aw}};
+  const float Rm[4][4] = {{bw, -bx, -by, -bz}, {bx, bw, bz, -by}, {by, -bz, bw, bx},
+                          {bz, by, -bx, bw}};
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float m = __fmul_rn(Rm[r][0], Lm[0][c]);
+#pragma unroll
+      for (int k = 1; k < 4; ++k) m = __fmaf_rn(Rm[r][k], Lm[k][c], m);
+      M[4 * r + c] = m;
+    }
+}
+
+// y = M v per block (row r: fma(M[r][3] v3, fma(M[r][2] v2, fma(M[r][1] v1,
+// M[r][0] v0)))), the matrices read from mats [d/4][16] (ch0 the thread's
+// first channel, a multiple of 4).
+template <int E>
+__device__ __forceinline__ void quat_mat_regs(float (&x)[E], const float* mats, int ch0) {
+#pragma unroll
+  for (int k = 0; k < E / 4; ++k) {
+    const float4* m4 = reinterpret_cast<const float4*>(mats + (ch0 / 4 + k) * 16);
+    const float v0 = x[4 * k], v1 = x[4 * k + 1], v2 = x[4 * k + 2], v3 = x[4 * k + 3];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float4 m = m4[r];
+      x[4 * k + r] = __fmaf_rn(m.w, v3, __fmaf_rn(m.z, v2, __fmaf_rn(m.y, v1, __fmul_rn(m.x, v0))));
+    }
+  }
+}
+
+// The same map with each block's matrix built from the quaternion table on
+// the spot (paths that rotate few rows); INV applies the transpose instead
+// (the inverse of the orthogonal map), in plain binary32 arithmetic.
+template <int E, bool INV = false>
+__device__ __forceinline__ void quat_mat_fly_regs(float (&x)[E], const float* tbl, int ch0) {
+#pragma unroll
+  for (int k = 0; k < E / 4; ++k) {
+    float M[16];
+    quat_matrix(tbl + (ch0 / 4 + k) * 8, M);
+    const float v[4] = {x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3]};
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int i0 = INV ? r : 4 * r, st = INV ? 4 : 1;
+      x[4 * k + r] = __fmaf_rn(M[i0 + 3 * st], v[3],
+                               __fmaf_rn(M[i0 + 2 * st], v[2],
+                                         __fmaf_rn(M[i0 + st], v[1], __fmul_rn(M[i0], v[0]))));
+    }
+  }
+}
+
 // Randomised-sign Hadamard: each channel times its fixed sign (+1 or -1,
 // exact); `signs` offset to the thread's first channel.
 template <int E>

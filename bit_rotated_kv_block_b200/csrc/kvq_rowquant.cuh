@@ -68,6 +68,8 @@ __device__ __forceinline__ uint32_t row_quantize(float (&x)[RowQuantShape<D>::CP
     quat_regs<CPL>(x, quat, rl * CPL);
   } else if (ROT == KVQ_ROT_QUAT_FAST) {
     quat_fast_regs<CPL>(x, quat, rl * CPL);
+  } else if (ROT == KVQ_ROT_QUAT_MAT) {
+    quat_mat_fly_regs<CPL>(x, quat, rl * CPL);
   }
 
   float mn = x[0], mx = x[0];

@@ -14,7 +14,8 @@ import torch
 
 from . import build as _build
 
-ROT_NONE, ROT_HADAMARD, ROT_QUAT, ROT_QUAT_FAST, ROT_HADAMARD_SIGNED = 0, 1, 2, 3, 4
+ROT_NONE, ROT_HADAMARD, ROT_QUAT, ROT_QUAT_FAST, ROT_HADAMARD_SIGNED, ROT_QUAT_MAT = \
+    0, 1, 2, 3, 4, 5
 ERRF_PAGE, ERRF_POS, ERRF_SEQ, ERRF_LEN = 1, 2, 4, 8
 STATUS = {0: "KVQ_OK", 1: "KVQ_ERR_INVALID_ARG", 2: "KVQ_ERR_UNSUPPORTED",
           3: "KVQ_ERR_MISALIGNED", 4: "KVQ_ERR_WORKSPACE", 5: "KVQ_ERR_CUDA"}
@@ -106,7 +107,7 @@ class Cache:
         self.d, self.H, self.P, self.NP = head_dim, num_kv_heads, page_size, num_pages
         self.rot_kind, self.rot_block = rot_kind, rot_block
         self.quat = None  # the rotation's table: quaternions, or signs
-        if rot_kind in (ROT_QUAT, ROT_QUAT_FAST, ROT_HADAMARD_SIGNED):
+        if rot_kind in (ROT_QUAT, ROT_QUAT_FAST, ROT_HADAMARD_SIGNED, ROT_QUAT_MAT):
             self.quat = torch.as_tensor(quat, dtype=torch.float32).contiguous().to(device)
         self.rope = None
         if rope is not None:

@@ -36,7 +36,8 @@ from typing import Optional
 
 import numpy as np
 
-ROT_NONE, ROT_HADAMARD, ROT_QUAT, ROT_QUAT_FAST, ROT_HADAMARD_SIGNED = 0, 1, 2, 3, 4
+ROT_NONE, ROT_HADAMARD, ROT_QUAT, ROT_QUAT_FAST, ROT_HADAMARD_SIGNED, ROT_QUAT_MAT = \
+    0, 1, 2, 3, 4, 5
 
 WORKLOAD_IDS = {"tiny": 1, "llama8b": 2, "long70b": 3, "prefill": 4, "ragged256": 5}
 
@@ -238,7 +239,8 @@ def ragged256(seed: int = 0, S: int = 128, lo: int = 512, hi: int = 16384,
     quat = unit_quaternions(rng(seed, "ragged256", S_QUAT), d // 4)
     return Workload("ragged256", d, H, 16, P, NP, rot_kind,
                     256 if rot_kind == ROT_HADAMARD else 0, lens, table,
-                    quat=quat if rot_kind == ROT_QUAT else None, channel_mult=mult, seed=seed)
+                    quat=quat if rot_kind in (ROT_QUAT, ROT_QUAT_FAST, ROT_QUAT_MAT) else None,
+                    channel_mult=mult, seed=seed)
 
 
 def random_quaternions(seed: int, d: int) -> np.ndarray:

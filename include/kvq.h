@@ -66,8 +66,12 @@ typedef enum {
                                   (IsoQuant-Full)                                */
   KVQ_ROT_QUAT_FAST = 3,       /* per 4-channel block v -> qL v: one isoclinic
                                   factor (IsoQuant-Fast)                         */
-  KVQ_ROT_HADAMARD_SIGNED = 4  /* channel i times a fixed sign s_i = +-1, then
+  KVQ_ROT_HADAMARD_SIGNED = 4, /* channel i times a fixed sign s_i = +-1, then
                                   the block Walsh-Hadamard rotation              */
+  KVQ_ROT_QUAT_MAT = 5         /* IsoQuant-Full folded into one binary32 4x4
+                                  matrix per block, M = Rm(conj qR) Lm(qL), built
+                                  from the quaternion table (16 multiply-adds per
+                                  block instead of 32; another rounding)         */
 } kvq_rot_kind;
 
 /* Bits OR-ed into *err_flags by the kernels. */
@@ -92,9 +96,11 @@ typedef enum {
  *               of two in [16, 256] dividing d (ignored otherwise).
  *  quat         the rotation's table, a device pointer (NULL for
  *               KVQ_ROT_NONE and KVQ_ROT_HADAMARD):
- *               KVQ_ROT_QUAT, KVQ_ROT_QUAT_FAST: float [d/4][2][4], per block
- *               j (qL[j], qR[j]) as (w, x, y, z); unit quaternions (the fast
- *               map uses qL only). Channels 4j..4j+3 form block j.
+ *               KVQ_ROT_QUAT, KVQ_ROT_QUAT_FAST, KVQ_ROT_QUAT_MAT: float
+ *               [d/4][2][4], per block j (qL[j], qR[j]) as (w, x, y, z); unit
+ *               quaternions (the fast map uses qL only; the matrix form builds
+ *               its matrices from the same table inside each launch).
+ *               Channels 4j..4j+3 form block j.
  *               KVQ_ROT_HADAMARD_SIGNED: float [d] of signs, each +1 or -1.
  *               The quaternion maps' Hamilton components are fused
  *               multiply-add chains in the term order of the quantize

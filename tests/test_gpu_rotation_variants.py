@@ -1,8 +1,9 @@
-"""GPU parity of the two further rotation kinds against the oracle:
+"""GPU parity of the further rotation kinds against the oracle:
 IsoQuant-Fast (page "IsoQuant: Hardware-Aligned SO(4) Isoclinic Rotations for
-LLM KV Cache Compression", Abstract: one isoclinic factor, v -> qL v) and the
-randomised-sign Hadamard (channels flipped by a fixed sign table, then the
-block Hadamard). Codes, scales and page placement bit-exact in the bulk and the
+LLM KV Cache Compression", Abstract: one isoclinic factor, v -> qL v), the
+full map folded into one 4x4 matrix per block (same page: the map is linear),
+and the randomised-sign Hadamard (channels flipped by a fixed sign table, then
+the block Hadamard). Codes, scales and page placement bit-exact in the bulk and the
 small-batch append kernels and in the fused decode step; decode attention
 within 2e-3; the un-rotated dense export against the oracle's."""
 
@@ -22,7 +23,8 @@ TOL = 2e-3
 
 KINDS = [(workloads.ROT_QUAT_FAST, 0, 128), (workloads.ROT_HADAMARD_SIGNED, 64, 128),
          (workloads.ROT_HADAMARD_SIGNED, 128, 128), (workloads.ROT_QUAT_FAST, 0, 256),
-         (workloads.ROT_HADAMARD_SIGNED, 256, 256)]
+         (workloads.ROT_HADAMARD_SIGNED, 256, 256), (workloads.ROT_QUAT_MAT, 0, 128),
+         (workloads.ROT_QUAT_MAT, 0, 256)]
 
 
 def workload(kind, b, d):
@@ -31,7 +33,8 @@ def workload(kind, b, d):
     else:
         w = workloads.ragged256(S=5, lo=300, hi=1500)
     w.rot_kind, w.rot_block = kind, b
-    w.quat = (workloads.random_quaternions(11, d) if kind == workloads.ROT_QUAT_FAST
+    w.quat = (workloads.random_quaternions(11, d)
+              if kind in (workloads.ROT_QUAT_FAST, workloads.ROT_QUAT_MAT)
               else workloads.random_signs(12, d))
     return w
 
