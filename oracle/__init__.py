@@ -32,6 +32,7 @@ import numpy as np
 from . import build as _build
 
 ROT_NONE, ROT_HADAMARD, ROT_QUAT, ROT_QUAT_FAST, ROT_HADAMARD_SIGNED, ROT_QUAT_MAT = 0, 1, 2, 3, 4, 5
+FMT_INT4, FMT_MXFP4 = 0, 1
 RN, RD, RU = 0, 1, 2
 ERR_PAGE, ERR_POS, ERR_SEQ, ERR_LEN = 1, 2, 4, 8
 
@@ -62,11 +63,19 @@ def lib():
             "orc_fwht_unscaled": (None, [P, i32]),
             "orc_quantize_rows": (None, [P, i64, i32, P, P, P]),
             "orc_quantize_append": (None, [i32, i32, i32, i32, i32, i32, P, i32, P, P, i64,
-                                           P, P, i32, P, i32, P, P, P, P, P, i32, P]),
+                                           P, P, i32, P, i32, P, P, P, P, P, i32, i32, P]),
             "orc_dequantize_pages": (None, [i32, i32, i32, i32, i32, i32, P, i32, P, i32, P,
-                                            i32, P, P, i32, i32, P, P]),
+                                            i32, P, P, i32, i32, P, i32, P]),
             "orc_paged_decode_attn": (None, [i32, i32, i32, i32, i32, i32, P, i32, i32, P, P,
-                                             i32, P, i32, dbl, P, P, P, P, P, i32, P, P]),
+                                             i32, P, i32, dbl, P, P, P, P, P, i32, i32, P,
+                                             P]),
+            "orc_mx_exponent": (i32, [ctypes.c_float, i32]),
+            "orc_e2m1_encode": (i32, [dbl]),
+            "orc_e2m1_value": (dbl, [i32]),
+            "orc_e4m3_encode": (i32, [dbl]),
+            "orc_e4m3_value": (dbl, [i32]),
+            "orc_mxfp4_quantize_row": (None, [P, i32, P, P]),
+            "orc_mxfp8_row_values": (None, [P, i32, P]),
             "orc_rope_row_f32": (None, [P, i32, P]),
             "orc_paged_decode_attn_fp16": (None, [i32, i32, i32, i32, i32, i32, P, P, i32, P,
                                                   i32, dbl, P, P, P, P]),
@@ -195,6 +204,56 @@ def unrotate_f64(x, kind, block=0, quat=None):
     return x
 
 
+# --- microscaled FP4 / FP8 -------------------------------------------------------
+
+def mx_exponent(amax, emax):
+    return lib().orc_mx_exponent(float(amax), int(emax))
+
+
+def e2m1_encode(t):
+    return lib().orc_e2m1_encode(float(t))
+
+
+def e2m1_value(code):
+    return lib().orc_e2m1_value(int(code))
+
+
+def e4m3_encode(t):
+    return lib().orc_e4m3_encode(float(t))
+
+
+def e4m3_value(code):
+    return lib().orc_e4m3_value(int(code))
+
+
+def mxfp4_quantize_rows(y):
+    """Rotated binary32 rows [..., d] -> (E2M1 codes uint8 [..., d/2], UE8M0
+    scales uint8 [..., d/32])."""
+    y = _c(y, np.float32)
+    d = y.shape[-1]
+    flat = y.reshape(-1, d)
+    codes = np.empty((flat.shape[0], d // 2), np.uint8)
+    scales = np.empty((flat.shape[0], d // 32), np.uint8)
+    for r in range(flat.shape[0]):
+        row = np.ascontiguousarray(flat[r])
+        cr, sr = codes[r], scales[r]
+        lib().orc_mxfp4_quantize_row(_p(row), d, _p(cr), _p(sr))
+    return codes.reshape(y.shape[:-1] + (d // 2,)), scales.reshape(y.shape[:-1] + (d // 32,))
+
+
+def mxfp8_values(y):
+    """Rotated binary32 rows [..., d] -> their MX E4M3 values (float64)."""
+    y = _c(y, np.float32)
+    d = y.shape[-1]
+    flat = y.reshape(-1, d)
+    out = np.empty(flat.shape, np.float64)
+    for r in range(flat.shape[0]):
+        row = np.ascontiguousarray(flat[r])
+        o = out[r]
+        lib().orc_mxfp8_row_values(_p(row), d, _p(o))
+    return out.reshape(y.shape)
+
+
 # --- quantizer ----------------------------------------------------------------
 
 def quantize_rows(y):
@@ -231,10 +290,13 @@ def dequantize_rows(codes, s16, m16):
 # --- cache-level operations (same contract as the library's entry points) ----
 
 class Cache:
-    """Geometry of one paged INT4 cache (head_dim d, KV heads H, page size P,
-    pool size NP, rotation kind / block / quaternion table)."""
+    """Geometry of one paged cache (head_dim d, KV heads H, page size P,
+    pool size NP, rotation kind / block / quaternion table) and its format:
+    FMT_INT4 (token-wise INT4, params (s16, m16)) or FMT_MXFP4 (E2M1 codes,
+    one UE8M0 byte per 32 channels, a 4-byte params row)."""
 
-    def __init__(self, d, H, P, NP, rot_kind, rot_block=0, quat=None, rope=None):
+    def __init__(self, d, H, P, NP, rot_kind, rot_block=0, quat=None, rope=None, fmt=FMT_INT4):
+        self.fmt = int(fmt)
         self.d, self.H, self.P, self.NP = int(d), int(H), int(P), int(NP)
         self.rot_kind, self.rot_block = int(rot_kind), int(rot_block)
         self.quat = _quat(quat)
@@ -244,8 +306,15 @@ class Cache:
 
     def alloc_pools(self, fill=0):
         codes = np.full((self.NP, self.H, self.P, self.d // 2), fill, np.uint8)
-        params = np.full((self.NP, self.H, self.P, 2), (fill << 8) | fill, np.uint16)
+        if self.fmt == FMT_MXFP4:
+            params = np.full((self.NP, self.H, self.P, max(4, self.d // 32)), fill, np.uint8)
+        else:
+            params = np.full((self.NP, self.H, self.P, 2), (fill << 8) | fill, np.uint16)
         return codes, params
+
+    def params_array(self, params):
+        """A params pool as the C code reads it (bytes for MX FP4)."""
+        return _c(params, np.uint8 if self.fmt == FMT_MXFP4 else np.uint16)
 
 
 def quantize_append(cache, k, v, token_seq, token_pos, block_table, k_codes, k_params,
@@ -269,7 +338,7 @@ def quantize_append(cache, k, v, token_seq, token_pos, block_table, k_codes, k_p
                               cache.rot_block, _p(cache.quat), T, _p(k), _p(v), tok_stride,
                               _p(ts), _p(tp), num_seqs, _p(bt), bt.shape[1], _p(k_codes),
                               _p(k_params), _p(v_codes), _p(v_params), _p(cache.rope),
-                              cache.rope_max_pos, _p(err))
+                              cache.rope_max_pos, cache.fmt, _p(err))
     return int(err[0])
 
 
@@ -277,7 +346,7 @@ def dequantize_pages(cache, seq_lens, max_seq_len, block_table, codes, params, u
                      out_fp32=True, out=None):
     bt = _c(block_table, np.int32)
     lens = _c(seq_lens, np.int32)
-    codes, params = _c(codes, np.uint8), _c(params, np.uint16)
+    codes, params = _c(codes, np.uint8), cache.params_array(params)
     S = bt.shape[0]
     shape = (S, max_seq_len, cache.H, cache.d)
     if out is None:
@@ -286,7 +355,7 @@ def dequantize_pages(cache, seq_lens, max_seq_len, block_table, codes, params, u
     lib().orc_dequantize_pages(cache.d, cache.H, cache.P, cache.NP, cache.rot_kind,
                                cache.rot_block, _p(cache.quat), S, _p(lens), max_seq_len, _p(bt),
                                bt.shape[1], _p(codes), _p(params), int(bool(unrotate)),
-                               int(bool(out_fp32)), _p(out), _p(err))
+                               int(bool(out_fp32)), _p(out), cache.fmt, _p(err))
     return out, int(err[0])
 
 
@@ -298,15 +367,15 @@ def paged_decode_attn(cache, q, seq_lens, max_seq_len, block_table, sm_scale, k_
     S, Hq, d = q.shape
     bt = _c(block_table, np.int32)
     lens = _c(seq_lens, np.int32)
-    kc, kp = _c(k_codes, np.uint8), _c(k_params, np.uint16)
-    vc, vp = _c(v_codes, np.uint8), _c(v_params, np.uint16)
+    kc, kp = _c(k_codes, np.uint8), cache.params_array(k_params)
+    vc, vp = _c(v_codes, np.uint8), cache.params_array(v_params)
     out = np.empty((S, Hq, d), np.float64)
     err = np.zeros(1, np.int32)
     lib().orc_paged_decode_attn(cache.d, cache.H, cache.P, cache.NP, cache.rot_kind,
                                 cache.rot_block, _p(cache.quat), S, Hq, _p(q), _p(lens),
                                 max_seq_len, _p(bt), bt.shape[1], float(sm_scale), _p(kc),
                                 _p(kp), _p(vc), _p(vp), _p(cache.rope), cache.rope_max_pos,
-                                _p(out), _p(err))
+                                cache.fmt, _p(out), _p(err))
     return out, int(err[0])
 
 

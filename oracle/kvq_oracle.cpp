@@ -369,6 +369,142 @@ void orc_unpack_row(const uint8_t* codes, int d, int* c) {
 }
 
 // ---------------------------------------------------------------------------
+// Microscaled FP4 cache, a second format of the same paged cache (UltraQuant
+// page, method section: FP4 KV tensors with UE8M0 group scales and FP8
+// queries, taken by the matrix cores' scaled multiply-accumulate).
+// Readings: the Open Compute Project microscaling (MX) formats, which both
+// scaled matrix-core paths implement: blocks of 32 consecutive channels of a
+// rotated (token, head) row share one power-of-two scale 2^X stored as the
+// UE8M0 byte X + 127, with X = floor(log2(amax)) - emax, amax the block's
+// largest |x| and emax the element format's largest exponent (2 for E2M1, 8
+// for E4M3); X is clamped to [-127, 127] and an all-zero block takes
+// X = -127. Each element x / 2^X (exact: a power-of-two scaling) is rounded
+// to the nearest value of the element format, ties to even, saturating at
+// the format's largest finite value (6 for E2M1, 448 for E4M3), keeping the
+// sign of x (a negative value that rounds to zero becomes -0). E2M1 codes:
+// bit 3 sign, bits 2-0 index into {0, 0.5, 1, 1.5, 2, 3, 4, 6}; packed two
+// per byte, the even channel in the low nibble. E4M3: bit 7 sign, 4 exponent
+// bits (bias 7), 3 mantissa bits, subnormals m 2^-9.
+// ---------------------------------------------------------------------------
+
+int orc_mx_exponent(float amax, int emax) {
+  if (!(amax > 0.0f)) return -127;
+  int e2;
+  std::frexp((double)amax, &e2);  // amax = f 2^e2 with f in [0.5, 1)
+  int x = e2 - 1 - emax;          // floor(log2 amax) - emax
+  if (x < -127) x = -127;
+  if (x > 127) x = 127;
+  return x;
+}
+
+// Nearest value, ties to even, of a >= 0 on a grid with `mbits` mantissa
+// bits and smallest normal exponent emin, saturating at vmax.
+static double round_minifloat(double a, int mbits, int emin, double vmax) {
+  if (a >= vmax) return vmax;
+  if (a == 0.0) return 0.0;
+  int e2;
+  std::frexp(a, &e2);
+  int E = e2 - 1;
+  if (E < emin) E = emin;
+  const double quantum = std::ldexp(1.0, E - mbits);
+  const double r = rint_half_even(a / quantum) * quantum;
+  return r > vmax ? vmax : r;
+}
+
+static const double kE2M1[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+int orc_e2m1_encode(double t) {
+  const double r = round_minifloat(std::fabs(t), 1, 0, 6.0);
+  int m = 0;
+  while (kE2M1[m] != r) ++m;
+  return (std::signbit(t) ? 8 : 0) | m;
+}
+
+double orc_e2m1_value(int code) {
+  const double v = kE2M1[code & 7];
+  return (code & 8) ? -v : v;
+}
+
+int orc_e4m3_encode(double t) {
+  const double r = round_minifloat(std::fabs(t), 3, -6, 448.0);
+  int bits = 0;
+  if (r != 0.0) {
+    int e2;
+    std::frexp(r, &e2);
+    const int E = e2 - 1;
+    if (E < -6) {
+      bits = (int)std::ldexp(r, 9);  // subnormal: m 2^-9
+    } else {
+      bits = ((E + 7) << 3) | (int)((std::ldexp(r, -E) - 1.0) * 8.0);
+    }
+  }
+  return (std::signbit(t) ? 0x80 : 0) | bits;
+}
+
+double orc_e4m3_value(int code) {
+  const int e = (code >> 3) & 15, m = code & 7;
+  const double v = e == 0 ? std::ldexp((double)m, -9) : std::ldexp(1.0 + m / 8.0, e - 7);
+  return (code & 0x80) ? -v : v;
+}
+
+// One rotated binary32 row -> d/2 bytes of E2M1 codes and d/32 UE8M0 bytes.
+void orc_mxfp4_quantize_row(const float* y, int d, uint8_t* codes, uint8_t* scales) {
+  std::vector<int> c(d);
+  for (int g = 0; g < d / 32; ++g) {
+    float amax = 0.0f;
+    for (int i = 0; i < 32; ++i) amax = std::max(amax, std::fabs(y[32 * g + i]));
+    const int X = orc_mx_exponent(amax, 2);
+    scales[g] = (uint8_t)(X + 127);
+    for (int i = 0; i < 32; ++i) c[32 * g + i] = orc_e2m1_encode(std::ldexp((double)y[32 * g + i], -X));
+  }
+  for (int k = 0; k < d / 2; ++k) codes[k] = (uint8_t)(c[2 * k] | (c[2 * k + 1] << 4));
+}
+
+// The query side: a rotated binary32 row -> its MX E4M3 values (exact, in
+// double), blocks of 32 channels with their own shared exponent.
+void orc_mxfp8_row_values(const float* y, int d, double* out) {
+  for (int g = 0; g < d / 32; ++g) {
+    float amax = 0.0f;
+    for (int i = 0; i < 32; ++i) amax = std::max(amax, std::fabs(y[32 * g + i]));
+    const int X = orc_mx_exponent(amax, 8);
+    for (int i = 0; i < 32; ++i) {
+      const int code = orc_e4m3_encode(std::ldexp((double)y[32 * g + i], -X));
+      out[32 * g + i] = std::ldexp(orc_e4m3_value(code), X);
+    }
+  }
+}
+
+enum { ORC_FMT_INT4 = 0, ORC_FMT_MXFP4 = 1 };
+
+// Bytes of one row's parameters: (s16, m16) for INT4, d/32 scale bytes for
+// MX FP4 (a params row of the pool is 4 bytes at d <= 128).
+static inline int params_row_bytes(int fmt, int d) {
+  return fmt == ORC_FMT_MXFP4 ? (d / 32 < 4 ? 4 : d / 32) : 4;
+}
+
+// Dequantized row (double) of one stored row in either format.
+static void deq_row(int fmt, const uint8_t* codes_row, const uint8_t* params_row, int d,
+                    double* x) {
+  if (fmt == ORC_FMT_MXFP4) {
+    for (int k = 0; k < d / 2; ++k)
+      for (int n = 0; n < 2; ++n) {
+        const int i = 2 * k + n;
+        const int code = n ? codes_row[k] >> 4 : codes_row[k] & 0xf;
+        x[i] = std::ldexp(orc_e2m1_value(code), (int)params_row[i / 32] - 127);
+      }
+  } else {
+    uint16_t s16, m16;
+    std::memcpy(&s16, params_row, 2);
+    std::memcpy(&m16, params_row + 2, 2);
+    const double s = orc_half_to_double(s16), m = orc_half_to_double(m16);
+    for (int k = 0; k < d / 2; ++k) {
+      x[2 * k] = (double)(codes_row[k] & 0xf) * s + m;
+      x[2 * k + 1] = (double)(codes_row[k] >> 4) * s + m;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Rotary position embedding, optionally applied to each key row and to the
 // query in front of the block rotation (the step before the method's path in
 // a decode step; the pages do not describe it, so this is a reading).
@@ -416,8 +552,8 @@ void orc_quantize_append(int d, int H, int P, int NP, int rot_kind, int rot_bloc
                          int64_t tok_stride, const int32_t* token_seq,
                          const int32_t* token_pos, int num_seqs,
                          const int32_t* block_table, int bt_stride, uint8_t* k_codes,
-                         uint16_t* k_params, uint8_t* v_codes, uint16_t* v_params,
-                         const float* rope, int rope_max_pos, int32_t* err) {
+                         void* k_params, uint8_t* v_codes, void* v_params,
+                         const float* rope, int rope_max_pos, int fmt, int32_t* err) {
   // Tokens are independent (each writes only its own slot), so they are
   // spread over threads; the arithmetic of every row is unchanged.
   int32_t flags = 0;
@@ -436,17 +572,22 @@ void orc_quantize_append(int d, int H, int P, int NP, int rot_kind, int rot_bloc
     for (int kv = 0; kv < 2; ++kv) {
       const uint16_t* src = kv == 0 ? k : v;
       uint8_t* codes = kv == 0 ? k_codes : v_codes;
-      uint16_t* params = kv == 0 ? k_params : v_params;
+      uint8_t* params = static_cast<uint8_t*>(kv == 0 ? k_params : v_params);
       for (int h = 0; h < H; ++h) {
         const uint16_t* x = src + (int64_t)t * tok_stride + (int64_t)h * d;
         for (int i = 0; i < d; ++i) row[i] = orc_half_to_float(x[i]);
         if (kv == 0 && rope != nullptr) orc_rope_row_f32(row.data(), d, rope + (int64_t)pos * d);
         orc_rotate_f32(row.data(), d, rot_kind, rot_block, quat);
         const int64_t r = ((int64_t)page * H + h) * P + slot;
-        uint16_t s16, m16;
-        orc_quantize_row(row.data(), d, codes + r * (d / 2), &s16, &m16);
-        params[2 * r] = s16;
-        params[2 * r + 1] = m16;
+        uint8_t* prow = params + r * params_row_bytes(fmt, d);
+        if (fmt == ORC_FMT_MXFP4) {
+          orc_mxfp4_quantize_row(row.data(), d, codes + r * (d / 2), prow);
+        } else {
+          uint16_t s16, m16;
+          orc_quantize_row(row.data(), d, codes + r * (d / 2), &s16, &m16);
+          std::memcpy(prow, &s16, 2);
+          std::memcpy(prow + 2, &m16, 2);
+        }
       }
     }
   }
@@ -571,11 +712,11 @@ static inline double deq(int c, uint16_t s16, uint16_t m16) {
 void orc_dequantize_pages(int d, int H, int P, int NP, int rot_kind, int rot_block,
                           const float* quat, int S, const int32_t* seq_lens,
                           int max_seq_len, const int32_t* block_table, int bt_stride,
-                          const uint8_t* codes, const uint16_t* params, int unrotate,
-                          int out_fp32, void* out, int32_t* err) {
+                          const uint8_t* codes, const void* params, int unrotate,
+                          int out_fp32, void* out, int fmt, int32_t* err) {
   int32_t flags = 0;
-  std::vector<int> c(d);
   std::vector<double> x(d);
+  const uint8_t* pb = static_cast<const uint8_t*>(params);
   for (int s = 0; s < S; ++s) {
     int L = seq_lens[s];
     if (L < 0 || L > max_seq_len || (L + P - 1) / P > bt_stride) { flags |= ORC_ERR_LEN; continue; }
@@ -584,8 +725,7 @@ void orc_dequantize_pages(int d, int H, int P, int NP, int rot_kind, int rot_blo
       if (page < 0 || page >= NP) { flags |= ORC_ERR_PAGE; continue; }
       for (int h = 0; h < H; ++h) {
         const int64_t r = ((int64_t)page * H + h) * P + j % P;
-        orc_unpack_row(codes + r * (d / 2), d, c.data());
-        for (int i = 0; i < d; ++i) x[i] = deq(c[i], params[2 * r], params[2 * r + 1]);
+        deq_row(fmt, codes + r * (d / 2), pb + r * params_row_bytes(fmt, d), d, x.data());
         if (unrotate) orc_unrotate_f64(x.data(), d, rot_kind, rot_block, quat);
         const int64_t o = (((int64_t)s * max_seq_len + j) * H + h) * d;
         if (out_fp32) {
@@ -625,9 +765,13 @@ void orc_paged_decode_attn(int d, int H, int P, int NP, int rot_kind, int rot_bl
                            const float* quat, int S, int Hq, const uint16_t* q,
                            const int32_t* seq_lens, int max_seq_len,
                            const int32_t* block_table, int bt_stride, double sm_scale,
-                           const uint8_t* k_codes, const uint16_t* k_params,
-                           const uint8_t* v_codes, const uint16_t* v_params,
-                           const float* rope, int rope_max_pos, double* out, int32_t* err) {
+                           const uint8_t* k_codes, const void* k_params,
+                           const uint8_t* v_codes, const void* v_params,
+                           const float* rope, int rope_max_pos, int fmt, double* out,
+                           int32_t* err) {
+  const uint8_t* kpb = static_cast<const uint8_t*>(k_params);
+  const uint8_t* vpb = static_cast<const uint8_t*>(v_params);
+  const int PB = params_row_bytes(fmt, d);
   const int G = Hq / H;
   int32_t flags = 0;
 #pragma omp parallel for schedule(dynamic) reduction(| : flags)
@@ -638,11 +782,20 @@ void orc_paged_decode_attn(int d, int H, int P, int NP, int rot_kind, int rot_bl
     const int L = seq_lens[s];
     if (L < 0 || L > max_seq_len || (L + P - 1) / P > bt_stride) { flags |= ORC_ERR_LEN; continue; }
     if (rope != nullptr && L > rope_max_pos) { flags |= ORC_ERR_LEN; continue; }
-    std::vector<double> qh(d), kh(d), acc(d, 0.0);
-    std::vector<int> c(d);
-    for (int i = 0; i < d; ++i) qh[i] = orc_half_to_double(q[(int64_t)sg * d + i]);
-    if (rope != nullptr && L >= 1) rope_row_f64(qh.data(), d, rope + (int64_t)(L - 1) * d);
-    orc_rotate_f64(qh.data(), d, rot_kind, rot_block, quat);
+    std::vector<double> qh(d), kh(d), vh(d), acc(d, 0.0);
+    if (fmt == ORC_FMT_MXFP4) {
+      // the query as the MX FP4 path takes it: turned and rotated in binary32
+      // (the quantize path's arithmetic), then MX E4M3 values
+      std::vector<float> qf(d);
+      for (int i = 0; i < d; ++i) qf[i] = orc_half_to_float(q[(int64_t)sg * d + i]);
+      if (rope != nullptr && L >= 1) orc_rope_row_f32(qf.data(), d, rope + (int64_t)(L - 1) * d);
+      orc_rotate_f32(qf.data(), d, rot_kind, rot_block, quat);
+      orc_mxfp8_row_values(qf.data(), d, qh.data());
+    } else {
+      for (int i = 0; i < d; ++i) qh[i] = orc_half_to_double(q[(int64_t)sg * d + i]);
+      if (rope != nullptr && L >= 1) rope_row_f64(qh.data(), d, rope + (int64_t)(L - 1) * d);
+      orc_rotate_f64(qh.data(), d, rot_kind, rot_block, quat);
+    }
     std::vector<double> z;
     std::vector<int64_t> rows;
     z.reserve(L);
@@ -651,9 +804,9 @@ void orc_paged_decode_attn(int d, int H, int P, int NP, int rot_kind, int rot_bl
       const int page = block_table[(int64_t)s * bt_stride + j / P];
       if (page < 0 || page >= NP) { flags |= ORC_ERR_PAGE; continue; }
       const int64_t r = ((int64_t)page * H + h) * P + j % P;
-      orc_unpack_row(k_codes + r * (d / 2), d, c.data());
+      deq_row(fmt, k_codes + r * (d / 2), kpb + r * PB, d, kh.data());
       double dot = 0.0;
-      for (int i = 0; i < d; ++i) dot += qh[i] * deq(c[i], k_params[2 * r], k_params[2 * r + 1]);
+      for (int i = 0; i < d; ++i) dot += qh[i] * kh[i];
       z.push_back(sm_scale * dot);
       rows.push_back(r);
     }
@@ -663,9 +816,9 @@ void orc_paged_decode_attn(int d, int H, int P, int NP, int rot_kind, int rot_bl
     for (size_t j = 0; j < z.size(); ++j) { z[j] = std::exp(z[j] - zmax); denom += z[j]; }
     for (size_t j = 0; j < z.size(); ++j) {
       const int64_t r = rows[j];
-      orc_unpack_row(v_codes + r * (d / 2), d, c.data());
+      deq_row(fmt, v_codes + r * (d / 2), vpb + r * PB, d, vh.data());
       const double p = z[j] / denom;
-      for (int i = 0; i < d; ++i) acc[i] += p * deq(c[i], v_params[2 * r], v_params[2 * r + 1]);
+      for (int i = 0; i < d; ++i) acc[i] += p * vh[i];
     }
     orc_unrotate_f64(acc.data(), d, rot_kind, rot_block, quat);
     for (int i = 0; i < d; ++i) o[i] = acc[i];
