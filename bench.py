@@ -65,7 +65,7 @@ def parse():
                     help="print one JSON line with the baseline comparisons (long-context INT4 with "
                          "and without rotation vs the binary16 cache; prefill append per Hadamard "
                          "block with reconstruction MSE) and exit")
-    ap.add_argument("--profile-case", choices=["append", "decode"], default=None,
+    ap.add_argument("--profile-case", choices=["append", "decode", "decode-mx"], default=None,
                     help="run a short fixed case for an ncu capture (4 launches) and exit")
     ap.add_argument("--profile-block", type=int, default=128,
                     help="Hadamard block size of the append profile case (0: no rotation)")
@@ -505,7 +505,8 @@ def profile_case(which, block=128, workload="llama8b"):
     append = 4 bulk appends of one prefill layer (65536 tokens, Hadamard block
     `block`, 268 MB in, 71 MB out); decode = 4 decode calls of the
     Llama-3-8B-shaped layer (143 MB of INT4 pages) or of the long-context
-    70B-shaped one (285 MB) after filling its cache with one append."""
+    70B-shaped one (285 MB) after filling its cache with one append; decode-mx
+    = the same decode calls over the microscaled FP4 cache."""
     from bit_rotated_kv_block_b200 import kvq, workloads
     torch.cuda.set_device(0)
     dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
@@ -514,7 +515,8 @@ def profile_case(which, block=128, workload="llama8b"):
     else:
         w = workloads.long70b() if workload == "long70b" else workloads.llama8b()
     k, v, ts, tp = w.prefill_tokens()
-    c = kvq.Cache(w.d, w.H, w.P, w.NP, w.rot_kind, w.rot_block)
+    fmt = kvq.FMT_MXFP4 if which == "decode-mx" else kvq.FMT_INT4
+    c = kvq.Cache(w.d, w.H, w.P, w.NP, w.rot_kind, w.rot_block, fmt=fmt)
     kc, kp = c.new_pools(fill=0)
     vc, vp = c.new_pools(fill=0)
     K, V, TS, TP, BT = dev(k), dev(v), dev(ts), dev(tp), dev(w.block_table)
@@ -599,7 +601,11 @@ def workload_records(device, seed=0):
       of the INT4 cache (GPU dequantization, un-rotated, against the input);
     * the ragged head_dim-256 workload (128 sequences, lengths 512-16384):
       one fused decode step (append + attention) with Hadamard b 256 and with
-      the quaternion rotation.
+      the quaternion rotation;
+    * the microscaled FP4 format (E2M1 codes, UE8M0 block scales, decode QK
+      on the block-scaled tensor-core MMA) against INT4 on the Llama-shaped
+      layer: bulk append, fused decode step, reconstruction MSE; and on the
+      long-context decode.
     """
     from bit_rotated_kv_block_b200 import kvq, workloads
     dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(device)
@@ -617,11 +623,13 @@ def workload_records(device, seed=0):
     out = torch.empty((w.S, w.Hq, w.d), dtype=torch.float32, device=device)
     n_th = int(w.seq_lens.sum()) * w.H
     rec = {"workload": "8 seqs x 32768 tokens, 8 KV heads, 64 q heads, d 128, page 32"}
-    for rot, blk, name in ((workloads.ROT_HADAMARD, 128, "int4_hadamard128"),
-                           (workloads.ROT_NONE, 0, "int4_no_rotation")):
+    for rot, blk, name, fmt in ((workloads.ROT_HADAMARD, 128, "int4_hadamard128", kvq.FMT_INT4),
+                                (workloads.ROT_NONE, 0, "int4_no_rotation", kvq.FMT_INT4),
+                                (workloads.ROT_HADAMARD, 128, "mxfp4_hadamard128",
+                                 kvq.FMT_MXFP4)):
         reps = []
         for _ in range(2):
-            c = kvq.Cache(w.d, w.H, w.P, w.NP, rot, blk, device=device)
+            c = kvq.Cache(w.d, w.H, w.P, w.NP, rot, blk, device=device, fmt=fmt)
             kc, kp = c.new_pools(device=device, fill=0)
             vc, vp = c.new_pools(device=device, fill=0)
             kvq.quantize_append(c, K, V, TS, TP, BT, kc, kp, vc, vp)
@@ -725,6 +733,47 @@ def workload_records(device, seed=0):
         del kc, kp, vc, vp, ws
         torch.cuda.empty_cache()
     res["ragged256_step"] = rec
+
+    # ---- the microscaled FP4 format on the Llama-shaped layer: bulk append,
+    # fused decode step, and the reconstruction MSE against INT4's
+    w = workloads.llama8b(seed=seed)
+    ts, tp = _all_tokens(w)
+    K, V = _device_kv(w, len(ts), gen, device)
+    TS, TP, BT = dev(ts), dev(tp), dev(w.block_table)
+    rec = {"workload": "32 seqs x 4096 tokens + 1, 8 KV heads, 32 q heads, d 128, page 16, "
+                       "Hadamard b 64"}
+    Lc = int(w.seq_lens[0])
+    lens_c = dev(np.full(w.S, Lc, np.int32))
+    for fmt, name in ((kvq.FMT_INT4, "int4"), (kvq.FMT_MXFP4, "mxfp4")):
+        c = kvq.Cache(w.d, w.H, w.P, w.NP, w.rot_kind, w.rot_block, device=device, fmt=fmt)
+        kc, kp = c.new_pools(device=device, fill=0)
+        vc, vp = c.new_pools(device=device, fill=0)
+        t = _device_time_us(lambda i: kvq.quantize_append(c, K, V, TS, TP, BT, kc, kp, vc, vp),
+                            n=10)
+        r = {"append": _rate(len(ts) * w.H * APPEND_BYTES_PER_TOKEN_HEAD, t, peak)}
+        mse = 0.0
+        for codes, params, src in ((kc, kp, K), (vc, vp, V)):
+            xh = kvq.dequantize_pages(c, lens_c, Lc, BT, codes, params, unrotate=True)
+            x = src.view(w.S, Lc, w.H, w.d).double()
+            mse += float(((xh.double() - x) ** 2).mean()) / 2
+            del xh, x
+        r["mse"] = mse
+        kn = torch.randn((w.S, w.H, w.d), generator=gen, device=device).half()
+        vn = torch.randn((w.S, w.H, w.d), generator=gen, device=device).half()
+        lens_np = (w.seq_lens + 1).astype(np.int32)
+        lens, L = dev(lens_np), int(lens_np.max())
+        q = dev(w.queries())
+        out = torch.empty((w.S, w.Hq, w.d), dtype=torch.float32, device=device)
+        ws = torch.zeros(kvq.decode_workspace_bytes(c, w.S, w.Hq, L), dtype=torch.uint8,
+                         device=device)
+        t = _device_time_us(lambda i: kvq.decode_step(c, q, kn, vn, lens, L, BT, kc, kp, vc, vp,
+                                                      out=out, workspace=ws))
+        r["step"] = _rate(int(lens_np.sum()) * w.H * BYTES_PER_TOKEN_HEAD, t, peak)
+        rec[name] = r
+        del kc, kp, vc, vp, ws
+        torch.cuda.empty_cache()
+    del K, V
+    res["mxfp4_llama8b"] = rec
     res["peak_gbs"] = peak
     res["nominal_gbs"] = NOMINAL_HBM_GBS
     return res

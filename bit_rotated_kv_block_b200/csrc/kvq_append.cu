@@ -79,7 +79,8 @@ __host__ __device__ constexpr int append_ctas_per_sm(int E) { return E == 64 ? 2
 // randomised-sign Hadamard (channels flipped before the butterflies).
 // PRE: the kernel turns rows (RoPE) or flips signs before the rotation; without
 // it the first butterfly stage is taken straight from binary16.
-template <int D, int ROT, int LGB, bool PRE>
+// MX: the microscaled FP4 format (kvq.h, KVQ_FMT_MXFP4) instead of INT4.
+template <int D, int ROT, int LGB, bool PRE, bool MX>
 __device__ __forceinline__ void quantize_row_part(const uint8_t* boxes, int box_stride,
                                                   int my_line, int my_part, const float* qtbl,
                                                   const float* cs, int64_t dst_cur,
@@ -129,6 +130,46 @@ __device__ __forceinline__ void quantize_row_part(const uint8_t* boxes, int box_
     quat_regs<E>(x, qtbl, my_part * E);
   } else if (ROT == KVQ_ROT_QUAT_MAT) {
     quat_mat_regs<E>(x, qtbl, my_part * E);  // the CTA's matrices
+  }
+
+  if constexpr (MX) {
+    // per block of 32 channels (all inside this thread): the shared
+    // exponent from the largest magnitude's exponent field, then E2M1 codes
+    // of x * 2^-X (exact scaling)
+    uint32_t packed[E / 8];
+    uint32_t sbytes = 0;
+#pragma unroll
+    for (int g = 0; g < E / 32; ++g) {
+      float amax = 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(x[32 * g + i]));
+      const int eb = (int)((__float_as_uint(amax) >> 23) & 0xFFu);
+      const uint32_t xb = eb > 2 ? (uint32_t)(eb - 2) : 0u;  // X + 127
+      const float inv = __uint_as_float((254u - xb) << 23);   // 2^-X
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t w = 0;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int i = 32 * g + 8 * c + 2 * q;
+          w |= e2m1x2(__fmul_rn(x[i], inv), __fmul_rn(x[i + 1], inv)) << (8 * q);
+        }
+        packed[4 * g + c] = w;
+      }
+      sbytes |= xb << (8 * g);
+    }
+    if (TPR == 2) {  // the row's second thread holds blocks E/32 .. 2E/32 - 1
+      const uint32_t other = __shfl_xor_sync(pair_mask, sbytes, 1);
+      if (my_part == 0) sbytes |= other << (8 * (E / 32));
+    }
+    if (dst_cur >= 0) {
+      uint4* dst = reinterpret_cast<uint4*>(codes + dst_cur * (D / 2) + my_part * (E / 2));
+#pragma unroll
+      for (int c = 0; c < E / 32; ++c)
+        dst[c] = make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+      if (my_part == 0) params[dst_cur] = sbytes;
+    }
+    return;
   }
 
   // row statistics
@@ -198,6 +239,7 @@ __device__ __forceinline__ void quantize_row_part(const uint8_t* boxes, int box_
 
 struct AppendArgs {
   int T, H, P, lg_page, NP, num_seqs, bt_stride, tok_per_tile, num_tiles;
+  int mx;  // the microscaled FP4 format (else INT4)
   int box_stride;  // bytes between TMA boxes in a tile buffer (multiple of 1024)
   const int32_t* token_seq;
   const int32_t* token_pos;
@@ -213,8 +255,9 @@ struct AppendArgs {
 };
 
 // D: head_dim, ROT: rotation kind, LGB: log2 of the Hadamard block, PRE: a
-// RoPE table or a sign table acts before the rotation.
-template <int D, int ROT, int LGB, bool PRE>
+// RoPE table or a sign table acts before the rotation, MX: the microscaled
+// FP4 format.
+template <int D, int ROT, int LGB, bool PRE, bool MX>
 __global__ void __launch_bounds__(append_threads(append_e(D, ROT, LGB)),
                                   append_ctas_per_sm(append_e(D, ROT, LGB)))
     append_kernel(const AppendArgs a, const __grid_constant__ CUtensorMap tmk,
@@ -354,7 +397,7 @@ __global__ void __launch_bounds__(append_threads(append_e(D, ROT, LGB)),
     if (active && tok < a.T) {
       const float* cs = (PRE && a.rope != nullptr && my_kv == 0 && dst_cur >= 0)
                             ? a.rope + (int64_t)pos_cur * D : nullptr;
-      quantize_row_part<D, ROT, LGB, PRE>(cur + my_kv * NH * a.box_stride, a.box_stride, my_line,
+      quantize_row_part<D, ROT, LGB, PRE, MX>(cur + my_kv * NH * a.box_stride, a.box_stride, my_line,
                                           my_part, rtbl, cs, dst_cur,
                                           my_kv ? a.v_codes : a.k_codes,
                                           my_kv ? a.v_params : a.k_params);
@@ -378,6 +421,7 @@ __global__ void __launch_bounds__(append_threads(append_e(D, ROT, LGB)),
 
 struct AppendRowsArgs {
   int T, H, P, lg_page, NP, num_seqs, bt_stride;
+  int mx;  // the microscaled FP4 format (else INT4)
   int64_t tok_stride;
   const __half* k;
   const __half* v;
@@ -426,7 +470,14 @@ __global__ void __launch_bounds__(kRowsWarps * kWarp) append_rows_kernel(const A
   row_load<D>(x, (kv ? a.v : a.k) + (int64_t)t * a.tok_stride + (int64_t)h * D + rl * CPL, active);
   if (a.rope != nullptr && kv == 0 && pos_ok) rope_regs<CPL>(x, a.rope + (int64_t)pos * D + rl * CPL);
   __half s16, m16;
-  const uint32_t packed = row_quantize<D, ROT, LGB>(x, rl, a.quat, s16, m16);
+  uint32_t pword = 0;
+  uint32_t packed;
+  if (a.mx) {
+    packed = row_quantize_mx<D, ROT, LGB>(x, rl, a.quat, pword);
+  } else {
+    packed = row_quantize<D, ROT, LGB>(x, rl, a.quat, s16, m16);
+    pword = (uint32_t)__half_as_ushort(s16) | ((uint32_t)__half_as_ushort(m16) << 16);
+  }
 
   if (!active || seq < 0) return;
   const bool lead = kv == 0 && h == 0 && rl == 0;
@@ -444,9 +495,7 @@ __global__ void __launch_bounds__(kRowsWarps * kWarp) append_rows_kernel(const A
   }
   const int64_t dst = (((int64_t)page * a.H + h) << a.lg_page) + (pos & ((1 << a.lg_page) - 1));
   row_store_codes<D>((kv ? a.v_codes : a.k_codes) + dst * (D / 2) + rl * (CPL / 2), packed);
-  if (rl == 0)
-    (kv ? a.v_params : a.k_params)[dst] =
-        (uint32_t)__half_as_ushort(s16) | ((uint32_t)__half_as_ushort(m16) << 16);
+  if (rl == 0) (kv ? a.v_params : a.k_params)[dst] = pword;
 }
 
 template <int D, int ROT, int LGB>
@@ -520,7 +569,13 @@ static cudaError_t launch_append(const AppendArgs& a, const CUtensorMap& tk, con
                                  int grid, cudaStream_t st) {
   const size_t smem = append_smem(D, ROT, a.box_stride);
   const bool pre = a.rope != nullptr || (ROT == KVQ_ROT_HADAMARD && a.quat != nullptr);
-  auto kern = pre ? append_kernel<D, ROT, LGB, true> : append_kernel<D, ROT, LGB, false>;
+  auto kern = pre ? append_kernel<D, ROT, LGB, true, false> : append_kernel<D, ROT, LGB, false, false>;
+  if (a.mx) {  // the microscaled FP4 format: head_dim 128 only
+    if constexpr (D == 128)
+      kern = pre ? append_kernel<D, ROT, LGB, true, true> : append_kernel<D, ROT, LGB, false, true>;
+    else
+      return cudaErrorInvalidValue;
+  }
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   e = launch_pdl(kern, grid, append_threads(append_e(D, ROT, LGB)), smem, st, a, tk, tv);
@@ -589,6 +644,7 @@ int append_launch(const kvq_cache_desc& d, int32_t T, const void* k, const void*
     r.k_codes = k_codes; r.v_codes = v_codes;
     r.k_params = static_cast<uint32_t*>(k_params); r.v_params = static_cast<uint32_t*>(v_params);
     r.quat = rot_table(d); r.rope = d.rope; r.rope_max_pos = d.rope_max_pos; r.err = err;
+    r.mx = d.format == KVQ_FMT_MXFP4;
     cudaError_t e;
     switch (D) {
       case 64: e = dispatch_rows<64>(r, rot_template(d), lgb, st); break;
@@ -626,6 +682,7 @@ int append_launch(const kvq_cache_desc& d, int32_t T, const void* k, const void*
   a.rope = d.rope;
   a.rope_max_pos = d.rope_max_pos;
   a.err = err;
+  a.mx = d.format == KVQ_FMT_MXFP4;
   CUtensorMap tk, tv;
   if (!encode_rows(&tk, k, D, a.H, T, tok_stride, a.H, tok) ||
       !encode_rows(&tv, v, D, a.H, T, tok_stride, a.H, tok))

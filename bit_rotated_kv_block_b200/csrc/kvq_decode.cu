@@ -183,46 +183,6 @@ struct DecCfg {
   static constexpr int STEP_B = (RAW_B + 2 * ROWB + 8 + 127) / 128 * 128;
   static constexpr int WARP_B = (NST * STAGE_B + STEP_B + 127) / 128 * 128;
 };
-// Rotation of a query row held as quarters: lane j of a group of four
-// consecutive lanes owns channels [j*QW, (j+1)*QW). Butterfly stages with
-// distance < QW run in registers, wider ones across the lanes (distance QW:
-// lane ^ 1, 2*QW: lane ^ 2); the lower-channel lane adds and the upper one
-// subtracts. All 32 lanes must call it. Binary32, not part of the bit-exact
-// quantize path. `tbl` is the rotation's table (quaternions or signs).
-template <int QW>
-__device__ __forceinline__ void rotate_quarter(float (&x)[QW], int j, int rot_kind, int lgb,
-                                               const float* tbl) {
-  if (rot_kind == KVQ_ROT_HADAMARD || rot_kind == KVQ_ROT_HADAMARD_SIGNED) {
-    if (rot_kind == KVQ_ROT_HADAMARD_SIGNED) sign_regs<QW>(x, tbl + j * QW);
-    constexpr int LQ = QW == 32 ? 5 : 6;
-    const int lin = lgb < LQ ? lgb : LQ;
-    switch (lin) {
-      case 4: fwht_regs<QW, 4>(x); break;
-      case 5: fwht_regs<QW, 5>(x); break;
-      default: fwht_regs<QW, (LQ > 5 ? 6 : 5)>(x); break;
-    }
-    for (int hs = QW; hs < (1 << lgb); hs <<= 1) {
-      const int m = hs / QW;  // 1 or 2: lane distance
-      const bool lower = (j & m) == 0;
-#pragma unroll
-      for (int i = 0; i < QW; ++i) {
-        const float o = __shfl_xor_sync(0xffffffffu, x[i], m);
-        x[i] = lower ? x[i] + o : o - x[i];
-      }
-    }
-    const float cb = hadamard_scale(lgb);
-#pragma unroll
-    for (int i = 0; i < QW; ++i) x[i] *= cb;
-  } else if (rot_kind == KVQ_ROT_QUAT) {
-    quat_regs<QW>(x, tbl, j * QW);
-  } else if (rot_kind == KVQ_ROT_QUAT_FAST) {
-    quat_fast_regs<QW>(x, tbl, j * QW);
-  } else if (rot_kind == KVQ_ROT_QUAT_MAT) {
-    quat_mat_fly_regs<QW>(x, tbl, j * QW);
-  }
-}
-
-
 // Online-softmax slack in base-2 logit units: a head's reference maximum M
 // moves only when a score exceeds it by more than this, so every weight
 // 2^(z - M) stays below 2^8 (binary16 weights and binary32 sums have room to
@@ -1007,6 +967,7 @@ static int resident_warps(int D, int P, int GP) {
 }
 
 DecodePlan decode_plan(const kvq_cache_desc& d, int32_t S, int32_t Hq, int32_t max_seq_len) {
+  if (d.format == KVQ_FMT_MXFP4) return decode_mx_plan(d, S, Hq, max_seq_len);
   DecodePlan pl{};
   const int P = d.page_size;
   pl.pages_max = (max_seq_len + P - 1) / P;
@@ -1056,6 +1017,10 @@ int decode_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, const void* q,
                   const void* k_params, const uint8_t* v_codes, const void* v_params,
                   float* out, void* workspace, size_t workspace_bytes, int32_t* err,
                   cudaStream_t st, const DecodeStepRows* step) {
+  if (d.format == KVQ_FMT_MXFP4)
+    return decode_mx_launch(d, S, Hq, q, seq_lens, max_seq_len, block_table, bt_stride, sm_scale,
+                            k_codes, k_params, v_codes, v_params, out, workspace,
+                            workspace_bytes, err, st, step);
   const int D = d.head_dim;
   const int G = Hq / d.num_kv_heads;
   const int GP = G <= 4 ? 4 : 8;
@@ -1088,12 +1053,20 @@ int decode_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, const void* q,
   cudaError_t e = launch_split_any(a, D, GP, st);
   if (e == cudaErrorInvalidValue) return KVQ_ERR_UNSUPPORTED;
   if (e != cudaSuccess) return KVQ_ERR_CUDA;
+  return decode_merge_launch(d, S, Hq, pl.splits, a.part, out, st);
+}
+
+int decode_merge_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, int splits,
+                        const float* part, float* out, cudaStream_t st) {
+  const int D = d.head_dim;
+  int lgb = 0;
+  while ((1 << lgb) < d.rot_block) ++lgb;
   MergeArgs mg;
-  mg.S = S; mg.Hq = Hq; mg.splits = pl.splits; mg.rot_kind = d.rot_kind; mg.lgb = lgb;
-  mg.quat = d.quat; mg.part = a.part; mg.out = out;
+  mg.S = S; mg.Hq = Hq; mg.splits = splits; mg.rot_kind = d.rot_kind; mg.lgb = lgb;
+  mg.quat = d.quat; mg.part = part; mg.out = out;
   const int mgrid = (S * Hq + kDecWarps - 1) / kDecWarps;
-  e = D == 128 ? launch_pdl(decode_merge_kernel<128>, mgrid, kDecWarps * kWarp, 0, st, mg)
-               : launch_pdl(decode_merge_kernel<256>, mgrid, kDecWarps * kWarp, 0, st, mg);
+  cudaError_t e = D == 128 ? launch_pdl(decode_merge_kernel<128>, mgrid, kDecWarps * kWarp, 0, st, mg)
+                           : launch_pdl(decode_merge_kernel<256>, mgrid, kDecWarps * kWarp, 0, st, mg);
   if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }

@@ -1,4 +1,5 @@
-// Dense export of cached rows: x = c * s16 + m16, optionally rotated back.
+// Dense export of cached rows: x = c * s16 + m16 (INT4) or x = e2m1(c) * 2^X
+// (microscaled FP4), optionally rotated back.
 //
 // The dequantization rule is the one of the token-wise asymmetric INT4 format
 // ("SAW-INT4: System-Aware 4-Bit KV-Cache Quantization for Real-World LLM
@@ -26,6 +27,7 @@ struct DequantArgs {
   const uint32_t* params;
   const float* quat;   // quaternion table (QUAT kinds)
   const float* signs;  // sign table of the randomised-sign Hadamard, or NULL
+  int mx;              // the microscaled FP4 format (else INT4)
   void* out;
   int32_t* err;
 };
@@ -58,15 +60,36 @@ __global__ void __launch_bounds__(128) dequant_kernel(const DequantArgs a, int u
   const float mn = __half2float(__ushort_as_half((unsigned short)(pr >> 16)));
   float x[E];
   const uint4* src = reinterpret_cast<const uint4*>(a.codes + prow * (D / 2) + part * (E / 2));
+  if (a.mx) {
+    // E2M1 value (exact in binary16) times 2^X of its 32-channel block:
+    // exact in binary32, subnormal results included (X = -127: 2^-127 is the
+    // binary32 bit pattern 0x00400000)
 #pragma unroll
-  for (int c = 0; c < E / 32; ++c) {
-    const uint4 u = src[c];
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    for (int c = 0; c < E / 32; ++c) {
+      const uint32_t xb = (pr >> (8 * ((part * E) / 32 + c))) & 0xFFu;
+      const float sx = __uint_as_float(xb ? xb << 23 : 0x00400000u);
+      const uint4 u = src[c];
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
+      for (int q = 0; q < 4; ++q)
 #pragma unroll
-      for (int n = 0; n < 8; ++n)
-        x[32 * c + 8 * q + n] = __fmaf_rn((float)((w[q] >> (4 * n)) & 0xfu), sc, mn);
+        for (int n = 0; n < 4; ++n) {
+          const float2 f = __half22float2(u32_as_h2(e2m1x2_to_h2((w[q] >> (8 * n)) & 0xFFu)));
+          x[32 * c + 8 * q + 2 * n] = __fmul_rn(f.x, sx);
+          x[32 * c + 8 * q + 2 * n + 1] = __fmul_rn(f.y, sx);
+        }
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < E / 32; ++c) {
+      const uint4 u = src[c];
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int n = 0; n < 8; ++n)
+          x[32 * c + 8 * q + n] = __fmaf_rn((float)((w[q] >> (4 * n)) & 0xfu), sc, mn);
+    }
   }
   if (unrotate) {
     const unsigned pair_mask = 3u << ((threadIdx.x % kWarp) & ~1);
@@ -134,6 +157,7 @@ int dequant_launch(const kvq_cache_desc& d, int32_t S, const int32_t* seq_lens,
   a.bt_stride = bt_stride; a.seq_lens = seq_lens; a.block_table = block_table;
   a.codes = codes; a.params = static_cast<const uint32_t*>(params); a.quat = d.quat;
   a.signs = d.rot_kind == KVQ_ROT_HADAMARD_SIGNED ? d.quat : nullptr;
+  a.mx = d.format == KVQ_FMT_MXFP4;
   a.out = out; a.err = err;
   int lgb = 0;
   while ((1 << lgb) < d.rot_block) ++lgb;

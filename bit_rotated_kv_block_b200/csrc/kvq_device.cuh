@@ -118,6 +118,11 @@ __device__ __forceinline__ void cp_async8(void* smem_dst, const void* gmem_src) 
                "l"(gmem_src)
                : "memory");
 }
+__device__ __forceinline__ void cp_async4(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)),
+               "l"(gmem_src)
+               : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
@@ -244,6 +249,43 @@ __device__ __forceinline__ uint32_t nib_c8(uint32_t z, uint32_t mask, int high) 
   asm("lop3.b32 %0, %1, %2, %3, 0xea;" : "=r"(t) : "r"(z), "r"(mask), "r"(0x64006400u));
   return high ? h2_as_u32(__hfma2(u32_as_h2(t), u32_as_h2(0x2C002C00u), u32_as_h2(0xD480D480u)))
               : h2_as_u32(__hsub2(u32_as_h2(t), u32_as_h2(0x64086408u)));
+}
+
+// ---------------------------------------------------------------------------
+// Microscaling (MX) element conversions with the hardware's converters:
+// round to nearest, ties to even, saturating at the largest finite value.
+// The sign of each input is OR-ed into its code so that a negative value
+// that rounds to zero is -0 whatever the converter does with it.
+// ---------------------------------------------------------------------------
+
+// Two binary32 values -> one byte of E2M1 codes, `lo` in bits 0-3.
+__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
+      "cvt.u32.u8 %0, t;\n\t}"
+      : "=r"(r)
+      : "f"(hi), "f"(lo));
+  return (r & 0xFFu) | ((__float_as_uint(lo) >> 31) << 3) | ((__float_as_uint(hi) >> 31) << 7);
+}
+
+// Two binary32 values -> two E4M3 bytes, `lo` in bits 0-7.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return (uint32_t)r | ((__float_as_uint(lo) >> 31) << 7) | ((__float_as_uint(hi) >> 31) << 15);
+}
+
+// One byte of two E2M1 codes (bits 0-3 and 4-7) -> the half2 of their values
+// (bits 0-3 in the low half); exact.
+__device__ __forceinline__ uint32_t e2m1x2_to_h2(uint32_t byte) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\t"
+      "cvt.u8.u32 t, %1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+      : "=r"(r)
+      : "r"(byte));
+  return r;
 }
 
 __device__ __forceinline__ float fast_exp2(float x) {

@@ -66,6 +66,21 @@ int decode_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, const void* q,
                   float* out, void* workspace, size_t workspace_bytes, int32_t* err,
                   cudaStream_t st, const DecodeStepRows* step = nullptr);
 
+// The merge kernel over split partial results [S][Hq][splits][d + 4] (the
+// running sums, then the base-2 maximum and total weight), rotated back.
+int decode_merge_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, int splits,
+                        const float* part, float* out, cudaStream_t st);
+
+// Decode attention over the microscaled FP4 cache (QK on the block-scaled
+// tensor-core MMA); plan (pages_per_split counts 128-token tiles) and launch.
+DecodePlan decode_mx_plan(const kvq_cache_desc& d, int32_t S, int32_t Hq, int32_t max_seq_len);
+int decode_mx_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, const void* q,
+                     const int32_t* seq_lens, int32_t max_seq_len, const int32_t* block_table,
+                     int32_t bt_stride, float sm_scale, const uint8_t* k_codes,
+                     const void* k_params, const uint8_t* v_codes, const void* v_params,
+                     float* out, void* workspace, size_t workspace_bytes, int32_t* err,
+                     cudaStream_t st, const DecodeStepRows* step);
+
 // Baseline decode attention over a binary16 paged cache.
 DecodePlan decode_fp16_plan(const kvq_cache_desc& d, int32_t S, int32_t Hq, int32_t max_seq_len);
 int decode_fp16_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, const void* q,

@@ -250,4 +250,43 @@ __device__ __forceinline__ void rope_regs(float (&x)[E], const float* cs) {
   }
 }
 
+// Rotation of a query row held as quarters: lane j of a group of four
+// consecutive lanes owns channels [j*QW, (j+1)*QW). Butterfly stages with
+// distance < QW run in registers, wider ones across the lanes (distance QW:
+// lane ^ 1, 2*QW: lane ^ 2); the lower-channel lane adds and the upper one
+// subtracts. All 32 lanes must call it. Binary32, not part of the bit-exact
+// quantize path. `tbl` is the rotation's table (quaternions or signs).
+template <int QW>
+__device__ __forceinline__ void rotate_quarter(float (&x)[QW], int j, int rot_kind, int lgb,
+                                               const float* tbl) {
+  if (rot_kind == KVQ_ROT_HADAMARD || rot_kind == KVQ_ROT_HADAMARD_SIGNED) {
+    if (rot_kind == KVQ_ROT_HADAMARD_SIGNED) sign_regs<QW>(x, tbl + j * QW);
+    constexpr int LQ = QW == 32 ? 5 : 6;
+    const int lin = lgb < LQ ? lgb : LQ;
+    switch (lin) {
+      case 4: fwht_regs<QW, 4>(x); break;
+      case 5: fwht_regs<QW, 5>(x); break;
+      default: fwht_regs<QW, (LQ > 5 ? 6 : 5)>(x); break;
+    }
+    for (int hs = QW; hs < (1 << lgb); hs <<= 1) {
+      const int m = hs / QW;  // 1 or 2: lane distance
+      const bool lower = (j & m) == 0;
+#pragma unroll
+      for (int i = 0; i < QW; ++i) {
+        const float o = __shfl_xor_sync(0xffffffffu, x[i], m);
+        x[i] = lower ? x[i] + o : o - x[i];
+      }
+    }
+    const float cb = hadamard_scale(lgb);
+#pragma unroll
+    for (int i = 0; i < QW; ++i) x[i] *= cb;
+  } else if (rot_kind == KVQ_ROT_QUAT) {
+    quat_regs<QW>(x, tbl, j * QW);
+  } else if (rot_kind == KVQ_ROT_QUAT_FAST) {
+    quat_fast_regs<QW>(x, tbl, j * QW);
+  } else if (rot_kind == KVQ_ROT_QUAT_MAT) {
+    quat_mat_fly_regs<QW>(x, tbl, j * QW);
+  }
+}
+
 }  // namespace kvq

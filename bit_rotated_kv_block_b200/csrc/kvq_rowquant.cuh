@@ -32,11 +32,11 @@ struct RowQuantShape {
 // sign table (HADAMARD with signs) or NULL. Every lane of the warp must call it (the
 // shuffles span the warp; rows never mix because lane distances stay below
 // LPR). Returns the lane's codes, channel i of the lane in bits 4i..4i+3.
+// The rotation alone (the first step of row_quantize and row_quantize_mx).
 template <int D, int ROT, int LGB>
-__device__ __forceinline__ uint32_t row_quantize(float (&x)[RowQuantShape<D>::CPL], int rl,
-                                                 const float* quat, __half& s16, __half& m16) {
+__device__ __forceinline__ void row_rotate(float (&x)[RowQuantShape<D>::CPL], int rl,
+                                           const float* quat) {
   constexpr int CPL = RowQuantShape<D>::CPL;
-  constexpr int LPR = RowQuantShape<D>::LPR;
   constexpr int B = 1 << LGB;
   if (ROT == KVQ_ROT_HADAMARD) {
     // randomised-sign Hadamard: `quat` is then the sign table (else NULL)
@@ -71,6 +71,14 @@ __device__ __forceinline__ uint32_t row_quantize(float (&x)[RowQuantShape<D>::CP
   } else if (ROT == KVQ_ROT_QUAT_MAT) {
     quat_mat_fly_regs<CPL>(x, quat, rl * CPL);
   }
+}
+
+template <int D, int ROT, int LGB>
+__device__ __forceinline__ uint32_t row_quantize(float (&x)[RowQuantShape<D>::CPL], int rl,
+                                                 const float* quat, __half& s16, __half& m16) {
+  constexpr int CPL = RowQuantShape<D>::CPL;
+  constexpr int LPR = RowQuantShape<D>::LPR;
+  row_rotate<D, ROT, LGB>(x, rl, quat);
 
   float mn = x[0], mx = x[0];
 #pragma unroll
@@ -101,6 +109,41 @@ __device__ __forceinline__ uint32_t row_quantize(float (&x)[RowQuantShape<D>::CP
       packed |= c << (4 * i);
     }
   }
+  return packed;
+}
+
+// The microscaled FP4 form of the same rotated row (kvq.h, KVQ_FMT_MXFP4):
+// per block of 32 channels (32 / CPL lanes) the maximum magnitude, the
+// shared exponent X = floor(log2 amax) - 2 clamped at -127 (its byte
+// X + 127 read off the binary32 exponent field), then each x * 2^-X (exact)
+// converted to E2M1. Returns the lane's codes as row_quantize does; `pword`
+// gets the row's params word (byte g = block g), valid in lane rl = 0.
+template <int D, int ROT, int LGB>
+__device__ __forceinline__ uint32_t row_quantize_mx(float (&x)[RowQuantShape<D>::CPL], int rl,
+                                                    const float* quat, uint32_t& pword) {
+  constexpr int CPL = RowQuantShape<D>::CPL;
+  constexpr int LPB = 32 / CPL;  // lanes per 32-channel block
+  static_assert(LPB >= 1 && 32 % CPL == 0, "a block spans whole lanes");
+  row_rotate<D, ROT, LGB>(x, rl, quat);
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < CPL; ++i) amax = fmaxf(amax, fabsf(x[i]));
+#pragma unroll
+  for (int m = 1; m < LPB; m <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, m));
+  const int eb = (int)((__float_as_uint(amax) >> 23) & 0xFFu);
+  const uint32_t xb = eb > 2 ? (uint32_t)(eb - 2) : 0u;  // X + 127
+  const float inv = __uint_as_float((254u - xb) << 23);   // 2^-X
+  uint32_t packed = 0;
+#pragma unroll
+  for (int i = 0; i < CPL; i += 2)
+    packed |= e2m1x2(__fmul_rn(x[i], inv), __fmul_rn(x[i + 1], inv)) << (4 * i);
+  // gather the blocks' bytes into the row's first lane
+  uint32_t w = xb;
+  constexpr int NB = D / 32;
+#pragma unroll
+  for (int g = 1; g < (NB < 4 ? NB : 4); ++g)
+    w |= __shfl_down_sync(0xffffffffu, xb, g * LPB) << (8 * g);
+  pword = w;
   return packed;
 }
 

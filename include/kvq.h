@@ -74,6 +74,26 @@ typedef enum {
                                   block instead of 32; another rounding)         */
 } kvq_rot_kind;
 
+/* Storage format of a rotated (token, head) row; both pools of a cache
+ * share it, with the same pool shapes (codes [NP][H][P][d/2] bytes, one
+ * 32-bit params word per row).
+ *  KVQ_FMT_INT4   token-wise asymmetric INT4 (SAW-INT4, Summary): codes
+ *                 c = nearest of (x - m16)/s16 in [0, 15]; params (s16, m16).
+ *  KVQ_FMT_MXFP4  microscaled FP4 (UltraQuant page, method section: FP4 KV
+ *                 tensors with UE8M0 group scales, FP8 queries, scaled
+ *                 matrix-core MMA), read as the OCP MX formats: each block of
+ *                 32 channels shares the scale 2^X, X = floor(log2 amax) - 2
+ *                 clamped to [-127, 127] (an all-zero block: -127), stored as
+ *                 the byte X + 127 (params byte g = block g); codes are E2M1
+ *                 (bit 3 sign, magnitude index into {0, 0.5, 1, 1.5, 2, 3, 4,
+ *                 6}) of x / 2^X, nearest with ties to even, saturating at 6,
+ *                 the sign kept (a negative value rounding to zero is -0).
+ *                 Decode quantizes the rotated query to MX E4M3 (X =
+ *                 floor(log2 amax) - 8 per 32 channels, nearest-even,
+ *                 saturating at 448, sign kept) and takes QK on the tensor
+ *                 cores' block-scaled MMA. head_dim 128 only. */
+typedef enum { KVQ_FMT_INT4 = 0, KVQ_FMT_MXFP4 = 1 } kvq_format;
+
 /* Bits OR-ed into *err_flags by the kernels. */
 #define KVQ_ERRF_PAGE 1 /* block-table entry outside [0, num_pages): page skipped */
 #define KVQ_ERRF_POS 2  /* position < 0 or position/page_size >= bt_stride       */
@@ -119,7 +139,9 @@ typedef enum {
  *               rows need not be turned by a separate kernel.
  *  rope_max_pos rows of the rope table (>= 1 when rope is set); a position at
  *               or past it is invalid (KVQ_ERRF_POS in an append, the row is
- *               skipped; KVQ_ERRF_LEN in a decode, the output is zero). */
+ *               skipped; KVQ_ERRF_LEN in a decode, the output is zero).
+ *  format       a kvq_format: how a rotated row is stored (0, the token-wise
+ *               INT4 of the pages, for a zero-initialised descriptor). */
 typedef struct {
   int32_t head_dim;
   int32_t num_kv_heads;
@@ -130,6 +152,7 @@ typedef struct {
   const float* quat;
   const float* rope;
   int32_t rope_max_pos;
+  int32_t format;
 } kvq_cache_desc;
 
 /*

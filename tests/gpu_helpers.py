@@ -16,9 +16,11 @@ class Pair:
     """One paged cache built twice: GPU pools through libkvq, host pools through
     the oracle, both started from the same sentinel bytes."""
 
-    def __init__(self, d, H, P, NP, rot_kind, rot_block=0, quat=None, fill=0xAA):
-        self.gpu = kvq.Cache(d, H, P, NP, rot_kind, rot_block, quat)
-        self.orc = oracle.Cache(d, H, P, NP, rot_kind, rot_block, quat)
+    def __init__(self, d, H, P, NP, rot_kind, rot_block=0, quat=None, fill=0xAA,
+                 fmt=kvq.FMT_INT4):
+        self.fmt = fmt
+        self.gpu = kvq.Cache(d, H, P, NP, rot_kind, rot_block, quat, fmt=fmt)
+        self.orc = oracle.Cache(d, H, P, NP, rot_kind, rot_block, quat, fmt=fmt)
         self.kc, self.kp = self.gpu.new_pools(fill=fill)
         self.vc, self.vp = self.gpu.new_pools(fill=fill)
         self.okc, self.okp = self.orc.alloc_pools(fill)
@@ -26,8 +28,14 @@ class Pair:
         self.err = torch.zeros(1, dtype=torch.int32, device="cuda")
 
     @classmethod
-    def for_workload(cls, w, fill=0xAA):
-        return cls(w.d, w.H, w.P, w.NP, w.rot_kind, w.rot_block, w.quat, fill)
+    def for_workload(cls, w, fill=0xAA, fmt=kvq.FMT_INT4):
+        return cls(w.d, w.H, w.P, w.NP, w.rot_kind, w.rot_block, w.quat, fill, fmt)
+
+    def okp_pool(self):
+        """The oracle's K params pool as its append writes it."""
+        if self.fmt == kvq.FMT_MXFP4:
+            return self.okp
+        return self.okp.reshape(self.orc.NP, self.orc.H, self.orc.P, 2)
 
     def append(self, k, v, token_seq, token_pos, block_table, oracle_too=True, tok_stride=None,
                k_dev=None, v_dev=None):
@@ -43,8 +51,8 @@ class Pair:
         if oracle_too:
             oerr = oracle.quantize_append(self.orc, k.view(np.uint16), v.view(np.uint16),
                                           token_seq, token_pos, block_table, self.okc,
-                                          self.okp.reshape(self.orc.NP, self.orc.H, self.orc.P, 2),
-                                          self.ovc, self.ovp, tok_stride=tok_stride)
+                                          self.okp_pool(), self.ovc, self.ovp,
+                                          tok_stride=tok_stride)
         torch.cuda.synchronize()
         return int(self.err.item()), oerr
 
@@ -56,7 +64,7 @@ class Pair:
                 bad = np.argwhere(gh != o)
                 raise AssertionError(f"code bytes differ at {len(bad)} places, first {bad[:5]}")
         for g, o in ((self.kp, self.okp), (self.vp, self.ovp)):
-            gh = g.cpu().numpy().view(np.uint16).reshape(o.shape)
+            gh = g.cpu().numpy().view(o.dtype).reshape(o.shape)
             if not np.array_equal(gh, o):
                 bad = np.argwhere(gh != o)
                 raise AssertionError(f"param words differ at {len(bad)} places, first {bad[:5]}")
@@ -76,9 +84,9 @@ class Pair:
         return out.cpu().numpy().astype(np.float64), int(self.err.item())
 
 
-def fill_workload(w, seqs=None, layer=0, oracle_too=True, fill=0xAA):
+def fill_workload(w, seqs=None, layer=0, oracle_too=True, fill=0xAA, fmt=kvq.FMT_INT4):
     """Pair cache holding the workload's cached tokens of the given sequences."""
-    p = Pair.for_workload(w, fill)
+    p = Pair.for_workload(w, fill, fmt)
     k, v, ts, tp = w.prefill_tokens(seqs, layer)
     e, oe = p.append(k, v, ts, tp, w.block_table, oracle_too=oracle_too)
     assert e == 0 and oe == 0
@@ -101,6 +109,6 @@ def fused_step_vs_oracle(p, k_new, v_new, lens, table, q, sm_scale):
                           err=p.err)
     torch.cuda.synchronize()
     oe = oracle.quantize_append(p.orc, k_new.view(np.uint16), v_new.view(np.uint16), ts, tp, table,
-                                p.okc, p.okp.reshape(p.orc.NP, p.orc.H, p.orc.P, 2), p.ovc, p.ovp)
+                                p.okc, p.okp_pool(), p.ovc, p.ovp)
     ref, oe2 = p.oracle_attention(q, lens, L, table, sm_scale)
     return out.cpu().numpy().astype(np.float64), ref, int(p.err.item()), oe | oe2

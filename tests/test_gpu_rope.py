@@ -46,6 +46,9 @@ class RopePair:
         assert np.array_equal(self.vp.cpu().numpy().view(np.uint16).reshape(self.ovp.shape), self.ovp)
 
     # gpu_helpers.fused_step_vs_oracle reads these names
+    def okp_pool(self):
+        return self.okp
+
     def oracle_attention(self, q, lens, L, table, sm):
         return oracle.paged_decode_attn(self.orc, q.view(np.uint16), lens, L, table,
                                         float(np.float32(sm)), self.okc, self.okp, self.ovc,
