@@ -32,7 +32,7 @@ import numpy as np
 from . import build as _build
 
 ROT_NONE, ROT_HADAMARD, ROT_QUAT, ROT_QUAT_FAST, ROT_HADAMARD_SIGNED, ROT_QUAT_MAT = 0, 1, 2, 3, 4, 5
-FMT_INT4, FMT_MXFP4 = 0, 1
+FMT_INT4, FMT_MXFP4, FMT_INT2, FMT_INT3, FMT_LUT4 = 0, 1, 2, 3, 4
 RN, RD, RU = 0, 1, 2
 ERR_PAGE, ERR_POS, ERR_SEQ, ERR_LEN = 1, 2, 4, 8
 
@@ -63,12 +63,14 @@ def lib():
             "orc_fwht_unscaled": (None, [P, i32]),
             "orc_quantize_rows": (None, [P, i64, i32, P, P, P]),
             "orc_quantize_append": (None, [i32, i32, i32, i32, i32, i32, P, i32, P, P, i64,
-                                           P, P, i32, P, i32, P, P, P, P, P, i32, i32, P]),
+                                           P, P, i32, P, i32, P, P, P, P, P, i32, i32, P, P]),
             "orc_dequantize_pages": (None, [i32, i32, i32, i32, i32, i32, P, i32, P, i32, P,
-                                            i32, P, P, i32, i32, P, i32, P]),
+                                            i32, P, P, i32, i32, P, i32, P, P]),
             "orc_paged_decode_attn": (None, [i32, i32, i32, i32, i32, i32, P, i32, i32, P, P,
                                              i32, P, i32, dbl, P, P, P, P, P, i32, i32, P,
-                                             P]),
+                                             P, P]),
+            "orc_quantize_rows_fmt": (None, [P, i64, i32, i32, P, P, P, P]),
+            "orc_unpack_codes_rows": (None, [P, i64, i32, i32, P]),
             "orc_mx_exponent": (i32, [ctypes.c_float, i32]),
             "orc_e2m1_encode": (i32, [dbl]),
             "orc_e2m1_value": (dbl, [i32]),
@@ -254,6 +256,30 @@ def mxfp8_values(y):
     return out.reshape(y.shape)
 
 
+def quantize_rows_fmt(y, fmt, levels=None):
+    """Rotated binary32 rows [..., d] -> (packed codes uint8 [..., d*bits/8],
+    s16 bits, m16 bits) for FMT_INT2 / FMT_INT3 / FMT_INT4 / FMT_LUT4."""
+    y = _c(y, np.float32)
+    d = y.shape[-1]
+    rows = y.size // d
+    bits = {FMT_INT2: 2, FMT_INT3: 3}.get(fmt, 4)
+    codes = np.empty(y.shape[:-1] + (d * bits // 8,), np.uint8)
+    s16 = np.empty(y.shape[:-1], np.uint16)
+    m16 = np.empty(y.shape[:-1], np.uint16)
+    lv = None if levels is None else _c(levels, np.float32)
+    lib().orc_quantize_rows_fmt(_p(y), rows, d, int(fmt), _p(lv), _p(codes), _p(s16), _p(m16))
+    return codes, s16, m16
+
+
+def unpack_codes_bits(codes, d, bits):
+    """Packed rows [..., d*bits/8] -> integer codes int32 [..., d]."""
+    codes = _c(codes, np.uint8)
+    rows = codes.size // (d * bits // 8)
+    out = np.empty(codes.shape[:-1] + (d,), np.int32)
+    lib().orc_unpack_codes_rows(_p(codes), rows, d, bits, _p(out))
+    return out
+
+
 # --- quantizer ----------------------------------------------------------------
 
 def quantize_rows(y):
@@ -295,8 +321,12 @@ class Cache:
     FMT_INT4 (token-wise INT4, params (s16, m16)) or FMT_MXFP4 (E2M1 codes,
     one UE8M0 byte per 32 channels, a 4-byte params row)."""
 
-    def __init__(self, d, H, P, NP, rot_kind, rot_block=0, quat=None, rope=None, fmt=FMT_INT4):
+    def __init__(self, d, H, P, NP, rot_kind, rot_block=0, quat=None, rope=None, fmt=FMT_INT4,
+                 levels=None):
         self.fmt = int(fmt)
+        # the LUT4 format's 16 levels (float32, binary16-exact, on the 1/16 grid)
+        self.levels = None if levels is None else _c(levels, np.float32).reshape(16)
+        assert (self.levels is not None) == (self.fmt == FMT_LUT4)
         self.d, self.H, self.P, self.NP = int(d), int(H), int(P), int(NP)
         self.rot_kind, self.rot_block = int(rot_kind), int(rot_block)
         self.quat = _quat(quat)
@@ -304,8 +334,11 @@ class Cache:
         self.rope = None if rope is None else _c(rope, np.float32).reshape(-1, self.d)
         self.rope_max_pos = 0 if rope is None else self.rope.shape[0]
 
+    def code_row_bytes(self):
+        return self.d * {FMT_INT2: 2, FMT_INT3: 3}.get(self.fmt, 4) // 8
+
     def alloc_pools(self, fill=0):
-        codes = np.full((self.NP, self.H, self.P, self.d // 2), fill, np.uint8)
+        codes = np.full((self.NP, self.H, self.P, self.code_row_bytes()), fill, np.uint8)
         if self.fmt == FMT_MXFP4:
             params = np.full((self.NP, self.H, self.P, max(4, self.d // 32)), fill, np.uint8)
         else:
@@ -338,7 +371,7 @@ def quantize_append(cache, k, v, token_seq, token_pos, block_table, k_codes, k_p
                               cache.rot_block, _p(cache.quat), T, _p(k), _p(v), tok_stride,
                               _p(ts), _p(tp), num_seqs, _p(bt), bt.shape[1], _p(k_codes),
                               _p(k_params), _p(v_codes), _p(v_params), _p(cache.rope),
-                              cache.rope_max_pos, cache.fmt, _p(err))
+                              cache.rope_max_pos, cache.fmt, _p(cache.levels), _p(err))
     return int(err[0])
 
 
@@ -355,7 +388,8 @@ def dequantize_pages(cache, seq_lens, max_seq_len, block_table, codes, params, u
     lib().orc_dequantize_pages(cache.d, cache.H, cache.P, cache.NP, cache.rot_kind,
                                cache.rot_block, _p(cache.quat), S, _p(lens), max_seq_len, _p(bt),
                                bt.shape[1], _p(codes), _p(params), int(bool(unrotate)),
-                               int(bool(out_fp32)), _p(out), cache.fmt, _p(err))
+                               int(bool(out_fp32)), _p(out), cache.fmt, _p(cache.levels),
+                               _p(err))
     return out, int(err[0])
 
 
@@ -375,7 +409,7 @@ def paged_decode_attn(cache, q, seq_lens, max_seq_len, block_table, sm_scale, k_
                                 cache.rot_block, _p(cache.quat), S, Hq, _p(q), _p(lens),
                                 max_seq_len, _p(bt), bt.shape[1], float(sm_scale), _p(kc),
                                 _p(kp), _p(vc), _p(vp), _p(cache.rope), cache.rope_max_pos,
-                                cache.fmt, _p(out), _p(err))
+                                cache.fmt, _p(cache.levels), _p(out), _p(err))
     return out, int(err[0])
 
 

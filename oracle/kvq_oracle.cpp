@@ -326,8 +326,33 @@ static double rint_half_even(double t) {
   return (std::fmod(fl, 2.0) == 0.0) ? fl : fl + 1.0;
 }
 
-void orc_quantize_row(const float* y, int d, uint8_t* codes,
-                      uint16_t* s16_out, uint16_t* m16_out) {
+// Codes of `bits` bits (2, 3 or 4) are packed into a little-endian bit
+// stream: code i of the row occupies bits [i*bits, (i+1)*bits) of the row's
+// d*bits/8 bytes (for 4 bits: the even channel in the low nibble).
+static void pack_codes(const int* c, int d, int bits, uint8_t* out) {
+  const int nbytes = d * bits / 8;
+  for (int k = 0; k < nbytes; ++k) out[k] = 0;
+  for (int i = 0; i < d; ++i) {
+    const int bit = i * bits;
+    const unsigned v = (unsigned)c[i] << (bit % 8);
+    out[bit / 8] |= (uint8_t)(v & 0xFF);
+    if ((bit % 8) + bits > 8) out[bit / 8 + 1] |= (uint8_t)(v >> 8);
+  }
+}
+
+void orc_unpack_codes(const uint8_t* codes, int d, int bits, int* c) {
+  for (int i = 0; i < d; ++i) {
+    const int bit = i * bits;
+    unsigned v = codes[bit / 8];
+    if ((bit % 8) + bits > 8) v |= (unsigned)codes[bit / 8 + 1] << 8;
+    c[i] = (int)((v >> (bit % 8)) & ((1u << bits) - 1));
+  }
+}
+
+// The row statistics shared by the integer and table formats: the minimum
+// rounded down to binary16 (m16) and the scale (max - m16)/Q rounded up at
+// every step (s16); Q = 2^bits - 1, or 15 for the 16-level table.
+static void row_stats(const float* y, int d, int Q, uint16_t* s16_out, uint16_t* m16_out) {
   float mn = y[0], mx = y[0];
   for (int i = 1; i < d; ++i) {
     if (y[i] < mn) mn = y[i];
@@ -338,9 +363,21 @@ void orc_quantize_row(const float* y, int d, uint8_t* codes,
   const uint16_t m16 = orc_float_to_half(mn, ORC_RD);
   const float m = orc_half_to_float(m16);
   const float diff = orc_sub_ru(mx, m);
-  const float s32 = orc_div_ru(diff, 15.0f);
-  const uint16_t s16 = orc_float_to_half(s32, ORC_RU);
-  const float s = orc_half_to_float(s16);
+  const float s32 = orc_div_ru(diff, (float)Q);
+  *s16_out = orc_float_to_half(s32, ORC_RU);
+  *m16_out = m16;
+}
+
+// Token-wise asymmetric integer codes of `bits` bits (2, 3 or 4; the 2- and
+// 3-bit forms follow IsoQuant's bit widths {2, 3, 4}, page "IsoQuant:
+// Hardware-Aligned SO(4) Isoclinic Rotations for LLM KV Cache Compression",
+// Abstract): as the INT4 rule above with Q = 2^bits - 1 levels above zero.
+void orc_quantize_row_bits(const float* y, int d, int bits, uint8_t* codes,
+                           uint16_t* s16_out, uint16_t* m16_out) {
+  const int Q = (1 << bits) - 1;
+  row_stats(y, d, Q, s16_out, m16_out);
+  const float m = orc_half_to_float(*m16_out);
+  const float s = orc_half_to_float(*s16_out);
   std::vector<int> c(d, 0);
   if (s != 0.0f) {
     const float inv = 1.0f / s;
@@ -349,15 +386,44 @@ void orc_quantize_row(const float* y, int d, uint8_t* codes,
       const double prod = (double)t0 * (double)inv;  // exact: 24 x 24 bits
       double r = rint_half_even(prod);
       if (r < 0.0) r = 0.0;
-      if (r > 15.0) r = 15.0;
+      if (r > Q) r = Q;
       c[i] = (int)r;
     }
   }
-  // Two 4-bit codes per byte, the even channel in the low nibble.
-  for (int k = 0; k < d / 2; ++k)
-    codes[k] = (uint8_t)(c[2 * k] | (c[2 * k + 1] << 4));
-  *s16_out = s16;
-  *m16_out = m16;
+  pack_codes(c.data(), d, bits, codes);
+}
+
+void orc_quantize_row(const float* y, int d, uint8_t* codes,
+                      uint16_t* s16_out, uint16_t* m16_out) {
+  orc_quantize_row_bits(y, d, 4, codes, s16_out, m16_out);
+}
+
+// Calibrated 16-entry table in place of the uniform INT4 levels (UltraQuant
+// page, method section: the 16 centroids refitted on activations instead of
+// the theoretical Lloyd-Max ones). Reading: the table replaces the levels
+// 0..15 of u = (x - m16)/s16 with the row statistics of INT4 unchanged;
+// `levels` holds 16 non-decreasing binary16-exact values in [0, 15] on the
+// 1/16 grid; the code is the index of the level nearest to the exact
+// u* = RN(x - m16) * RN(1/s16), a tie going to the lower index (the count of
+// midpoints (t_k + t_k+1)/2 that u* exceeds); x^ = t[c] s16 + m16.
+void orc_quantize_row_lut(const float* y, int d, const float* levels, uint8_t* codes,
+                          uint16_t* s16_out, uint16_t* m16_out) {
+  row_stats(y, d, 15, s16_out, m16_out);
+  const float m = orc_half_to_float(*m16_out);
+  const float s = orc_half_to_float(*s16_out);
+  std::vector<int> c(d, 0);
+  if (s != 0.0f) {
+    const float inv = 1.0f / s;
+    for (int i = 0; i < d; ++i) {
+      const float t0 = y[i] - m;
+      const double u = (double)t0 * (double)inv;  // exact
+      int code = 0;
+      for (int k = 0; k < 15; ++k)
+        if (u > 0.5 * ((double)levels[k] + (double)levels[k + 1])) code = k + 1;
+      c[i] = code;
+    }
+  }
+  pack_codes(c.data(), d, 4, codes);
 }
 
 // Unpacks one row of codes (d/2 bytes) into d integers.
@@ -474,17 +540,25 @@ void orc_mxfp8_row_values(const float* y, int d, double* out) {
   }
 }
 
-enum { ORC_FMT_INT4 = 0, ORC_FMT_MXFP4 = 1 };
+// Storage formats (same numbering as the library's public enum, restated).
+enum { ORC_FMT_INT4 = 0, ORC_FMT_MXFP4 = 1, ORC_FMT_INT2 = 2, ORC_FMT_INT3 = 3,
+       ORC_FMT_LUT4 = 4 };
 
-// Bytes of one row's parameters: (s16, m16) for INT4, d/32 scale bytes for
-// MX FP4 (a params row of the pool is 4 bytes at d <= 128).
+// Bits per code and bytes of one row's codes and parameters: (s16, m16) for
+// the integer and table formats, d/32 scale bytes for MX FP4 (a params row of
+// the pool is 4 bytes at d <= 128).
+static inline int code_bits(int fmt) {
+  return fmt == ORC_FMT_INT2 ? 2 : (fmt == ORC_FMT_INT3 ? 3 : 4);
+}
+static inline int code_row_bytes(int fmt, int d) { return d * code_bits(fmt) / 8; }
 static inline int params_row_bytes(int fmt, int d) {
   return fmt == ORC_FMT_MXFP4 ? (d / 32 < 4 ? 4 : d / 32) : 4;
 }
 
-// Dequantized row (double) of one stored row in either format.
-static void deq_row(int fmt, const uint8_t* codes_row, const uint8_t* params_row, int d,
-                    double* x) {
+// Dequantized row (double) of one stored row in any format (`levels`: the
+// table of the LUT4 format).
+static void deq_row(int fmt, const float* levels, const uint8_t* codes_row,
+                    const uint8_t* params_row, int d, double* x) {
   if (fmt == ORC_FMT_MXFP4) {
     for (int k = 0; k < d / 2; ++k)
       for (int n = 0; n < 2; ++n) {
@@ -497,10 +571,10 @@ static void deq_row(int fmt, const uint8_t* codes_row, const uint8_t* params_row
     std::memcpy(&s16, params_row, 2);
     std::memcpy(&m16, params_row + 2, 2);
     const double s = orc_half_to_double(s16), m = orc_half_to_double(m16);
-    for (int k = 0; k < d / 2; ++k) {
-      x[2 * k] = (double)(codes_row[k] & 0xf) * s + m;
-      x[2 * k + 1] = (double)(codes_row[k] >> 4) * s + m;
-    }
+    std::vector<int> c(d);
+    orc_unpack_codes(codes_row, d, code_bits(fmt), c.data());
+    for (int i = 0; i < d; ++i)
+      x[i] = (fmt == ORC_FMT_LUT4 ? (double)levels[c[i]] : (double)c[i]) * s + m;
   }
 }
 
@@ -553,7 +627,8 @@ void orc_quantize_append(int d, int H, int P, int NP, int rot_kind, int rot_bloc
                          const int32_t* token_pos, int num_seqs,
                          const int32_t* block_table, int bt_stride, uint8_t* k_codes,
                          void* k_params, uint8_t* v_codes, void* v_params,
-                         const float* rope, int rope_max_pos, int fmt, int32_t* err) {
+                         const float* rope, int rope_max_pos, int fmt, const float* levels,
+                         int32_t* err) {
   // Tokens are independent (each writes only its own slot), so they are
   // spread over threads; the arithmetic of every row is unchanged.
   int32_t flags = 0;
@@ -580,11 +655,15 @@ void orc_quantize_append(int d, int H, int P, int NP, int rot_kind, int rot_bloc
         orc_rotate_f32(row.data(), d, rot_kind, rot_block, quat);
         const int64_t r = ((int64_t)page * H + h) * P + slot;
         uint8_t* prow = params + r * params_row_bytes(fmt, d);
+        uint8_t* crow = codes + r * code_row_bytes(fmt, d);
         if (fmt == ORC_FMT_MXFP4) {
-          orc_mxfp4_quantize_row(row.data(), d, codes + r * (d / 2), prow);
+          orc_mxfp4_quantize_row(row.data(), d, crow, prow);
         } else {
           uint16_t s16, m16;
-          orc_quantize_row(row.data(), d, codes + r * (d / 2), &s16, &m16);
+          if (fmt == ORC_FMT_LUT4)
+            orc_quantize_row_lut(row.data(), d, levels, crow, &s16, &m16);
+          else
+            orc_quantize_row_bits(row.data(), d, code_bits(fmt), crow, &s16, &m16);
           std::memcpy(prow, &s16, 2);
           std::memcpy(prow + 2, &m16, 2);
         }
@@ -713,7 +792,8 @@ void orc_dequantize_pages(int d, int H, int P, int NP, int rot_kind, int rot_blo
                           const float* quat, int S, const int32_t* seq_lens,
                           int max_seq_len, const int32_t* block_table, int bt_stride,
                           const uint8_t* codes, const void* params, int unrotate,
-                          int out_fp32, void* out, int fmt, int32_t* err) {
+                          int out_fp32, void* out, int fmt, const float* levels,
+                          int32_t* err) {
   int32_t flags = 0;
   std::vector<double> x(d);
   const uint8_t* pb = static_cast<const uint8_t*>(params);
@@ -725,7 +805,8 @@ void orc_dequantize_pages(int d, int H, int P, int NP, int rot_kind, int rot_blo
       if (page < 0 || page >= NP) { flags |= ORC_ERR_PAGE; continue; }
       for (int h = 0; h < H; ++h) {
         const int64_t r = ((int64_t)page * H + h) * P + j % P;
-        deq_row(fmt, codes + r * (d / 2), pb + r * params_row_bytes(fmt, d), d, x.data());
+        deq_row(fmt, levels, codes + r * code_row_bytes(fmt, d), pb + r * params_row_bytes(fmt, d),
+                d, x.data());
         if (unrotate) orc_unrotate_f64(x.data(), d, rot_kind, rot_block, quat);
         const int64_t o = (((int64_t)s * max_seq_len + j) * H + h) * d;
         if (out_fp32) {
@@ -767,11 +848,12 @@ void orc_paged_decode_attn(int d, int H, int P, int NP, int rot_kind, int rot_bl
                            const int32_t* block_table, int bt_stride, double sm_scale,
                            const uint8_t* k_codes, const void* k_params,
                            const uint8_t* v_codes, const void* v_params,
-                           const float* rope, int rope_max_pos, int fmt, double* out,
+                           const float* rope, int rope_max_pos, int fmt, const float* levels,
+                           double* out,
                            int32_t* err) {
   const uint8_t* kpb = static_cast<const uint8_t*>(k_params);
   const uint8_t* vpb = static_cast<const uint8_t*>(v_params);
-  const int PB = params_row_bytes(fmt, d);
+  const int PB = params_row_bytes(fmt, d), CB = code_row_bytes(fmt, d);
   const int G = Hq / H;
   int32_t flags = 0;
 #pragma omp parallel for schedule(dynamic) reduction(| : flags)
@@ -804,7 +886,7 @@ void orc_paged_decode_attn(int d, int H, int P, int NP, int rot_kind, int rot_bl
       const int page = block_table[(int64_t)s * bt_stride + j / P];
       if (page < 0 || page >= NP) { flags |= ORC_ERR_PAGE; continue; }
       const int64_t r = ((int64_t)page * H + h) * P + j % P;
-      deq_row(fmt, k_codes + r * (d / 2), kpb + r * PB, d, kh.data());
+      deq_row(fmt, levels, k_codes + r * CB, kpb + r * PB, d, kh.data());
       double dot = 0.0;
       for (int i = 0; i < d; ++i) dot += qh[i] * kh[i];
       z.push_back(sm_scale * dot);
@@ -816,7 +898,7 @@ void orc_paged_decode_attn(int d, int H, int P, int NP, int rot_kind, int rot_bl
     for (size_t j = 0; j < z.size(); ++j) { z[j] = std::exp(z[j] - zmax); denom += z[j]; }
     for (size_t j = 0; j < z.size(); ++j) {
       const int64_t r = rows[j];
-      deq_row(fmt, v_codes + r * (d / 2), vpb + r * PB, d, vh.data());
+      deq_row(fmt, levels, v_codes + r * CB, vpb + r * PB, d, vh.data());
       const double p = z[j] / denom;
       for (int i = 0; i < d; ++i) acc[i] += p * vh[i];
     }
@@ -912,6 +994,25 @@ void orc_rotate_rows_f64(double* x, int64_t rows, int d, int kind, int b, const 
 
 void orc_unrotate_rows_f64(double* x, int64_t rows, int d, int kind, int b, const float* quat) {
   for (int64_t r = 0; r < rows; ++r) orc_unrotate_f64(x + r * d, d, kind, b, quat);
+}
+
+void orc_quantize_rows_fmt(const float* y, int64_t rows, int d, int fmt, const float* levels,
+                           uint8_t* codes, uint16_t* s16, uint16_t* m16) {
+  const int cb = code_row_bytes(fmt, d);
+  for (int64_t r = 0; r < rows; ++r) {
+    if (fmt == ORC_FMT_LUT4)
+      orc_quantize_row_lut(y + r * d, d, levels, codes + r * cb, s16 + r, m16 + r);
+    else
+      orc_quantize_row_bits(y + r * d, d, code_bits(fmt), codes + r * cb, s16 + r, m16 + r);
+  }
+}
+
+void orc_unpack_codes_rows(const uint8_t* codes, int64_t rows, int d, int bits, int32_t* c) {
+  std::vector<int> t(d);
+  for (int64_t r = 0; r < rows; ++r) {
+    orc_unpack_codes(codes + r * (d * bits / 8), d, bits, t.data());
+    for (int i = 0; i < d; ++i) c[r * d + i] = t[i];
+  }
 }
 
 void orc_quantize_rows(const float* y, int64_t rows, int d, uint8_t* codes, uint16_t* s16,
