@@ -34,8 +34,10 @@ static int check_desc(const kvq_cache_desc* d) {
     return KVQ_ERR_INVALID_ARG;
   if (d->head_dim != 64 && d->head_dim != 128 && d->head_dim != 256) return KVQ_ERR_UNSUPPORTED;
   if (d->page_size != 16 && d->page_size != 32 && d->page_size != 64) return KVQ_ERR_UNSUPPORTED;
-  if (d->format != KVQ_FMT_INT4 && d->format != KVQ_FMT_MXFP4) return KVQ_ERR_INVALID_ARG;
-  if (d->format == KVQ_FMT_MXFP4 && d->head_dim != 128) return KVQ_ERR_UNSUPPORTED;
+  if (d->format < KVQ_FMT_INT4 || d->format > KVQ_FMT_LUT4) return KVQ_ERR_INVALID_ARG;
+  if (d->format != KVQ_FMT_INT4 && d->head_dim != 128) return KVQ_ERR_UNSUPPORTED;
+  if ((d->format == KVQ_FMT_LUT4) != (d->levels != nullptr)) return KVQ_ERR_INVALID_ARG;
+  if (d->levels != nullptr && !aligned4(d->levels)) return KVQ_ERR_MISALIGNED;
   switch (d->rot_kind) {
     case KVQ_ROT_NONE:
       break;

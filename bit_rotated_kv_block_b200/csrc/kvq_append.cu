@@ -67,6 +67,97 @@ __host__ __device__ constexpr int append_table_bytes(int D, int rot) {
 }
 __host__ __device__ constexpr int append_ctas_per_sm(int E) { return E == 64 ? 2 : 1; }
 
+// Row-part encodings of the tile kernel (template argument FMT).
+constexpr int kAppInt4 = 0, kAppMx = 1, kAppGen = 2;
+
+// The 2-bit, 3-bit and level-table formats of one thread's E channels: the
+// row statistics of INT4 with Q = 3, 7 or 15 levels above zero (the two
+// threads of a row combine theirs), then each code from the exact product
+// RN(x - m16) * RN(1/s16): the nearest integer (one fused multiply-add with
+// 1.5 * 2^23, as for INT4) or the index of the nearest table level (the count
+// of level midpoints below it, each decided exactly by the sign of one fused
+// multiply-add); codes packed as a little-endian bit stream.
+// Codes of one thread's E channels as a little-endian bit stream of BITS
+// bits per code (LUT: the level-table rule), into w[E * BITS / 32].
+template <int E, int BITS, bool LUT>
+__device__ __forceinline__ void gen_codes(const float (&x)[E], float m, float inv,
+                                          const float* levels, uint32_t (&w)[E / 8]) {
+  float mid[15];
+  if (LUT) {
+#pragma unroll
+    for (int k = 0; k < 15; ++k) mid[k] = 0.5f * (__ldg(levels + k) + __ldg(levels + k + 1));
+  }
+#pragma unroll
+  for (int i = 0; i < E; ++i) {
+    const float t0 = __fsub_rn(x[i], m);
+    uint32_t c;
+    if (LUT) {
+      c = 0;
+#pragma unroll
+      for (int k = 0; k < 15; ++k) c += __fmaf_rn(t0, inv, -mid[k]) > 0.f ? 1u : 0u;
+    } else {
+      c = __float_as_uint(__fmaf_rn(t0, inv, 12582912.0f)) & ((1u << BITS) - 1u);
+    }
+    const int bit = i * BITS;
+    w[bit >> 5] |= c << (bit & 31);
+    if ((bit & 31) + BITS > 32) w[(bit >> 5) + 1] |= c >> (32 - (bit & 31));
+  }
+}
+
+// The 2-bit, 3-bit and level-table formats of one thread's E channels: the
+// row statistics of INT4 with Q = 3, 7 or 15 levels above zero (the two
+// threads of a row combine theirs), then each code from the exact product
+// RN(x - m16) * RN(1/s16): the nearest integer (one fused multiply-add with
+// 1.5 * 2^23, as for INT4) or the index of the nearest table level (the count
+// of level midpoints below it, each decided exactly by the sign of one fused
+// multiply-add); codes packed as a little-endian bit stream.
+template <int D, int E, int TPR>
+__device__ __forceinline__ void gen_encode_store(float (&x)[E], int fmt, const float* levels,
+                                                 int my_part, unsigned pair_mask,
+                                                 int64_t dst_cur, uint8_t* codes,
+                                                 uint32_t* params) {
+  const int bits = fmt == KVQ_FMT_INT2 ? 2 : (fmt == KVQ_FMT_INT3 ? 3 : 4);
+  const float Q = fmt == KVQ_FMT_INT2 ? 3.f : (fmt == KVQ_FMT_INT3 ? 7.f : 15.f);
+  float mn = x[0], mx = x[0];
+#pragma unroll
+  for (int i = 1; i < E; ++i) {
+    mn = fminf(mn, x[i]);
+    mx = fmaxf(mx, x[i]);
+  }
+  if (TPR == 2) {
+    mn = fminf(mn, __shfl_xor_sync(pair_mask, mn, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(pair_mask, mx, 1));
+  }
+  mn = __fadd_rn(mn, 0.0f);
+  mx = __fadd_rn(mx, 0.0f);
+  const __half m16 = __float2half_rd(mn);
+  const float m = __half2float(m16);
+  const __half s16 = __float2half_ru(__fdiv_ru(__fsub_ru(mx, m), Q));
+  const float s = __half2float(s16);
+  uint32_t w[E / 8];  // E * bits / 32 words used
+#pragma unroll
+  for (int i = 0; i < E / 8; ++i) w[i] = 0u;
+  if (s != 0.0f) {
+    const float inv = __frcp_rn(s);
+    if (fmt == KVQ_FMT_INT2)
+      gen_codes<E, 2, false>(x, m, inv, levels, w);
+    else if (fmt == KVQ_FMT_INT3)
+      gen_codes<E, 3, false>(x, m, inv, levels, w);
+    else
+      gen_codes<E, 4, true>(x, m, inv, levels, w);
+  }
+  if (dst_cur >= 0) {
+    const int rb = D * bits / 8;  // code bytes of the row
+    const int pb = E * bits / 8;  // this thread's code bytes (a multiple of 8)
+    uint2* dst = reinterpret_cast<uint2*>(codes + dst_cur * rb + my_part * pb);
+#pragma unroll
+    for (int j = 0; j < E / 16; ++j)
+      if (8 * j < pb) dst[j] = make_uint2(w[2 * j], w[2 * j + 1]);
+    if (my_part == 0)
+      params[dst_cur] = (uint32_t)__half_as_ushort(s16) | ((uint32_t)__half_as_ushort(m16) << 16);
+  }
+}
+
 // One thread's part of one row: E channels of a (token, head) row of K or
 // V, read from the row's line of the 128-byte swizzled TMA boxes (channel
 // block c of the row sits in box my_part * E/64 + c/8, 16-byte chunk c % 8 at
@@ -79,12 +170,16 @@ __host__ __device__ constexpr int append_ctas_per_sm(int E) { return E == 64 ? 2
 // randomised-sign Hadamard (channels flipped before the butterflies).
 // PRE: the kernel turns rows (RoPE) or flips signs before the rotation; without
 // it the first butterfly stage is taken straight from binary16.
-// MX: the microscaled FP4 format (kvq.h, KVQ_FMT_MXFP4) instead of INT4.
-template <int D, int ROT, int LGB, bool PRE, bool MX>
+// FMT: kAppInt4 (INT4), kAppMx (microscaled FP4, KVQ_FMT_MXFP4) or kAppGen
+// (the 2-bit, 3-bit and level-table formats, chosen by `fmt` at run time,
+// `levels` the table).
+template <int D, int ROT, int LGB, bool PRE, int FMT>
 __device__ __forceinline__ void quantize_row_part(const uint8_t* boxes, int box_stride,
                                                   int my_line, int my_part, const float* qtbl,
                                                   const float* cs, int64_t dst_cur,
-                                                  uint8_t* codes, uint32_t* params) {
+                                                  uint8_t* codes, uint32_t* params, int fmt,
+                                                  const float* levels) {
+  constexpr bool MX = FMT == kAppMx;
   constexpr bool fused1 = ROT == KVQ_ROT_HADAMARD && !PRE;
   constexpr int E = append_e(D, ROT, LGB);  // channels per thread
   constexpr int TPR = D / E;                // threads per row
@@ -130,6 +225,11 @@ __device__ __forceinline__ void quantize_row_part(const uint8_t* boxes, int box_
     quat_regs<E>(x, qtbl, my_part * E);
   } else if (ROT == KVQ_ROT_QUAT_MAT) {
     quat_mat_regs<E>(x, qtbl, my_part * E);  // the CTA's matrices
+  }
+
+  if constexpr (FMT == kAppGen) {
+    gen_encode_store<D, E, TPR>(x, fmt, levels, my_part, pair_mask, dst_cur, codes, params);
+    return;
   }
 
   if constexpr (MX) {
@@ -239,7 +339,8 @@ __device__ __forceinline__ void quantize_row_part(const uint8_t* boxes, int box_
 
 struct AppendArgs {
   int T, H, P, lg_page, NP, num_seqs, bt_stride, tok_per_tile, num_tiles;
-  int mx;  // the microscaled FP4 format (else INT4)
+  int fmt;  // kvq_format
+  const float* levels;  // the level table (KVQ_FMT_LUT4)
   int box_stride;  // bytes between TMA boxes in a tile buffer (multiple of 1024)
   const int32_t* token_seq;
   const int32_t* token_pos;
@@ -255,9 +356,9 @@ struct AppendArgs {
 };
 
 // D: head_dim, ROT: rotation kind, LGB: log2 of the Hadamard block, PRE: a
-// RoPE table or a sign table acts before the rotation, MX: the microscaled
-// FP4 format.
-template <int D, int ROT, int LGB, bool PRE, bool MX>
+// RoPE table or a sign table acts before the rotation, FMT: the row-part
+// encoding (kAppInt4, kAppMx, kAppGen).
+template <int D, int ROT, int LGB, bool PRE, int FMT>
 __global__ void __launch_bounds__(append_threads(append_e(D, ROT, LGB)),
                                   append_ctas_per_sm(append_e(D, ROT, LGB)))
     append_kernel(const AppendArgs a, const __grid_constant__ CUtensorMap tmk,
@@ -397,10 +498,10 @@ __global__ void __launch_bounds__(append_threads(append_e(D, ROT, LGB)),
     if (active && tok < a.T) {
       const float* cs = (PRE && a.rope != nullptr && my_kv == 0 && dst_cur >= 0)
                             ? a.rope + (int64_t)pos_cur * D : nullptr;
-      quantize_row_part<D, ROT, LGB, PRE, MX>(cur + my_kv * NH * a.box_stride, a.box_stride, my_line,
-                                          my_part, rtbl, cs, dst_cur,
-                                          my_kv ? a.v_codes : a.k_codes,
-                                          my_kv ? a.v_params : a.k_params);
+      quantize_row_part<D, ROT, LGB, PRE, FMT>(cur + my_kv * NH * a.box_stride, a.box_stride,
+                                               my_line, my_part, rtbl, cs, dst_cur,
+                                               my_kv ? a.v_codes : a.k_codes,
+                                               my_kv ? a.v_params : a.k_params, a.fmt, a.levels);
     }
     dst_cur = resolve(seq_n, pos_n);  // next tile's destination (its loads were in flight)
     pos_cur = pos_n;
@@ -421,7 +522,8 @@ __global__ void __launch_bounds__(append_threads(append_e(D, ROT, LGB)),
 
 struct AppendRowsArgs {
   int T, H, P, lg_page, NP, num_seqs, bt_stride;
-  int mx;  // the microscaled FP4 format (else INT4)
+  int fmt;  // kvq_format
+  const float* levels;  // the level table (KVQ_FMT_LUT4)
   int64_t tok_stride;
   const __half* k;
   const __half* v;
@@ -472,30 +574,41 @@ __global__ void __launch_bounds__(kRowsWarps * kWarp) append_rows_kernel(const A
   __half s16, m16;
   uint32_t pword = 0;
   uint32_t packed;
-  if (a.mx) {
+  if (a.fmt == KVQ_FMT_MXFP4) {
     packed = row_quantize_mx<D, ROT, LGB>(x, rl, a.quat, pword);
   } else {
-    packed = row_quantize<D, ROT, LGB>(x, rl, a.quat, s16, m16);
+    packed = a.fmt == KVQ_FMT_INT4
+                 ? row_quantize<D, ROT, LGB>(x, rl, a.quat, s16, m16)
+                 : row_quantize_gen<D, ROT, LGB>(x, rl, a.quat, a.fmt, a.levels, s16, m16);
     pword = (uint32_t)__half_as_ushort(s16) | ((uint32_t)__half_as_ushort(m16) << 16);
   }
-
-  if (!active || seq < 0) return;
+  const int bits = a.fmt == KVQ_FMT_INT2 ? 2 : (a.fmt == KVQ_FMT_INT3 ? 3 : 4);
+  // 3-bit codes pair lanes for their stores: every lane of a row stays until then
+  const bool ok_row = active && seq >= 0;
   const bool lead = kv == 0 && h == 0 && rl == 0;
-  if (!seq_ok) {
+  bool store = ok_row;
+  if (ok_row && !seq_ok) {
     if (lead) raise_flag(a.err, KVQ_ERRF_SEQ);
-    return;
-  }
-  if (!pos_ok) {
+    store = false;
+  } else if (ok_row && !pos_ok) {
     if (lead) raise_flag(a.err, KVQ_ERRF_POS);
-    return;
-  }
-  if (page < 0 || page >= a.NP) {
+    store = false;
+  } else if (ok_row && (page < 0 || page >= a.NP)) {
     if (lead) raise_flag(a.err, KVQ_ERRF_PAGE);
-    return;
+    store = false;
   }
-  const int64_t dst = (((int64_t)page * a.H + h) << a.lg_page) + (pos & ((1 << a.lg_page) - 1));
-  row_store_codes<D>((kv ? a.v_codes : a.k_codes) + dst * (D / 2) + rl * (CPL / 2), packed);
-  if (rl == 0) (kv ? a.v_params : a.k_params)[dst] = pword;
+  const int64_t dst =
+      store ? (((int64_t)page * a.H + h) << a.lg_page) + (pos & ((1 << a.lg_page) - 1)) : 0;
+  if (bits == 4) {
+    if (store)
+      row_store_codes<D>((kv ? a.v_codes : a.k_codes) + dst * (D / 2) + rl * (CPL / 2), packed);
+  } else {
+    // the pairing shuffle inside involves every lane of the row (a row's
+    // lanes share `store`)
+    row_store_bits<D>((kv ? a.v_codes : a.k_codes) + dst * (D * bits / 8), packed, bits, rl,
+                      store);
+  }
+  if (store && rl == 0) (kv ? a.v_params : a.k_params)[dst] = pword;
 }
 
 template <int D, int ROT, int LGB>
@@ -569,12 +682,19 @@ static cudaError_t launch_append(const AppendArgs& a, const CUtensorMap& tk, con
                                  int grid, cudaStream_t st) {
   const size_t smem = append_smem(D, ROT, a.box_stride);
   const bool pre = a.rope != nullptr || (ROT == KVQ_ROT_HADAMARD && a.quat != nullptr);
-  auto kern = pre ? append_kernel<D, ROT, LGB, true, false> : append_kernel<D, ROT, LGB, false, false>;
-  if (a.mx) {  // the microscaled FP4 format: head_dim 128 only
-    if constexpr (D == 128)
-      kern = pre ? append_kernel<D, ROT, LGB, true, true> : append_kernel<D, ROT, LGB, false, true>;
-    else
+  auto kern = pre ? append_kernel<D, ROT, LGB, true, kAppInt4>
+                  : append_kernel<D, ROT, LGB, false, kAppInt4>;
+  if (a.fmt != KVQ_FMT_INT4) {  // the other formats: head_dim 128 only
+    if constexpr (D == 128) {
+      if (a.fmt == KVQ_FMT_MXFP4)
+        kern = pre ? append_kernel<D, ROT, LGB, true, kAppMx>
+                   : append_kernel<D, ROT, LGB, false, kAppMx>;
+      else
+        kern = pre ? append_kernel<D, ROT, LGB, true, kAppGen>
+                   : append_kernel<D, ROT, LGB, false, kAppGen>;
+    } else {
       return cudaErrorInvalidValue;
+    }
   }
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -644,7 +764,8 @@ int append_launch(const kvq_cache_desc& d, int32_t T, const void* k, const void*
     r.k_codes = k_codes; r.v_codes = v_codes;
     r.k_params = static_cast<uint32_t*>(k_params); r.v_params = static_cast<uint32_t*>(v_params);
     r.quat = rot_table(d); r.rope = d.rope; r.rope_max_pos = d.rope_max_pos; r.err = err;
-    r.mx = d.format == KVQ_FMT_MXFP4;
+    r.fmt = d.format;
+    r.levels = d.levels;
     cudaError_t e;
     switch (D) {
       case 64: e = dispatch_rows<64>(r, rot_template(d), lgb, st); break;
@@ -682,7 +803,8 @@ int append_launch(const kvq_cache_desc& d, int32_t T, const void* k, const void*
   a.rope = d.rope;
   a.rope_max_pos = d.rope_max_pos;
   a.err = err;
-  a.mx = d.format == KVQ_FMT_MXFP4;
+  a.fmt = d.format;
+  a.levels = d.levels;
   CUtensorMap tk, tv;
   if (!encode_rows(&tk, k, D, a.H, T, tok_stride, a.H, tok) ||
       !encode_rows(&tv, v, D, a.H, T, tok_stride, a.H, tok))

@@ -968,6 +968,7 @@ static int resident_warps(int D, int P, int GP) {
 
 DecodePlan decode_plan(const kvq_cache_desc& d, int32_t S, int32_t Hq, int32_t max_seq_len) {
   if (d.format == KVQ_FMT_MXFP4) return decode_mx_plan(d, S, Hq, max_seq_len);
+  if (d.format != KVQ_FMT_INT4) return decode_gen_plan(d, S, Hq, max_seq_len);
   DecodePlan pl{};
   const int P = d.page_size;
   pl.pages_max = (max_seq_len + P - 1) / P;
@@ -1021,6 +1022,10 @@ int decode_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, const void* q,
     return decode_mx_launch(d, S, Hq, q, seq_lens, max_seq_len, block_table, bt_stride, sm_scale,
                             k_codes, k_params, v_codes, v_params, out, workspace,
                             workspace_bytes, err, st, step);
+  if (d.format != KVQ_FMT_INT4)
+    return decode_gen_launch(d, S, Hq, q, seq_lens, max_seq_len, block_table, bt_stride,
+                             sm_scale, k_codes, k_params, v_codes, v_params, out, workspace,
+                             workspace_bytes, err, st, step);
   const int D = d.head_dim;
   const int G = Hq / d.num_kv_heads;
   const int GP = G <= 4 ? 4 : 8;

@@ -10,7 +10,7 @@
 //    K-major operand layout for 4-bit elements (each 16-byte chunk holds 16
 //    codes in its low 8 bytes), its 4 K block-scale bytes into the scale-
 //    factor copy layout, its V codes and V scale word as plain rows;
-//    cp.async, a 3-stage ring;
+//    cp.async, a 2-stage ring (4 CTAs per SM for G <= 4);
 //  * one thread copies the K scales into tensor memory and issues four
 //    tcgen05.mma kind::mxf8f6f4.block_scale (M = 128 tokens, N = 16 query
 //    rows, K = 32 channels each): S = (K e2m1 x 2^Xk)(q e4m3 x 2^Xq)^T, fp32
@@ -49,7 +49,7 @@ constexpr int kMxD = 128;        // head_dim
 constexpr int kMxThreads = 128;  // 4 warps; thread t stages and scores token t of a tile
 constexpr int kMxTile = 128;     // tokens per tile: the MMA's M
 constexpr int kMxN = 16;         // the MMA's N: query rows of B (G used, the rest zero)
-constexpr int kMxStages = 3;
+constexpr int kMxStages = 2;
 constexpr uint32_t kMxTmemCols = 32;
 constexpr uint32_t kColD = 0, kColSFA = 16, kColSFB = 20;  // tensor-memory columns
 constexpr float kMxSlack = 8.f;
@@ -67,9 +67,12 @@ constexpr int kStage_B = kVS_OFF + kMxTile * 4;
 constexpr int kB_OFF = kMxStages * kStage_B;  // query E4M3: 2 row groups x 8 chunks x 128 B
 constexpr int kB_B = 2048;
 constexpr int kSFB_OFF = kB_OFF + kB_B;       // query block scales (rows 0-15 used)
-constexpr int kP_OFF = kSFB_OFF + kSF_B;      // per-warp weights [4][8 heads][32 tokens] fp32
-constexpr int kP_B = 4 * 8 * 32 * 4;
-constexpr int kBar_OFF = kP_OFF + kP_B;       // mbarrier, then the tensor-memory base
+constexpr int kBar_OFF = kSFB_OFF + kSF_B;    // mbarrier, then the tensor-memory base
+// per-warp weights [8 heads][32 tokens] fp32 live in the K region of the
+// stage being consumed (free once its MMA has completed, refilled only after
+// the next barrier)
+constexpr int kP_B = 8 * 32 * 4;
+static_assert(4 * kP_B <= kA_B, "weights fit in the consumed K region");
 constexpr int kMxSmem = kBar_OFF + 16;
 static_assert(kStage_B % 128 == 0 && kB_OFF % 1024 == 0, "operand alignment");
 // the four warps' states at the end reuse stage 0: [4][8][128] acc + [4][8] M, L
@@ -242,7 +245,6 @@ __global__ void __launch_bounds__(kMxThreads) decode_mx_kernel(const MxDecodeArg
     for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[nb][mt][e] = 0.f;
-  float* pw = reinterpret_cast<float*>(smem + kP_OFF) + warp * 8 * 32;
   bool timed_out = false;
   int it_out = 0;  // the iteration whose wait ran out
 
@@ -286,6 +288,7 @@ __global__ void __launch_bounds__(kMxThreads) decode_mx_kernel(const MxDecodeArg
 
     // ---- scores of token tid for the G heads, the warp's online softmax
     const bool valid = (vbits >> stage) & 1u;
+    float* pw = reinterpret_cast<float*>(st + kA_OFF) + warp * 8 * 32;
     float z[8];
 #pragma unroll
     for (int g = 0; g < 8; ++g)
@@ -334,9 +337,16 @@ __global__ void __launch_bounds__(kMxThreads) decode_mx_kernel(const MxDecodeArg
     }
     __syncwarp();
 
-    // ---- PV over the warp's 32 tokens, two k-steps of 16
+    // ---- PV over the warp's 32 tokens, two k-steps of 16. For NB = 1 the
+    // tile's two k-steps accumulate in the MMA from zero and join the running
+    // sums once; for NB = 2 (hi and lo products) each k-step does.
     const uint8_t* vst = st + kV_OFF;
     const uint32_t* vsw = reinterpret_cast<const uint32_t*>(st + kVS_OFF);
+    float tacc[8][4];
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) tacc[mt][e] = 0.f;
 #pragma unroll
     for (int ks = 0; ks < 2; ++ks) {
       const int tb = warp * 32 + ks * 16;  // first token of the k-step in the tile
@@ -389,11 +399,13 @@ __global__ void __launch_bounds__(kMxThreads) decode_mx_kernel(const MxDecodeArg
           av[1] = h2_as_u32(__hmul2(u32_as_h2(e2m1x2_to_h2((o0 >> (8 * m4)) & 0xFFu)), sAB));
           av[2] = h2_as_u32(__hmul2(u32_as_h2(e2m1x2_to_h2((e1 >> (8 * m4)) & 0xFFu)), sCD));
           av[3] = h2_as_u32(__hmul2(u32_as_h2(e2m1x2_to_h2((o1 >> (8 * m4)) & 0xFFu)), sCD));
-          float t4[4] = {0.f, 0.f, 0.f, 0.f};
-          mma16816(t4, av, b0, b1);
+          if (NB == 1) {
+            mma16816(tacc[mt], av, b0, b1);
+          } else {
+            float t4[4] = {0.f, 0.f, 0.f, 0.f};
+            mma16816(t4, av, b0, b1);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) acc[0][mt][e] += t4[e];
-          if (NB == 2) {
+            for (int e = 0; e < 4; ++e) acc[0][mt][e] += t4[e];
             float u4[4] = {0.f, 0.f, 0.f, 0.f};
             mma16816(u4, av, bl0, bl1);
 #pragma unroll
@@ -401,6 +413,12 @@ __global__ void __launch_bounds__(kMxThreads) decode_mx_kernel(const MxDecodeArg
           }
         }
       }
+    }
+    if (NB == 1) {
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[0][mt][e] += tacc[mt][e];
     }
   }
   cp_async_wait<0>();
@@ -550,12 +568,14 @@ static cudaError_t dispatch_mx_step(const MxStepArgs& a, int rot, int lgb, cudaS
   return cudaErrorInvalidValue;
 }
 
+template <int NB>
 static int mx_resident_ctas() {
   static int cached = -1;
   if (cached < 0) {
     int blocks = 0;
-    cudaFuncSetAttribute(decode_mx_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMxSmem);
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, decode_mx_kernel<1>, kMxThreads,
+    cudaFuncSetAttribute(decode_mx_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         kMxSmem);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, decode_mx_kernel<NB>, kMxThreads,
                                                       kMxSmem) != cudaSuccess ||
         blocks < 1)
       blocks = 1;
@@ -566,13 +586,16 @@ static int mx_resident_ctas() {
 }
 
 DecodePlan decode_mx_plan(const kvq_cache_desc& d, int32_t S, int32_t Hq, int32_t max_seq_len) {
-  (void)Hq;
   DecodePlan pl{};
   int tiles = (max_seq_len + kMxTile - 1) / kMxTile;
   if (tiles < 1) tiles = 1;
   pl.pages_max = tiles;
+  const int G = Hq / (d.num_kv_heads > 0 ? d.num_kv_heads : 1);
+  const int resident = G <= 4 ? mx_resident_ctas<1>() : mx_resident_ctas<2>();
   const int pairs = S * d.num_kv_heads;
-  int splits = (2 * mx_resident_ctas()) / (pairs > 0 ? pairs : 1);
+  // about one CTA per resident slot (a single wave), at least one split per
+  // 64 tiles
+  int splits = (resident + (pairs > 0 ? pairs : 1) / 2) / (pairs > 0 ? pairs : 1);
   const int min_splits = (tiles + 63) / 64;
   if (splits < min_splits) splits = min_splits;
   if (splits < 1) splits = 1;

@@ -1,5 +1,6 @@
-// Dense export of cached rows: x = c * s16 + m16 (INT4) or x = e2m1(c) * 2^X
-// (microscaled FP4), optionally rotated back.
+// Dense export of cached rows: x = c * s16 + m16 (the integer formats),
+// t[c] * s16 + m16 (the level table) or e2m1(c) * 2^X (microscaled FP4),
+// optionally rotated back.
 //
 // The dequantization rule is the one of the token-wise asymmetric INT4 format
 // ("SAW-INT4: System-Aware 4-Bit KV-Cache Quantization for Real-World LLM
@@ -27,7 +28,8 @@ struct DequantArgs {
   const uint32_t* params;
   const float* quat;   // quaternion table (QUAT kinds)
   const float* signs;  // sign table of the randomised-sign Hadamard, or NULL
-  int mx;              // the microscaled FP4 format (else INT4)
+  int fmt;             // kvq_format
+  const float* levels; // the level table (KVQ_FMT_LUT4)
   void* out;
   int32_t* err;
 };
@@ -60,7 +62,21 @@ __global__ void __launch_bounds__(128) dequant_kernel(const DequantArgs a, int u
   const float mn = __half2float(__ushort_as_half((unsigned short)(pr >> 16)));
   float x[E];
   const uint4* src = reinterpret_cast<const uint4*>(a.codes + prow * (D / 2) + part * (E / 2));
-  if (a.mx) {
+  if (a.fmt == KVQ_FMT_INT2 || a.fmt == KVQ_FMT_INT3 || a.fmt == KVQ_FMT_LUT4) {
+    // c (or the table's level t[c]) times s16 plus m16, one rounding; the
+    // codes of this thread's E channels as a little-endian bit stream
+    const int bits = a.fmt == KVQ_FMT_INT2 ? 2 : (a.fmt == KVQ_FMT_INT3 ? 3 : 4);
+    const uint8_t* cb = a.codes + prow * (D * bits / 8) + part * (E * bits / 8);
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+      const int bit = i * bits;
+      uint32_t v = cb[bit >> 3];
+      if ((bit & 7) + bits > 8) v |= (uint32_t)cb[(bit >> 3) + 1] << 8;
+      const uint32_t c = (v >> (bit & 7)) & ((1u << bits) - 1u);
+      const float lv = a.fmt == KVQ_FMT_LUT4 ? __ldg(a.levels + c) : (float)c;
+      x[i] = __fmaf_rn(lv, sc, mn);
+    }
+  } else if (a.fmt == KVQ_FMT_MXFP4) {
     // E2M1 value (exact in binary16) times 2^X of its 32-channel block:
     // exact in binary32, subnormal results included (X = -127: 2^-127 is the
     // binary32 bit pattern 0x00400000)
@@ -157,7 +173,8 @@ int dequant_launch(const kvq_cache_desc& d, int32_t S, const int32_t* seq_lens,
   a.bt_stride = bt_stride; a.seq_lens = seq_lens; a.block_table = block_table;
   a.codes = codes; a.params = static_cast<const uint32_t*>(params); a.quat = d.quat;
   a.signs = d.rot_kind == KVQ_ROT_HADAMARD_SIGNED ? d.quat : nullptr;
-  a.mx = d.format == KVQ_FMT_MXFP4;
+  a.fmt = d.format;
+  a.levels = d.levels;
   a.out = out; a.err = err;
   int lgb = 0;
   while ((1 << lgb) < d.rot_block) ++lgb;

@@ -81,6 +81,17 @@ int decode_mx_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, const void*
                      float* out, void* workspace, size_t workspace_bytes, int32_t* err,
                      cudaStream_t st, const DecodeStepRows* step);
 
+// Decode attention over the 2-bit, 3-bit and level-table caches (QK on the
+// tensor cores' integer MMA); plan (pages_per_split counts 128-token tiles)
+// and launch.
+DecodePlan decode_gen_plan(const kvq_cache_desc& d, int32_t S, int32_t Hq, int32_t max_seq_len);
+int decode_gen_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, const void* q,
+                      const int32_t* seq_lens, int32_t max_seq_len, const int32_t* block_table,
+                      int32_t bt_stride, float sm_scale, const uint8_t* k_codes,
+                      const void* k_params, const uint8_t* v_codes, const void* v_params,
+                      float* out, void* workspace, size_t workspace_bytes, int32_t* err,
+                      cudaStream_t st, const DecodeStepRows* step);
+
 // Baseline decode attention over a binary16 paged cache.
 DecodePlan decode_fp16_plan(const kvq_cache_desc& d, int32_t S, int32_t Hq, int32_t max_seq_len);
 int decode_fp16_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, const void* q,

@@ -147,6 +147,91 @@ __device__ __forceinline__ uint32_t row_quantize_mx(float (&x)[RowQuantShape<D>:
   return packed;
 }
 
+// The 2-bit, 3-bit and level-table forms of the same rotated row (kvq.h,
+// KVQ_FMT_INT2 / INT3 / LUT4): the INT4 statistics with Q = 3, 7 or 15, each
+// code the nearest integer of the exact product RN(x - m16) * RN(1/s16) (one
+// fused multiply-add with 1.5 * 2^23) or the index of the nearest table level
+// (the count of level midpoints below the exact product, each decided by the
+// sign of one fused multiply-add). Returns the lane's codes, channel i of the
+// lane at bits [i*bits, (i+1)*bits).
+template <int D, int ROT, int LGB>
+__device__ __forceinline__ uint32_t row_quantize_gen(float (&x)[RowQuantShape<D>::CPL], int rl,
+                                                     const float* quat, int fmt,
+                                                     const float* levels, __half& s16,
+                                                     __half& m16) {
+  constexpr int CPL = RowQuantShape<D>::CPL;
+  constexpr int LPR = RowQuantShape<D>::LPR;
+  row_rotate<D, ROT, LGB>(x, rl, quat);
+  const int bits = fmt == KVQ_FMT_INT2 ? 2 : (fmt == KVQ_FMT_INT3 ? 3 : 4);
+  const float Q = fmt == KVQ_FMT_INT2 ? 3.f : (fmt == KVQ_FMT_INT3 ? 7.f : 15.f);
+  float mn = x[0], mx = x[0];
+#pragma unroll
+  for (int i = 1; i < CPL; ++i) {
+    mn = fminf(mn, x[i]);
+    mx = fmaxf(mx, x[i]);
+  }
+#pragma unroll
+  for (int m = 1; m < LPR; m <<= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, m));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
+  }
+  mn = __fadd_rn(mn, 0.0f);
+  mx = __fadd_rn(mx, 0.0f);
+  m16 = __float2half_rd(mn);
+  const float m = __half2float(m16);
+  s16 = __float2half_ru(__fdiv_ru(__fsub_ru(mx, m), Q));
+  const float s = __half2float(s16);
+  uint32_t packed = 0;
+  if (s != 0.0f) {
+    const float inv = __frcp_rn(s);
+    if (fmt == KVQ_FMT_LUT4) {
+      float mid[15];
+#pragma unroll
+      for (int k = 0; k < 15; ++k) mid[k] = 0.5f * (__ldg(levels + k) + __ldg(levels + k + 1));
+#pragma unroll
+      for (int i = 0; i < CPL; ++i) {
+        const float t0 = __fsub_rn(x[i], m);
+        uint32_t c = 0;
+#pragma unroll
+        for (int k = 0; k < 15; ++k) c += __fmaf_rn(t0, inv, -mid[k]) > 0.f ? 1u : 0u;
+        packed |= c << (4 * i);
+      }
+    } else {
+      const uint32_t mask = (1u << bits) - 1u;
+#pragma unroll
+      for (int i = 0; i < CPL; ++i) {
+        const uint32_t c =
+            __float_as_uint(__fmaf_rn(__fsub_rn(x[i], m), inv, 12582912.0f)) & mask;
+        packed |= c << (bits * i);
+      }
+    }
+  }
+  return packed;
+}
+
+// Stores the lane's packed codes of a row of `bits`-bit codes (row_bytes =
+// D * bits / 8 at `row`). With 12 bits per lane (3-bit codes, 4 channels per
+// lane) the even lane of each pair writes both lanes' 24 bits; every lane of
+// the warp must call it (nothing is written where `store` is false).
+template <int D>
+__device__ __forceinline__ void row_store_bits(uint8_t* row, uint32_t packed, int bits, int rl,
+                                               bool store) {
+  constexpr int CPL = RowQuantShape<D>::CPL;
+  const int lb = CPL * bits;  // bits per lane
+  if (lb % 8 == 0) {
+    uint8_t* p = row + rl * (lb / 8);
+    if (store)
+      for (int k = 0; k < lb / 8; ++k) p[k] = (uint8_t)(packed >> (8 * k));
+  } else {  // 12 bits per lane: lane pairs
+    const uint32_t other = __shfl_xor_sync(0xffffffffu, packed, 1);
+    if (store && (rl & 1) == 0) {
+      const uint32_t v = packed | (other << lb);
+      uint8_t* p = row + (rl / 2) * (2 * lb / 8);
+      for (int k = 0; k < 2 * lb / 8; ++k) p[k] = (uint8_t)(v >> (8 * k));
+    }
+  }
+}
+
 // Loads this lane's CPL channels of a binary16 row (zeros when !active).
 template <int D>
 __device__ __forceinline__ void row_load(float (&x)[RowQuantShape<D>::CPL], const __half* src,

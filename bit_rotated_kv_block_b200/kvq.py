@@ -16,7 +16,7 @@ from . import build as _build
 
 ROT_NONE, ROT_HADAMARD, ROT_QUAT, ROT_QUAT_FAST, ROT_HADAMARD_SIGNED, ROT_QUAT_MAT = \
     0, 1, 2, 3, 4, 5
-FMT_INT4, FMT_MXFP4 = 0, 1
+FMT_INT4, FMT_MXFP4, FMT_INT2, FMT_INT3, FMT_LUT4 = 0, 1, 2, 3, 4
 ERRF_PAGE, ERRF_POS, ERRF_SEQ, ERRF_LEN = 1, 2, 4, 8
 STATUS = {0: "KVQ_OK", 1: "KVQ_ERR_INVALID_ARG", 2: "KVQ_ERR_UNSUPPORTED",
           3: "KVQ_ERR_MISALIGNED", 4: "KVQ_ERR_WORKSPACE", 5: "KVQ_ERR_CUDA"}
@@ -56,7 +56,8 @@ class CacheDesc(ctypes.Structure):
                 ("page_size", ctypes.c_int32), ("num_pages", ctypes.c_int32),
                 ("rot_kind", ctypes.c_int32), ("rot_block", ctypes.c_int32),
                 ("quat", ctypes.c_void_p), ("rope", ctypes.c_void_p),
-                ("rope_max_pos", ctypes.c_int32), ("format", ctypes.c_int32)]
+                ("rope_max_pos", ctypes.c_int32), ("format", ctypes.c_int32),
+                ("levels", ctypes.c_void_p)]
 
 
 _lib = None
@@ -103,10 +104,13 @@ class Cache:
     (kept alive here because the descriptor points at it)."""
 
     def __init__(self, head_dim, num_kv_heads, page_size, num_pages, rot_kind=ROT_HADAMARD,
-                 rot_block=0, quat=None, device="cuda", rope=None, fmt=FMT_INT4):
+                 rot_block=0, quat=None, device="cuda", rope=None, fmt=FMT_INT4, levels=None):
         """``rope``: optional RoPE table float32 [max_pos][d/2][2] of (cos, sin);
-        ``fmt``: FMT_INT4 or FMT_MXFP4 (the pools have the same shapes)."""
+        ``fmt``: a kvq_format; ``levels``: the 16-entry table of FMT_LUT4."""
         self.fmt = fmt
+        self.levels = None
+        if levels is not None:
+            self.levels = torch.as_tensor(levels, dtype=torch.float32).contiguous().to(device)
         self.d, self.H, self.P, self.NP = head_dim, num_kv_heads, page_size, num_pages
         self.rot_kind, self.rot_block = rot_kind, rot_block
         self.quat = None  # the rotation's table: quaternions, or signs
@@ -118,12 +122,18 @@ class Cache:
         self.desc = CacheDesc(head_dim, num_kv_heads, page_size, num_pages, rot_kind, rot_block,
                               None if self.quat is None else self.quat.data_ptr(),
                               None if self.rope is None else self.rope.data_ptr(),
-                              0 if self.rope is None else int(self.rope.shape[0]), fmt)
+                              0 if self.rope is None else int(self.rope.shape[0]), fmt,
+                              None if self.levels is None else self.levels.data_ptr())
+
+    def code_row_bytes(self):
+        return self.d * {FMT_INT2: 2, FMT_INT3: 3}.get(self.fmt, 4) // 8
 
     def new_pools(self, device="cuda", fill=None):
-        """(codes uint8 [NP][H][P][d/2], params int32 [NP][H][P]) for one of K / V;
-        each params word is the binary16 pair (scale, minimum), scale in the low half."""
-        codes = torch.empty((self.NP, self.H, self.P, self.d // 2), dtype=torch.uint8, device=device)
+        """(codes uint8 [NP][H][P][d * bits / 8], params int32 [NP][H][P]) for one
+        of K / V; each params word is the binary16 pair (scale, minimum), scale in
+        the low half (MX FP4: the four block-scale bytes)."""
+        codes = torch.empty((self.NP, self.H, self.P, self.code_row_bytes()), dtype=torch.uint8,
+                            device=device)
         params = torch.empty((self.NP, self.H, self.P), dtype=torch.int32, device=device)
         if fill is not None:
             codes.fill_(fill)

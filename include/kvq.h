@@ -75,8 +75,9 @@ typedef enum {
 } kvq_rot_kind;
 
 /* Storage format of a rotated (token, head) row; both pools of a cache
- * share it, with the same pool shapes (codes [NP][H][P][d/2] bytes, one
- * 32-bit params word per row).
+ * share it: codes [NP][H][P][d * bits / 8] bytes (bits 4 except for the
+ * 2- and 3-bit formats), one 32-bit params word per row. Every format but
+ * INT4 needs head_dim 128.
  *  KVQ_FMT_INT4   token-wise asymmetric INT4 (SAW-INT4, Summary): codes
  *                 c = nearest of (x - m16)/s16 in [0, 15]; params (s16, m16).
  *  KVQ_FMT_MXFP4  microscaled FP4 (UltraQuant page, method section: FP4 KV
@@ -91,8 +92,22 @@ typedef enum {
  *                 Decode quantizes the rotated query to MX E4M3 (X =
  *                 floor(log2 amax) - 8 per 32 channels, nearest-even,
  *                 saturating at 448, sign kept) and takes QK on the tensor
- *                 cores' block-scaled MMA. head_dim 128 only. */
-typedef enum { KVQ_FMT_INT4 = 0, KVQ_FMT_MXFP4 = 1 } kvq_format;
+ *                 cores' block-scaled MMA. */
+typedef enum {
+  KVQ_FMT_INT4 = 0,
+  KVQ_FMT_MXFP4 = 1,
+  KVQ_FMT_INT2 = 2,  /* the INT4 rule with 2-bit codes (Q = 3 levels above zero;
+                        IsoQuant page, Abstract: bit widths {2, 3, 4}); a row's
+                        codes are a little-endian bit stream of d/4 bytes      */
+  KVQ_FMT_INT3 = 3,  /* 3-bit codes (Q = 7), 3d/8 bytes per row; the codes
+                        pool is [NP][H][P][d * bits / 8] for every format      */
+  KVQ_FMT_LUT4 = 4   /* a calibrated 16-entry level table in place of the
+                        uniform INT4 levels (UltraQuant page, method section:
+                        the refitted 16-entry table): the INT4 statistics, the
+                        code the index of the level t nearest to the exact
+                        RN(x - m16) * RN(1/s16) (ties to the lower index),
+                        x^ = t[c] s16 + m16                                    */
+} kvq_format;
 
 /* Bits OR-ed into *err_flags by the kernels. */
 #define KVQ_ERRF_PAGE 1 /* block-table entry outside [0, num_pages): page skipped */
@@ -141,7 +156,11 @@ typedef enum { KVQ_FMT_INT4 = 0, KVQ_FMT_MXFP4 = 1 } kvq_format;
  *               or past it is invalid (KVQ_ERRF_POS in an append, the row is
  *               skipped; KVQ_ERRF_LEN in a decode, the output is zero).
  *  format       a kvq_format: how a rotated row is stored (0, the token-wise
- *               INT4 of the pages, for a zero-initialised descriptor). */
+ *               INT4 of the pages, for a zero-initialised descriptor).
+ *  levels       KVQ_FMT_LUT4 only (NULL otherwise): device float [16], the
+ *               level table, strictly increasing, each level a multiple of
+ *               1/16 in [0, 15] (16 t an integer in [0, 240]); 4-byte aligned.
+ *               A table that breaks these rules gives unspecified codes. */
 typedef struct {
   int32_t head_dim;
   int32_t num_kv_heads;
@@ -153,6 +172,7 @@ typedef struct {
   const float* rope;
   int32_t rope_max_pos;
   int32_t format;
+  const float* levels;
 } kvq_cache_desc;
 
 /*

@@ -17,10 +17,10 @@ class Pair:
     the oracle, both started from the same sentinel bytes."""
 
     def __init__(self, d, H, P, NP, rot_kind, rot_block=0, quat=None, fill=0xAA,
-                 fmt=kvq.FMT_INT4):
+                 fmt=kvq.FMT_INT4, levels=None):
         self.fmt = fmt
-        self.gpu = kvq.Cache(d, H, P, NP, rot_kind, rot_block, quat, fmt=fmt)
-        self.orc = oracle.Cache(d, H, P, NP, rot_kind, rot_block, quat, fmt=fmt)
+        self.gpu = kvq.Cache(d, H, P, NP, rot_kind, rot_block, quat, fmt=fmt, levels=levels)
+        self.orc = oracle.Cache(d, H, P, NP, rot_kind, rot_block, quat, fmt=fmt, levels=levels)
         self.kc, self.kp = self.gpu.new_pools(fill=fill)
         self.vc, self.vp = self.gpu.new_pools(fill=fill)
         self.okc, self.okp = self.orc.alloc_pools(fill)
@@ -28,8 +28,8 @@ class Pair:
         self.err = torch.zeros(1, dtype=torch.int32, device="cuda")
 
     @classmethod
-    def for_workload(cls, w, fill=0xAA, fmt=kvq.FMT_INT4):
-        return cls(w.d, w.H, w.P, w.NP, w.rot_kind, w.rot_block, w.quat, fill, fmt)
+    def for_workload(cls, w, fill=0xAA, fmt=kvq.FMT_INT4, levels=None):
+        return cls(w.d, w.H, w.P, w.NP, w.rot_kind, w.rot_block, w.quat, fill, fmt, levels)
 
     def okp_pool(self):
         """The oracle's K params pool as its append writes it."""
@@ -84,9 +84,10 @@ class Pair:
         return out.cpu().numpy().astype(np.float64), int(self.err.item())
 
 
-def fill_workload(w, seqs=None, layer=0, oracle_too=True, fill=0xAA, fmt=kvq.FMT_INT4):
+def fill_workload(w, seqs=None, layer=0, oracle_too=True, fill=0xAA, fmt=kvq.FMT_INT4,
+                  levels=None):
     """Pair cache holding the workload's cached tokens of the given sequences."""
-    p = Pair.for_workload(w, fill, fmt)
+    p = Pair.for_workload(w, fill, fmt, levels)
     k, v, ts, tp = w.prefill_tokens(seqs, layer)
     e, oe = p.append(k, v, ts, tp, w.block_table, oracle_too=oracle_too)
     assert e == 0 and oe == 0

@@ -165,7 +165,7 @@ def test_cache_desc_mirrors_the_header_struct():
             assert t is ctypes.c_void_p, n
         else:
             assert f[-2] == "int32_t" and t is ctypes.c_int32, n
-    # the C layout on a 64-bit host: six int32, two pointers, two int32
+    # the C layout on a 64-bit host: six int32, two pointers, two int32, a pointer
     assert kvq.CacheDesc.quat.offset == 24 and kvq.CacheDesc.rope.offset == 32
     assert kvq.CacheDesc.rope_max_pos.offset == 40 and kvq.CacheDesc.format.offset == 44
-    assert ctypes.sizeof(kvq.CacheDesc) == 48
+    assert kvq.CacheDesc.levels.offset == 48 and ctypes.sizeof(kvq.CacheDesc) == 56
