@@ -65,7 +65,8 @@ def parse():
                     help="print one JSON line with the baseline comparisons (long-context INT4 with "
                          "and without rotation vs the binary16 cache; prefill append per Hadamard "
                          "block with reconstruction MSE) and exit")
-    ap.add_argument("--profile-case", choices=["append", "decode", "decode-mx"], default=None,
+    ap.add_argument("--profile-case", choices=["append", "decode", "decode-mx", "decode-int3",
+                                               "decode-lut4"], default=None,
                     help="run a short fixed case for an ncu capture (4 launches) and exit")
     ap.add_argument("--profile-block", type=int, default=128,
                     help="Hadamard block size of the append profile case (0: no rotation)")
@@ -505,8 +506,9 @@ def profile_case(which, block=128, workload="llama8b"):
     append = 4 bulk appends of one prefill layer (65536 tokens, Hadamard block
     `block`, 268 MB in, 71 MB out); decode = 4 decode calls of the
     Llama-3-8B-shaped layer (143 MB of INT4 pages) or of the long-context
-    70B-shaped one (285 MB) after filling its cache with one append; decode-mx
-    = the same decode calls over the microscaled FP4 cache."""
+    70B-shaped one (285 MB) after filling its cache with one append; decode-mx,
+    decode-int3, decode-lut4 = the same decode calls over the microscaled FP4,
+    3-bit and level-table caches."""
     from bit_rotated_kv_block_b200 import kvq, workloads
     torch.cuda.set_device(0)
     dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
@@ -515,8 +517,14 @@ def profile_case(which, block=128, workload="llama8b"):
     else:
         w = workloads.long70b() if workload == "long70b" else workloads.llama8b()
     k, v, ts, tp = w.prefill_tokens()
-    fmt = kvq.FMT_MXFP4 if which == "decode-mx" else kvq.FMT_INT4
-    c = kvq.Cache(w.d, w.H, w.P, w.NP, w.rot_kind, w.rot_block, fmt=fmt)
+    fmt = {"decode-mx": kvq.FMT_MXFP4, "decode-int3": kvq.FMT_INT3,
+           "decode-lut4": kvq.FMT_LUT4}.get(which, kvq.FMT_INT4)
+    levels = None
+    if fmt == kvq.FMT_LUT4:
+        from bit_rotated_kv_block_b200 import calibrate
+        levels = calibrate.calibrate_levels(np.random.default_rng(77).standard_normal((4000, w.d)),
+                                            w.rot_block)
+    c = kvq.Cache(w.d, w.H, w.P, w.NP, w.rot_kind, w.rot_block, fmt=fmt, levels=levels)
     kc, kp = c.new_pools(fill=0)
     vc, vp = c.new_pools(fill=0)
     K, V, TS, TP, BT = dev(k), dev(v), dev(ts), dev(tp), dev(w.block_table)
@@ -602,10 +610,11 @@ def workload_records(device, seed=0):
     * the ragged head_dim-256 workload (128 sequences, lengths 512-16384):
       one fused decode step (append + attention) with Hadamard b 256 and with
       the quaternion rotation;
-    * the microscaled FP4 format (E2M1 codes, UE8M0 block scales, decode QK
-      on the block-scaled tensor-core MMA) against INT4 on the Llama-shaped
-      layer: bulk append, fused decode step, reconstruction MSE; and on the
-      long-context decode.
+    * the cache formats against INT4 on the Llama-shaped layer -- microscaled
+      FP4 (E2M1 codes, UE8M0 block scales, decode QK on the block-scaled
+      tensor-core MMA), 3- and 2-bit codes and the calibrated level table
+      (decode QK on the integer tensor-core MMA): bulk append, fused decode
+      step, reconstruction MSE; FP4 also on the long-context decode.
     """
     from bit_rotated_kv_block_b200 import kvq, workloads
     dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(device)
@@ -734,9 +743,14 @@ def workload_records(device, seed=0):
         torch.cuda.empty_cache()
     res["ragged256_step"] = rec
 
-    # ---- the microscaled FP4 format on the Llama-shaped layer: bulk append,
-    # fused decode step, and the reconstruction MSE against INT4's
+    # ---- the cache formats on the Llama-shaped layer (INT4, microscaled FP4,
+    # 3- and 2-bit codes, the calibrated level table): bulk append, fused
+    # decode step, reconstruction MSE; bytes per token-head from each
+    # format's row size
+    from bit_rotated_kv_block_b200 import calibrate
     w = workloads.llama8b(seed=seed)
+    levels = calibrate.calibrate_levels(
+        np.random.default_rng([seed, 77]).standard_normal((4000, w.d)), w.rot_block)
     ts, tp = _all_tokens(w)
     K, V = _device_kv(w, len(ts), gen, device)
     TS, TP, BT = dev(ts), dev(tp), dev(w.block_table)
@@ -744,13 +758,17 @@ def workload_records(device, seed=0):
                        "Hadamard b 64"}
     Lc = int(w.seq_lens[0])
     lens_c = dev(np.full(w.S, Lc, np.int32))
-    for fmt, name in ((kvq.FMT_INT4, "int4"), (kvq.FMT_MXFP4, "mxfp4")):
-        c = kvq.Cache(w.d, w.H, w.P, w.NP, w.rot_kind, w.rot_block, device=device, fmt=fmt)
+    for fmt, name in ((kvq.FMT_INT4, "int4"), (kvq.FMT_MXFP4, "mxfp4"), (kvq.FMT_INT3, "int3"),
+                      (kvq.FMT_INT2, "int2"), (kvq.FMT_LUT4, "lut4_calibrated")):
+        c = kvq.Cache(w.d, w.H, w.P, w.NP, w.rot_kind, w.rot_block, device=device, fmt=fmt,
+                      levels=levels if fmt == kvq.FMT_LUT4 else None)
+        row_b = 2 * (c.code_row_bytes() + 4)  # K and V codes + params per token-head
         kc, kp = c.new_pools(device=device, fill=0)
         vc, vp = c.new_pools(device=device, fill=0)
         t = _device_time_us(lambda i: kvq.quantize_append(c, K, V, TS, TP, BT, kc, kp, vc, vp),
                             n=10)
-        r = {"append": _rate(len(ts) * w.H * APPEND_BYTES_PER_TOKEN_HEAD, t, peak)}
+        r = {"append": _rate(len(ts) * w.H * (4 * w.d + row_b), t, peak),
+             "bytes_per_token_head": row_b}
         mse = 0.0
         for codes, params, src in ((kc, kp, K), (vc, vp, V)):
             xh = kvq.dequantize_pages(c, lens_c, Lc, BT, codes, params, unrotate=True)
@@ -768,12 +786,13 @@ def workload_records(device, seed=0):
                          device=device)
         t = _device_time_us(lambda i: kvq.decode_step(c, q, kn, vn, lens, L, BT, kc, kp, vc, vp,
                                                       out=out, workspace=ws))
-        r["step"] = _rate(int(lens_np.sum()) * w.H * BYTES_PER_TOKEN_HEAD, t, peak)
+        r["step"] = _rate(int(lens_np.sum()) * w.H * row_b, t, peak)
         rec[name] = r
         del kc, kp, vc, vp, ws
         torch.cuda.empty_cache()
     del K, V
-    res["mxfp4_llama8b"] = rec
+    rec["levels"] = [float(x) for x in levels]
+    res["formats_llama8b"] = rec
     res["peak_gbs"] = peak
     res["nominal_gbs"] = NOMINAL_HBM_GBS
     return res

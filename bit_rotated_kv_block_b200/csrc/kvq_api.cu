@@ -23,6 +23,30 @@ int device_sm_count() {
   return n;
 }
 
+// CTAs of `kern` that fit on one SM at once, from its registers and shared
+// memory and the device's limits (the occupancy query reports one CTA for
+// the tensor-memory kernels although several run side by side).
+int resident_ctas_per_sm(const void* kern, int threads, size_t dyn_smem) {
+  cudaFuncAttributes fa;
+  int dev = 0, smem_sm = 0, res_blk = 0, regs_sm = 0, max_blk = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaFuncGetAttributes(&fa, kern) != cudaSuccess ||
+      cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) !=
+          cudaSuccess ||
+      cudaDeviceGetAttribute(&res_blk, cudaDevAttrReservedSharedMemoryPerBlock, dev) !=
+          cudaSuccess ||
+      cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev) !=
+          cudaSuccess ||
+      cudaDeviceGetAttribute(&max_blk, cudaDevAttrMaxBlocksPerMultiprocessor, dev) != cudaSuccess)
+    return 1;
+  const size_t per_blk = dyn_smem + fa.sharedSizeBytes + (size_t)res_blk;
+  int n = per_blk > 0 ? (int)((size_t)smem_sm / per_blk) : max_blk;
+  const int warps = (threads + 31) / 32;
+  const int regs_blk = warps * ((fa.numRegs * 32 + 255) / 256 * 256);
+  if (regs_blk > 0 && regs_sm / regs_blk < n) n = regs_sm / regs_blk;
+  if (n > max_blk) n = max_blk;
+  return n < 1 ? 1 : n;
+}
+
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 static bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 static bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }

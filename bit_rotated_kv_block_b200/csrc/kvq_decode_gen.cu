@@ -679,13 +679,9 @@ template <int BITS, bool LUT, int NB>
 static int gen_resident_ctas() {
   static int cached = -1;
   if (cached < 0) {
-    auto kern = decode_gen_kernel<BITS, LUT, NB>;
-    int blocks = 0;
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GenCfg<BITS>::SMEM);
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, kern, kGThreads,
-                                                      GenCfg<BITS>::SMEM) != cudaSuccess ||
-        blocks < 1)
-      blocks = 1;
+    const int blocks = resident_ctas_per_sm(
+        reinterpret_cast<const void*>(decode_gen_kernel<BITS, LUT, NB>), kGThreads,
+        GenCfg<BITS>::SMEM);
     const int sms = device_sm_count();
     cached = blocks * (sms > 0 ? sms : 148);
   }
@@ -707,7 +703,7 @@ DecodePlan decode_gen_plan(const kvq_cache_desc& d, int32_t S, int32_t Hq, int32
                        : d.format == KVQ_FMT_INT3 ? gen_resident<3, false>(G)
                                                   : gen_resident<4, true>(G);
   const int pairs = S * d.num_kv_heads > 0 ? S * d.num_kv_heads : 1;
-  int splits = (resident + pairs / 2) / pairs;
+  int splits = resident / pairs;  // a single wave of CTAs
   const int min_splits = (tiles + 63) / 64;
   if (splits < min_splits) splits = min_splits;
   if (splits < 1) splits = 1;

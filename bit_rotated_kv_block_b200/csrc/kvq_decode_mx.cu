@@ -572,13 +572,9 @@ template <int NB>
 static int mx_resident_ctas() {
   static int cached = -1;
   if (cached < 0) {
-    int blocks = 0;
-    cudaFuncSetAttribute(decode_mx_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         kMxSmem);
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, decode_mx_kernel<NB>, kMxThreads,
-                                                      kMxSmem) != cudaSuccess ||
-        blocks < 1)
-      blocks = 1;
+    const int blocks =
+        resident_ctas_per_sm(reinterpret_cast<const void*>(decode_mx_kernel<NB>), kMxThreads,
+                             kMxSmem);
     const int sms = device_sm_count();
     cached = blocks * (sms > 0 ? sms : 148);
   }
@@ -593,9 +589,9 @@ DecodePlan decode_mx_plan(const kvq_cache_desc& d, int32_t S, int32_t Hq, int32_
   const int G = Hq / (d.num_kv_heads > 0 ? d.num_kv_heads : 1);
   const int resident = G <= 4 ? mx_resident_ctas<1>() : mx_resident_ctas<2>();
   const int pairs = S * d.num_kv_heads;
-  // about one CTA per resident slot (a single wave), at least one split per
-  // 64 tiles
-  int splits = (resident + (pairs > 0 ? pairs : 1) / 2) / (pairs > 0 ? pairs : 1);
+  // at most one CTA per resident slot (a single wave: a second, partial one
+  // would double the time), at least one split per 64 tiles
+  int splits = resident / (pairs > 0 ? pairs : 1);
   const int min_splits = (tiles + 63) / 64;
   if (splits < min_splits) splits = min_splits;
   if (splits < 1) splits = 1;

@@ -12,6 +12,8 @@ namespace kvq {
 
 // Streaming multiprocessors of the current device (cached per device).
 int device_sm_count();
+// CTAs of `kern` (threads per CTA, dynamic shared memory) resident per SM.
+int resident_ctas_per_sm(const void* kern, int threads, size_t dyn_smem);
 
 int append_launch(const kvq_cache_desc& d, int32_t T, const void* k, const void* v,
                   int64_t tok_stride, const int32_t* token_seq, const int32_t* token_pos,
