@@ -92,9 +92,7 @@ __device__ __forceinline__ void gen_codes(const float (&x)[E], float m, float in
     const float t0 = __fsub_rn(x[i], m);
     uint32_t c;
     if (LUT) {
-      c = 0;
-#pragma unroll
-      for (int k = 0; k < 15; ++k) c += __fmaf_rn(t0, inv, -mid[k]) > 0.f ? 1u : 0u;
+      c = lut_code(t0, inv, mid);
     } else {
       c = __float_as_uint(__fmaf_rn(t0, inv, 12582912.0f)) & ((1u << BITS) - 1u);
     }

@@ -147,6 +147,23 @@ __device__ __forceinline__ uint32_t row_quantize_mx(float (&x)[RowQuantShape<D>:
   return packed;
 }
 
+// Index of the table level nearest to the exact product t0 * inv (ties to
+// the lower index), given the 15 sorted level midpoints: a four-step binary
+// search, each step decided exactly by the sign of one fused multiply-add
+// (t0 * inv - mid); the same count of midpoints below t0 * inv as a linear
+// scan. The next midpoint is picked with selects, so `mid` stays in registers.
+__device__ __forceinline__ uint32_t lut_code(float t0, float inv, const float (&mid)[15]) {
+  const bool b3 = __fmaf_rn(t0, inv, -mid[7]) > 0.f;
+  const float m2 = b3 ? mid[11] : mid[3];
+  const bool b2 = __fmaf_rn(t0, inv, -m2) > 0.f;
+  const float m1 = b3 ? (b2 ? mid[13] : mid[9]) : (b2 ? mid[5] : mid[1]);
+  const bool b1 = __fmaf_rn(t0, inv, -m1) > 0.f;
+  const float m0 = b3 ? (b2 ? (b1 ? mid[14] : mid[12]) : (b1 ? mid[10] : mid[8]))
+                      : (b2 ? (b1 ? mid[6] : mid[4]) : (b1 ? mid[2] : mid[0]));
+  const bool b0 = __fmaf_rn(t0, inv, -m0) > 0.f;
+  return (b3 ? 8u : 0u) | (b2 ? 4u : 0u) | (b1 ? 2u : 0u) | (b0 ? 1u : 0u);
+}
+
 // The 2-bit, 3-bit and level-table forms of the same rotated row (kvq.h,
 // KVQ_FMT_INT2 / INT3 / LUT4): the INT4 statistics with Q = 3, 7 or 15, each
 // code the nearest integer of the exact product RN(x - m16) * RN(1/s16) (one
@@ -191,10 +208,7 @@ __device__ __forceinline__ uint32_t row_quantize_gen(float (&x)[RowQuantShape<D>
 #pragma unroll
       for (int i = 0; i < CPL; ++i) {
         const float t0 = __fsub_rn(x[i], m);
-        uint32_t c = 0;
-#pragma unroll
-        for (int k = 0; k < 15; ++k) c += __fmaf_rn(t0, inv, -mid[k]) > 0.f ? 1u : 0u;
-        packed |= c << (4 * i);
+        packed |= lut_code(t0, inv, mid) << (4 * i);
       }
     } else {
       const uint32_t mask = (1u << bits) - 1u;
