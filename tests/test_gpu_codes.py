@@ -109,3 +109,24 @@ def test_llama8b_full_size_lut4_step():
     assert e == 0 and oe == 0
     p.assert_pools_equal()
     assert np.max(np.abs(out - ref)) <= TOL
+
+
+def test_format_arguments_are_checked():
+    # host-side rejections (status 1 invalid argument, 2 unsupported), nothing
+    # launched: an unknown format, the formats other than INT4 at head_dim 256,
+    # the table format without its table and a table given to another format
+    w = workload(workloads.ROT_HADAMARD, 64, S=1, ctx=32)
+    k, v, ts, tp = w.prefill_tokens()
+    for fmt, d, lv, want in ((7, 128, None, 1),
+                             (kvq.FMT_INT3, 256, None, 2),
+                             (kvq.FMT_LUT4, 128, None, 1),
+                             (kvq.FMT_INT2, 128, np.arange(16, dtype=np.float32),
+                              1)):
+        c = kvq.Cache(d, w.H, w.P, w.NP, workloads.ROT_HADAMARD, 64, fmt=fmt if fmt != 7 else 0,
+                      levels=lv)
+        c.desc.format = fmt
+        kc, kp = c.new_pools(fill=0)
+        kk = dev(np.zeros((len(ts), w.H, d), np.float16))
+        with pytest.raises(kvq.KvqError) as ei:
+            kvq.quantize_append(c, kk, kk, dev(ts), dev(tp), dev(w.block_table), kc, kp, kc, kp)
+        assert ei.value.status == want
