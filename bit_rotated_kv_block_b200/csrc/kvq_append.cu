@@ -256,7 +256,7 @@ __device__ __forceinline__ void quantize_row_part(const uint8_t* boxes, int box_
       }
       sbytes |= xb << (8 * g);
     }
-    if (TPR == 2) {  // the row's second thread holds blocks E/32 .. 2E/32 - 1
+    if constexpr (TPR == 2) {  // the row's second thread holds blocks E/32 .. 2E/32 - 1
       const uint32_t other = __shfl_xor_sync(pair_mask, sbytes, 1);
       if (my_part == 0) sbytes |= other << (8 * (E / 32));
     }
