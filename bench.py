@@ -297,26 +297,50 @@ def run_ours(args, world, rank, local):
     # end to end through the public API with host buffers: pinned inputs in,
     # result out, every step
     # the step's inputs (new K and V rows, queries) travel in one pinned
-    # buffer and one copy; the result comes back in one copy
+    # buffer and one copy; the result comes back in one copy. As a serving
+    # loop would, the copies run on their own streams (one per direction) and
+    # overlap the neighbouring steps' kernels: inputs and outputs are double
+    # buffered, step i reads input buffer i % 2 once its copy has landed and
+    # its result leaves while step i + 1 runs
     nk, nv, nq = ks.size, vs.size, q.size
     hin = torch.empty(nk + nv + nq, dtype=torch.float16).pin_memory()
     hin[:nk] = torch.from_numpy(ks.reshape(-1))
     hin[nk:nk + nv] = torch.from_numpy(vs.reshape(-1))
     hin[nk + nv:] = torch.from_numpy(q.reshape(-1))
-    din = torch.empty(nk + nv + nq, dtype=torch.float16, device=device)
-    SK = din[:nk].view(ks.shape)
-    SV = din[nk:nk + nv].view(vs.shape)
-    Q = din[nk + nv:].view(q.shape)
-    hout = torch.empty((S, Hq, d), dtype=torch.float32).pin_memory()
+    dins = [torch.empty(nk + nv + nq, dtype=torch.float16, device=device) for _ in range(2)]
+    views = [(dn[:nk].view(ks.shape), dn[nk:nk + nv].view(vs.shape), dn[nk + nv:].view(q.shape))
+             for dn in dins]
+    outs = [torch.empty((S, Hq, d), dtype=torch.float32, device=device) for _ in range(2)]
+    houts = [torch.empty((S, Hq, d), dtype=torch.float32).pin_memory() for _ in range(2)]
     h2d = hin.numel() * 2
-    d2h = hout.numel() * 4
+    d2h = houts[0].numel() * 4
     e2e_steps = min(steps, 500)
+    up, down = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    issued = [False, False]
 
     def e2e_step(i):
-        c, kc, kp, vc, vp = caches[i % 2]
-        din.copy_(hin, non_blocking=True)
-        kvq.decode_step(c, Q, SK, SV, LENS, L, BT, kc, kp, vc, vp, out=out, workspace=ws, err=err)
-        hout.copy_(out, non_blocking=True)
+        b = i % 2
+        c, kc, kp, vc, vp = caches[b]
+        with torch.cuda.stream(up):
+            if issued[b]:
+                up.wait_event(ev_done[b])  # step i - 2 has read this buffer
+            dins[b].copy_(hin, non_blocking=True)
+            ev_in[b].record(up)
+        stream.wait_event(ev_in[b])
+        if issued[b]:
+            stream.wait_event(ev_out[b])  # step i - 2's result has left this buffer
+        SKb, SVb, Qb = views[b]
+        kvq.decode_step(c, Qb, SKb, SVb, LENS, L, BT, kc, kp, vc, vp, out=outs[b], workspace=ws,
+                        err=err)
+        ev_done[b].record(stream)
+        with torch.cuda.stream(down):
+            down.wait_event(ev_done[b])
+            houts[b].copy_(outs[b], non_blocking=True)
+            ev_out[b].record(down)
+        issued[b] = True
 
     for i in range(3):
         e2e_step(i)
@@ -325,8 +349,14 @@ def run_ours(args, world, rank, local):
     a0 = torch.cuda.Event(enable_timing=True)
     a1 = torch.cuda.Event(enable_timing=True)
     a0.record(stream)
+    ev_start = torch.cuda.Event()
+    ev_start.record(stream)
+    up.wait_event(ev_start)  # no copy of the timed steps starts before the region
+    down.wait_event(ev_start)
     for i in range(e2e_steps):
         e2e_step(i)
+    stream.wait_event(ev_out[(e2e_steps - 1) % 2])  # the last result is on the host
+    stream.wait_event(ev_out[e2e_steps % 2])
     a1.record(stream)
     torch.cuda.synchronize()
     barrier(world)
