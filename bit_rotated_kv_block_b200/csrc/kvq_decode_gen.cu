@@ -99,6 +99,79 @@ __device__ __forceinline__ uint32_t lut_byte(const uint32_t (&lut)[4], uint32_t 
   return ((c & 8u) ? hi : lo) & 0xFFu;
 }
 
+// Bytes t[c0..c3] of a 16-byte table held in four registers, for the four
+// 4-bit codes of `sel` (code k in bits 4k..4k+3 of its low 16 bits), in
+// bytes 0-3: two 8-entry lookups (byte permutes of the low and high halves of
+// the table) and a byte mask from the codes' top bits (the sign-replicating
+// permute of 0x80 bytes gives 0xFF where a code is >= 8 and 0x80 elsewhere;
+// m & (m << 1 | 0x01010101) turns that into 0xFF / 0x00).
+__device__ __forceinline__ uint32_t lut16x4(const uint32_t (&t)[4], uint32_t sel) {
+  const uint32_t s7 = sel & 0x7777u;
+  const uint32_t lo = __byte_perm(t[0], t[1], s7);
+  const uint32_t hi = __byte_perm(t[2], t[3], s7);
+  uint32_t m;  // the PTX permute itself: __byte_perm ignores the selectors' top bits
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(m) : "r"(0x80808080u), "r"(0x80808080u), "r"(sel & 0xFFFFu));
+  const uint32_t mask = m & ((m << 1) | 0x01010101u);
+  return (hi & mask) | (lo & ~mask);
+}
+
+// Eight 4-bit codes (code i in bits 4i..4i+3) -> eight bytes in code order.
+__device__ __forceinline__ uint2 nibbles_to_bytes(uint32_t w) {
+  const uint32_t ev = w & 0x0F0F0F0Fu;         // codes 0, 2, 4, 6
+  const uint32_t od = (w >> 4) & 0x0F0F0F0Fu;  // codes 1, 3, 5, 7
+  return make_uint2(__byte_perm(ev, od, 0x5140), __byte_perm(ev, od, 0x7362));
+}
+
+// Eight 2-bit codes (bits 0-15) -> the same codes in 4-bit fields.
+__device__ __forceinline__ uint32_t crumbs_to_nibbles(uint32_t v) {
+  v &= 0xFFFFu;
+  v = (v | (v << 8)) & 0x00FF00FFu;
+  v = (v | (v << 4)) & 0x0F0F0F0Fu;
+  return (v | (v << 2)) & 0x33333333u;
+}
+
+// The 16 codes of channels [16 k, 16 k + 16) of one row as 16 bytes in
+// channel order (the code, or 16 t[code] for the table); `lo`, `hi`: the 64
+// bits starting at the block's first code (the low BITS * 16 used).
+template <int BITS, bool LUT>
+__device__ __forceinline__ void codes16_bytes(uint32_t lo, uint32_t hi, const uint32_t (&lut)[4],
+                                              uint32_t (&o)[4]) {
+  if (BITS == 4) {
+    if (LUT) {
+      o[0] = lut16x4(lut, lo);
+      o[1] = lut16x4(lut, lo >> 16);
+      o[2] = lut16x4(lut, hi);
+      o[3] = lut16x4(lut, hi >> 16);
+    } else {
+      const uint2 a = nibbles_to_bytes(lo), b = nibbles_to_bytes(hi);
+      o[0] = a.x; o[1] = a.y; o[2] = b.x; o[3] = b.y;
+    }
+  } else if (BITS == 2) {
+    const uint2 a = nibbles_to_bytes(crumbs_to_nibbles(lo));
+    const uint2 b = nibbles_to_bytes(crumbs_to_nibbles(lo >> 16));
+    o[0] = a.x; o[1] = a.y; o[2] = b.x; o[3] = b.y;
+  } else {  // 3 bits: code i at bits 3 i of the 48-bit field
+    const uint32_t w2[2] = {lo, hi};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t v = 0;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) v |= code_at<3, 2>(w2, 4 * q + b) << (8 * b);
+      o[q] = v;
+    }
+  }
+}
+
+// Bits [pos, pos + 32) of a little-endian word array (pos a compile-time
+// multiple of 16 after unrolling).
+template <int NW>
+__device__ __forceinline__ uint32_t bits32(const uint32_t (&w)[NW], int pos) {
+  const int i = pos >> 5, sh = pos & 31;
+  const uint32_t a = w[i];
+  const uint32_t b = i + 1 < NW ? w[i + 1] : 0u;
+  return sh ? __funnelshift_r(a, b, sh) : a;
+}
+
 // NB as in the FP4 decode (1: G <= 4, hi and lo weights in one MMA; 2: G <= 8).
 template <int BITS, bool LUT, int NB>
 __global__ void __launch_bounds__(kGThreads) decode_gen_kernel(const GenDecodeArgs a) {
@@ -309,18 +382,8 @@ __global__ void __launch_bounds__(kGThreads) decode_gen_kernel(const GenDecodeAr
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) {  // 16 channels per 16-byte chunk
         uint32_t o[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t v = 0;
-#pragma unroll
-          for (int b = 0; b < 4; ++b) {
-            const uint32_t c = code_at<BITS, NW>(w, 16 * ch + 4 * q + b);
-            uint32_t byte = c;
-            if (LUT) byte = lut_byte(lut, c);
-            v |= byte << (8 * b);
-          }
-          o[q] = v;
-        }
+        codes16_bytes<BITS, LUT>(bits32<NW>(w, 16 * BITS * ch), bits32<NW>(w, 16 * BITS * ch + 32),
+                                 lut, o);
         *reinterpret_cast<uint4*>(arow + ch * 128) = make_uint4(o[0], o[1], o[2], o[3]);
       }
     }
@@ -475,6 +538,14 @@ __global__ void __launch_bounds__(kGThreads) decode_gen_kernel(const GenDecodeAr
           cw[k][1] = s16[2];
         }
       }
+      // each token's 16 codes as 16 bytes in channel order (3-bit codes are
+      // taken one by one below: spreading them to bytes first costs more)
+      uint32_t cb[4][4];
+      if (BITS != 3) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) codes16_bytes<BITS, LUT>(cw[k][0], cw[k][1], lut, cb[k]);
+      }
+      const __half2 bias = __half2half2(__ushort_as_half((unsigned short)(0x6400u + C0)));
       float tacc[8][4];
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt)
@@ -488,17 +559,20 @@ __global__ void __launch_bounds__(kGThreads) decode_gen_kernel(const GenDecodeAr
 #pragma unroll
           for (int pp = 0; pp < 2; ++pp) {    // token pairs (A, B), (C, D)
             const int ci = 2 * mt + rr;
-            uint32_t va = code_at<BITS, 2>(cw[2 * pp], ci);
-            uint32_t vb = code_at<BITS, 2>(cw[2 * pp + 1], ci);
-            if (LUT) {
-              va = lut_byte(lut, va);
-              vb = lut_byte(lut, vb);
+            // byte ci of each token of the pair into bytes 0 and 2, then
+            // binary16 1024 + v (v < 1024 exact in the mantissa) minus 1024 + C0
+            uint32_t hv;
+            if (BITS == 3) {
+              hv = 0x64006400u | code_at<3, 2>(cw[2 * pp], ci) |
+                   (code_at<3, 2>(cw[2 * pp + 1], ci) << 16);
+            } else {
+              const uint32_t pr =
+                  __byte_perm(cb[2 * pp][ci >> 2], cb[2 * pp + 1][ci >> 2],
+                              (uint32_t)(ci & 3) | ((uint32_t)(4 + (ci & 3)) << 8));
+              asm("lop3.b32 %0, %1, %2, %3, 0xea;" : "=r"(hv) : "r"(pr), "r"(0x00FF00FFu),
+                  "r"(0x64006400u));
             }
-            // binary16 1024 + v (v < 1024 exact in the mantissa), minus 1024 + C0
-            const uint32_t hv = 0x64006400u | va | (vb << 16);
-            av[2 * pp + rr] = h2_as_u32(__hsub2(u32_as_h2(hv),
-                                                __half2half2(__ushort_as_half(
-                                                    (unsigned short)(0x6400u + C0)))));
+            av[2 * pp + rr] = h2_as_u32(__hsub2(u32_as_h2(hv), bias));
           }
         }
         if (NB == 1) {
