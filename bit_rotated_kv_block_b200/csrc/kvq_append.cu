@@ -209,13 +209,20 @@ __device__ __forceinline__ void quantize_row_part(const uint8_t* boxes, int box_
 
   // the two threads of a d = 256 row are lanes 2i, 2i+1 of one warp
   const unsigned pair_mask = 3u << ((threadIdx.x % kWarp) & ~1);
+  // For b a power of 4 the Hadamard scale 2^-(lg b)/2 is exact, and for the
+  // INT4 codes it is folded into the row's scalars instead of the E values:
+  // min and max of the scaled row are the scaled min and max, and with x the
+  // unscaled value, RN(x cb - m) * inv = RN(x - m / cb) * (inv cb) exactly
+  // (every operand a multiple of 2^-24 far above the subnormal range), so
+  // statistics, parameters and codes come out bit for bit the same.
+  constexpr bool FOLD = ROT == KVQ_ROT_HADAMARD && (LGB % 2) == 0 && FMT == kAppInt4;
   if (PRE && cs != nullptr) rope_regs<E>(x, cs + my_part * E);
   if (ROT == KVQ_ROT_HADAMARD) {
     if (fused1) {
-      hadamard_regs<E, LGB, true>(x, my_part, pair_mask);  // first stage done on load
+      hadamard_regs<E, LGB, true, !FOLD>(x, my_part, pair_mask);  // first stage done on load
     } else {
       if (PRE && qtbl != nullptr) sign_regs<E>(x, qtbl + my_part * E);
-      hadamard_regs<E, LGB, false>(x, my_part, pair_mask);
+      hadamard_regs<E, LGB, false, !FOLD>(x, my_part, pair_mask);
     }
   } else if (ROT == KVQ_ROT_QUAT_FAST) {
     quat_fast_regs<E>(x, qtbl, my_part * E);
@@ -286,6 +293,13 @@ __device__ __forceinline__ void quantize_row_part(const uint8_t* boxes, int box_
     mn = fminf(mn, __shfl_xor_sync(pair_mask, mn, 1));
     mx = fmaxf(mx, __shfl_xor_sync(pair_mask, mx, 1));
   }
+  // the folded scale cb = 2^-(LGB/2) and its inverse, both exact
+  const float cb = FOLD ? __int_as_float((127 - LGB / 2) << 23) : 1.0f;
+  const float rcb = FOLD ? __int_as_float((127 + LGB / 2) << 23) : 1.0f;
+  if (FOLD) {
+    mn = __fmul_rn(mn, cb);
+    mx = __fmul_rn(mx, cb);
+  }
   mn = __fadd_rn(mn, 0.0f);
   mx = __fadd_rn(mx, 0.0f);
   const __half m16 = __float2half_rd(mn);
@@ -296,8 +310,9 @@ __device__ __forceinline__ void quantize_row_part(const uint8_t* boxes, int box_
 
   uint32_t packed[E / 8];
   if (s != 0.0f) {
-    const float inv = __frcp_rn(s);
-    const uint64_t m2 = pk(m, m), inv2 = pk(inv, inv);
+    const float inv = __fmul_rn(__frcp_rn(s), cb);  // times cb: exact
+    const float mq = __fmul_rn(m, rcb);              // exact
+    const uint64_t m2 = pk(mq, mq), inv2 = pk(inv, inv);
     const uint64_t magic2 = pk(12582912.0f, 12582912.0f);  // 1.5 * 2^23
 #pragma unroll
     for (int c = 0; c < E / 8; ++c) {

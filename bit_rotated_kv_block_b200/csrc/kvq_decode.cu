@@ -20,23 +20,25 @@
 //     lanes j by shuffles. Each rotated head is then held as a fixed point
 //     qint = RN(qhat * 2^k), 2^k the power of two that brings the head's
 //     largest |qhat| just below 2^26 (so qhat * 2^k is exact in binary32),
-//     split into four signed 8-bit limbs (even channels as 16 qint).
+//     split into four signed 8-bit limbs (even channels of a code byte as
+//     16 qint_e - qint_o, odd ones as qint_o).
 //  2. The sequence's pages are dealt out to its splits as contiguous ranges
 //     of near-equal size. The warp streams its (page, KV head) chunks (codes
 //     + params of K and V, contiguous in the pool) into a 2-4 stage
 //     shared-memory ring with cp.async and runs both contractions on tensor
 //     cores (mma.sync):
 //       QK^T: m16n8k32 s8 x u8 -> s32, A = the query limbs (one row per
-//             (head, limb)), B = the K codes as bytes (even channels c, odd
-//             channels 16 c, one AND per word each); the limb dots
-//             recombine exactly into 16 sum_i (c_i - 8) qint_i, and the score
+//             (head, limb)), B = the K codes as bytes (even slots the low
+//             nibble c_e of a code byte, one AND per word; odd slots the
+//             byte itself, c_e + 16 c_o); the limb dots recombine exactly
+//             into 16 sum_i (c_i - 8) qint_i, and the score
 //               z = sm_scale log2(e) 2^-k (s_k dot + (m_k + 8 s_k) sum qint)
 //             is formed in binary32;
 //       PV:   m16n8k16 f16 x f16 -> f32, A = V codes transposed (channels x
 //             tokens) as c - 8, exact in binary16 (a logic operation and a
 //             half2 subtract per pair of codes after a byte interleave),
-//             B = p * s_v split into binary16 hi + lo; each 16-token product
-//             joins the running sum through a round-to-nearest add, and
+//             B = p * s_v split into binary16 hi + lo, accumulated in the
+//             tensor core's binary32 accumulators across the split;
 //             sum p (m_v + 8 s_v) is kept aside. Online softmax in base 2
 //             against a per-head reference maximum that moves only when a
 //             score exceeds it by more than 8.
@@ -407,9 +409,10 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : (GP == 8 ? 3
   // as a 26-bit fixed point qint = RN(qhat * 2^k) (2^k the power of two that
   // brings the head's largest |qhat| just below 2^26, so qhat * 2^k is exact
   // in binary32) and split into four signed 8-bit limbs for the int8 tensor
-  // cores. Even channels enter as 16 qint: the K codes of odd channels are
-  // then used in place as 16 c (the high nibble of each byte masked, never
-  // shifted), and the contraction gives 16 sum_i c_i qint_i exactly.
+  // cores. The code byte of channels (e, o) = (2i, 2i + 1) enters twice,
+  // masked to c_e against 16 qint_e - qint_o and whole (c_e + 16 c_o, never
+  // shifted) against qint_o, so the contraction gives 16 sum_i c_i qint_i
+  // exactly with one AND per word of codes.
   // score z = (s_k zs) dot_c + (m_k + 8 s_k) zq in base-2 logit units, with
   // dot_c = 16 sum_i (c_i - 8) qint_i = dot' - 128 qsum: centred codes keep
   // both terms near the score's own size instead of two large ones that
@@ -455,12 +458,20 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : (GP == 8 ? 3
       // each of the three low bytes), q = sum_k (T_k - 128 [k < 3]) 256^k for
       // the bytes T_k of t, so the signed limbs are the bytes of
       // t ^ 0x00808080, byte k = limb k (|q| <= 2^30 keeps the top limb in s8)
+      int qi[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        qi[c] = __float2int_rn(x[8 * kk + c] * mulf);
+        qs_l += qi[c];
+      }
+      // the K operand of an even slot is its byte's low nibble c_e, of an odd
+      // slot the whole byte c_e + 16 c_o: with 16 q_e - q_o against the first
+      // and q_o against the second, c_e q_o cancels and the pair contributes
+      // 16 (c_e q_e + c_o q_o) (|16 q_e - q_o| < 17 * 2^26 stays in 4 limbs)
       uint32_t u[8];
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        const int q = __float2int_rn(x[8 * kk + c] * mulf);
-        qs_l += q;
-        const int qe = (c & 1) ? q : q * 16;
+        const int qe = (c & 1) ? qi[c] : 16 * qi[c] - qi[c + 1];
         u[c] = (uint32_t)(qe + 0x808080) ^ 0x00808080u;
       }
       // limb `lb` (0 = lowest) of channels {o, o+2, o+4, o+6} as one s8x4 word
@@ -564,10 +575,9 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : (GP == 8 ? 3
           }
 #pragma unroll
           for (int kk = 0; kk < C::NKS8; ++kk) {
-            const uint32_t b0 = w[kk] & 0x0F0F0F0Fu;  // even channels: c
-            const uint32_t b1 = w[kk] & 0xF0F0F0F0u;  // odd channels: 16 c
+            const uint32_t b0 = w[kk] & 0x0F0F0F0Fu;  // even slots: c_e
 #pragma unroll
-            for (int t = 0; t < C::NQT; ++t) mma16832_s8u8(ci[t][nt], qa[t][kk], b0, b1);
+            for (int t = 0; t < C::NQT; ++t) mma16832_s8u8(ci[t][nt], qa[t][kk], b0, w[kk]);
           }
         }
         // dot' = 16 sum_i c_i qint_i of head hr with each of the lane's
@@ -736,15 +746,12 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : (GP == 8 ? 3
             av[1] = nib_c8(pr[0][1][sh], mask, e8 & 1);  // row slot r+8, k slots 0, 1
             av[2] = nib_c8(pr[1][0][sh], mask, e8 & 1);  // row slot r,   k slots 2, 3
             av[3] = nib_c8(pr[1][1][sh], mask, e8 & 1);  // row slot r+8, k slots 2, 3
-            // each 16-token product starts from zero and joins the running
-            // sum through a round-to-nearest add: the tensor core truncates
-            // every product against its accumulator, which, fed the running
-            // sum of non-negative terms, would bias the sum low
-            float t4[4] = {0.f, 0.f, 0.f, 0.f};
-            mma16816(t4, av, bh[0], bh[1]);
-            if (GP == 8) mma16816(t4, av, bl[0], bl[1]);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acc[mt][e] += t4[e];
+            // the running sum stays in the tensor core's accumulator: the
+            // centred codes keep it within 8 sum w, so its truncation per
+            // product (a unit in the last place of the accumulator) stays
+            // near 2^-20 of the weight sum over a whole split
+            mma16816(acc[mt], av, bh[0], bh[1]);
+            if (GP == 8) mma16816(acc[mt], av, bl[0], bl[1]);
           }
         }
       }

@@ -95,8 +95,9 @@ __device__ __forceinline__ void quat_regs(float (&x)[E], const float* tbl, int c
 // Full Hadamard rotation of a thread's E channels, block 2^LGB. Blocks wider
 // than E (b = 256 with E = 128) finish with one stage across the lane pair
 // (2i, 2i+1) given by pair_mask; part 0 holds the lower channels. With
-// STAGE1_DONE the first butterfly stage (h = 1) has already been applied.
-template <int E, int LGB, bool STAGE1_DONE = false>
+// STAGE1_DONE the first butterfly stage (h = 1) has already been applied;
+// without SCALE the 1/sqrt(b) factor is left to the caller.
+template <int E, int LGB, bool STAGE1_DONE = false, bool SCALE = true>
 __device__ __forceinline__ void hadamard_regs(float (&x)[E], int part, unsigned pair_mask) {
   constexpr int B = 1 << LGB;
   constexpr int LGIN = (B <= E) ? LGB : (E == 128 ? 7 : 6);
@@ -108,7 +109,7 @@ __device__ __forceinline__ void hadamard_regs(float (&x)[E], int part, unsigned 
       x[i] = part == 0 ? __fadd_rn(x[i], o) : __fsub_rn(o, x[i]);
     }
   }
-  scale_regs<E, LGB>(x, hadamard_scale(LGB));
+  if (SCALE) scale_regs<E, LGB>(x, hadamard_scale(LGB));
 }
 
 // Inverse quaternion rotation w -> conj(qL) w qR (the inverse of
