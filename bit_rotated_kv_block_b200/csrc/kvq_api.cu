@@ -57,6 +57,8 @@ static int check_desc(const kvq_cache_desc* d) {
   if (d->head_dim <= 0 || d->num_kv_heads <= 0 || d->page_size <= 0 || d->num_pages <= 0)
     return KVQ_ERR_INVALID_ARG;
   if (d->head_dim != 64 && d->head_dim != 128 && d->head_dim != 256) return KVQ_ERR_UNSUPPORTED;
+  // page strides of a pool (heads x page bytes) stay 32-bit products
+  if (d->num_kv_heads > 65536) return KVQ_ERR_UNSUPPORTED;
   if (d->page_size != 16 && d->page_size != 32 && d->page_size != 64) return KVQ_ERR_UNSUPPORTED;
   if (d->format < KVQ_FMT_INT4 || d->format > KVQ_FMT_LUT4) return KVQ_ERR_INVALID_ARG;
   if (d->format != KVQ_FMT_INT4 && d->head_dim != 128) return KVQ_ERR_UNSUPPORTED;

@@ -24,8 +24,9 @@
 //     16 qint_e - qint_o, odd ones as qint_o).
 //  2. The sequence's pages are dealt out to its splits as contiguous ranges
 //     of near-equal size. The warp streams its (page, KV head) chunks (codes
-//     + params of K and V, contiguous in the pool) into a 2-4 stage
-//     shared-memory ring with cp.async and runs both contractions on tensor
+//     + params of K and V, contiguous in the pool) into a two-stage
+//     shared-memory ring of 64-token stages (32 at d = 256) with cp.async
+//     and runs both contractions on tensor
 //     cores (mma.sync):
 //       QK^T: m16n8k32 s8 x u8 -> s32, A = the query limbs (one row per
 //             (head, limb)), B = the K codes as bytes (even slots the low
@@ -37,11 +38,11 @@
 //       PV:   m16n8k16 f16 x f16 -> f32, A = V codes transposed (channels x
 //             tokens) as c - 8, exact in binary16 (a logic operation and a
 //             half2 subtract per pair of codes after a byte interleave),
-//             B = p * s_v split into binary16 hi + lo, accumulated in the
-//             tensor core's binary32 accumulators across the split;
-//             sum p (m_v + 8 s_v) is kept aside. Online softmax in base 2
-//             against a per-head reference maximum that moves only when a
-//             score exceeds it by more than 8.
+//             B = p * s_v split into binary16 hi + lo, summed over a
+//             64-token stage in the tensor core and added to the running
+//             sum once per stage; sum p (m_v + 8 s_v) is kept aside.
+//             Online softmax in base 2 against a per-head reference maximum
+//             that moves only when a score exceeds it by more than 8.
 //  3. It writes (acc, max, sum) per query head to the workspace.
 // Merge kernel, one warp per (sequence, query head): combines the splits
 // (log-sum-exp), normalises, rotates back in registers and writes the
@@ -173,11 +174,14 @@ struct DecCfg {
   static constexpr int ROWB = D / 2;           // code bytes per token
   static constexpr int CODE_B = P * ROWB;      // code bytes per (page, head)
   static constexpr int PAGE_B = 2 * CODE_B + 8 * P;  // K codes, V codes, K and V params
-  static constexpr int PG = P == 16 ? 2 : 1;         // pages per pipeline stage
+  // pages per pipeline stage: 64 tokens at d = 128 (32 at d = 256), so a
+  // stage's fixed costs (copy issue, wait, page checks) spread over 4 (2)
+  // tiles whatever the page size
+  static constexpr int PG = (D == 128 ? 64 : 32) / P > 1 ? (D == 128 ? 64 : 32) / P : 1;
   static constexpr int TPG = TILES * PG;             // 16-token tiles per stage
   static constexpr int STAGE_B = PG * PAGE_B;
-  // pipeline depth: about 8-13 KB of pages in flight per warp
-  static constexpr int NST = STAGE_B <= 2304 ? 4 : (STAGE_B <= 4608 ? 3 : 2);
+  // pipeline depth: one stage (8.5 KB) in flight while the other computes
+  static constexpr int NST = 2;
   // behind the ring, for a fused decode step: the new token's binary16 K and
   // V rows as copied in, then its K and V code rows and parameter words,
   // kept until its page is staged
@@ -192,7 +196,7 @@ struct DecCfg {
 constexpr float kMaxSlack = 8.f;
 
 template <int D, int P, int GP>
-__global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : (GP == 8 ? 3 : 4))
+__global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : 3)
     decode_split_kernel(const DecodeArgs a) {
   static_assert(D == 128 || D == 256, "decode attention supports head_dim 128 and 256");
   using C = DecCfg<D, P, GP>;
@@ -288,7 +292,9 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : (GP == 8 ? 3
   constexpr int KU = C::CODE_B / 16;  // units of codes per pool (a multiple of 32)
   constexpr int PU = P / 4;           // units of params per pool (<= 16)
   static_assert(KU % kWarp == 0 && 2 * PU <= kWarp, "page block does not tile the warp");
-  const int64_t cstride = (int64_t)a.H * C::CODE_B, pstride = (int64_t)a.H * P * 4;
+  // page strides of the code and parameter pools (H * 8 KB at most: 32-bit
+  // products, widened once into the 64-bit address)
+  const uint32_t cstride = (uint32_t)a.H * C::CODE_B, pstride = (uint32_t)a.H * P * 4;
   const uint8_t* const kc_l = a.k_codes + (int64_t)h * C::CODE_B + lane * 16;
   const uint8_t* const vc_l = a.v_codes + (int64_t)h * C::CODE_B + lane * 16;
   const uint8_t* const par_l =
@@ -313,13 +319,13 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : (GP == 8 ? 3
       const int id = __shfl_sync(0xffffffffu, ids_a, (gn * C::PG + q) & 31);
       if (id < 0) continue;  // past the range or skipped
       okbits |= 1u << (slot * C::PG + q);
-      const int64_t co = (int64_t)id * cstride;
+      const uint64_t co = (uint64_t)(uint32_t)id * cstride;
       uint8_t* dst = ring + slot * C::STAGE_B + q * C::PAGE_B + lane * 16;
 #pragma unroll
       for (int m = 0; m < KU / kWarp; ++m) cp_async16(dst + m * 512, kc_l + co + m * 512);
 #pragma unroll
       for (int m = 0; m < KU / kWarp; ++m) cp_async16(dst + C::CODE_B + m * 512, vc_l + co + m * 512);
-      if (lane < 2 * PU) cp_async16(dst + 2 * C::CODE_B, par_l + (int64_t)id * pstride);
+      if (lane < 2 * PU) cp_async16(dst + 2 * C::CODE_B, par_l + (uint64_t)(uint32_t)id * pstride);
     }
     cp_async_commit();
   };
@@ -418,7 +424,7 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : (GP == 8 ? 3
   // both terms near the score's own size instead of two large ones that
   // cancel. 128 qsum = QA * 2^16 + QB (0 <= QB < 2^16) comes off the limb
   // halves before they are combined.
-  float zs, zq;
+  float zs, zq, zq8, zA, zB;
   int QA, QB;
   // A fragments per k-step kk: the lane's 8 channels j*QW + 8kk + [0, 8),
   // even ones in a[0]/a[1], odd ones in a[2]/a[3]. Rows:
@@ -501,6 +507,12 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : (GP == 8 ? 3
     qs_l += __shfl_xor_sync(0xffffffffu, qs_l, 2);
     zs = zk * 0.0625f;          // exact: the factor 16 of dot'
     zq = zk * (float)qs_l;      // sum of qint over the head's channels
+    zq8 = 8.f * zq;             // exact
+    // weights of the two halves of dot_c; for GP = 4 a lane's own half is
+    // the high one (r < 4) or the low one (r >= 4)
+    const float zhi = zs * 65536.f, zlo = zs;
+    zA = (GP == 4 && lo_row) ? zlo : zhi;
+    zB = (GP == 4 && lo_row) ? zhi : zlo;
     const long long q128 = qs_l * 128;  // |qsum| < 2^26 d: no overflow
     QA = (int)(q128 >> 16);             // floor division
     QB = (int)(q128 - ((long long)QA << 16));
@@ -563,10 +575,6 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : (GP == 8 ? 3
         int ci[C::NQT][2][4];
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-          for (int t = 0; t < C::NQT; ++t)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) ci[t][nt][e] = 0;
           uint32_t w[D / 32];
 #pragma unroll
           for (int u = 0; u < D / 128; ++u) {
@@ -577,41 +585,47 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : (GP == 8 ? 3
           for (int kk = 0; kk < C::NKS8; ++kk) {
             const uint32_t b0 = w[kk] & 0x0F0F0F0Fu;  // even slots: c_e
 #pragma unroll
-            for (int t = 0; t < C::NQT; ++t) mma16832_s8u8(ci[t][nt], qa[t][kk], b0, w[kk]);
+            for (int t = 0; t < C::NQT; ++t) {
+              if (kk == 0)
+                mma16832_s8u8_z(ci[t][nt], qa[t][kk], b0, w[kk]);
+              else
+                mma16832_s8u8(ci[t][nt], qa[t][kk], b0, w[kk]);
+            }
           }
         }
         // dot' = 16 sum_i c_i qint_i of head hr with each of the lane's
         // tokens: the limb dots combine as (l3*256 + l2) * 2^16 + (l1*256 + l0)
-        // halves of dot_c: l3*256 + l2 - QA and l1*256 + l0 - QB (|.| < 2^31)
-        int hA[NE], hB[NE];
+        // halves of dot_c: hA = l3*256 + l2 - QA and hB = l1*256 + l0 - QB
+        // (|.| < 2^31), weighted in binary32 by zA = 2^16 zs and zB = zs
+        float fA[NE], fB[NE];
         if (GP == 8) {
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int nt = e >> 1, c = e & 1;
-            hA[e] = ci[0][nt][c] * 256 + (ci[0][nt][2 + c] - QA);
-            hB[e] = ci[C::NQT - 1][nt][c] * 256 + (ci[C::NQT - 1][nt][2 + c] - QB);
+            fA[e] = (float)(ci[0][nt][c] * 256 + (ci[0][nt][2 + c] - QA));
+            fB[e] = (float)(ci[C::NQT - 1][nt][c] * 256 + (ci[C::NQT - 1][nt][2 + c] - QB));
           }
         } else {
-          // lanes r < 4 hold the (l3, l2) rows and form l3*256 + l2 - QA,
-          // lanes r + 4 the (l1, l0) rows and form l1*256 + l0 - QB, for both
-          // token halves; each sends its partner the half that partner scores
+          // lanes r < 4 hold the (l3, l2) rows and form hA, lanes r + 4 the
+          // (l1, l0) rows and form hB, for both token halves; each sends its
+          // partner the half that partner scores (zA, zB swap with the role)
           const int Qh = lo_row ? QB : QA;
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             const int loc0 = ci[0][0][c] * 256 + (ci[0][0][2 + c] - Qh);
             const int loc1 = ci[0][1][c] * 256 + (ci[0][1][2 + c] - Qh);
             const int got = __shfl_xor_sync(0xffffffffu, lo_row ? loc0 : loc1, 16);
-            const int mine = lo_row ? loc1 : loc0;
-            hA[c] = lo_row ? got : mine;
-            hB[c] = lo_row ? mine : got;
+            fA[c] = (float)(lo_row ? loc1 : loc0);  // this lane's own half
+            fB[c] = (float)got;
           }
         }
 #pragma unroll
         for (int e = 0; e < NE; ++e) {
-          const float dotf = fmaf((float)hA[e], 65536.f, (float)hB[e]);
+          // zs dot_c + 8 zq, then z = s (zs dot_c + 8 zq) + m zq
+          const float zd = fmaf(fA[e], zA, fmaf(fB[e], zB, zq8));
           const uint32_t kpw = *reinterpret_cast<const uint32_t*>(st + kps[e] + pofs);
           const float2 sm = __half22float2(u32_as_h2(kpw));  // (scale, min)
-          const float sc = fmaf(sm.x * zs, dotf, fmaf(8.f, sm.x, sm.y) * zq);
+          const float sc = fmaf(sm.x, zd, sm.y * zq);
           if (MASKED) {
             const int tok = tok0 + (tt / C::TILES) * P + (tt % C::TILES) * 16 + tks[e];
             z[tt][e] = tok < L ? sc : -INFINITY;
@@ -649,7 +663,20 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : (GP == 8 ? 3
         }
       }
 
-      // ---- PV per tile
+      // ---- PV per tile, summed over the stage's tiles in the tensor core
+      // from zero (the first tile's product writes the stage sum; a masked
+      // stage, whose first tile may be skipped, starts from explicit zeros)
+      // and then added to the running sum with one round-to-nearest add: the
+      // tensor core truncates each product sum against its accumulator, so
+      // the bias of a chain grows with its length, and a chain is kept to
+      // one stage whatever the length of the split
+      float t4[C::NMT][4];
+      if (MASKED) {
+#pragma unroll
+        for (int mt = 0; mt < C::NMT; ++mt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) t4[mt][e] = 0.f;
+      }
 #pragma unroll
       for (int tt = 0; tt < C::TPG; ++tt) {
         if (MASKED && !pgok[tt / C::TILES]) continue;
@@ -746,15 +773,18 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : (GP == 8 ? 3
             av[1] = nib_c8(pr[0][1][sh], mask, e8 & 1);  // row slot r+8, k slots 0, 1
             av[2] = nib_c8(pr[1][0][sh], mask, e8 & 1);  // row slot r,   k slots 2, 3
             av[3] = nib_c8(pr[1][1][sh], mask, e8 & 1);  // row slot r+8, k slots 2, 3
-            // the running sum stays in the tensor core's accumulator: the
-            // centred codes keep it within 8 sum w, so its truncation per
-            // product (a unit in the last place of the accumulator) stays
-            // near 2^-20 of the weight sum over a whole split
-            mma16816(acc[mt], av, bh[0], bh[1]);
-            if (GP == 8) mma16816(acc[mt], av, bl[0], bl[1]);
+            if (!MASKED && tt == 0)
+              mma16816_z(t4[mt], av, bh[0], bh[1]);
+            else
+              mma16816(t4[mt], av, bh[0], bh[1]);
+            if (GP == 8) mma16816(t4[mt], av, bl[0], bl[1]);
           }
         }
       }
+#pragma unroll
+      for (int mt = 0; mt < C::NMT; ++mt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[mt][e] += t4[mt][e];
     };
     if (full)
       body(std::false_type{});

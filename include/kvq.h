@@ -123,7 +123,7 @@ typedef enum {
 
 /* Geometry of one paged cache (both pools share it).
  *  head_dim     d: 64, 128 or 256.
- *  num_kv_heads H: >= 1.
+ *  num_kv_heads H: 1 .. 65536 (larger counts return KVQ_ERR_UNSUPPORTED).
  *  page_size    P: tokens per page; 16, 32 or 64.
  *  num_pages    NP: pool capacity in pages (>= 1).
  *  rot_kind     a kvq_rot_kind.
