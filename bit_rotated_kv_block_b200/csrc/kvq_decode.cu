@@ -62,6 +62,7 @@ constexpr int kDecWarps = 4;
 
 struct DecodeArgs {
   int S, Hq, H, G, P, NP, bt_stride, max_seq_len, splits;
+  int nhi;  // (sequence, KV head) pairs with `splits` splits; the rest have splits - 1
   int rot_kind, lgb;
   float scale2;   // sm_scale * log2(e)
   const __half* q;  // [S][Hq][D]
@@ -209,11 +210,24 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : 3)
   const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
   const int r = lane >> 2, j = lane & 3;
   const int item = blockIdx.x * kDecWarps + warp;
-  const int per_seq = a.H * a.splits;
-  if (item >= a.S * per_seq) return;
-  const int s = item / per_seq;
-  const int h = (item / a.splits) % a.H;
-  const int split = item % a.splits;
+  // items: the first nhi (sequence, KV head) pairs with `splits` splits
+  // each, then the others with splits - 1
+  const int hi_items = a.nhi * a.splits;
+  int pair, split, nspl;
+  if (item < hi_items) {
+    pair = item / a.splits;
+    split = item - pair * a.splits;
+    nspl = a.splits;
+  } else {
+    nspl = a.splits - 1;
+    const int r = item - hi_items;
+    const int k = nspl > 0 ? r / nspl : 0;
+    pair = a.nhi + k;
+    split = r - k * nspl;
+  }
+  if (pair >= a.S * a.H || nspl < 1) return;
+  const int s = pair / a.H;
+  const int h = pair - s * a.H;
   uint8_t* ring = smem + warp * C::WARP_B;
 
   // ---- independent loads first: the sequence length and the query rows
@@ -237,8 +251,8 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : 3)
   const int npages = (L + P - 1) / P;
   // this warp's pages: a contiguous range; the sequence's pages are dealt
   // out evenly over its splits (range sizes differ by at most one page)
-  const int pg_lo = (int)(((int64_t)split * npages) / a.splits);
-  const int pg_hi = (int)(((int64_t)(split + 1) * npages) / a.splits);
+  const int pg_lo = (int)(((int64_t)split * npages) / nspl);
+  const int pg_hi = (int)(((int64_t)(split + 1) * npages) / nspl);
   const int ngrp = (pg_hi - pg_lo + C::PG - 1) / C::PG;  // stage groups
   const int32_t* const bt_row = a.block_table + (int64_t)s * a.bt_stride;
   // fused step: the warp whose range holds the page of position L - 1
@@ -669,9 +683,11 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : 3)
       // and then added to the running sum with one round-to-nearest add: the
       // tensor core truncates each product sum against its accumulator, so
       // the bias of a chain grows with its length, and a chain is kept to
-      // one stage whatever the length of the split
+      // one stage whatever the length of the split. At d = 256 (no registers
+      // for a second set of sums) each tile's product is added on its own.
+      constexpr bool SSUM = D == 128;
       float t4[C::NMT][4];
-      if (MASKED) {
+      if (SSUM && MASKED) {
 #pragma unroll
         for (int mt = 0; mt < C::NMT; ++mt)
 #pragma unroll
@@ -773,18 +789,28 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : 3)
             av[1] = nib_c8(pr[0][1][sh], mask, e8 & 1);  // row slot r+8, k slots 0, 1
             av[2] = nib_c8(pr[1][0][sh], mask, e8 & 1);  // row slot r,   k slots 2, 3
             av[3] = nib_c8(pr[1][1][sh], mask, e8 & 1);  // row slot r+8, k slots 2, 3
-            if (!MASKED && tt == 0)
-              mma16816_z(t4[mt], av, bh[0], bh[1]);
-            else
-              mma16816(t4[mt], av, bh[0], bh[1]);
-            if (GP == 8) mma16816(t4[mt], av, bl[0], bl[1]);
+            if (SSUM) {
+              if (!MASKED && tt == 0)
+                mma16816_z(t4[mt], av, bh[0], bh[1]);
+              else
+                mma16816(t4[mt], av, bh[0], bh[1]);
+              if (GP == 8) mma16816(t4[mt], av, bl[0], bl[1]);
+            } else {
+              float u4[4];
+              mma16816_z(u4, av, bh[0], bh[1]);
+              if (GP == 8) mma16816(u4, av, bl[0], bl[1]);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) acc[mt][e] += u4[e];
+            }
           }
         }
       }
+      if (SSUM) {
 #pragma unroll
-      for (int mt = 0; mt < C::NMT; ++mt)
+        for (int mt = 0; mt < C::NMT; ++mt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) acc[mt][e] += t4[mt][e];
+          for (int e = 0; e < 4; ++e) acc[mt][e] += t4[mt][e];
+      }
     };
     if (full)
       body(std::false_type{});
@@ -853,7 +879,7 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : 3)
 // ---------------------------------------------------------------------------
 
 struct MergeArgs {
-  int S, Hq, splits, rot_kind, lgb;
+  int S, Hq, G, splits, nhi, rot_kind, lgb;
   const float* quat;
   const float* part;  // [S][Hq][splits][D + 4]
   float* out;         // [S][Hq][D]
@@ -913,18 +939,20 @@ __global__ void __launch_bounds__(kDecWarps * kWarp) decode_merge_kernel(const M
   const int gw = blockIdx.x * kDecWarps + threadIdx.x / kWarp;
   if (gw >= m.S * m.Hq) return;
   const float* src = m.part + (int64_t)gw * m.splits * (D + 4);
+  // the query head's (sequence, KV head) pair and its number of splits
+  const int nspl = gw / m.G < m.nhi ? m.splits : m.splits - 1;
   float Mr = -INFINITY, Ls = 0.f;
   float x[CPL];
 #pragma unroll
   for (int c = 0; c < CPL; ++c) x[c] = 0.f;
-  for (int i0 = 0; i0 < m.splits; i0 += RB) {
+  for (int i0 = 0; i0 < nspl; i0 += RB) {
     float4 f[RB][CPL / 4];
     float2 ml[RB];  // (M, L) of each split
 #pragma unroll
     for (int rb = 0; rb < RB; ++rb) {
       const int i = i0 + rb;
       const float* pi = src + (int64_t)i * (D + 4);
-      const bool in = i < m.splits;
+      const bool in = i < nspl;
       ml[rb] = in ? __ldcg(reinterpret_cast<const float2*>(pi + D)) : make_float2(-INFINITY, 0.f);
 #pragma unroll
       for (int c = 0; c < CPL / 4; ++c)
@@ -1013,17 +1041,32 @@ DecodePlan decode_plan(const kvq_cache_desc& d, int32_t S, int32_t Hq, int32_t m
   const int G = Hq / d.num_kv_heads;
   const int GP = G <= 4 ? 4 : 8;
   const int target = resident_warps(d.head_dim, P, GP);
-  const int pairs = S * d.num_kv_heads;
-  int splits = target / (pairs > 0 ? pairs : 1);
+  const int pairs = S * d.num_kv_heads > 0 ? S * d.num_kv_heads : 1;
+  // one wave of the resident warps: `extra` pairs get one split more than
+  // the others, so every resident slot holds a warp of near-equal work
+  // (whole splits per pair would leave up to pairs - 1 slots empty, and the
+  // SMs that hold one CTA more than the rest set the launch time)
+  int splits = target / pairs;
+  int extra = target - splits * pairs;
   // long contexts get at least one split per 256 pages: with lengths that
   // vary across the batch this puts more warps on the long sequences' pairs
   // (short pairs' warps leave the GPU early and the next CTAs take their place)
   const int min_splits = (pl.pages_max + 255) / 256;
-  if (splits < min_splits) splits = min_splits;
-  if (splits < 1) splits = 1;
-  if (splits > pl.pages_max) splits = pl.pages_max;
+  if (splits < min_splits) {
+    splits = min_splits;
+    extra = 0;
+  }
+  if (splits < 1) {
+    splits = 1;
+    extra = 0;
+  }
+  if (splits >= pl.pages_max) {
+    splits = pl.pages_max;
+    extra = 0;
+  }
+  pl.splits = extra > 0 ? splits + 1 : splits;
+  pl.nhi = extra > 0 ? extra : pairs;
   pl.pages_per_split = (pl.pages_max + splits - 1) / splits;
-  pl.splits = (pl.pages_max + pl.pages_per_split - 1) / pl.pages_per_split;
   pl.workspace = (size_t)S * Hq * pl.splits * (d.head_dim + 4) * sizeof(float);
   return pl;
 }
@@ -1034,7 +1077,7 @@ static cudaError_t launch_split(const DecodeArgs& a, cudaStream_t st) {
   const size_t smem = split_smem<D, P, GP>();
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const int items = a.S * a.H * a.splits;
+  const int items = a.nhi * a.splits + (a.S * a.H - a.nhi) * (a.splits - 1);
   const int grid = (items + kDecWarps - 1) / kDecWarps;
   e = launch_pdl(kern, grid, kDecWarps * kWarp, smem, st, a);
   if (e != cudaSuccess) return e;
@@ -1074,7 +1117,7 @@ int decode_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, const void* q,
 
   DecodeArgs a;
   a.S = S; a.Hq = Hq; a.H = d.num_kv_heads; a.G = G; a.P = d.page_size; a.NP = d.num_pages;
-  a.bt_stride = bt_stride; a.max_seq_len = max_seq_len; a.splits = pl.splits;
+  a.bt_stride = bt_stride; a.max_seq_len = max_seq_len; a.splits = pl.splits; a.nhi = pl.nhi;
   a.rot_kind = d.rot_kind; a.lgb = lgb;
   a.scale2 = (float)((double)sm_scale * 1.4426950408889634074);
   a.q = static_cast<const __half*>(q); a.quat = d.quat;
@@ -1095,16 +1138,17 @@ int decode_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, const void* q,
   cudaError_t e = launch_split_any(a, D, GP, st);
   if (e == cudaErrorInvalidValue) return KVQ_ERR_UNSUPPORTED;
   if (e != cudaSuccess) return KVQ_ERR_CUDA;
-  return decode_merge_launch(d, S, Hq, pl.splits, a.part, out, st);
+  return decode_merge_launch(d, S, Hq, pl.splits, pl.nhi, a.part, out, st);
 }
 
-int decode_merge_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, int splits,
+int decode_merge_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, int splits, int nhi,
                         const float* part, float* out, cudaStream_t st) {
   const int D = d.head_dim;
   int lgb = 0;
   while ((1 << lgb) < d.rot_block) ++lgb;
   MergeArgs mg;
-  mg.S = S; mg.Hq = Hq; mg.splits = splits; mg.rot_kind = d.rot_kind; mg.lgb = lgb;
+  mg.S = S; mg.Hq = Hq; mg.G = Hq / d.num_kv_heads; mg.splits = splits; mg.nhi = nhi;
+  mg.rot_kind = d.rot_kind; mg.lgb = lgb;
   mg.quat = d.quat; mg.part = part; mg.out = out;
   const int mgrid = (S * Hq + kDecWarps - 1) / kDecWarps;
   cudaError_t e = D == 128 ? launch_pdl(decode_merge_kernel<128>, mgrid, kDecWarps * kWarp, 0, st, mg)

@@ -427,6 +427,7 @@ DecodePlan decode_fp16_plan(const kvq_cache_desc& d, int32_t S, int32_t Hq, int3
   if (splits > pl.pages_max) splits = pl.pages_max;
   pl.pages_per_split = (pl.pages_max + splits - 1) / splits;
   pl.splits = (pl.pages_max + pl.pages_per_split - 1) / pl.pages_per_split;
+  pl.nhi = S * d.num_kv_heads;  // every pair has `splits` splits
   const size_t counters = (size_t)S * d.num_kv_heads * sizeof(int32_t);
   const size_t parts = (size_t)S * Hq * pl.splits * (d.head_dim + 4) * sizeof(float);
   pl.workspace = (counters + 255) / 256 * 256 + parts;

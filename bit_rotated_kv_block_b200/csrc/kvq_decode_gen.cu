@@ -784,6 +784,7 @@ DecodePlan decode_gen_plan(const kvq_cache_desc& d, int32_t S, int32_t Hq, int32
   if (splits > tiles) splits = tiles;
   pl.pages_per_split = (tiles + splits - 1) / splits;
   pl.splits = (tiles + pl.pages_per_split - 1) / pl.pages_per_split;
+  pl.nhi = S * d.num_kv_heads;  // every pair has `splits` splits
   pl.workspace = (size_t)S * Hq * pl.splits * (d.head_dim + 4) * sizeof(float);
   return pl;
 }
@@ -855,7 +856,7 @@ int decode_gen_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, const void
   else
     e = launch_gen<4, true>(a, grid, st);
   if (e != cudaSuccess) return KVQ_ERR_CUDA;
-  return decode_merge_launch(d, S, Hq, pl.splits, a.part, out, st);
+  return decode_merge_launch(d, S, Hq, pl.splits, S * d.num_kv_heads, a.part, out, st);
 }
 
 }  // namespace kvq

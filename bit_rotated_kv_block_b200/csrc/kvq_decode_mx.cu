@@ -598,6 +598,7 @@ DecodePlan decode_mx_plan(const kvq_cache_desc& d, int32_t S, int32_t Hq, int32_
   if (splits > tiles) splits = tiles;
   pl.pages_per_split = (tiles + splits - 1) / splits;
   pl.splits = (tiles + pl.pages_per_split - 1) / pl.pages_per_split;
+  pl.nhi = S * d.num_kv_heads;  // every pair has `splits` splits
   pl.workspace = (size_t)S * Hq * pl.splits * (d.head_dim + 4) * sizeof(float);
   return pl;
 }
@@ -657,7 +658,7 @@ int decode_mx_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, const void*
   e = launch_pdl(kern, S * d.num_kv_heads * pl.splits, kMxThreads, kMxSmem, st, a);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return KVQ_ERR_CUDA;
-  return decode_merge_launch(d, S, Hq, pl.splits, a.part, out, st);
+  return decode_merge_launch(d, S, Hq, pl.splits, S * d.num_kv_heads, a.part, out, st);
 }
 
 }  // namespace kvq

@@ -46,7 +46,10 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), int grid, int threads, siz
 
 struct DecodePlan {
   int pages_max;        // ceil(max_seq_len / P)
-  int splits;           // work items per (sequence, KV head)
+  int splits;           // work items per (sequence, KV head): the first `nhi`
+                        // (sequence, KV head) pairs have `splits`, the others
+                        // splits - 1 (so the total can match the resident warps)
+  int nhi;
   int pages_per_split;  // pages per split (contiguous ranges; an even share for interleaved groups)
   size_t workspace;     // bytes of partial results
 };
@@ -70,7 +73,9 @@ int decode_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, const void* q,
 
 // The merge kernel over split partial results [S][Hq][splits][d + 4] (the
 // running sums, then the base-2 maximum and total weight), rotated back.
-int decode_merge_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, int splits,
+// Query heads of the first `nhi` (sequence, KV head) pairs combine `splits`
+// partials, the others splits - 1.
+int decode_merge_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, int splits, int nhi,
                         const float* part, float* out, cudaStream_t st);
 
 // Decode attention over the microscaled FP4 cache (QK on the block-scaled
