@@ -63,6 +63,7 @@ constexpr int kDecWarps = 4;
 struct DecodeArgs {
   int S, Hq, H, G, P, NP, bt_stride, max_seq_len, splits;
   int nhi;  // (sequence, KV head) pairs with `splits` splits; the rest have splits - 1
+  int lead;  // pages the last split gives up to the others
   int rot_kind, lgb;
   float scale2;   // sm_scale * log2(e)
   const __half* q;  // [S][Hq][D]
@@ -251,8 +252,16 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : 3)
   const int npages = (L + P - 1) / P;
   // this warp's pages: a contiguous range; the sequence's pages are dealt
   // out evenly over its splits (range sizes differ by at most one page)
-  const int pg_lo = (int)(((int64_t)split * npages) / nspl);
-  const int pg_hi = (int)(((int64_t)(split + 1) * npages) / nspl);
+  // In a fused step the last split also quantizes the new token first: it
+  // takes `lead` pages fewer than an even share (as if the sequence had
+  // npages + lead pages and its last ones were that work), so it does not
+  // finish after the others. Plain decode attention uses the same ranges,
+  // so both calls sum in the same order. Short sequences keep even shares,
+  // so the last split always holds the last page.
+  const int lead = npages >= 4 * nspl ? a.lead : 0;
+  const int64_t vpages = (int64_t)npages + lead;
+  const int pg_lo = split == 0 ? 0 : (int)min((int64_t)npages, (split * vpages) / nspl);
+  const int pg_hi = split + 1 == nspl ? npages : (int)min((int64_t)npages, ((split + 1) * vpages) / nspl);
   const int ngrp = (pg_hi - pg_lo + C::PG - 1) / C::PG;  // stage groups
   const int32_t* const bt_row = a.block_table + (int64_t)s * a.bt_stride;
   // fused step: the warp whose range holds the page of position L - 1
@@ -1128,6 +1137,7 @@ int decode_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, const void* q,
   a.out = out;
   a.part = static_cast<float*>(workspace);
   a.err = err;
+  a.lead = (128 + d.page_size - 1) / d.page_size;  // 128 tokens: measured best of 48-208
   a.k_new = step ? static_cast<const __half*>(step->k_new) : nullptr;
   a.v_new = step ? static_cast<const __half*>(step->v_new) : nullptr;
   a.new_stride = step ? step->new_stride : 0;
