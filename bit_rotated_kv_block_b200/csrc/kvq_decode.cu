@@ -336,20 +336,28 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : 3)
       ++cidx;
       ids_b = load_ids(cidx + 1);
     }
-    okbits &= ~(((1u << C::PG) - 1) << (slot * C::PG));
+    // a page past the range or skipped (id < 0) is not read: its copies
+    // zero-fill from page 0's address and its okbits bit stays clear (no
+    // branch, so no divergence bookkeeping for a warp-uniform condition)
+    uint32_t okm = 0;
 #pragma unroll
     for (int q = 0; q < C::PG; ++q) {
       const int id = __shfl_sync(0xffffffffu, ids_a, (gn * C::PG + q) & 31);
-      if (id < 0) continue;  // past the range or skipped
-      okbits |= 1u << (slot * C::PG + q);
-      const uint64_t co = (uint64_t)(uint32_t)id * cstride;
+      const bool ok = id >= 0;
+      okm |= (uint32_t)ok << q;
+      const uint32_t idc = ok ? (uint32_t)id : 0u;
+      const uint32_t nb = ok ? 16u : 0u;
+      const uint64_t co = (uint64_t)idc * cstride;
       uint8_t* dst = ring + slot * C::STAGE_B + q * C::PAGE_B + lane * 16;
 #pragma unroll
-      for (int m = 0; m < KU / kWarp; ++m) cp_async16(dst + m * 512, kc_l + co + m * 512);
+      for (int m = 0; m < KU / kWarp; ++m) cp_async16_zf(dst + m * 512, kc_l + co + m * 512, nb);
 #pragma unroll
-      for (int m = 0; m < KU / kWarp; ++m) cp_async16(dst + C::CODE_B + m * 512, vc_l + co + m * 512);
-      if (lane < 2 * PU) cp_async16(dst + 2 * C::CODE_B, par_l + (uint64_t)(uint32_t)id * pstride);
+      for (int m = 0; m < KU / kWarp; ++m)
+        cp_async16_zf(dst + C::CODE_B + m * 512, vc_l + co + m * 512, nb);
+      if (lane < 2 * PU)
+        cp_async16_zf(dst + 2 * C::CODE_B, par_l + (uint64_t)idc * pstride, nb);
     }
+    okbits = (okbits & ~(((1u << C::PG) - 1) << (slot * C::PG))) | (okm << (slot * C::PG));
     cp_async_commit();
   };
 

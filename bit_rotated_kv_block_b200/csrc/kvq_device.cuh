@@ -113,6 +113,15 @@ __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src)
                "l"(gmem_src)
                : "memory");
 }
+// 16 bytes of which the first `src_bytes` (0 or 16) are read from global
+// memory and the rest zero-filled: a copy switched off without a branch
+// (gmem_src must still be a valid address).
+__device__ __forceinline__ void cp_async16_zf(void* smem_dst, const void* gmem_src,
+                                              uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)),
+               "l"(gmem_src), "r"(src_bytes)
+               : "memory");
+}
 __device__ __forceinline__ void cp_async8(void* smem_dst, const void* gmem_src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(smem_dst)),
                "l"(gmem_src)
