@@ -64,7 +64,8 @@ struct GenCfg {
 }  // namespace
 
 struct GenDecodeArgs {
-  int S, Hq, H, G, P, lg_page, NP, bt_stride, max_seq_len, splits, tiles_per_split;
+  int S, Hq, H, G, P, lg_page, NP, bt_stride, max_seq_len, splits;
+  int nhi;  // (sequence, KV head) pairs with `splits` splits; the rest have splits - 1
   int rot_kind, lgb;
   float scale2;
   const __half* q;
@@ -181,8 +182,21 @@ __global__ void __launch_bounds__(kGThreads) decode_gen_kernel(const GenDecodeAr
   constexpr int C0 = LUT ? 128 : (1 << (BITS - 1));  // centre, in operand units
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid / kWarp, lane = tid % kWarp;
-  const int split = blockIdx.x % a.splits;
-  const int sh = blockIdx.x / a.splits;
+  // blocks: the first nhi (sequence, KV head) pairs with `splits` splits
+  // each, then the others with splits - 1
+  const int hi_items = a.nhi * a.splits;
+  int sh, split, nspl;
+  if ((int)blockIdx.x < hi_items) {
+    sh = blockIdx.x / a.splits;
+    split = blockIdx.x - sh * a.splits;
+    nspl = a.splits;
+  } else {
+    nspl = a.splits - 1;
+    const int r = blockIdx.x - hi_items;
+    const int k = nspl > 0 ? r / nspl : 0;
+    sh = a.nhi + k;
+    split = r - k * nspl;
+  }
   const int h = sh % a.H, s = sh / a.H;
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::BAR_OFF + 8);
@@ -195,8 +209,9 @@ __global__ void __launch_bounds__(kGThreads) decode_gen_kernel(const GenDecodeAr
                       ((L + a.P - 1) >> a.lg_page) <= a.bt_stride &&
                       (a.rope == nullptr || L <= a.rope_max_pos);
   const int ntiles = len_ok ? (L + kGTile - 1) / kGTile : 0;
-  const int t0 = split * a.tiles_per_split;
-  const int t1 = min(ntiles, t0 + a.tiles_per_split);
+  // the sequence's tiles dealt out evenly over its splits
+  const int t0 = (int)(((int64_t)split * ntiles) / nspl);
+  const int t1 = (int)(((int64_t)(split + 1) * ntiles) / nspl);
   const int64_t base = ((int64_t)s * a.Hq + (int64_t)h * a.G) * a.splits + split;
   if (t0 >= t1) {
     if (!len_ok && split == 0 && h == 0 && tid == 0) raise_flag(a.err, KVQ_ERRF_LEN);
@@ -779,12 +794,24 @@ DecodePlan decode_gen_plan(const kvq_cache_desc& d, int32_t S, int32_t Hq, int32
   const int pairs = S * d.num_kv_heads > 0 ? S * d.num_kv_heads : 1;
   int splits = resident / pairs;  // a single wave of CTAs
   const int min_splits = (tiles + 63) / 64;
-  if (splits < min_splits) splits = min_splits;
-  if (splits < 1) splits = 1;
-  if (splits > tiles) splits = tiles;
+  // `extra` pairs get one split more, so the CTAs fill the resident slots
+  int extra = resident - splits * pairs;
+  if (splits < min_splits) {
+    splits = min_splits;
+    extra = 0;
+  }
+  if (splits < 1) {
+    splits = 1;
+    extra = 0;
+  }
+  if (splits >= tiles) {
+    splits = tiles;
+    extra = 0;
+  }
+  if (extra < 0) extra = 0;
   pl.pages_per_split = (tiles + splits - 1) / splits;
-  pl.splits = (tiles + pl.pages_per_split - 1) / pl.pages_per_split;
-  pl.nhi = S * d.num_kv_heads;  // every pair has `splits` splits
+  pl.splits = extra > 0 ? splits + 1 : splits;
+  pl.nhi = extra > 0 ? extra : S * d.num_kv_heads;
   pl.workspace = (size_t)S * Hq * pl.splits * (d.head_dim + 4) * sizeof(float);
   return pl;
 }
@@ -838,7 +865,7 @@ int decode_gen_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, const void
   GenDecodeArgs a;
   a.S = S; a.Hq = Hq; a.H = d.num_kv_heads; a.G = G; a.P = d.page_size; a.lg_page = lg_page;
   a.NP = d.num_pages; a.bt_stride = bt_stride; a.max_seq_len = max_seq_len;
-  a.splits = pl.splits; a.tiles_per_split = pl.pages_per_split;
+  a.splits = pl.splits; a.nhi = pl.nhi;
   a.rot_kind = d.rot_kind; a.lgb = lgb;
   a.scale2 = (float)((double)sm_scale * 1.4426950408889634074);
   a.q = static_cast<const __half*>(q); a.quat = d.quat;
@@ -848,7 +875,7 @@ int decode_gen_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, const void
   a.v_codes = v_codes; a.v_params = static_cast<const uint32_t*>(v_params);
   a.part = static_cast<float*>(workspace);
   a.err = err;
-  const int grid = S * d.num_kv_heads * pl.splits;
+  const int grid = pl.nhi * pl.splits + (S * d.num_kv_heads - pl.nhi) * (pl.splits - 1);
   if (d.format == KVQ_FMT_INT2)
     e = launch_gen<2, false>(a, grid, st);
   else if (d.format == KVQ_FMT_INT3)
@@ -856,7 +883,7 @@ int decode_gen_launch(const kvq_cache_desc& d, int32_t S, int32_t Hq, const void
   else
     e = launch_gen<4, true>(a, grid, st);
   if (e != cudaSuccess) return KVQ_ERR_CUDA;
-  return decode_merge_launch(d, S, Hq, pl.splits, S * d.num_kv_heads, a.part, out, st);
+  return decode_merge_launch(d, S, Hq, pl.splits, pl.nhi, a.part, out, st);
 }
 
 }  // namespace kvq
