@@ -256,8 +256,11 @@ __global__ void __launch_bounds__(kDecWarps * kWarp, D == 256 ? 2 : 3)
   // takes `lead` pages fewer than an even share (as if the sequence had
   // npages + lead pages and its last ones were that work), so it does not
   // finish after the others. Plain decode attention uses the same ranges,
-  // so both calls sum in the same order. Short sequences keep even shares,
-  // so the last split always holds the last page.
+  // so both calls sum in the same order. Sequences with fewer than 4 pages
+  // per split keep even shares. Between that and (n - 1) lead + n pages the
+  // last split can come out empty: the split before it then holds the last
+  // page and quantizes the new token (the owner is whichever split holds
+  // that page), and every page is still in exactly one range.
   const int lead = npages >= 4 * nspl ? a.lead : 0;
   const int64_t vpages = (int64_t)npages + lead;
   const int pg_lo = split == 0 ? 0 : (int)min((int64_t)npages, (split * vpages) / nspl);
