@@ -203,3 +203,25 @@ def test_calibration_is_a_lloyd_max_fixed_point_and_beats_uniform():
     mse_t = np.mean((u - t[cell]) ** 2)
     mse_u = np.mean((u - np.clip(np.rint(u), 0, 15)) ** 2)
     assert mse_t < mse_u
+
+
+def test_level_table_rounding_keeps_strictly_increasing_grid_levels():
+    # the decode's integer path needs 16 t integral and strictly increasing
+    # levels: crowded inputs move up one grid step, and down from the top
+    # when the grid runs out
+    lo = calibrate.round_to_grid(np.zeros(16))
+    assert np.array_equal(lo * 16, np.arange(16))
+    hi = calibrate.round_to_grid(np.full(16, 15.0))
+    assert np.array_equal(hi * 16, np.arange(225, 241))
+    g = np.random.default_rng(3)
+    for _ in range(200):
+        t = calibrate.round_to_grid(g.uniform(-2, 17, 16) ** g.choice([1, 2]) % 15.5)
+        assert t.dtype == np.float32 and np.all(np.diff(t) > 0)
+        assert np.all(t >= 0) and np.all(t <= 15) and np.all(t * 16 == np.round(t * 16))
+    # Lloyd-Max on 16 separated clusters (symmetric about the integers 1..14,
+    # point masses at 0 and 15) moves a perturbed start onto the cluster
+    # means, the integers
+    u = np.concatenate([k + np.linspace(-0.45, 0.45, 99) for k in range(1, 15)] +
+                       [np.zeros(99), np.full(99, 15.0)])
+    t = calibrate.lloyd_max(u, init=np.arange(16) + 0.04 * (-1.0) ** np.arange(16))
+    assert np.max(np.abs(t - np.arange(16))) < 1e-9
